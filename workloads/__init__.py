@@ -1,0 +1,142 @@
+"""Seeded synthetic inputs shaped like the pages' workloads.
+
+This module is shared by the tests, the oracle side and the benchmark.  It generates numbers and
+shapes only: it contains none of the attention arithmetic.  Every tensor is drawn in fp32 from a
+seeded generator, scaled, and rounded once to bf16 (round-to-nearest-even, done by
+``Tensor.to(torch.bfloat16)``); both the CUDA path and the oracle read that single copy (the
+oracle upcasts it to fp64, which is exact).
+
+Workloads (sizes from the pages: h_q = 32, d_h = 128, T = 8192 and the 32/8/1 KV-head sweep from
+the MHA/MQA/GQA walkthrough's parameter table; 64 query / 8 KV heads from 第三章 §3.3):
+
+* ``prefill_small``   causal prefill, B=1, h_q=4, h_kv=2, T=256, d_h=64, N(0,1).
+* ``decode_8k``       decode, B=8, h_q=32, d_h=128, T=8192, h_kv in {32, 8, 1}, N(0,1);
+                      the query sits at position 8191 and sees every key.
+* ``prefill_4k``      causal prefill, B=1, h_q=32, h_kv=8, T=4096, d_h=128, N(0,1)*0.5.
+* ``ragged_decode``   decode, B=64, h_q=64, h_kv=8, d_h=128, lengths uniform integers on
+                      [1024, 32768] (inclusive), cache allocated at 32768, tail filled with NaN.
+* ``chunked_prefill`` B=1, h_q=32, h_kv=8, d_h=128: 32256 cached positions, then 512 new
+                      queries at positions 32256..32767 over T=32768 after appending their K/V.
+"""
+
+from __future__ import annotations
+
+import dataclasses
+
+import numpy as np
+import torch
+
+DEFAULT_SEED = 0
+PAGES_SEED = 1949  # the seed the 第 09 章 checks were recorded with (§09.6)
+
+
+@dataclasses.dataclass(frozen=True)
+class PrefillShape:
+    B: int
+    h_q: int
+    h_kv: int
+    S_q: int
+    T_max: int
+    d_h: int
+    q_start: int
+    kv_len: int
+    std: float = 1.0
+
+
+@dataclasses.dataclass(frozen=True)
+class DecodeShape:
+    B: int
+    h_q: int
+    h_kv: int
+    T_max: int
+    d_h: int
+    std: float = 1.0
+    ragged: bool = False
+    len_lo: int = 0
+    len_hi: int = 0
+
+
+PREFILL_SMALL = PrefillShape(B=1, h_q=4, h_kv=2, S_q=256, T_max=256, d_h=64, q_start=0, kv_len=256)
+PREFILL_4K = PrefillShape(B=1, h_q=32, h_kv=8, S_q=4096, T_max=4096, d_h=128, q_start=0,
+                          kv_len=4096, std=0.5)
+CHUNKED_PREFILL = PrefillShape(B=1, h_q=32, h_kv=8, S_q=512, T_max=32768, d_h=128, q_start=32256,
+                               kv_len=32768)
+DECODE_8K = {h_kv: DecodeShape(B=8, h_q=32, h_kv=h_kv, T_max=8192, d_h=128) for h_kv in (32, 8, 1)}
+RAGGED_DECODE = DecodeShape(B=64, h_q=64, h_kv=8, T_max=32768, d_h=128, ragged=True,
+                            len_lo=1024, len_hi=32768)
+
+
+def ragged_lengths(seed: int, B: int = 64, lo: int = 1024, hi: int = 32768) -> np.ndarray:
+    """Per-request cached lengths, uniform integers on [lo, hi] inclusive."""
+    return np.random.default_rng(seed).integers(lo, hi + 1, size=B).astype(np.int32)
+
+
+def _generator(seed: int, device) -> torch.Generator:
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    return g
+
+
+def randn_bf16(shape, gen: torch.Generator, std: float = 1.0, device="cpu",
+               dtype=torch.bfloat16) -> torch.Tensor:
+    """N(0, std^2) drawn in fp32 from ``gen``, rounded once to ``dtype``."""
+    x = torch.randn(shape, generator=gen, dtype=torch.float32, device=device)
+    if std != 1.0:
+        x.mul_(std)
+    return x.to(dtype)
+
+
+def prefill_inputs(shape: PrefillShape, seed: int = DEFAULT_SEED, device="cpu",
+                   dtype=torch.bfloat16):
+    """Q (B,h_q,S_q,d_h) and the K/V cache (B,h_kv,T_max,d_h); draw order Q, K, V."""
+    g = _generator(seed, device)
+    q = randn_bf16((shape.B, shape.h_q, shape.S_q, shape.d_h), g, shape.std, device, dtype)
+    k = randn_bf16((shape.B, shape.h_kv, shape.T_max, shape.d_h), g, shape.std, device, dtype)
+    v = randn_bf16((shape.B, shape.h_kv, shape.T_max, shape.d_h), g, shape.std, device, dtype)
+    return q, k, v
+
+
+def chunked_prefill_inputs(shape: PrefillShape = CHUNKED_PREFILL, seed: int = DEFAULT_SEED,
+                           device="cpu", dtype=torch.bfloat16):
+    """Cache with positions < q_start filled (rest zero), the new K/V chunk and the new queries.
+
+    Draw order: K cache, V cache, K new, V new, Q.
+    """
+    g = _generator(seed, device)
+    B, h_kv, T, d = shape.B, shape.h_kv, shape.T_max, shape.d_h
+    k = torch.zeros((B, h_kv, T, d), dtype=dtype, device=device)
+    v = torch.zeros((B, h_kv, T, d), dtype=dtype, device=device)
+    k[:, :, :shape.q_start] = randn_bf16((B, h_kv, shape.q_start, d), g, shape.std, device, dtype)
+    v[:, :, :shape.q_start] = randn_bf16((B, h_kv, shape.q_start, d), g, shape.std, device, dtype)
+    k_new = randn_bf16((B, h_kv, shape.S_q, d), g, shape.std, device, dtype)
+    v_new = randn_bf16((B, h_kv, shape.S_q, d), g, shape.std, device, dtype)
+    q = randn_bf16((B, shape.h_q, shape.S_q, d), g, shape.std, device, dtype)
+    return k, v, k_new, v_new, q
+
+
+def decode_inputs(shape: DecodeShape, seed: int = DEFAULT_SEED, device="cpu",
+                  dtype=torch.bfloat16, nan_tail: bool = True):
+    """q (B,h_q,d_h), K/V cache (B,h_kv,T_max,d_h), kv_len (B,) int32.
+
+    Draw order: q, K, V.  For ragged shapes the positions at or beyond each request's length
+    are overwritten with NaN (a sentinel that must never reach an output).
+    """
+    g = _generator(seed, device)
+    q = randn_bf16((shape.B, shape.h_q, shape.d_h), g, shape.std, device, dtype)
+    k = randn_bf16((shape.B, shape.h_kv, shape.T_max, shape.d_h), g, shape.std, device, dtype)
+    v = randn_bf16((shape.B, shape.h_kv, shape.T_max, shape.d_h), g, shape.std, device, dtype)
+    if shape.ragged:
+        lens = ragged_lengths(seed, shape.B, shape.len_lo, shape.len_hi)
+        if nan_tail:
+            for b in range(shape.B):
+                k[b, :, int(lens[b]):] = float("nan")
+                v[b, :, int(lens[b]):] = float("nan")
+    else:
+        lens = np.full(shape.B, shape.T_max, np.int32)
+    kv_len = torch.from_numpy(lens).to(device)
+    return q, k, v, kv_len
+
+
+def to_f64(t: torch.Tensor) -> np.ndarray:
+    """Exact upcast of a (bf16 or fp32) tensor to a float64 NumPy array on the host."""
+    return t.detach().to("cpu").to(torch.float64).numpy()

@@ -1,0 +1,469 @@
+"""Benchmark: decode KV-read bandwidth (and causal prefill TFLOPS) of the GQA library on B200.
+
+Default workload (``decode_8k``): B=8, h_q=32, d_h=128, T=8192, swept over h_kv in {32, 8, 1}
+(MHA / GQA / MQA). One step = for each variant, one ``kv_append`` of the new token's K/V at
+position 8191 followed by one ``gqa_decode`` over the 8192 cached keys. ``value`` is the KV bytes
+the decodes must read (2 * B * h_kv * T * d_h * 2 per variant) divided by the device time of the
+whole step, in GB/s. L2 is flushed (a 256 MiB write) between steps, outside the timed events.
+
+``--impl reference`` times the fp64 CPU oracle on a bounded sample of the same workload.
+Run with no flags for N=1; under torchrun every rank runs an independent replica (the path needs
+no exchange between GPUs) and rank 0 prints one JSON line with the max-over-ranks time.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "GQA decode KV-read GB/s vs HBM peak; causal prefill TFLOPS vs bf16 peak"
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+L2_FLUSH_BYTES = 256 << 20
+
+
+# ---------------------------------------------------------------------------------------------
+# helpers
+# ---------------------------------------------------------------------------------------------
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), "measured"
+    return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, FALLBACK_BF16_TFLOPS, "fallback"
+
+
+def decode_kv_bytes(B, h_kv, lengths, d_h, s=2):
+    """Algorithmic KV bytes one decode reads: 2 * h_kv * len * d_h * s per sequence."""
+    return sum(2 * h_kv * int(n) * d_h * s for n in lengths)
+
+
+def prefill_flops(B, h_q, d_h, S_q, q_start, kv_len):
+    """Algorithmic causal prefill FLOPs: 4 * d_h per visible (query, key) pair per head."""
+    pairs = 0
+    for i in range(S_q):
+        pairs += min(kv_len, q_start + i + 1)
+    return 4 * d_h * B * h_q * pairs
+
+
+def source_digest(paths):
+    h = hashlib.sha256()
+    for p in sorted(paths):
+        h.update(open(os.path.join(ROOT, p), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(summary_name, digest):
+    """DRAM bytes per launch recorded in profiles/<summary_name> for the kernel source `digest`,
+    or None when absent or taken on a different version of the kernel."""
+    p = os.path.join(ROOT, "profiles", summary_name)
+    if not os.path.exists(p):
+        return None
+    text = open(p).read()
+    m = re.search(r"kernel_source_digest:\s*([0-9a-f]+)", text)
+    if not m or m.group(1) != digest:
+        return None
+    out = {}
+    for key, val in re.findall(r"traffic_bytes_per_launch\[([^\]]+)\]:\s*([0-9]+)", text):
+        out[key] = int(val)
+    return out or None
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu_index = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu_index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), parts))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        for _, _, p in rows:
+            for nm, v in zip(names, p[5:9]):
+                if v.lower() in ("active", "1"):
+                    reasons.add(nm)
+        busy = [r[0] for r in rows if r[0] > 0] or [r[0] for r in rows]
+        return {"sm_mhz": statistics.median(busy), "sm_max_mhz": max(r[1] for r in rows),
+                "samples": len(rows), "reasons": sorted(reasons)}
+
+
+# ---------------------------------------------------------------------------------------------
+# our implementation
+# ---------------------------------------------------------------------------------------------
+
+def run_ours(args, rank, world, dist):
+    import torch
+
+    import kv_cache_attention_gqa_b200 as gqa
+    import workloads
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    hbm_peak, tf_peak, tf_sust, peak_kind = load_peaks()
+
+    variants = []
+    for h_kv in (32, 8, 1):
+        shape = workloads.DECODE_8K[h_kv]
+        q, k, v, kv_len = workloads.decode_inputs(shape, seed=args.seed + rank, device=dev)
+        # the new token: its K/V row is appended at position T-1, then the query attends
+        g = torch.Generator(device=dev)
+        g.manual_seed(10_000 + args.seed + rank + h_kv)
+        k_new = torch.randn(shape.B, h_kv, 1, shape.d_h, generator=g, device=dev).to(torch.bfloat16)
+        v_new = torch.randn(shape.B, h_kv, 1, shape.d_h, generator=g, device=dev).to(torch.bfloat16)
+        pos = (kv_len - 1).contiguous()
+        out = torch.empty_like(q)
+        ws = torch.zeros(gqa.decode_workspace_size(shape.B, shape.h_q, h_kv, shape.T_max, shape.d_h),
+                         dtype=torch.uint8, device=dev)
+        variants.append(dict(h_kv=h_kv, shape=shape, q=q, k=k, v=v, kv_len=kv_len, k_new=k_new,
+                             v_new=v_new, pos=pos, out=out, ws=ws,
+                             bytes=decode_kv_bytes(shape.B, h_kv, [shape.T_max] * shape.B, shape.d_h)))
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def step(record=None):
+        for i, var in enumerate(variants):
+            gqa.kv_append(var["k"], var["v"], var["k_new"], var["v_new"], var["pos"])
+            if record is not None:
+                record[i][0].record(stream)
+            gqa.decode(var["q"], var["k"], var["v"], kv_len=var["kv_len"], out=var["out"], ws=var["ws"])
+            if record is not None:
+                record[i][1].record(stream)
+
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        step()
+    torch.cuda.synchronize()
+    if gqa.get_device_error() != 0:
+        raise RuntimeError("device error during warm-up")
+
+    E = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    step_ev = [(E(), E()) for _ in range(args.steps)]
+    dec_ev = [[(E(), E()) for _ in variants] for _ in range(args.steps)]
+    sampler = ClockSampler(local)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    t0 = time.perf_counter()
+    for s in range(args.steps):
+        flush.fill_(s & 0xFF)  # evict the caches from L2 (outside the step's events)
+        step_ev[s][0].record(stream)
+        step(dec_ev[s])
+        step_ev[s][1].record(stream)
+    torch.cuda.synchronize()
+    wall = time.perf_counter() - t0
+    clocks = sampler.stop()
+    if dist is not None:
+        dist.barrier()
+    step_ms = [a.elapsed_time(b) for a, b in step_ev]
+    dec_ms = [[a.elapsed_time(b) for a, b in row] for row in dec_ev]
+    total_ms = sum(step_ms)
+    if dist is not None:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    if gqa.get_device_error() != 0:
+        raise RuntimeError("device error during the timed steps")
+
+    step_bytes = sum(var["bytes"] for var in variants)
+    value = step_bytes * args.steps * world / (total_ms / 1e3) / 1e9
+    per_variant = {}
+    for i, var in enumerate(variants):
+        ms = statistics.mean(row[i] for row in dec_ms)
+        per_variant[f"h_kv={var['h_kv']}"] = {"decode_us": round(ms * 1e3, 2),
+                                              "kv_bytes": var["bytes"],
+                                              "GB_s": round(var["bytes"] / (ms / 1e3) / 1e9, 1),
+                                              "frac_of_hbm_peak": round(var["bytes"] / (ms / 1e3) / 1e9 / hbm_peak, 4)}
+    dec_total_ms = sum(sum(row) for row in dec_ms) / args.steps
+    achieved = step_bytes / (dec_total_ms / 1e3) / 1e9
+    digest = source_digest(["kv_cache_attention_gqa_b200/csrc/decode.cu", "kv_cache_attention_gqa_b200/csrc/common.cuh"])
+    traffic = recorded_traffic("decode_splitkv_decode_8k.md", digest)
+    traffic_per_launch = None
+    if traffic and all(f"h_kv={v['h_kv']}" in traffic for v in variants):
+        traffic_per_launch = round(sum(traffic[f"h_kv={v['h_kv']}"] for v in variants) / len(variants))
+    roofline = {"bound": "hbm", "kernel": "decode_bf16_kernel (split-KV decode + fused combine)",
+                "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
+                "frac": round(achieved / hbm_peak, 4), "peak_kind": f"hbm_gbs of {peak_kind}",
+                "traffic": traffic_per_launch,
+                "algorithmic_bytes_per_launch": round(step_bytes / len(variants)),
+                "kernel_source_digest": digest}
+
+    e2e = run_e2e(args, variants, dev, stream, dist, world)
+    prefill = run_prefill(args, dev, stream, tf_peak, peak_kind) if not args.skip_prefill else None
+
+    result = {
+        "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic: seeded N(0,1) bf16 (no dataset)",
+        "config": {"workload": "decode_8k: B=8, h_q=32, d_h=128, T=8192, h_kv in {32,8,1}; per step and variant one "
+                               "kv_append (1 token at position 8191) + one gqa_decode over 8192 keys",
+                   "B": 8, "h_q": 32, "d_h": 128, "T": 8192, "h_kv": [32, 8, 1],
+                   "l2": "flushed between steps (256 MiB write, outside the timed events)",
+                   "parallelism": f"replicas x{world} (no exchange)"},
+        "roofline": roofline,
+        "per_variant": per_variant,
+        "gpu_launches": args.steps * 2 * len(variants),
+        "clocks": clocks,
+        "e2e": e2e,
+        "wall_s_timed_region": round(wall, 3),
+    }
+    if prefill is not None:
+        result["prefill"] = prefill
+    if rank == 0 and world == 1 and not args.skip_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(args)
+    return result
+
+
+def run_e2e(args, variants, dev, stream, dist, world):
+    """The same step through the public API with host buffers: per step and variant, copy q and the
+    new K/V from pinned host memory, append + decode, copy O back to the host."""
+    import torch
+
+    import kv_cache_attention_gqa_b200 as gqa
+
+    host = []
+    for var in variants:
+        host.append(dict(q=var["q"].cpu().pin_memory(), kn=var["k_new"].cpu().pin_memory(),
+                         vn=var["v_new"].cpu().pin_memory(), o=torch.empty_like(var["out"], device="cpu").pin_memory(),
+                         qd=torch.empty_like(var["q"]), knd=torch.empty_like(var["k_new"]),
+                         vnd=torch.empty_like(var["v_new"])))
+    h2d = sum(h["q"].nbytes + h["kn"].nbytes + h["vn"].nbytes for h in host)
+    d2h = sum(h["o"].nbytes for h in host)
+
+    def step():
+        for var, h in zip(variants, host):
+            h["qd"].copy_(h["q"], non_blocking=True)
+            h["knd"].copy_(h["kn"], non_blocking=True)
+            h["vnd"].copy_(h["vn"], non_blocking=True)
+            gqa.kv_append(var["k"], var["v"], h["knd"], h["vnd"], var["pos"])
+            gqa.decode(h["qd"], var["k"], var["v"], kv_len=var["kv_len"], out=var["out"], ws=var["ws"])
+            h["o"].copy_(var["out"], non_blocking=True)
+
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for s in range(args.steps):
+        flush.fill_(s & 0xFF)
+        evs[s][0].record(stream)
+        step()
+        evs[s][1].record(stream)
+    torch.cuda.synchronize()
+    total = sum(a.elapsed_time(b) for a, b in evs)
+    if dist is not None:
+        t = torch.tensor([total], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total = float(t.item())
+    step_bytes = sum(var["bytes"] for var in variants)
+    return {"value": round(step_bytes * args.steps * world / (total / 1e3) / 1e9, 1), "unit": "GB/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "ms_per_step": round(total / args.steps, 4)}
+
+
+def run_prefill(args, dev, stream, tf_peak, peak_kind):
+    """Secondary line: causal prefill prefill_4k (B=1, h_q=32, h_kv=8, T=4096, d_h=128), TFLOPS."""
+    import torch
+
+    import kv_cache_attention_gqa_b200 as gqa
+    import workloads
+
+    shape = workloads.PREFILL_4K
+    q, k, v = workloads.prefill_inputs(shape, seed=args.seed, device=dev)
+    out = torch.empty_like(q)
+    try:
+        gqa.prefill(q, k, v, out=out)
+    except gqa.GQAError as e:
+        return {"unavailable": str(e)}
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    for _ in range(max(3, args.warmup)):
+        gqa.prefill(q, k, v, out=out)
+    torch.cuda.synchronize()
+    n = max(5, args.steps)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    for i in range(n):
+        flush.fill_(i & 0xFF)
+        evs[i][0].record(stream)
+        gqa.prefill(q, k, v, out=out)
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
+    flops = prefill_flops(1, 32, 128, 4096, 0, 4096)
+    tflops = flops / (ms / 1e3) / 1e12
+    return {"workload": "prefill_4k: B=1, h_q=32, h_kv=8, S_q=T=4096, d_h=128, causal",
+            "value": round(tflops, 1), "unit": "TFLOP/s", "ms": round(ms, 4),
+            "roofline": {"bound": "tensor", "achieved": round(tflops, 1), "peak": tf_peak, "unit": "TFLOP/s",
+                         "frac": round(tflops / tf_peak, 4), "peak_kind": f"bf16_tflops of {peak_kind}",
+                         "algorithmic_flops_per_launch": flops}}
+
+
+# ---------------------------------------------------------------------------------------------
+# the oracle on the host cores
+# ---------------------------------------------------------------------------------------------
+
+def _oracle_sample_inputs(seed=0):
+    import workloads
+
+    out = []
+    for h_kv in (32, 8, 1):
+        shape = workloads.DECODE_8K[h_kv]
+        small = workloads.DecodeShape(B=1, h_q=shape.h_q, h_kv=h_kv, T_max=shape.T_max, d_h=shape.d_h)
+        q, k, v, kv_len = workloads.decode_inputs(small, seed=seed)
+        out.append((h_kv, workloads.to_f64(q), workloads.to_f64(k), workloads.to_f64(v), kv_len.numpy()))
+    return out
+
+
+def _threads():
+    try:
+        from threadpoolctl import threadpool_info
+
+        n = [i.get("num_threads", 1) for i in threadpool_info()]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(args, budget_s=10.0):
+    """fp64 oracle on a bounded sample of decode_8k: sequence 0 of each h_kv variant, repeated
+    until about `budget_s` seconds of CPU work."""
+    import oracle
+
+    samples = _oracle_sample_inputs(args.seed)
+    nbytes, t_total, reps = 0, 0.0, 0
+    while t_total < budget_s and reps < 1000:
+        for h_kv, q, k, v, kv_len in samples:
+            t0 = time.perf_counter()
+            oracle.decode_ref(q, k, v, kv_len=kv_len)
+            t_total += time.perf_counter() - t0
+            nbytes += decode_kv_bytes(1, h_kv, kv_len, 128)
+        reps += 1
+    return {"value": round(nbytes / t_total / 1e9, 4), "unit": "GB/s", "cores": _threads(), "kind": "oracle",
+            "sample": f"decode_8k, sequence 0 of each h_kv variant (all 32 query heads, 8192 keys), "
+                      f"{reps} repetitions, {t_total:.1f} s of fp64 NumPy"}
+
+
+def run_reference(args, rank):
+    """The reference arm: the oracle, as it stands, on the host cores; one step = the decode of one
+    sequence of each h_kv variant (a bounded sample of decode_8k)."""
+    import oracle
+
+    samples = _oracle_sample_inputs(args.seed)
+    step_bytes = sum(decode_kv_bytes(1, h_kv, kv_len, 128) for h_kv, _, _, _, kv_len in samples)
+    for _ in range(args.warmup):
+        for h_kv, q, k, v, kv_len in samples:
+            oracle.decode_ref(q, k, v, kv_len=kv_len)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        for h_kv, q, k, v, kv_len in samples:
+            oracle.decode_ref(q, k, v, kv_len=kv_len)
+    dt = time.perf_counter() - t0
+    value = step_bytes * args.steps / dt / 1e9
+    sample = "decode_8k, sequence 0 of each h_kv variant (32 query heads, 8192 keys) per step, fp64 NumPy"
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic: seeded N(0,1) bf16 upcast to fp64",
+            "config": {"workload": "decode_8k: B=8, h_q=32, d_h=128, T=8192, h_kv in {32,8,1} (sampled)",
+                       "B": 8, "h_q": 32, "d_h": 128, "T": 8192, "h_kv": [32, 8, 1]},
+            "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": _threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+# ---------------------------------------------------------------------------------------------
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--skip-prefill", action="store_true")
+    ap.add_argument("--skip-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args, rank)), flush=True)
+        return
+
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as tdist
+
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        dist = tdist
+    try:
+        res = run_ours(args, rank, world, dist)
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+    finally:
+        if dist is not None:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,166 @@
+/*
+ * gqa.h - C ABI of the B200 (sm_100a) causal grouped-query attention library.
+ *
+ * The operation (all citations name the source page by title and section):
+ *
+ *   h_q query heads share h_kv K/V heads, h_q divisible by h_kv, r = h_q / h_kv. Query head a
+ *   reads K/V head g(a) = floor(a / r); the r heads of one group are adjacent
+ *   [序列计算与存储, section 分组查询注意力; 第 09 章 GQA、MLA 与跨层 KV 共享, section 09.2].
+ *   h_kv = h_q is MHA, h_kv = 1 is MQA [序列计算与存储, the head-sharing table].
+ *
+ *   O_a = softmax(Q_a K_{g(a)}^T * scale + M) V_{g(a)}
+ *   [序列计算与存储, display equation of section 分组查询注意力; section 分块注意力],
+ *   evaluated block by block with an online softmax (running max m, running sum l, rescaled
+ *   output u) so the score matrix never reaches memory [序列计算与存储, section 在线 softmax;
+ *   第三章：MHA 的局限与 MQA、GQA、Flash Attention, section 3.5].
+ *
+ *   M masks by absolute position and by length: query row i of sequence b sits at position
+ *   q_start[b] + i and sees key j iff j <= q_start[b] + i (causal) and j < kv_len[b]
+ *   [第 09 章, section 09.2 on ptr_current_pos; 第三章, section 3.3 on is_causal].
+ *
+ *   The K/V cache is kept unexpanded as (B, h_kv, T_max, d_h) [序列计算与存储, section 缓存字节].
+ *
+ * Conventions shared by every entry point:
+ *   - All tensors are dense, row-major (C order), with the shapes given per call. Element type is
+ *     bf16 (GQA_BF16) or fp32 (GQA_FP32, the check mode: scalar FFMA, no tensor cores).
+ *   - Tensor pointers are DEVICE pointers on the current CUDA device. Small integer arrays
+ *     (q_start, kv_len, q_pos, pos) are device int32 arrays of length B, or NULL for the default.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream). Every call is
+ *     asynchronous on that stream; the library keeps no per-request state and allocates nothing
+ *     per call (tensor-map descriptors are encoded on the host and passed by value).
+ *   - Buffers are owned by the caller. The library never frees or retains them after the call.
+ *   - Host-detectable argument errors return a status without launching anything. Errors that only
+ *     the device can see (a length or position out of range, a query with no visible key) never
+ *     trap: the kernel writes zeros for the affected output rows, records the first such error in
+ *     a sticky device word, and returns; read it with gqa_get_device_error().
+ */
+#ifndef GQA_B200_H
+#define GQA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  GQA_OK = 0,
+  GQA_ERR_INVALID_ARG = 1, /* null pointer, non-positive size, h_q % h_kv != 0, bad scale ...   */
+  GQA_ERR_UNSUPPORTED = 2, /* a valid request this build does not implement (e.g. bf16 d_h 96)  */
+  GQA_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed (launch, symbol, tensor map)      */
+  GQA_ERR_DEVICE = 4,      /* returned by gqa_get_device_error when the device word was set       */
+  GQA_ERR_WORKSPACE = 5    /* workspace pointer missing, too small or not 256-byte aligned        */
+} gqa_status;
+
+typedef enum {
+  GQA_BF16 = 0, /* bf16 in, fp32 accumulate (tcgen05 / mma), bf16 out                        */
+  GQA_FP32 = 1  /* check mode: fp32 in, fp32 scalar FFMA arithmetic, fp32 out                 */
+} gqa_dtype;
+
+/* Device error codes (the value of the sticky word read by gqa_get_device_error). */
+enum {
+  GQA_DEVERR_NONE = 0,
+  GQA_DEVERR_KV_LEN = 1,      /* kv_len[b] < 1 or kv_len[b] > T_max                               */
+  GQA_DEVERR_POSITION = 2,    /* q_start/q_pos < 0, or an append that does not fit in T_max       */
+  GQA_DEVERR_NO_VISIBLE = 3,  /* a query row that sees no key (e.g. q_start + i < 0 is impossible,
+                                 but kv_len = 0 with a valid position is)                          */
+  GQA_DEVERR_TIMEOUT = 4      /* a bounded pipeline wait ran out (the kernel returned early)      */
+};
+
+/*
+ * gqa_prefill - causal (or full) grouped-query attention of S_q new queries over a cache.
+ *
+ *   q        (B, h_q, S_q, d_h)    queries, already position-encoded.
+ *   k_cache  (B, h_kv, T_max, d_h) keys;   only rows j < kv_len[b] are read.
+ *   v_cache  (B, h_kv, T_max, d_h) values; only rows j < kv_len[b] are read.
+ *   o        (B, h_q, S_q, d_h)    output (written).
+ *   lse      (B, h_q, S_q) fp32 or NULL: natural-log sum over visible keys of exp(score * scale)
+ *            (the softmax normaliser; written when non-NULL).
+ *   q_start  device int32[B] or NULL (= all 0): absolute position of query row 0.
+ *   kv_len   device int32[B] or NULL (= all T_max): keys present, 1 <= kv_len[b] <= T_max.
+ *   scale    finite, > 0; pass 1/sqrt(d_h) for the standard scaling.
+ *   causal   1: key j visible to row i iff j <= q_start[b] + i and j < kv_len[b];
+ *            0: iff j < kv_len[b].
+ *   dtype    GQA_BF16: d_h in {64, 128}, tcgen05 tensor-core kernel (sm_100a);
+ *            GQA_FP32: 1 <= d_h <= 256, scalar check-mode kernel.
+ *
+ * A chunked prefill over an existing cache is kv_append(...) of the chunk's K/V at position p,
+ * then gqa_prefill with q_start[b] = p and kv_len[b] = p + S_q.
+ * Errors: INVALID_ARG (nulls, sizes <= 0, h_q % h_kv, scale), UNSUPPORTED (bf16 d_h), CUDA.
+ */
+gqa_status gqa_prefill(const void* q, const void* k_cache, const void* v_cache, void* o,
+                       float* lse, const int32_t* q_start, const int32_t* kv_len,
+                       int B, int h_q, int h_kv, int S_q, int T_max, int d_h,
+                       float scale, int causal, gqa_dtype dtype, void* stream);
+
+/*
+ * gqa_decode_workspace_size - bytes of device workspace gqa_decode needs for this shape with
+ * `num_splits` work partitions (0 = the automatic choice gqa_decode makes on the current device).
+ * The workspace holds per-partition partial results and one completion counter per
+ * (sequence, KV head) unit. It must be zero-filled before its first use; every gqa_decode call
+ * that completes leaves the counters at zero again, so it can be reused without clearing.
+ * Returns 0 on invalid arguments.
+ */
+size_t gqa_decode_workspace_size(int B, int h_q, int h_kv, int T_max, int d_h, gqa_dtype dtype,
+                                 int num_splits);
+
+/*
+ * gqa_decode - one new query per sequence attending over its cached keys (split-KV decode).
+ *
+ *   q        (B, h_q, d_h)          the new token's queries.
+ *   k_cache, v_cache (B, h_kv, T_max, d_h); rows j < min(kv_len[b], q_pos[b] + 1) are read,
+ *            each exactly once from HBM per call.
+ *   o        (B, h_q, d_h)          output.  lse: (B, h_q) fp32 or NULL, as in gqa_prefill.
+ *   kv_len   device int32[B] or NULL (= all T_max).
+ *   q_pos    device int32[B] or NULL (= kv_len[b] - 1: the token's own K/V was appended first,
+ *            so it sees every cached key [MHA/MQA/GQA walkthrough, section 4]).
+ *   workspace, workspace_bytes: caller-owned device memory, >= gqa_decode_workspace_size(...),
+ *            256-byte aligned, zero-filled before first use (see above). Calls that share one
+ *            workspace must not overlap in time (use one stream, or one workspace per stream).
+ *   num_splits: number of work partitions the visible keys of all (sequence, KV head) units are
+ *            cut into, contiguous and of equal size; 0 = automatic (one per SM). Results do not
+ *            depend on it beyond floating-point rounding.
+ *   dtype    GQA_BF16: d_h in {64, 128}; GQA_FP32: 1 <= d_h <= 256 (check mode).
+ * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA.
+ */
+gqa_status gqa_decode(const void* q, const void* k_cache, const void* v_cache, void* o, float* lse,
+                      const int32_t* kv_len, const int32_t* q_pos,
+                      int B, int h_q, int h_kv, int T_max, int d_h, float scale, gqa_dtype dtype,
+                      void* workspace, size_t workspace_bytes, int num_splits, void* stream);
+
+/*
+ * kv_append - copy new K/V rows into the cache: cache[b, g, pos[b] + t, :] = new[b, g, t, :]
+ * for t < S_new. Bit-exact; no other byte of the cache is written.
+ * [第三章, section 3.1: the new token's K/V join the cache; MHA/MQA/GQA walkthrough, section 4].
+ *
+ *   k_cache, v_cache (B, h_kv, T_max, d_h), written in place.
+ *   k_new, v_new     (B, h_kv, S_new, d_h), read.
+ *   pos      device int32[B] (required): first cache row written for sequence b.
+ *            Rows that would fall outside [0, T_max) are not written; the device error word is
+ *            set to GQA_DEVERR_POSITION.
+ *   dtype    element type of all four tensors (bf16: 2 bytes, fp32: 4 bytes); any d_h >= 1.
+ * Errors: INVALID_ARG, CUDA.
+ */
+gqa_status kv_append(void* k_cache, void* v_cache, const void* k_new, const void* v_new,
+                     const int32_t* pos, int B, int h_kv, int S_new, int T_max, int d_h,
+                     gqa_dtype dtype, void* stream);
+
+/*
+ * gqa_get_device_error - synchronise `stream`, then read and clear the sticky device error word
+ * of the current device. *code receives a GQA_DEVERR_* value. Returns GQA_ERR_DEVICE when the word
+ * was non-zero, GQA_OK when it was zero, GQA_ERR_CUDA if the read failed.
+ */
+gqa_status gqa_get_device_error(int* code, void* stream);
+
+/* Human-readable name of a status. Never NULL. */
+const char* gqa_status_string(gqa_status s);
+
+/* Library version string, e.g. "gqa-b200 0.1.0 (sm_100a)". */
+const char* gqa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GQA_B200_H */

@@ -1,0 +1,19 @@
+"""Causal grouped-query attention on B200 (sm_100a): prefill, split-KV decode and KV append.
+
+The computation lives in the CUDA library ``libgqa_b200.so`` behind the C ABI of
+``include/gqa.h``; this package is a thin ctypes binding over it (``_lib``) plus the build script
+(``build``). Importing the package fails if the library has not been built: there is no CPU path.
+"""
+
+from ._lib import (  # noqa: F401
+    GQAError,
+    LIB_PATH,
+    decode,
+    decode_workspace_size,
+    get_device_error,
+    kv_append,
+    prefill,
+    status_string,
+    version,
+    workspace,
+)

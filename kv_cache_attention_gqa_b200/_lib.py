@@ -1,0 +1,223 @@
+"""ctypes binding of the C ABI in ``include/gqa.h``: argument marshalling only.
+
+Every step of the computation runs in the CUDA library ``libgqa_b200.so``; this module checks
+tensor shapes and dtypes, allocates outputs with PyTorch (device memory is plumbing), passes raw
+device pointers and the current CUDA stream, and turns status codes into exceptions.  There is no
+fallback: if the library is missing, importing this module raises.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import threading
+
+import torch
+
+_PKG_DIR = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG_DIR, "libgqa_b200.so")
+
+GQA_OK = 0
+STATUS_NAMES = {
+    0: "GQA_OK",
+    1: "GQA_ERR_INVALID_ARG",
+    2: "GQA_ERR_UNSUPPORTED",
+    3: "GQA_ERR_CUDA",
+    4: "GQA_ERR_DEVICE",
+    5: "GQA_ERR_WORKSPACE",
+}
+GQA_BF16, GQA_FP32 = 0, 1
+DEVERR_NAMES = {0: "none", 1: "kv_len out of range", 2: "position out of range",
+                3: "query with no visible key", 4: "pipeline wait timed out"}
+
+# name -> (restype, argtypes), mirroring include/gqa.h
+_P, _I, _F, _Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+SIGNATURES = {
+    "gqa_prefill": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _I, _P]),
+    "gqa_decode_workspace_size": (_Z, [_I, _I, _I, _I, _I, _I, _I]),
+    "gqa_decode": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _P, _Z, _I, _P]),
+    "kv_append": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P]),
+    "gqa_get_device_error": (_I, [ctypes.POINTER(_I), _P]),
+    "gqa_status_string": (ctypes.c_char_p, [_I]),
+    "gqa_version": (ctypes.c_char_p, []),
+}
+
+
+class GQAError(RuntimeError):
+    """A non-OK status returned by the library."""
+
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn} returned {STATUS_NAMES.get(status, status)}")
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    if not os.path.exists(path):
+        raise ImportError(
+            f"{path} is missing: build it with `python -c 'import __graft_entry__ as g; g.build()'` "
+            "(or `python kv_cache_attention_gqa_b200/build.py`). There is no fallback implementation."
+        )
+    lib = ctypes.CDLL(path)
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+_lib = load_library()
+
+
+def _check(fn: str, status: int) -> None:
+    if status != GQA_OK:
+        raise GQAError(fn, status)
+
+
+def version() -> str:
+    return _lib.gqa_version().decode()
+
+
+def status_string(status: int) -> str:
+    return _lib.gqa_status_string(status).decode()
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return GQA_BF16
+    if t.dtype == torch.float32:
+        return GQA_FP32
+    raise TypeError(f"unsupported dtype {t.dtype}: bf16 (tensor-core path) or fp32 (check mode)")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is None:
+            continue
+        if not t.is_cuda:
+            raise ValueError("tensors must live on a CUDA device")
+        if not t.is_contiguous():
+            raise ValueError("tensors must be contiguous (row-major)")
+
+
+def _int_vec(x, B: int, device, name: str):
+    """Device int32[B] from None / int / sequence / tensor (None stays None = library default)."""
+    if x is None:
+        return None
+    if isinstance(x, int):
+        x = [x] * B
+    t = torch.as_tensor(x, dtype=torch.int32, device=device).contiguous()
+    if t.numel() != B:
+        raise ValueError(f"{name} must have {B} entries")
+    return t
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def get_device_error() -> int:
+    """Synchronise the current stream, read and clear the sticky device error word."""
+    code = ctypes.c_int(0)
+    st = _lib.gqa_get_device_error(ctypes.byref(code), _stream())
+    if st not in (GQA_OK, 4):
+        raise GQAError("gqa_get_device_error", st)
+    return code.value
+
+
+def kv_append(k_cache: torch.Tensor, v_cache: torch.Tensor, k_new: torch.Tensor,
+              v_new: torch.Tensor, pos) -> None:
+    """cache[b, g, pos[b] + t] = new[b, g, t] for t < S_new (in place, bit-exact)."""
+    _need_cuda(k_cache, v_cache, k_new, v_new)
+    B, h_kv, T_max, d_h = k_cache.shape
+    if v_cache.shape != k_cache.shape or k_new.shape != v_new.shape:
+        raise ValueError("shape mismatch")
+    if k_new.dim() != 4 or k_new.shape[0] != B or k_new.shape[1] != h_kv or k_new.shape[3] != d_h:
+        raise ValueError("k_new must be (B, h_kv, S_new, d_h)")
+    dt = _dtype_code(k_cache)
+    if any(t.dtype != k_cache.dtype for t in (v_cache, k_new, v_new)):
+        raise TypeError("all four tensors must share one dtype")
+    pos_t = _int_vec(pos, B, k_cache.device, "pos")
+    _check("kv_append", _lib.kv_append(_ptr(k_cache), _ptr(v_cache), _ptr(k_new), _ptr(v_new),
+                                       _ptr(pos_t), B, h_kv, k_new.shape[2], T_max, d_h, dt, _stream()))
+
+
+def prefill(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, *, q_start=None,
+            kv_len=None, scale: float | None = None, causal: bool = True, out=None,
+            return_lse: bool = False):
+    """Grouped-query attention of q (B, h_q, S_q, d_h) over the cache (B, h_kv, T_max, d_h)."""
+    _need_cuda(q, k_cache, v_cache, out)
+    B, h_q, S_q, d_h = q.shape
+    Bk, h_kv, T_max, dk = k_cache.shape
+    if (Bk, dk) != (B, d_h) or v_cache.shape != k_cache.shape:
+        raise ValueError("q / k_cache / v_cache shapes disagree")
+    dt = _dtype_code(q)
+    if k_cache.dtype != q.dtype or v_cache.dtype != q.dtype:
+        raise TypeError("q, k_cache and v_cache must share one dtype")
+    if out is None:
+        out = torch.empty_like(q)
+    lse = torch.empty((B, h_q, S_q), dtype=torch.float32, device=q.device) if return_lse else None
+    qs = _int_vec(q_start, B, q.device, "q_start")
+    kl = _int_vec(kv_len, B, q.device, "kv_len")
+    scale = 1.0 / math.sqrt(d_h) if scale is None else float(scale)
+    _check("gqa_prefill", _lib.gqa_prefill(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(out), _ptr(lse),
+                                           _ptr(qs), _ptr(kl), B, h_q, h_kv, S_q, T_max, d_h, scale,
+                                           1 if causal else 0, dt, _stream()))
+    return (out, lse) if return_lse else out
+
+
+def decode_workspace_size(B: int, h_q: int, h_kv: int, T_max: int, d_h: int, dtype=torch.bfloat16,
+                          num_splits: int = 0) -> int:
+    dt = GQA_BF16 if dtype == torch.bfloat16 else GQA_FP32
+    n = _lib.gqa_decode_workspace_size(B, h_q, h_kv, T_max, d_h, dt, num_splits)
+    if n == 0:
+        raise GQAError("gqa_decode_workspace_size", 1)
+    return n
+
+
+_ws_lock = threading.Lock()
+_ws_cache: dict = {}
+
+
+def workspace(nbytes: int, device) -> torch.Tensor:
+    """A zero-filled, 256-byte aligned device workspace of at least ``nbytes``, cached per device
+    and stream (the decode kernels leave it zeroed again after every completed call)."""
+    dev = torch.device(device)
+    key = (dev.index, torch.cuda.current_stream(dev).cuda_stream)
+    with _ws_lock:
+        buf = _ws_cache.get(key)
+        if buf is None or buf.numel() < nbytes:
+            buf = torch.zeros(max(nbytes, 1 << 20), dtype=torch.uint8, device=dev)
+            _ws_cache[key] = buf
+    return buf
+
+
+def decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, *, kv_len=None,
+           q_pos=None, scale: float | None = None, num_splits: int = 0, out=None,
+           return_lse: bool = False, ws: torch.Tensor | None = None):
+    """Split-KV decode of q (B, h_q, d_h) over the cache (B, h_kv, T_max, d_h)."""
+    _need_cuda(q, k_cache, v_cache, out)
+    B, h_q, d_h = q.shape
+    Bk, h_kv, T_max, dk = k_cache.shape
+    if (Bk, dk) != (B, d_h) or v_cache.shape != k_cache.shape:
+        raise ValueError("q / k_cache / v_cache shapes disagree")
+    dt = _dtype_code(q)
+    if k_cache.dtype != q.dtype or v_cache.dtype != q.dtype:
+        raise TypeError("q, k_cache and v_cache must share one dtype")
+    if out is None:
+        out = torch.empty_like(q)
+    lse = torch.empty((B, h_q), dtype=torch.float32, device=q.device) if return_lse else None
+    kl = _int_vec(kv_len, B, q.device, "kv_len")
+    qp = _int_vec(q_pos, B, q.device, "q_pos")
+    scale = 1.0 / math.sqrt(d_h) if scale is None else float(scale)
+    need = decode_workspace_size(B, h_q, h_kv, T_max, d_h, q.dtype, num_splits)
+    if ws is None:
+        ws = workspace(need, q.device)
+    _check("gqa_decode", _lib.gqa_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(out), _ptr(lse),
+                                         _ptr(kl), _ptr(qp), B, h_q, h_kv, T_max, d_h, scale, dt,
+                                         _ptr(ws), ws.numel(), num_splits, _stream()))
+    return (out, lse) if return_lse else out

@@ -1,0 +1,245 @@
+// C ABI of the library (declared in include/gqa.h): host-side argument checks, TMA descriptor
+// encoding and dispatch to the kernels. No per-call allocation; no per-request state.
+
+#include <cudaTypedefs.h>
+#include <math.h>
+#include <mutex>
+#include <string.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace gqa {
+
+// Sticky device error word (one per device that loads the library). Kernels receive its address.
+__device__ unsigned g_device_error_word;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+unsigned* device_error_ptr() {
+  static unsigned* ptrs[kMaxDevices] = {nullptr};
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!ptrs[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_error_word) != cudaSuccess) return nullptr;
+    ptrs[dev] = reinterpret_cast<unsigned*>(p);
+  }
+  return ptrs[dev];
+}
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return n;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// Encode a bf16 tensor map over a row-major matrix viewed as (rows, inner) with a 128-byte
+// swizzle. Dimensions are listed innermost first, as the driver expects.
+bool encode_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
+                 const uint64_t* strides_bytes, const uint32_t* box) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  uint32_t elem_strides[5] = {1, 1, 1, 1, 1};
+  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank,
+                        const_cast<void*>(base), dims, strides_bytes, box, elem_strides,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool valid_scale(float s) { return isfinite(s) && s > 0.f; }
+
+gqa_status from_cuda(cudaError_t e) { return e == cudaSuccess ? GQA_OK : GQA_ERR_CUDA; }
+
+}  // namespace
+
+int decode_auto_splits() { return sm_count(); }
+
+}  // namespace gqa
+
+using namespace gqa;
+
+extern "C" {
+
+const char* gqa_status_string(gqa_status s) {
+  switch (s) {
+    case GQA_OK: return "GQA_OK";
+    case GQA_ERR_INVALID_ARG: return "GQA_ERR_INVALID_ARG";
+    case GQA_ERR_UNSUPPORTED: return "GQA_ERR_UNSUPPORTED";
+    case GQA_ERR_CUDA: return "GQA_ERR_CUDA";
+    case GQA_ERR_DEVICE: return "GQA_ERR_DEVICE";
+    case GQA_ERR_WORKSPACE: return "GQA_ERR_WORKSPACE";
+  }
+  return "GQA_ERR_UNKNOWN";
+}
+
+const char* gqa_version(void) { return "gqa-b200 0.1.0 (sm_100a)"; }
+
+gqa_status gqa_get_device_error(int* code, void* stream) {
+  if (!code) return GQA_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  unsigned v = 0;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return GQA_ERR_CUDA;
+  if (cudaMemcpyFromSymbol(&v, g_device_error_word, sizeof(v)) != cudaSuccess) return GQA_ERR_CUDA;
+  *code = (int)v;
+  if (v != 0) {
+    const unsigned zero = 0;
+    if (cudaMemcpyToSymbol(g_device_error_word, &zero, sizeof(zero)) != cudaSuccess)
+      return GQA_ERR_CUDA;
+    return GQA_ERR_DEVICE;
+  }
+  return GQA_OK;
+}
+
+gqa_status kv_append(void* k_cache, void* v_cache, const void* k_new, const void* v_new,
+                     const int32_t* pos, int B, int h_kv, int S_new, int T_max, int d_h,
+                     gqa_dtype dtype, void* stream) {
+  if (!k_cache || !v_cache || !k_new || !v_new || !pos) return GQA_ERR_INVALID_ARG;
+  if (B <= 0 || h_kv <= 0 || S_new < 0 || T_max <= 0 || d_h <= 0) return GQA_ERR_INVALID_ARG;
+  if (dtype != GQA_BF16 && dtype != GQA_FP32) return GQA_ERR_INVALID_ARG;
+  if (S_new > T_max) return GQA_ERR_INVALID_ARG;
+  AppendArgs a;
+  a.k_cache = k_cache;
+  a.v_cache = v_cache;
+  a.k_new = k_new;
+  a.v_new = v_new;
+  a.pos = pos;
+  a.B = B;
+  a.h_kv = h_kv;
+  a.S_new = S_new;
+  a.T_max = T_max;
+  a.d_h = d_h;
+  a.elem_bytes = dtype == GQA_BF16 ? 2 : 4;
+  a.err = device_error_ptr();
+  if (!a.err) return GQA_ERR_CUDA;
+  return from_cuda(launch_kv_append(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+gqa_status gqa_prefill(const void* q, const void* k_cache, const void* v_cache, void* o,
+                       float* lse, const int32_t* q_start, const int32_t* kv_len,
+                       int B, int h_q, int h_kv, int S_q, int T_max, int d_h,
+                       float scale, int causal, gqa_dtype dtype, void* stream) {
+  if (!q || !k_cache || !v_cache || !o) return GQA_ERR_INVALID_ARG;
+  if (B <= 0 || h_q <= 0 || h_kv <= 0 || S_q <= 0 || T_max <= 0 || d_h <= 0)
+    return GQA_ERR_INVALID_ARG;
+  if (h_q % h_kv != 0 || !valid_scale(scale)) return GQA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return GQA_ERR_INVALID_ARG;
+  PrefillArgs a;
+  a.q = q;
+  a.k = k_cache;
+  a.v = v_cache;
+  a.o = o;
+  a.lse = lse;
+  a.q_start = q_start;
+  a.kv_len = kv_len;
+  a.B = B;
+  a.h_q = h_q;
+  a.h_kv = h_kv;
+  a.S_q = S_q;
+  a.T_max = T_max;
+  a.d_h = d_h;
+  a.scale = scale;
+  a.causal = causal;
+  a.err = device_error_ptr();
+  if (!a.err) return GQA_ERR_CUDA;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (dtype == GQA_FP32) {
+    if (d_h > 256) return GQA_ERR_UNSUPPORTED;
+    return from_cuda(launch_prefill_fp32(a, s));
+  }
+  if (dtype != GQA_BF16) return GQA_ERR_INVALID_ARG;
+  if (d_h != 64 && d_h != 128) return GQA_ERR_UNSUPPORTED;
+  if ((long long)B * h_kv * T_max >= (1ll << 31) || (long long)B * h_q * S_q >= (1ll << 31))
+    return GQA_ERR_UNSUPPORTED;
+  // TMA views: Q as rows (B*h_q*S_q, d_h); K, V as rows (B*h_kv*T_max, d_h); 64-column boxes.
+  CUtensorMap maps[3];
+  const uint64_t qdims[2] = {(uint64_t)d_h, (uint64_t)B * h_q * S_q};
+  const uint64_t kdims[2] = {(uint64_t)d_h, (uint64_t)B * h_kv * T_max};
+  const uint64_t strides[1] = {(uint64_t)d_h * 2};
+  const uint32_t box[2] = {64, 128};
+  if (!encode_bf16(&maps[0], q, 2, qdims, strides, box) ||
+      !encode_bf16(&maps[1], k_cache, 2, kdims, strides, box) ||
+      !encode_bf16(&maps[2], v_cache, 2, kdims, strides, box))
+    return GQA_ERR_CUDA;
+  return from_cuda(launch_prefill_bf16(a, maps, sm_count(), s));
+}
+
+size_t gqa_decode_workspace_size(int B, int h_q, int h_kv, int T_max, int d_h, gqa_dtype dtype,
+                                 int num_splits) {
+  if (B <= 0 || h_q <= 0 || h_kv <= 0 || T_max <= 0 || d_h <= 0 || h_q % h_kv != 0) return 0;
+  if (num_splits < 0) return 0;
+  const int G = num_splits > 0 ? num_splits : decode_auto_splits();
+  if (G <= 0) return 0;
+  return decode_workspace_bytes(B, h_q, h_kv, d_h, dtype == GQA_BF16, G);
+}
+
+gqa_status gqa_decode(const void* q, const void* k_cache, const void* v_cache, void* o, float* lse,
+                      const int32_t* kv_len, const int32_t* q_pos,
+                      int B, int h_q, int h_kv, int T_max, int d_h, float scale, gqa_dtype dtype,
+                      void* workspace, size_t workspace_bytes, int num_splits, void* stream) {
+  if (!q || !k_cache || !v_cache || !o) return GQA_ERR_INVALID_ARG;
+  if (B <= 0 || h_q <= 0 || h_kv <= 0 || T_max <= 0 || d_h <= 0 || num_splits < 0)
+    return GQA_ERR_INVALID_ARG;
+  if (h_q % h_kv != 0 || !valid_scale(scale)) return GQA_ERR_INVALID_ARG;
+  if (dtype != GQA_BF16 && dtype != GQA_FP32) return GQA_ERR_INVALID_ARG;
+  if (B > decode_max_batch()) return GQA_ERR_UNSUPPORTED;
+  if (dtype == GQA_FP32 && d_h > 256) return GQA_ERR_UNSUPPORTED;
+  if (dtype == GQA_BF16 && d_h != 64 && d_h != 128) return GQA_ERR_UNSUPPORTED;
+  if ((long long)B * h_kv * T_max >= (1ll << 31)) return GQA_ERR_UNSUPPORTED;
+  const int G = num_splits > 0 ? num_splits : decode_auto_splits();
+  if (G <= 0) return GQA_ERR_CUDA;
+  const size_t need = decode_workspace_bytes(B, h_q, h_kv, d_h, dtype == GQA_BF16, G);
+  if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return GQA_ERR_WORKSPACE;
+  DecodeArgs a;
+  a.q = q;
+  a.k = k_cache;
+  a.v = v_cache;
+  a.o = o;
+  a.lse = lse;
+  a.kv_len = kv_len;
+  a.q_pos = q_pos;
+  a.B = B;
+  a.h_q = h_q;
+  a.h_kv = h_kv;
+  a.T_max = T_max;
+  a.d_h = d_h;
+  a.scale = scale;
+  a.workspace = workspace;
+  a.workspace_bytes = workspace_bytes;
+  a.num_splits = G;
+  a.err = device_error_ptr();
+  if (!a.err) return GQA_ERR_CUDA;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (dtype == GQA_FP32) return from_cuda(launch_decode_fp32(a, s));
+  CUtensorMap maps[2];
+  const uint64_t kdims[2] = {(uint64_t)d_h, (uint64_t)B * h_kv * T_max};
+  const uint64_t strides[1] = {(uint64_t)d_h * 2};
+  const uint32_t box[2] = {64, 64};
+  if (!encode_bf16(&maps[0], k_cache, 2, kdims, strides, box) ||
+      !encode_bf16(&maps[1], v_cache, 2, kdims, strides, box))
+    return GQA_ERR_CUDA;
+  return from_cuda(launch_decode_bf16(a, maps, s));
+}
+
+}  // extern "C"

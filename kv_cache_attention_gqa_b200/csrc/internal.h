@@ -1,0 +1,69 @@
+// Internal launcher interface between the C ABI (api.cu) and the kernel translation units.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "gqa.h"
+
+namespace gqa {
+
+struct AppendArgs {
+  void* k_cache;
+  void* v_cache;
+  const void* k_new;
+  const void* v_new;
+  const int32_t* pos;
+  int B, h_kv, S_new, T_max, d_h;
+  int elem_bytes;
+  unsigned* err;
+};
+cudaError_t launch_kv_append(const AppendArgs& a, cudaStream_t s);
+
+struct PrefillArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  void* o;
+  float* lse;
+  const int32_t* q_start;
+  const int32_t* kv_len;
+  int B, h_q, h_kv, S_q, T_max, d_h;
+  float scale;
+  int causal;
+  unsigned* err;
+};
+// fp32 check mode (scalar FFMA)
+cudaError_t launch_prefill_fp32(const PrefillArgs& a, cudaStream_t s);
+// bf16 tcgen05 path (sm_100a). tmaps: [0] = Q, [1] = K, [2] = V (encoded by the caller).
+cudaError_t launch_prefill_bf16(const PrefillArgs& a, const CUtensorMap* tmaps, int num_sms,
+                                cudaStream_t s);
+
+struct DecodeArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  void* o;
+  float* lse;
+  const int32_t* kv_len;
+  const int32_t* q_pos;
+  int B, h_q, h_kv, T_max, d_h;
+  float scale;
+  void* workspace;
+  size_t workspace_bytes;
+  int num_splits;  // resolved (> 0)
+  unsigned* err;
+};
+
+// Workspace layout shared by both decode variants (see decode.cu).
+size_t decode_workspace_bytes(int B, int h_q, int h_kv, int d_h, bool bf16, int num_splits);
+int decode_heads_per_unit(int h_q, int h_kv, bool bf16);
+int decode_max_batch();
+
+cudaError_t launch_decode_fp32(const DecodeArgs& a, cudaStream_t s);
+// tmaps: [0] = K cache, [1] = V cache, 2-D views (d_h, B*h_kv*T_max), box (64, 64), SWIZZLE_128B.
+cudaError_t launch_decode_bf16(const DecodeArgs& a, const CUtensorMap* tmaps, cudaStream_t s);
+
+}  // namespace gqa

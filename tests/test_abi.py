@@ -1,0 +1,95 @@
+"""The C-ABI library loads on a machine without a GPU and exports every symbol gqa.h declares;
+host-side argument checks run before any CUDA call. No compute is launched here."""
+
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gqa.h")
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][\w]*\s*\**\s+\**([A-Za-z_]\w*)\s*\(", text, flags=re.M)
+    return sorted(set(n for n in names if n not in ("if", "while")))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from kv_cache_attention_gqa_b200 import _lib
+
+    return _lib._lib
+
+
+def test_header_declares_the_three_entry_points():
+    names = _declared_functions()
+    for n in ("gqa_prefill", "gqa_decode", "kv_append", "gqa_decode_workspace_size",
+              "gqa_get_device_error", "gqa_status_string", "gqa_version"):
+        assert n in names, names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    from kv_cache_attention_gqa_b200 import _lib
+
+    out = subprocess.run(["nm", "-D", "--defined-only", _lib.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(line.split()[-1] for line in out.splitlines() if line.strip())
+    for n in _declared_functions():
+        assert n in exported, f"{n} not exported"
+        assert hasattr(lib, n)
+    assert set(_lib.SIGNATURES) == set(_declared_functions())
+
+
+def test_status_strings_and_version(lib):
+    from kv_cache_attention_gqa_b200 import _lib
+
+    for code, name in _lib.STATUS_NAMES.items():
+        assert lib.gqa_status_string(code).decode() == name
+    assert b"sm_100a" in lib.gqa_version()
+
+
+def test_host_side_argument_errors(lib):
+    P = ctypes.c_void_p
+    fake = P(0x1000)
+    null = None
+    s = None
+    # null pointers
+    assert lib.gqa_prefill(null, fake, fake, fake, null, null, null, 1, 4, 2, 8, 8, 64, 0.125, 1, 0, s) == 1
+    # h_q not a multiple of h_kv
+    assert lib.gqa_prefill(fake, fake, fake, fake, null, null, null, 1, 6, 4, 8, 8, 64, 0.125, 1, 0, s) == 1
+    # non-positive sizes, bad scale, bad causal flag
+    assert lib.gqa_prefill(fake, fake, fake, fake, null, null, null, 0, 4, 2, 8, 8, 64, 0.125, 1, 0, s) == 1
+    assert lib.gqa_prefill(fake, fake, fake, fake, null, null, null, 1, 4, 2, 8, 8, 64, float("nan"), 1, 0, s) == 1
+    assert lib.gqa_prefill(fake, fake, fake, fake, null, null, null, 1, 4, 2, 8, 8, 64, -1.0, 1, 0, s) == 1
+    assert lib.gqa_prefill(fake, fake, fake, fake, null, null, null, 1, 4, 2, 8, 8, 64, 0.1, 2, 0, s) == 1
+    # decode
+    assert lib.gqa_decode(null, fake, fake, fake, null, null, null, 1, 4, 2, 8, 64, 0.1, 0, fake, 1 << 20, 1, s) == 1
+    assert lib.gqa_decode(fake, fake, fake, fake, null, null, null, 1, 4, 3, 8, 64, 0.1, 0, fake, 1 << 20, 1, s) == 1
+    assert lib.gqa_decode(fake, fake, fake, fake, null, null, null, 1, 4, 2, 8, 64, 0.1, 0, fake, 1 << 20, -1, s) == 1
+    assert lib.gqa_decode(fake, fake, fake, fake, null, null, null, 1, 4, 2, 8, 64, 0.1, 7, fake, 1 << 20, 1, s) == 1
+    # unsupported: bf16 with d_h = 96; batch beyond the decode limit
+    assert lib.gqa_decode(fake, fake, fake, fake, null, null, null, 1, 4, 2, 8, 96, 0.1, 0, fake, 1 << 20, 1, s) == 2
+    assert lib.gqa_decode(fake, fake, fake, fake, null, null, null, 5000, 4, 2, 8, 64, 0.1, 0, fake, 1 << 20, 1, s) == 2
+    # workspace: missing, too small, misaligned (num_splits given, so no device query is needed)
+    assert lib.gqa_decode(fake, fake, fake, fake, null, null, null, 1, 4, 2, 8, 64, 0.1, 0, null, 1 << 20, 1, s) == 5
+    assert lib.gqa_decode(fake, fake, fake, fake, null, null, null, 1, 4, 2, 8, 64, 0.1, 0, fake, 16, 1, s) == 5
+    assert lib.gqa_decode(fake, fake, fake, fake, null, null, null, 1, 4, 2, 8, 64, 0.1, 0, P(0x1004), 1 << 20, 1, s) == 5
+    # kv_append
+    assert lib.kv_append(fake, fake, fake, fake, null, 1, 2, 1, 8, 64, 0, s) == 1
+    assert lib.kv_append(fake, fake, fake, fake, fake, 1, 2, 9, 8, 64, 0, s) == 1
+    assert lib.kv_append(fake, fake, fake, fake, fake, 1, 2, 1, 8, 64, 9, s) == 1
+    assert lib.gqa_get_device_error(None, s) == 1
+
+
+def test_workspace_size(lib):
+    assert lib.gqa_decode_workspace_size(1, 6, 4, 8, 64, 0, 4) == 0
+    assert lib.gqa_decode_workspace_size(0, 4, 2, 8, 64, 0, 4) == 0
+    a = lib.gqa_decode_workspace_size(8, 32, 8, 8192, 128, 0, 148)
+    b = lib.gqa_decode_workspace_size(8, 32, 8, 8192, 128, 0, 296)
+    assert 0 < a < b
+    # partials: (splits + units) slots of r heads x (d_h + 1) floats, plus one counter per unit
+    assert a >= (148 + 64) * 4 * 129 * 4 + 64 * 4

@@ -4,7 +4,8 @@ Default workload (``decode_8k``): B=8, h_q=32, d_h=128, T=8192, swept over h_kv 
 (MHA / GQA / MQA). One step = for each variant, one ``kv_append`` of the new token's K/V at
 position 8191 followed by one ``gqa_decode`` over the 8192 cached keys. ``value`` is the KV bytes
 the decodes must read (2 * B * h_kv * T * d_h * 2 per variant) divided by the device time of the
-whole step, in GB/s. L2 is flushed (a 256 MiB write) between steps, outside the timed events.
+whole step, in GB/s. L2 is flushed (a 256 MiB write, then a 256 MiB read) between steps, outside
+the timed events.
 
 ``--impl reference`` times the fp64 CPU oracle on a bounded sample of the same workload.
 Run with no flags for N=1; under torchrun every rank runs an independent replica (the path needs
@@ -84,6 +85,22 @@ def recorded_traffic(summary_name, digest):
     return out or None
 
 
+class L2Flush:
+    """Evict L2 between timed steps: write a 256 MiB buffer (twice the 126 MB L2), then read a
+    second one, so the dirty lines of the write are written back here and not during the next
+    timed kernel. Both run outside the timed events."""
+
+    def __init__(self, dev):
+        import torch
+
+        self.a = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+        self.b = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+
+    def __call__(self, i):
+        self.a.fill_(i & 0xFF)
+        self.b.sum()
+
+
 class ClockSampler:
     """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
 
@@ -156,7 +173,7 @@ def run_ours(args, rank, world, dist):
     hbm_peak, tf_peak, tf_sust, peak_kind = load_peaks()
 
     variants = []
-    for h_kv in (32, 8, 1):
+    for h_kv in args.h_kv:
         shape = workloads.DECODE_8K[h_kv]
         q, k, v, kv_len = workloads.decode_inputs(shape, seed=args.seed + rank, device=dev)
         # the new token: its K/V row is appended at position T-1, then the query attends
@@ -171,27 +188,46 @@ def run_ours(args, rank, world, dist):
         variants.append(dict(h_kv=h_kv, shape=shape, q=q, k=k, v=v, kv_len=kv_len, k_new=k_new,
                              v_new=v_new, pos=pos, out=out, ws=ws,
                              bytes=decode_kv_bytes(shape.B, h_kv, [shape.T_max] * shape.B, shape.d_h)))
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
 
     def step(record=None):
         for i, var in enumerate(variants):
             gqa.kv_append(var["k"], var["v"], var["k_new"], var["v_new"], var["pos"])
             if record is not None:
-                record[i][0].record(stream)
+                record[i][0].record()
             gqa.decode(var["q"], var["k"], var["v"], kv_len=var["kv_len"], out=var["out"], ws=var["ws"])
             if record is not None:
-                record[i][1].record(stream)
+                record[i][1].record()
 
     for _ in range(args.warmup):
-        flush.fill_(1)
+        flush(1)
         step()
     torch.cuda.synchronize()
     if gqa.get_device_error() != 0:
         raise RuntimeError("device error during warm-up")
 
-    E = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    # The step is captured once in a CUDA graph (as a decode loop would run it), with timing
+    # events recorded inside the graph around each decode launch; each replay is preceded by an
+    # L2 flush outside the timed events. Falls back to eager launches if capture fails.
+    E = lambda **kw: torch.cuda.Event(enable_timing=True, **kw)  # noqa: E731
+    inner = [(E(external=True), E(external=True)) for _ in variants]
+    graph = None
+    if not args.eager:
+        try:
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):
+                step(inner)
+            graph.replay()
+            torch.cuda.synchronize()
+            inner[0][0].elapsed_time(inner[0][1])
+        except Exception as exc:  # pragma: no cover - depends on the driver/runtime
+            print(f"graph capture unavailable ({exc}); timing eager launches", file=sys.stderr)
+            graph = None
+            torch.cuda.synchronize()
+    mode = "cuda_graph" if graph is not None else "eager"
+
     step_ev = [(E(), E()) for _ in range(args.steps)]
-    dec_ev = [[(E(), E()) for _ in variants] for _ in range(args.steps)]
+    dec_ms = []
     sampler = ClockSampler(local)
     if dist is not None:
         dist.barrier()
@@ -199,17 +235,20 @@ def run_ours(args, rank, world, dist):
     sampler.start()
     t0 = time.perf_counter()
     for s in range(args.steps):
-        flush.fill_(s & 0xFF)  # evict the caches from L2 (outside the step's events)
+        flush(s)  # evict the caches from L2 (outside the step's events)
         step_ev[s][0].record(stream)
-        step(dec_ev[s])
+        if graph is not None:
+            graph.replay()
+        else:
+            step(inner)
         step_ev[s][1].record(stream)
-    torch.cuda.synchronize()
+        torch.cuda.synchronize()
+        dec_ms.append([a.elapsed_time(b) for a, b in inner])
     wall = time.perf_counter() - t0
     clocks = sampler.stop()
     if dist is not None:
         dist.barrier()
     step_ms = [a.elapsed_time(b) for a, b in step_ev]
-    dec_ms = [[a.elapsed_time(b) for a, b in row] for row in dec_ev]
     total_ms = sum(step_ms)
     if dist is not None:
         t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
@@ -217,6 +256,7 @@ def run_ours(args, rank, world, dist):
         total_ms = float(t.item())
     if gqa.get_device_error() != 0:
         raise RuntimeError("device error during the timed steps")
+    del graph
 
     step_bytes = sum(var["bytes"] for var in variants)
     value = step_bytes * args.steps * world / (total_ms / 1e3) / 1e9
@@ -241,7 +281,7 @@ def run_ours(args, rank, world, dist):
                 "algorithmic_bytes_per_launch": round(step_bytes / len(variants)),
                 "kernel_source_digest": digest}
 
-    e2e = run_e2e(args, variants, dev, stream, dist, world)
+    e2e = run_e2e(args, variants, dev, stream, dist, world) if not args.skip_e2e else None
     prefill = run_prefill(args, dev, stream, tf_peak, peak_kind) if not args.skip_prefill else None
 
     result = {
@@ -252,7 +292,8 @@ def run_ours(args, rank, world, dist):
         "config": {"workload": "decode_8k: B=8, h_q=32, d_h=128, T=8192, h_kv in {32,8,1}; per step and variant one "
                                "kv_append (1 token at position 8191) + one gqa_decode over 8192 keys",
                    "B": 8, "h_q": 32, "d_h": 128, "T": 8192, "h_kv": [32, 8, 1],
-                   "l2": "flushed between steps (256 MiB write, outside the timed events)",
+                   "l2": "flushed between steps (256 MiB write then 256 MiB read, outside the timed events)",
+                   "launch": mode,
                    "parallelism": f"replicas x{world} (no exchange)"},
         "roofline": roofline,
         "per_variant": per_variant,
@@ -293,13 +334,13 @@ def run_e2e(args, variants, dev, stream, dist, world):
             gqa.decode(h["qd"], var["k"], var["v"], kv_len=var["kv_len"], out=var["out"], ws=var["ws"])
             h["o"].copy_(var["out"], non_blocking=True)
 
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     for s in range(args.steps):
-        flush.fill_(s & 0xFF)
+        flush(s)
         evs[s][0].record(stream)
         step()
         evs[s][1].record(stream)
@@ -329,14 +370,14 @@ def run_prefill(args, dev, stream, tf_peak, peak_kind):
         gqa.prefill(q, k, v, out=out)
     except gqa.GQAError as e:
         return {"unavailable": str(e)}
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
     for _ in range(max(3, args.warmup)):
         gqa.prefill(q, k, v, out=out)
     torch.cuda.synchronize()
     n = max(5, args.steps)
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
     for i in range(n):
-        flush.fill_(i & 0xFF)
+        flush(i)
         evs[i][0].record(stream)
         gqa.prefill(q, k, v, out=out)
         evs[i][1].record(stream)
@@ -435,6 +476,10 @@ def main():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--skip-prefill", action="store_true")
     ap.add_argument("--skip-cpu-baseline", action="store_true")
+    ap.add_argument("--skip-e2e", action="store_true")
+    ap.add_argument("--eager", action="store_true", help="time eager launches instead of a CUDA graph")
+    ap.add_argument("--h-kv", dest="h_kv", type=int, nargs="+", default=[32, 8, 1],
+                    help="decode_8k variants to run (default: all three); fewer only for profiling")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

@@ -96,11 +96,11 @@ gqa_status gqa_prefill(const void* q, const void* k_cache, const void* v_cache, 
 
 /*
  * gqa_decode_workspace_size - bytes of device workspace gqa_decode needs for this shape with
- * `num_splits` work partitions (0 = the automatic choice gqa_decode makes on the current device).
- * The workspace holds per-partition partial results and one completion counter per
- * (sequence, KV head) unit. It must be zero-filled before its first use; every gqa_decode call
- * that completes leaves the counters at zero again, so it can be reused without clearing.
- * Returns 0 on invalid arguments.
+ * `num_splits` (0 = the automatic choice gqa_decode makes on the current device).
+ * The workspace holds a small header (a work ticket), the per-sequence visible lengths and their
+ * prefix sums, and per-piece partial results. It must be zero-filled before its first use; every
+ * gqa_decode call that completes leaves the ticket at zero again, so one workspace can be reused,
+ * for any shape it is large enough for, without clearing. Returns 0 on invalid arguments.
  */
 size_t gqa_decode_workspace_size(int B, int h_q, int h_kv, int T_max, int d_h, gqa_dtype dtype,
                                  int num_splits);
@@ -118,9 +118,11 @@ size_t gqa_decode_workspace_size(int B, int h_q, int h_kv, int T_max, int d_h, g
  *   workspace, workspace_bytes: caller-owned device memory, >= gqa_decode_workspace_size(...),
  *            256-byte aligned, zero-filled before first use (see above). Calls that share one
  *            workspace must not overlap in time (use one stream, or one workspace per stream).
- *   num_splits: number of work partitions the visible keys of all (sequence, KV head) units are
- *            cut into, contiguous and of equal size; 0 = automatic (one per SM). Results do not
- *            depend on it beyond floating-point rounding.
+ *   num_splits: the visible keys of all (sequence, KV head) units, laid end to end, are cut into
+ *            at most this many contiguous chunks of equal size; 0 = automatic (one chunk per SM,
+ *            at least 128 keys and at least 16 keys per query head in a chunk). Results do not depend on it beyond floating-point
+ *            rounding. The call launches two kernels: the split-KV pass over the chunks and a merge
+ *            of the rows whose keys fell into more than one chunk.
  *   dtype    GQA_BF16: d_h in {64, 128}; GQA_FP32: 1 <= d_h <= 256 (check mode).
  * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA.
  */

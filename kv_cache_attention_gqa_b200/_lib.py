@@ -108,6 +108,10 @@ def _int_vec(x, B: int, device, name: str):
     """Device int32[B] from None / int / sequence / tensor (None stays None = library default)."""
     if x is None:
         return None
+    if isinstance(x, torch.Tensor) and x.is_cuda and x.dtype == torch.int32 and x.is_contiguous():
+        if x.numel() != B:
+            raise ValueError(f"{name} must have {B} entries")
+        return x
     if isinstance(x, int):
         x = [x] * B
     t = torch.as_tensor(x, dtype=torch.int32, device=device).contiguous()
@@ -181,11 +185,12 @@ def decode_workspace_size(B: int, h_q: int, h_kv: int, T_max: int, d_h: int, dty
 
 _ws_lock = threading.Lock()
 _ws_cache: dict = {}
+_ws_sizes: dict = {}
 
 
 def workspace(nbytes: int, device) -> torch.Tensor:
     """A zero-filled, 256-byte aligned device workspace of at least ``nbytes``, cached per device
-    and stream (the decode kernels leave it zeroed again after every completed call)."""
+    and stream (every completed decode leaves its counter region at zero again)."""
     dev = torch.device(device)
     key = (dev.index, torch.cuda.current_stream(dev).cuda_stream)
     with _ws_lock:
@@ -214,7 +219,10 @@ def decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, *, kv_
     kl = _int_vec(kv_len, B, q.device, "kv_len")
     qp = _int_vec(q_pos, B, q.device, "q_pos")
     scale = 1.0 / math.sqrt(d_h) if scale is None else float(scale)
-    need = decode_workspace_size(B, h_q, h_kv, T_max, d_h, q.dtype, num_splits)
+    key = (B, h_q, h_kv, T_max, d_h, dt, num_splits, q.device.index)
+    need = _ws_sizes.get(key)
+    if need is None:
+        need = _ws_sizes[key] = decode_workspace_size(B, h_q, h_kv, T_max, d_h, q.dtype, num_splits)
     if ws is None:
         ws = workspace(need, q.device)
     _check("gqa_decode", _lib.gqa_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(out), _ptr(lse),

@@ -33,9 +33,12 @@ unsigned* device_error_ptr() {
 }
 
 int sm_count() {
+  static int cached[kMaxDevices] = {0};
   int dev = 0, n = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (dev >= 0 && dev < kMaxDevices && cached[dev] > 0) return cached[dev];
   if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  if (dev >= 0 && dev < kMaxDevices) cached[dev] = n;
   return n;
 }
 
@@ -72,8 +75,6 @@ bool valid_scale(float s) { return isfinite(s) && s > 0.f; }
 gqa_status from_cuda(cudaError_t e) { return e == cudaSuccess ? GQA_OK : GQA_ERR_CUDA; }
 
 }  // namespace
-
-int decode_auto_splits() { return sm_count(); }
 
 }  // namespace gqa
 
@@ -187,10 +188,10 @@ gqa_status gqa_prefill(const void* q, const void* k_cache, const void* v_cache, 
 size_t gqa_decode_workspace_size(int B, int h_q, int h_kv, int T_max, int d_h, gqa_dtype dtype,
                                  int num_splits) {
   if (B <= 0 || h_q <= 0 || h_kv <= 0 || T_max <= 0 || d_h <= 0 || h_q % h_kv != 0) return 0;
-  if (num_splits < 0) return 0;
-  const int G = num_splits > 0 ? num_splits : decode_auto_splits();
-  if (G <= 0) return 0;
-  return decode_workspace_bytes(B, h_q, h_kv, d_h, dtype == GQA_BF16, G);
+  if (num_splits < 0 || (dtype != GQA_BF16 && dtype != GQA_FP32)) return 0;
+  const int sms = num_splits > 0 ? 1 : sm_count();
+  if (sms <= 0) return 0;
+  return decode_workspace_bytes(B, h_q, h_kv, T_max, d_h, num_splits, sms);
 }
 
 gqa_status gqa_decode(const void* q, const void* k_cache, const void* v_cache, void* o, float* lse,
@@ -205,11 +206,15 @@ gqa_status gqa_decode(const void* q, const void* k_cache, const void* v_cache, v
   if (B > decode_max_batch()) return GQA_ERR_UNSUPPORTED;
   if (dtype == GQA_FP32 && d_h > 256) return GQA_ERR_UNSUPPORTED;
   if (dtype == GQA_BF16 && d_h != 64 && d_h != 128) return GQA_ERR_UNSUPPORTED;
-  if ((long long)B * h_kv * T_max >= (1ll << 31)) return GQA_ERR_UNSUPPORTED;
-  const int G = num_splits > 0 ? num_splits : decode_auto_splits();
-  if (G <= 0) return GQA_ERR_CUDA;
-  const size_t need = decode_workspace_bytes(B, h_q, h_kv, d_h, dtype == GQA_BF16, G);
-  if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+  if ((long long)B * h_kv * T_max >= (1ll << 31) || (long long)B * h_q >= (1ll << 31))
+    return GQA_ERR_UNSUPPORTED;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return GQA_ERR_WORKSPACE;
+  // the workspace check needs no device query when num_splits is given
+  if (num_splits > 0 && workspace_bytes < decode_workspace_bytes(B, h_q, h_kv, T_max, d_h, num_splits, 1))
+    return GQA_ERR_WORKSPACE;
+  const int sms = sm_count();
+  if (sms <= 0) return GQA_ERR_CUDA;
+  if (workspace_bytes < decode_workspace_bytes(B, h_q, h_kv, T_max, d_h, num_splits, sms))
     return GQA_ERR_WORKSPACE;
   DecodeArgs a;
   a.q = q;
@@ -227,17 +232,23 @@ gqa_status gqa_decode(const void* q, const void* k_cache, const void* v_cache, v
   a.scale = scale;
   a.workspace = workspace;
   a.workspace_bytes = workspace_bytes;
-  a.num_splits = G;
+  a.num_splits = num_splits;
+  a.num_sms = sms;
   a.err = device_error_ptr();
   if (!a.err) return GQA_ERR_CUDA;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (dtype == GQA_FP32) return from_cuda(launch_decode_fp32(a, s));
-  CUtensorMap maps[2];
+  const int r = h_q / h_kv;
+  const uint32_t qrows = r > 16 ? 32 : 16;
+  CUtensorMap maps[3];
   const uint64_t kdims[2] = {(uint64_t)d_h, (uint64_t)B * h_kv * T_max};
+  const uint64_t qdims[2] = {(uint64_t)d_h, (uint64_t)B * h_q};
   const uint64_t strides[1] = {(uint64_t)d_h * 2};
   const uint32_t box[2] = {64, 64};
+  const uint32_t qbox[2] = {64, qrows};
   if (!encode_bf16(&maps[0], k_cache, 2, kdims, strides, box) ||
-      !encode_bf16(&maps[1], v_cache, 2, kdims, strides, box))
+      !encode_bf16(&maps[1], v_cache, 2, kdims, strides, box) ||
+      !encode_bf16(&maps[2], q, 2, qdims, strides, qbox))
     return GQA_ERR_CUDA;
   return from_cuda(launch_decode_bf16(a, maps, s));
 }

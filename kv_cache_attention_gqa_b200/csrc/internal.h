@@ -53,17 +53,19 @@ struct DecodeArgs {
   float scale;
   void* workspace;
   size_t workspace_bytes;
-  int num_splits;  // resolved (> 0)
+  int num_splits;  // 0 = automatic chunking, else the number of chunks to cut the keys into
+  int num_sms;     // persistent grid size
   unsigned* err;
 };
 
-// Workspace layout shared by both decode variants (see decode.cu).
-size_t decode_workspace_bytes(int B, int h_q, int h_kv, int d_h, bool bf16, int num_splits);
-int decode_heads_per_unit(int h_q, int h_kv, bool bf16);
+// Workspace bytes for a decode of this shape (layout in decode.cu).
+size_t decode_workspace_bytes(int B, int h_q, int h_kv, int T_max, int d_h, int num_splits,
+                              int num_sms);
 int decode_max_batch();
 
 cudaError_t launch_decode_fp32(const DecodeArgs& a, cudaStream_t s);
-// tmaps: [0] = K cache, [1] = V cache, 2-D views (d_h, B*h_kv*T_max), box (64, 64), SWIZZLE_128B.
+// tmaps: [0] = K cache, [1] = V cache as 2-D views (d_h, B*h_kv*T_max) with box (64, 64);
+// [2] = queries as (d_h, B*h_q) with box (64, 16 or 32 rows: 32 when r > 16); SWIZZLE_128B.
 cudaError_t launch_decode_bf16(const DecodeArgs& a, const CUtensorMap* tmaps, cudaStream_t s);
 
 }  // namespace gqa

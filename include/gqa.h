@@ -132,6 +132,28 @@ gqa_status gqa_decode(const void* q, const void* k_cache, const void* v_cache, v
                       void* workspace, size_t workspace_bytes, int num_splits, void* stream);
 
 /*
+ * gqa_decode_noalloc - gqa_decode for callers that cannot allocate device memory. (The source
+ * pages have no counterpart; this is a library convenience.) Some callers run where cudaMalloc is
+ * unavailable or forbidden: a plugin inside a host framework that owns all device memory and hands
+ * over only inputs and outputs, or a latency-critical loop that must not risk the synchronisation
+ * an allocation can bring. This entry point takes the same arguments as gqa_decode minus the
+ * workspace, and uses a fixed 16 MiB scratch array that the library itself holds in device memory
+ * (every GPU that loads the library keeps it until the process exits). It allocates nothing.
+ *   - Shapes whose workspace (gqa_decode_workspace_size) exceeds 16 MiB are rejected with
+ *     GQA_ERR_WORKSPACE; use gqa_decode with your own workspace for those.
+ *   - The first call on a device looks up the scratch array's device address and caches it; make
+ *     that first call before any stream capture.
+ *   - All calls share the one array, which keeps the previous call's contents; the part that must
+ *     start at zero is cleared on `stream` before each launch. Calls that overlap on the GPU (on
+ *     different streams or from different host threads) race on the array: serialise them.
+ * Errors: as gqa_decode.
+ */
+gqa_status gqa_decode_noalloc(const void* q, const void* k_cache, const void* v_cache, void* o,
+                              float* lse, const int32_t* kv_len, const int32_t* q_pos,
+                              int B, int h_q, int h_kv, int T_max, int d_h, float scale,
+                              gqa_dtype dtype, int num_splits, void* stream);
+
+/*
  * kv_append - copy new K/V rows into the cache: cache[b, g, pos[b] + t, :] = new[b, g, t, :]
  * for t < S_new. Bit-exact; no other byte of the cache is written.
  * [第三章, section 3.1: the new token's K/V join the cache; MHA/MQA/GQA walkthrough, section 4].

@@ -9,6 +9,7 @@ from ._lib import (  # noqa: F401
     GQAError,
     LIB_PATH,
     decode,
+    decode_noalloc,
     decode_workspace_size,
     get_device_error,
     kv_append,

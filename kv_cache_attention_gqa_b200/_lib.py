@@ -37,6 +37,7 @@ SIGNATURES = {
     "gqa_prefill": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _I, _P]),
     "gqa_decode_workspace_size": (_Z, [_I, _I, _I, _I, _I, _I, _I]),
     "gqa_decode": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _P, _Z, _I, _P]),
+    "gqa_decode_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _I, _P]),
     "kv_append": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P]),
     "gqa_get_device_error": (_I, [ctypes.POINTER(_I), _P]),
     "gqa_status_string": (ctypes.c_char_p, [_I]),
@@ -228,4 +229,30 @@ def decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, *, kv_
     _check("gqa_decode", _lib.gqa_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(out), _ptr(lse),
                                          _ptr(kl), _ptr(qp), B, h_q, h_kv, T_max, d_h, scale, dt,
                                          _ptr(ws), ws.numel(), num_splits, _stream()))
+    return (out, lse) if return_lse else out
+
+
+def decode_noalloc(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, *, kv_len=None,
+                   q_pos=None, scale: float | None = None, num_splits: int = 0, out=None,
+                   return_lse: bool = False):
+    """gqa_decode_noalloc: the decode with the library's fixed device scratch array instead of a
+    caller workspace, for callers that cannot allocate device memory (the output buffer may be
+    passed in as ``out``). Overlapping calls on different streams race on that array."""
+    _need_cuda(q, k_cache, v_cache, out)
+    B, h_q, d_h = q.shape
+    Bk, h_kv, T_max, dk = k_cache.shape
+    if (Bk, dk) != (B, d_h) or v_cache.shape != k_cache.shape:
+        raise ValueError("q / k_cache / v_cache shapes disagree")
+    dt = _dtype_code(q)
+    if k_cache.dtype != q.dtype or v_cache.dtype != q.dtype:
+        raise TypeError("q, k_cache and v_cache must share one dtype")
+    if out is None:
+        out = torch.empty_like(q)
+    lse = torch.empty((B, h_q), dtype=torch.float32, device=q.device) if return_lse else None
+    kl = _int_vec(kv_len, B, q.device, "kv_len")
+    qp = _int_vec(q_pos, B, q.device, "q_pos")
+    scale = 1.0 / math.sqrt(d_h) if scale is None else float(scale)
+    _check("gqa_decode_noalloc", _lib.gqa_decode_noalloc(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(out),
+                                                         _ptr(lse), _ptr(kl), _ptr(qp), B, h_q, h_kv, T_max,
+                                                         d_h, scale, dt, num_splits, _stream()))
     return (out, lse) if return_lse else out

@@ -172,13 +172,18 @@ gqa_status gqa_prefill(const void* q, const void* k_cache, const void* v_cache, 
   if (d_h != 64 && d_h != 128) return GQA_ERR_UNSUPPORTED;
   if ((long long)B * h_kv * T_max >= (1ll << 31) || (long long)B * h_q * S_q >= (1ll << 31))
     return GQA_ERR_UNSUPPORTED;
-  // TMA views: Q as rows (B*h_q*S_q, d_h); K, V as rows (B*h_kv*T_max, d_h); 64-column boxes.
+  // TMA views: Q as (d_h, S_q, B*h_q) with box (64, P, H): one box holds the H heads x P
+  // positions of a tile, head-major; K, V as rows (B*h_kv*T_max, d_h) with box (64, 128).
+  const int H = prefill_heads_per_tile(h_q, h_kv);
+  const uint32_t P = (uint32_t)(128 / H);
   CUtensorMap maps[3];
-  const uint64_t qdims[2] = {(uint64_t)d_h, (uint64_t)B * h_q * S_q};
+  const uint64_t qdims[3] = {(uint64_t)d_h, (uint64_t)S_q, (uint64_t)B * h_q};
+  const uint64_t qstrides[2] = {(uint64_t)d_h * 2, (uint64_t)S_q * d_h * 2};
+  const uint32_t qbox[3] = {64, P, (uint32_t)H};
   const uint64_t kdims[2] = {(uint64_t)d_h, (uint64_t)B * h_kv * T_max};
   const uint64_t strides[1] = {(uint64_t)d_h * 2};
   const uint32_t box[2] = {64, 128};
-  if (!encode_bf16(&maps[0], q, 2, qdims, strides, box) ||
+  if (!encode_bf16(&maps[0], q, 3, qdims, qstrides, qbox) ||
       !encode_bf16(&maps[1], k_cache, 2, kdims, strides, box) ||
       !encode_bf16(&maps[2], v_cache, 2, kdims, strides, box))
     return GQA_ERR_CUDA;

@@ -37,9 +37,12 @@ struct PrefillArgs {
 };
 // fp32 check mode (scalar FFMA)
 cudaError_t launch_prefill_fp32(const PrefillArgs& a, cudaStream_t s);
-// bf16 tcgen05 path (sm_100a). tmaps: [0] = Q, [1] = K, [2] = V (encoded by the caller).
+// bf16 tcgen05 path (sm_100a). tmaps: [0] = Q as a 3-D view (d_h, S_q, B*h_q) with box
+// (64, 128 / H, H); [1] = K, [2] = V as 2-D views (d_h, B*h_kv*T_max) with box (64, 128).
 cudaError_t launch_prefill_bf16(const PrefillArgs& a, const CUtensorMap* tmaps, int num_sms,
                                 cudaStream_t s);
+// query heads per prefill tile (H); a tile holds H heads x floor(128 / H) positions
+int prefill_heads_per_tile(int h_q, int h_kv);
 
 struct DecodeArgs {
   const void* q;

@@ -1,0 +1,101 @@
+"""bf16 tcgen05 prefill on the GPU against the fp64 oracle (max |d| <= 2e-2, mean |d| <= 2e-3)."""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from _tol import assert_bf16_close
+
+pytestmark = pytest.mark.gpu
+
+
+def _f64(t):
+    return workloads.to_f64(t)
+
+
+def _run(B, h_q, h_kv, S_q, T, d, q_start, kv_len, causal=True, seed=0, nan_tail=False, std=1.0):
+    import kv_cache_attention_gqa_b200 as gqa
+
+    shape = workloads.PrefillShape(B=B, h_q=h_q, h_kv=h_kv, S_q=S_q, T_max=T, d_h=d, q_start=0,
+                                   kv_len=T, std=std)
+    q, k, v = workloads.prefill_inputs(shape, seed=seed)
+    if nan_tail:
+        for b in range(B):
+            k[b, :, kv_len[b]:] = float("nan")
+            v[b, :, kv_len[b]:] = float("nan")
+    o, lse = gqa.prefill(q.cuda(), k.cuda(), v.cuda(), q_start=list(q_start), kv_len=list(kv_len),
+                         causal=causal, return_lse=True)
+    ref, lref = oracle.attention_ref(_f64(q), _f64(k), _f64(v), q_start=q_start, kv_len=kv_len,
+                                     causal=causal)
+    assert_bf16_close(_f64(o), ref, f"prefill B={B} h_q={h_q} h_kv={h_kv} S_q={S_q} T={T} d={d}")
+    assert np.abs(lse.cpu().double().numpy() - lref).max() < 2e-2
+    assert gqa.get_device_error() == 0
+
+
+def test_prefill_small_workload():
+    """prefill_small: B=1, h_q=4, h_kv=2, T=256, d_h=64, causal, N(0,1)."""
+    _run(1, 4, 2, 256, 256, 64, [0], [256])
+
+
+@pytest.mark.parametrize("h_q,h_kv", [(4, 4), (8, 4), (16, 4), (32, 4), (6, 2), (8, 1)])
+@pytest.mark.parametrize("d", [64, 128])
+def test_prefill_group_widths_ragged(h_q, h_kv, d):
+    # S_q not a multiple of any tile; kv_len not a multiple of the 128-key block
+    _run(2, h_q, h_kv, 77, 200, d, [0, 50], [77, 127], seed=h_q + d)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_prefill_offset_and_nan_tail(d):
+    # queries at absolute positions q_start.. over a longer cache; keys past kv_len are NaN
+    _run(2, 8, 2, 130, 600, d, [300, 460], [431, 590], seed=7, nan_tail=True)
+
+
+def test_prefill_not_causal():
+    _run(1, 8, 2, 100, 300, 128, [0], [260], causal=False, seed=3)
+
+
+def test_prefill_4k_full_size_sampled():
+    """prefill_4k at full size (B=1, h_q=32, h_kv=8, T=4096, d_h=128, N(0,1)*0.5), in the bench's
+    launch configuration; the oracle checks every row of four heads (two of one group)."""
+    import kv_cache_attention_gqa_b200 as gqa
+
+    shape = workloads.PREFILL_4K
+    q, k, v = workloads.prefill_inputs(shape, seed=0, device="cuda")
+    o = gqa.prefill(q, k, v)
+    assert gqa.get_device_error() == 0
+    for a in (0, 1, 17, 31):
+        g = oracle.group_of(a, 32, 8)
+        ref, _ = oracle.head_attention(_f64(q[0, a]), _f64(k[0, g]), _f64(v[0, g]), np.arange(4096), 4096,
+                                       1.0 / np.sqrt(128))
+        assert_bf16_close(_f64(o[0, a]), ref, f"prefill_4k head {a}")
+
+
+def test_chunked_prefill_full_size_sampled():
+    """chunked_prefill: kv_append of 512 new K/V rows at 32256, then prefill of the 512 queries at
+    absolute positions 32256.. over T=32768; sampled heads against the oracle."""
+    import kv_cache_attention_gqa_b200 as gqa
+
+    shape = workloads.CHUNKED_PREFILL
+    k, v, k_new, v_new, q = workloads.chunked_prefill_inputs(shape, seed=0, device="cuda")
+    gqa.kv_append(k, v, k_new, v_new, [shape.q_start])
+    o = gqa.prefill(q, k, v, q_start=[shape.q_start], kv_len=[shape.kv_len])
+    assert gqa.get_device_error() == 0
+    for a in (0, 13, 31):
+        g = oracle.group_of(a, 32, 8)
+        pos = shape.q_start + np.arange(shape.S_q)
+        ref, _ = oracle.head_attention(_f64(q[0, a]), _f64(k[0, g]), _f64(v[0, g]), pos, shape.kv_len,
+                                       1.0 / np.sqrt(128))
+        assert_bf16_close(_f64(o[0, a]), ref, f"chunked prefill head {a}")
+
+
+def test_prefill_equals_rows_of_decode():
+    """The last prefill row equals a decode of the same query at position T-1."""
+    import kv_cache_attention_gqa_b200 as gqa
+
+    shape = workloads.PrefillShape(B=2, h_q=16, h_kv=4, S_q=300, T_max=300, d_h=128, q_start=0, kv_len=300)
+    q, k, v = workloads.prefill_inputs(shape, seed=11, device="cuda")
+    o = gqa.prefill(q, k, v)
+    od = gqa.decode(q[:, :, -1].contiguous(), k, v)
+    assert (o[:, :, -1].float() - od.float()).abs().max().item() < 2e-2

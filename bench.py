@@ -171,6 +171,8 @@ def run_ours(args, rank, world, dist):
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream(dev)
     hbm_peak, tf_peak, tf_sust, peak_kind = load_peaks()
+    if args.prefill_only:  # profiling aid: the prefill_4k line alone
+        return {"prefill": run_prefill(args, dev, stream, tf_peak, peak_kind)}
 
     variants = []
     for h_kv in args.h_kv:
@@ -478,6 +480,7 @@ def main():
     ap.add_argument("--skip-cpu-baseline", action="store_true")
     ap.add_argument("--skip-e2e", action="store_true")
     ap.add_argument("--eager", action="store_true", help="time eager launches instead of a CUDA graph")
+    ap.add_argument("--prefill-only", action="store_true", help="only the prefill_4k line (profiling aid)")
     ap.add_argument("--h-kv", dest="h_kv", type=int, nargs="+", default=[32, 8, 1],
                     help="decode_8k variants to run (default: all three); fewer only for profiling")
     args = ap.parse_args()

@@ -156,6 +156,31 @@ class ClockSampler:
                 "samples": len(rows), "reasons": sorted(reasons)}
 
 
+def decode_config(world, launch="cuda_graph"):
+    """The `config` object of the decode_8k line (shared by both arms)."""
+    return {"workload": "decode_8k: B=8, h_q=32, d_h=128, T=8192, h_kv in {32,8,1}; per step and variant one "
+                        "kv_append (1 token at position 8191) + one gqa_decode over 8192 keys",
+            "B": 8, "h_q": 32, "d_h": 128, "T": 8192, "h_kv": [32, 8, 1],
+            "l2": "flushed between steps (256 MiB write then 256 MiB read, outside the timed events)",
+            "launch": launch, "parallelism": f"replicas x{world} (no exchange)"}
+
+
+def max_over_ranks(x, dist, device):
+    """The largest value of `x` over all ranks (the job's time is its slowest replica's)."""
+    if dist is None:
+        return float(x)
+    import torch
+
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(unit_per_step, steps, world, total_ms):
+    """Whole-job rate: the units all ranks processed divided by the (max-over-ranks) time."""
+    return unit_per_step * steps * world / (total_ms / 1e3)
+
+
 # ---------------------------------------------------------------------------------------------
 # our implementation
 # ---------------------------------------------------------------------------------------------
@@ -251,17 +276,13 @@ def run_ours(args, rank, world, dist):
     if dist is not None:
         dist.barrier()
     step_ms = [a.elapsed_time(b) for a, b in step_ev]
-    total_ms = sum(step_ms)
-    if dist is not None:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(step_ms), dist, dev)
     if gqa.get_device_error() != 0:
         raise RuntimeError("device error during the timed steps")
     del graph
 
     step_bytes = sum(var["bytes"] for var in variants)
-    value = step_bytes * args.steps * world / (total_ms / 1e3) / 1e9
+    value = job_throughput(step_bytes, args.steps, world, total_ms) / 1e9
     per_variant = {}
     for i, var in enumerate(variants):
         ms = statistics.mean(row[i] for row in dec_ms)
@@ -291,12 +312,7 @@ def run_ours(args, rank, world, dist):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic: seeded N(0,1) bf16 (no dataset)",
-        "config": {"workload": "decode_8k: B=8, h_q=32, d_h=128, T=8192, h_kv in {32,8,1}; per step and variant one "
-                               "kv_append (1 token at position 8191) + one gqa_decode over 8192 keys",
-                   "B": 8, "h_q": 32, "d_h": 128, "T": 8192, "h_kv": [32, 8, 1],
-                   "l2": "flushed between steps (256 MiB write then 256 MiB read, outside the timed events)",
-                   "launch": mode,
-                   "parallelism": f"replicas x{world} (no exchange)"},
+        "config": decode_config(world, mode),
         "roofline": roofline,
         "per_variant": per_variant,
         "gpu_launches": args.steps * 2 * len(variants),
@@ -347,13 +363,9 @@ def run_e2e(args, variants, dev, stream, dist, world):
         step()
         evs[s][1].record(stream)
     torch.cuda.synchronize()
-    total = sum(a.elapsed_time(b) for a, b in evs)
-    if dist is not None:
-        t = torch.tensor([total], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total = float(t.item())
+    total = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs), dist, dev)
     step_bytes = sum(var["bytes"] for var in variants)
-    return {"value": round(step_bytes * args.steps * world / (total / 1e3) / 1e9, 1), "unit": "GB/s",
+    return {"value": round(job_throughput(step_bytes, args.steps, world, total) / 1e9, 1), "unit": "GB/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "ms_per_step": round(total / args.steps, 4)}
 
@@ -460,8 +472,7 @@ def run_reference(args, rank):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic: seeded N(0,1) bf16 upcast to fp64",
-            "config": {"workload": "decode_8k: B=8, h_q=32, d_h=128, T=8192, h_kv in {32,8,1} (sampled)",
-                       "B": 8, "h_q": 32, "d_h": 128, "T": 8192, "h_kv": [32, 8, 1]},
+            "config": decode_config(1),
             "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": _threads(), "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}

@@ -119,7 +119,7 @@ class ClockSampler:
             os.close(fd)
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu_index}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
+                 "--format=csv,noheader,nounits", "-lms", "20"],
                 stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
@@ -297,7 +297,7 @@ def run_ours(args, rank, world, dist):
     traffic_per_launch = None
     if traffic and all(f"h_kv={v['h_kv']}" in traffic for v in variants):
         traffic_per_launch = round(sum(traffic[f"h_kv={v['h_kv']}"] for v in variants) / len(variants))
-    roofline = {"bound": "hbm", "kernel": "decode_bf16_kernel (split-KV decode + fused combine)",
+    roofline = {"bound": "hbm", "kernel": "decode_bf16_kernel + merge_kernel (events bracket both launches of one gqa_decode)",
                 "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
                 "frac": round(achieved / hbm_peak, 4), "peak_kind": f"hbm_gbs of {peak_kind}",
                 "traffic": traffic_per_launch,
@@ -315,7 +315,7 @@ def run_ours(args, rank, world, dist):
         "config": decode_config(world, mode),
         "roofline": roofline,
         "per_variant": per_variant,
-        "gpu_launches": args.steps * 2 * len(variants),
+        "gpu_launches": args.steps * 3 * len(variants),  # kv_append, decode, merge per variant
         "clocks": clocks,
         "e2e": e2e,
         "wall_s_timed_region": round(wall, 3),

@@ -9,40 +9,47 @@
 // Work tile. Rows of one tile are (query position, query head) pairs of ONE KV group: H heads
 // (H = min(r, 128)) times P = floor(128 / H) consecutive positions, head-major, so every K/V block
 // staged in shared memory serves all r heads of the group [MHA/MQA/GQA walkthrough, section 7:
-// e.g. 32 positions x 4 heads = 128 rows; the mask still uses each row's own position]. A CTA owns
-// two such 128-row sub-tiles (positions q0 .. q0 + 2P) that share every K/V block.
+// e.g. 32 positions x 4 heads = 128 rows; the mask still uses each row's own position].
 //
-// Roles (384 threads):
-//   warp 0      TMA producer: the two Q sub-tiles once, then 128-key K and V blocks into a 2-stage
-//               ring (cp.async.bulk.tensor, 128-byte swizzle, no multicast).
-//   warp 1      allocates 512 TMEM columns and issues the MMAs from one thread:
-//               S_t = Q_t K_j^T  (tcgen05.mma kind::f16, A and B from shared memory, K-major),
-//               O_t += P_t V_j   (A = P from TMEM, B = V from shared memory, MN-major),
-//               ping-ponging the two sub-tiles so one sub-tile's softmax overlaps the other's MMAs.
-//   warps 4-7   softmax of sub-tile 0, warps 8-11 of sub-tile 1: one thread per row (TMEM lane).
-//               Each reads its score row from TMEM, masks by absolute position, updates (m, l),
-//               writes P = 2^(s - m) as bf16 back into the same TMEM columns, and rescales its O
-//               row only when the running maximum grew by more than 8 (base 2): between rescales
-//               P and l share the stale maximum, which leaves O = u / l unchanged.
-// TMEM columns: S0 [0,128), S1 [128,256), O0 [256, 256+D), O1 [256+D, 256+2D); P_t aliases the
-// first 64 columns of S_t. MMAs issued by one thread execute in order, so S_t of block j+1 is
-// written only after O_t += P_t V_j has read P_t.
+// Roles (256 threads, one 128-row tile per CTA):
+//   warp 0      TMA producer: the tile's Q rows once, then 128-key K blocks and V blocks into two
+//               3-deep rings (cp.async.bulk.tensor, 128-byte swizzle, no multicast).
+//   warp 1      allocates 512 TMEM columns and issues every MMA from one thread:
+//               S_j = Q K_j^T  (tcgen05.mma kind::f16, A = Q from TMEM, B = K from shared memory),
+//               O  += P_j V_j  (A = P_j from TMEM, B = V from shared memory, MN-major).
+//               S is double-buffered: S_{j+2} is issued right after O += P_j V_j, so the scores of
+//               the next block are ready when the softmax finishes the current one. Both MMAs read
+//               only one operand from shared memory (a 128x128x16 MMA with both operands there
+//               would need the whole shared-memory bandwidth).
+//   warps 4-7   softmax, one thread per row (TMEM lane). Each first copies its Q row from shared
+//               memory into TMEM, then per block reads its score row, masks by absolute position,
+//               updates (m, l), writes P = 2^(s - m) as bf16 into the block's S columns, and
+//               rescales its O row only when the running maximum grew by more than 8 (base 2):
+//               between rescales P and l share the stale maximum, which leaves O = u / l unchanged.
+// TMEM columns: S_0 [0,128), S_1 [128,256), O [256, 256+D), Q [256+D, 256+3D/2); P_b aliases the
+// first 64 columns of S_b. MMAs issued by one thread execute in order, so S_b of block j+2 is
+// written only after O += P_j V_j has read P_j.
 
 #include <math.h>
 
 #include "common.cuh"
+#include "exp2_poly.cuh"
 #include "internal.h"
 #include "tcgen05.cuh"
 
 namespace gqa {
 namespace pf {
 
-constexpr int kBM = 128;     // rows per sub-tile (= TMEM lanes)
+constexpr int kBM = 128;     // rows per tile (= TMEM lanes)
 constexpr int kBN = 128;     // keys per K/V block
-constexpr int kStages = 2;   // K/V ring depth
+constexpr int kKStages = 3;  // K ring depth (K_j is read two blocks before V_j)
+constexpr int kVStages = 2;  // V ring depth
 constexpr int kThreads = 384;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // base-2 units: P <= 2^8 between rescales
+#ifndef GQA_PREFILL_POLY_EVERY
+#define GQA_PREFILL_POLY_EVERY 0  // one exponential pair in this many goes to the polynomial (0: none)
+#endif
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -50,17 +57,19 @@ template <int D>
 struct Cfg {
   static constexpr int kNch = D / 64;                  // 64-column (128-byte) chunks
   static constexpr int kQChunk = kBM * 128;            // bytes of one Q chunk (128 rows)
-  static constexpr int kQBytes = kNch * kQChunk;       // one sub-tile of Q
+  static constexpr int kQBytes = kNch * kQChunk;
   static constexpr int kKVChunk = kBN * 128;
   static constexpr int kKVBytes = kNch * kKVChunk;     // one K (or V) block
   static constexpr int kOffQ = 0;
-  static constexpr int kOffK = 2 * kQBytes;
-  static constexpr int kOffV = kOffK + kStages * kKVBytes;
-  static constexpr int kOffBar = kOffV + kStages * kKVBytes;
+  static constexpr int kOffK = kQBytes;
+  static constexpr int kOffV = kOffK + kKStages * kKVBytes;
+  static constexpr int kOffX = kOffV + kVStages * kKVBytes;  // 6 x 128 floats
+  static constexpr int kOffBar = kOffX + 6 * 128 * 4;
   // barriers + slack for 1024-byte alignment; at least 120 KiB so that only one CTA (which
   // allocates all 512 TMEM columns) is resident per SM
   static constexpr int kSmem = kOffBar + 256 + 1024 > 120 * 1024 ? kOffBar + 256 + 1024 : 120 * 1024;
-  static constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO0 = 256, kColO1 = 256 + D;
+  static_assert(kSmem <= 227 * 1024, "shared memory budget");
+  static constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256, kColQ = 256 + D;
 };
 
 struct PArgs {
@@ -77,15 +86,17 @@ struct PArgs {
 
 // barrier indices inside the barrier block
 enum {
-  kBarQ = 0,
-  kBarKFull = 1,    // + stage
-  kBarVFull = 3,    // + stage
-  kBarKVEmpty = 5,  // + stage
-  kBarS = 7,        // + sub-tile
-  kBarP = 9,        // + sub-tile
-  kBarO = 11,       // + sub-tile
-  kBarDone = 13,
-  kNumBars = 14
+  kBarQ = 0,          // Q rows landed in shared memory (TMA)
+  kBarQT = 1,         // Q rows copied into TMEM (128 softmax threads)
+  kBarKFull = 2,      // + K stage (3)
+  kBarKEmpty = 5,     // + K stage
+  kBarVFull = 8,      // + V stage (3)
+  kBarVEmpty = 11,    // + V stage
+  kBarS = 14,         // + S buffer (2): scores of a block are in TMEM
+  kBarP = 16,         // + S buffer (2): P of a block is in TMEM
+  kBarO = 18,         // O += P V of a block completed
+  kBarDone = 19,
+  kNumBars = 20
 };
 
 // Bounded wait that also gives up as soon as another thread of the CTA has aborted.
@@ -107,7 +118,7 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile
 }
 
 struct Tile {
-  int b, g, hb, q0;  // q0: first query position (index into S_q) of sub-tile 0
+  int b, g, hb, q0;  // q0: first query position (index into S_q) of the tile
   int nh;            // heads of this head block
   int qs, kv;        // q_start[b], kv_len[b]
   int nb;            // K/V blocks to visit
@@ -124,7 +135,7 @@ __device__ __forceinline__ Tile make_tile(const PArgs& a) {
   const int gh = rem - t.b * (a.h_kv * a.hblocks);
   t.g = gh / a.hblocks;
   t.hb = gh - t.g * a.hblocks;
-  t.q0 = qt * 2 * a.P;
+  t.q0 = qt * a.P;
   t.nh = min(a.H, a.r - t.hb * a.H);
   t.kv = a.kv_len ? a.kv_len[t.b] : a.T_max;
   t.qs = a.q_start ? a.q_start[t.b] : 0;
@@ -132,7 +143,7 @@ __device__ __forceinline__ Tile make_tile(const PArgs& a) {
   t.nb = 0;
   if (t.valid) {
     if (a.causal) {
-      const int last_row = min(t.q0 + 2 * a.P, a.S_q) - 1;
+      const int last_row = min(t.q0 + a.P, a.S_q) - 1;
       const long long pos_max = (long long)t.qs + last_row;
       const long long last_key = pos_max < t.kv - 1 ? pos_max : (long long)(t.kv - 1);
       t.nb = (int)(last_key / kBN) + 1;
@@ -143,121 +154,185 @@ __device__ __forceinline__ Tile make_tile(const PArgs& a) {
   return t;
 }
 
-// One thread per row of sub-tile t (warps 4-7: t = 0, warps 8-11: t = 1).
+#ifndef GQA_PREFILL_EXP_F16X2
+#define GQA_PREFILL_EXP_F16X2 0  // two exponentials per special-function op, in f16
+#endif
+// 2^x0, 2^x1 with one packed f16x2 special-function op: the arguments (<= 8) are rounded to f16,
+// the results widened back to fp32 (they are rounded to bf16 for P in any case).
+__device__ __forceinline__ void exp2_f16x2(float x0, float x1, float& y0, float& y1) {
+  uint32_t h;
+  asm("{\n\t.reg .b32 t;\n\tcvt.rn.f16x2.f32 t, %2, %1;\n\tex2.approx.f16x2 %0, t;\n\t}"
+      : "=r"(h) : "f"(x0), "f"(x1));
+  asm("{\n\t.reg .f16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\tcvt.f32.f16 %0, lo;\n\tcvt.f32.f16 %1, hi;\n\t}"
+      : "=f"(y0), "=f"(y1) : "r"(h));
+}
+#ifndef GQA_PREFILL_PACKED
+#define GQA_PREFILL_PACKED 1  // packed fp32x2 FMA/ADD in the softmax
+#endif
+// packed fp32x2 helpers (sm_100): d = a * b + c and s += a, on register pairs
+__device__ __forceinline__ void ffma2(float& d0, float& d1, float a0, float a1, float b, float c) {
+#if !GQA_PREFILL_PACKED
+  d0 = fmaf(a0, b, c);
+  d1 = fmaf(a1, b, c);
+  return;
+#endif
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %4};\n\t"
+      "mov.b64 rc, {%5, %5};\n\tfma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b), "f"(c));
+}
+__device__ __forceinline__ void fadd2(float& s0, float& s1, float a0, float a1) {
+#if !GQA_PREFILL_PACKED
+  s0 += a0;
+  s1 += a1;
+  return;
+#endif
+  asm("{\n\t.reg .b64 ra, rs;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rs, {%0, %1};\n\t"
+      "add.rn.f32x2 rs, rs, ra;\n\tmov.b64 {%0, %1}, rs;\n\t}"
+      : "+f"(s0), "+f"(s1)
+      : "f"(a0), "f"(a1));
+}
+
+// Two warpgroups share the tile's rows: warps 4-7 take the first half of every block's columns
+// (keys 0-63) and warps 8-11 the second half (keys 64-127), so each SM sub-partition runs two
+// independent softmax warps. A thread owns one row (its TMEM lane, warp % 4 selects the lane
+// quarter) and half of the row's columns; the two halves of a row exchange their block maximum
+// through shared memory once per block, and their partial sums at the end.
 template <int D>
 __device__ __forceinline__ void softmax_role(const PArgs& a, const Tile& tile, int warp, int lane,
-                                             uint32_t tmem, uint32_t sV, uint64_t* bars,
-                                             volatile int* abort) {
+                                             uint32_t tmem, uint32_t sQ, uint32_t sV, uint64_t* bars,
+                                             float* xbuf, volatile int* abort) {
   using C = Cfg<D>;
   auto bar = [&](int i) { return smem_u32(&bars[i]); };
-  const int t = (warp - 4) >> 2;
-  const int wq = warp & 3;                   // TMEM lane quarter this warp may access
-  const int row = wq * 32 + lane;            // TMEM lane = tile row
+  const int half = (warp - 4) >> 2;           // which 64 columns of each block
+  const int wq = warp & 3;
+  const int row = wq * 32 + lane;             // TMEM lane = tile row
+  const int sm_tid = (warp - 4) * 32 + lane;  // 0..255
   const uint32_t lane_addr = tmem + ((uint32_t)(wq * 32) << 16);
-  const uint32_t colS = t == 0 ? C::kColS0 : C::kColS1;
-  const uint32_t colO = t == 0 ? C::kColO0 : C::kColO1;
   const int h = row / a.P, p = row - h * a.P;
-  const int qi = tile.q0 + t * a.P + p;      // query index into S_q
+  const int qi = tile.q0 + p;                 // query index into S_q
   const bool store_row = h < tile.nh && row < a.H * a.P && qi < a.S_q;
   const long long pos = (long long)tile.qs + qi;
-  const long long pos_min = (long long)tile.qs + tile.q0 + t * a.P;  // smallest position in t
+  const long long pos_min = (long long)tile.qs + tile.q0;  // smallest position in the tile
   const int nb = tile.nb;
+  const float c = a.scale_log2;
+  const long long orow = ((long long)tile.b * a.h_q + tile.g * a.r + tile.hb * a.H + h) * a.S_q + qi;
+  constexpr int kOHalf = D / 2;               // O columns (and Q columns) of this half
+  float* xmax = xbuf;                         // [2 buffers][2 halves][128 rows]
+
+  // ---- this half of this row of Q: shared memory (128-byte swizzled) -> TMEM (A of Q K^T)
+  bool ok = nb > 0 && wait_bar(bar(kBarQ), 0, abort, a.err);
+  if (ok) {
+#pragma unroll
+    for (int ch = 0; ch < C::kNch; ++ch) {
+      if ((C::kNch == 2 && ch != half) || (C::kNch == 1 && half != 0)) continue;
+      uint32_t qr[32];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const uint32_t addr = swz128(sQ + ch * C::kQChunk, row, k);
+        asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(qr[4 * k]), "=r"(qr[4 * k + 1]), "=r"(qr[4 * k + 2]), "=r"(qr[4 * k + 3])
+                     : "r"(addr));
+      }
+      tc::st32(lane_addr + C::kColQ + ch * 32, qr);
+    }
+    tc::wait_st();
+  }
+  tc::fence_before_sync();
+  mbar_arrive(bar(kBarQT));
 
   float m = -INFINITY, l = 0.f;
-  bool ok = true;
   for (int j = 0; j < nb && ok; ++j) {
-    if (!wait_bar(bar(kBarS + t), (uint32_t)(j & 1), abort, a.err)) { ok = false; break; }
+    const int buf = j & 1;
+    const uint32_t colS = buf ? C::kColS1 : C::kColS0;
+    if (!wait_bar(bar(kBarS + buf), (uint32_t)((j >> 1) & 1), abort, a.err)) { ok = false; break; }
     tc::fence_after_sync();
-    uint32_t sr[4][32];
-#pragma unroll
-    for (int c = 0; c < 4; ++c) tc::ld32(lane_addr + colS + c * 32, sr[c]);
+    uint32_t su[2][32];
+    tc::ld32(lane_addr + colS + half * 64, su[0]);
+    tc::ld32(lane_addr + colS + half * 64 + 32, su[1]);
     tc::wait_ld();
-    const int key0 = j * kBN;
+    float sr[64];
+#pragma unroll
+    for (int i = 0; i < 64; ++i) sr[i] = __uint_as_float(su[i >> 5][i & 31]);
+    const int key0 = j * kBN + half * 64;     // first key of this half
     const bool need_mask =
-        (a.causal && (long long)key0 + kBN - 1 > pos_min) || key0 + kBN > tile.kv;
-    float mx = -INFINITY;
+        (a.causal && (long long)key0 + 63 > pos_min) || key0 + 64 > tile.kv;
     if (need_mask) {
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int key = key0 + c * 32 + i;
-          const bool vis = key < tile.kv && (!a.causal || key <= pos);
-          const float x = vis ? __uint_as_float(sr[c][i]) * a.scale_log2 : -INFINITY;
-          sr[c][i] = __float_as_uint(x);
-          mx = fmaxf(mx, x);
-        }
-    } else {
-#pragma unroll
-      for (int c = 0; c < 4; ++c)
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float x = __uint_as_float(sr[c][i]) * a.scale_log2;
-          sr[c][i] = __float_as_uint(x);
-          mx = fmaxf(mx, x);
-        }
+      for (int i = 0; i < 64; ++i) {
+        const int key = key0 + i;
+        const bool vis = key < tile.kv && (!a.causal || key <= pos);
+        sr[i] = vis ? sr[i] : -INFINITY;
+      }
     }
-    // running maximum with lazy rescaling
+    float mx0 = sr[0], mx1 = sr[1];
+#pragma unroll
+    for (int i = 2; i < 64; i += 2) {
+      mx0 = fmaxf(mx0, sr[i]);
+      mx1 = fmaxf(mx1, sr[i + 1]);
+    }
+    // block maximum over both halves of the row
+    xmax[(buf * 2 + half) * 128 + row] = fmaxf(mx0, mx1);
+    named_barrier_sync(1, 256);
+    const float mx = fmaxf(xmax[(buf * 2 + half) * 128 + row], xmax[(buf * 2 + (half ^ 1)) * 128 + row]) * c;
+    // running maximum with lazy rescaling (both halves take the same decision)
     const float m_new = fmaxf(m, mx);
     float m_use = m, alpha = 1.f;
     bool rescale_o = false;
     if (m == -INFINITY) {
-      m_use = m_new;  // first block with a visible key: nothing accumulated yet
+      m_use = m_new;  // first block: nothing accumulated yet
     } else if (m_new > m + kRescaleThreshold) {
       m_use = m_new;
       alpha = fast_exp2(m - m_new);
       rescale_o = true;
     }
-    // P = 2^(x - m_use) as bf16 pairs into the first 64 columns of S_t; row sum in fp32
-    float sum = 0.f;
+    // P = 2^(s c - m_use) as bf16 pairs: this half's keys go to 32 of the first 64 S columns
+    float sum0 = 0.f, sum1 = 0.f;
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
+    for (int cc = 0; cc < 2; ++cc) {
       uint32_t pk[16];
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
-        const float p0 = fast_exp2(__uint_as_float(sr[c][2 * i]) - m_use);
-        const float p1 = fast_exp2(__uint_as_float(sr[c][2 * i + 1]) - m_use);
-        sum += p0 + p1;
+        float x0, x1;
+        ffma2(x0, x1, sr[cc * 32 + 2 * i], sr[cc * 32 + 2 * i + 1], c, -m_use);
+        const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+        fadd2(sum0, sum1, p0, p1);
         pk[i] = pack_bf16x2(p0, p1);
       }
-      tc::st16(lane_addr + colS + c * 16, pk);
+      tc::st16(lane_addr + colS + half * 32 + cc * 16, pk);
     }
-    l = l * alpha + sum;
+    l = l * alpha + (sum0 + sum1);
     m = m_use;
-    if (rescale_o) {
-      // O_t must hold the result of every earlier block before it is rescaled
-      if (!wait_bar(bar(kBarO + t), (uint32_t)((j - 1) & 1), abort, a.err)) { ok = false; }
+    if (rescale_o && j > 0) {
+      // O must hold every earlier block's contribution before it is rescaled
+      if (!wait_bar(bar(kBarO), (uint32_t)((j - 1) & 1), abort, a.err)) ok = false;
       if (ok) {
         tc::fence_after_sync();
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
+        for (int cc = 0; cc < kOHalf / 32; ++cc) {
           uint32_t o[32];
-          tc::ld32(lane_addr + colO + c * 32, o);
+          tc::ld32(lane_addr + C::kColO + half * kOHalf + cc * 32, o);
           tc::wait_ld();
 #pragma unroll
           for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-          tc::st32(lane_addr + colO + c * 32, o);
+          tc::st32(lane_addr + C::kColO + half * kOHalf + cc * 32, o);
         }
       }
     }
     tc::wait_st();
-    if (t == 0 && j == nb - 1 && key0 + kBN > tile.kv) {
+    const int bkey0 = j * kBN;
+    if (ok && j == nb - 1 && bkey0 + kBN > tile.kv && (C::kNch == 2 || half == 0)) {
       // V rows at or past kv_len get weight 0 but may hold anything (NaN included): zero them in
-      // shared memory so 0 * V stays 0. The block's V must have landed first.
-      const int s = j & 1;
-      if (wait_bar(bar(kBarVFull + s), (uint32_t)((j >> 1) & 1), abort, a.err)) {
-        const int first_bad = tile.kv - key0;
-        if (row >= first_bad) {
-          const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+      // shared memory so 0 * V stays 0 (each half zeroes its own 64-column chunk). The block's V
+      // must have landed first.
+      const int vs = j % kVStages;
+      if (wait_bar(bar(kBarVFull + vs), (uint32_t)((j / kVStages) & 1), abort, a.err)) {
+        if (row >= tile.kv - bkey0) {
 #pragma unroll
-          for (int ch = 0; ch < C::kNch; ++ch)
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              const uint32_t addr = sV + s * C::kKVBytes + ch * C::kKVChunk + row * 128 + i * 16;
-              asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(z.x),
-                           "r"(z.y), "r"(z.z), "r"(z.w)
-                           : "memory");
-            }
+          for (int k = 0; k < 8; ++k) {
+            const uint32_t addr = sV + vs * C::kKVBytes + (C::kNch == 2 ? half : 0) * C::kKVChunk + row * 128 + k * 16;
+            asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(addr), "r"(0u) : "memory");
+          }
         }
         tc::fence_proxy_async_smem();
       } else {
@@ -265,27 +340,32 @@ __device__ __forceinline__ void softmax_role(const PArgs& a, const Tile& tile, i
       }
     }
     tc::fence_before_sync();
-    mbar_arrive(bar(kBarP + t));
+    mbar_arrive(bar(kBarP + buf));
   }
-  if (!ok || nb == 0) {
-    if (nb == 0 && store_row) {  // invalid request: zero row
-      __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(a.o) +
-                           (((long long)tile.b * a.h_q + tile.g * a.r + tile.hb * a.H + h) * a.S_q + qi) * D;
-      for (int c = 0; c < D; ++c) out[c] = __float2bfloat16_rn(0.f);
-      if (a.lse) a.lse[((long long)tile.b * a.h_q + tile.g * a.r + tile.hb * a.H + h) * a.S_q + qi] = -INFINITY;
+  if (nb == 0) {  // invalid request: zero row
+    if (store_row) {
+      __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(a.o) + orow * D;
+      for (int cc = half * kOHalf; cc < (half + 1) * kOHalf; ++cc) out[cc] = __float2bfloat16_rn(0.f);
+      if (a.lse && half == 0) a.lse[orow] = -INFINITY;
     }
     return;
   }
-  // epilogue: O / l -> bf16 -> global; lse = (m + log2 l) * ln 2
-  if (!wait_bar(bar(kBarO + t), (uint32_t)((nb - 1) & 1), abort, a.err)) return;
+  // row sum over both halves (every softmax thread reaches this barrier, aborted or not)
+  float* xsum = xbuf + 4 * 128;
+  xsum[half * 128 + row] = l;
+  named_barrier_sync(1, 256);
+  l += xsum[(half ^ 1) * 128 + row];
+  (void)sm_tid;
+  if (!ok) return;
+  // epilogue: this half of O / l -> bf16 -> global; lse = (m + log2 l) * ln 2
+  if (!wait_bar(bar(kBarO), (uint32_t)((nb - 1) & 1), abort, a.err)) return;
   tc::fence_after_sync();
   const float inv = 1.f / l;
-  const long long orow = ((long long)tile.b * a.h_q + tile.g * a.r + tile.hb * a.H + h) * a.S_q + qi;
-  uint4* out = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.o) + orow * D);
+  uint4* out = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.o) + orow * D + half * kOHalf);
 #pragma unroll
-  for (int c = 0; c < D / 32; ++c) {
+  for (int cc = 0; cc < kOHalf / 32; ++cc) {
     uint32_t o[32];
-    tc::ld32(lane_addr + colO + c * 32, o);
+    tc::ld32(lane_addr + C::kColO + half * kOHalf + cc * 32, o);
     tc::wait_ld();
     uint32_t pk[16];
 #pragma unroll
@@ -294,10 +374,10 @@ __device__ __forceinline__ void softmax_role(const PArgs& a, const Tile& tile, i
     if (store_row) {
 #pragma unroll
       for (int v = 0; v < 4; ++v)
-        out[c * 4 + v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+        out[cc * 4 + v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
     }
   }
-  if (store_row && a.lse) a.lse[orow] = (m + __log2f(l)) * kLn2;
+  if (store_row && a.lse && half == 0) a.lse[orow] = (m + __log2f(l)) * kLn2;
 }
 
 template <int D>
@@ -312,6 +392,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kNumBars);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* xbuf = reinterpret_cast<float*>(smem + C::kOffX);  // softmax max/sum exchange
   const uint32_t sQ = smem_u32(smem + C::kOffQ);
   const uint32_t sK = smem_u32(smem + C::kOffK);
   const uint32_t sV = smem_u32(smem + C::kOffV);
@@ -322,16 +403,20 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(bar(kBarQ), 1);
-    for (int s = 0; s < kStages; ++s) {
+    mbar_init(bar(kBarQT), 256);
+    for (int s = 0; s < kKStages; ++s) {
       mbar_init(bar(kBarKFull + s), 1);
+      mbar_init(bar(kBarKEmpty + s), 1);
+    }
+    for (int s = 0; s < kVStages; ++s) {
       mbar_init(bar(kBarVFull + s), 1);
-      mbar_init(bar(kBarKVEmpty + s), 1);
+      mbar_init(bar(kBarVEmpty + s), 1);
     }
-    for (int t = 0; t < 2; ++t) {
-      mbar_init(bar(kBarS + t), 1);
-      mbar_init(bar(kBarP + t), 128);
-      mbar_init(bar(kBarO + t), 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar(kBarS + b), 1);
+      mbar_init(bar(kBarP + b), 256);
     }
+    mbar_init(bar(kBarO), 1);
     mbar_init(bar(kBarDone), 1);
     *abort = 0;
     fence_barrier_init();
@@ -354,99 +439,83 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&tmk);
     tma_prefetch_desc(&tmv);
     const int zq = tile.b * a.h_q + tile.g * a.r + tile.hb * a.H;  // first head of the block
-    const uint32_t qbytes = (uint32_t)(C::kNch * a.H * a.P * 128);
-    mbar_arrive_expect_tx(bar(kBarQ), 2 * qbytes);
-    for (int t = 0; t < 2; ++t)
-      for (int ch = 0; ch < C::kNch; ++ch)
-        tma_load_3d(sQ + t * C::kQBytes + ch * C::kQChunk, &tmq, bar(kBarQ), ch * 64,
-                    tile.q0 + t * a.P, zq);
+    mbar_arrive_expect_tx(bar(kBarQ), (uint32_t)(C::kNch * a.H * a.P * 128));
+    for (int ch = 0; ch < C::kNch; ++ch)
+      tma_load_3d(sQ + ch * C::kQChunk, &tmq, bar(kBarQ), ch * 64, tile.q0, zq);
     const int row0 = (tile.b * a.h_kv + tile.g) * a.T_max;
-    int last_fill[kStages] = {-1, -1};
-    bool ok = true;
-    for (int j = 0; j < nb && ok; ++j) {
-      const int s = j & 1, n = j >> 1;
-      if (n > 0 && !wait_bar(bar(kBarKVEmpty + s), (uint32_t)((n - 1) & 1), abort, a.err)) {
-        ok = false;
-        break;
-      }
-      mbar_arrive_expect_tx(bar(kBarKFull + s), C::kKVBytes);
+    int last_k[kKStages], last_v[kVStages];
+    for (int s = 0; s < kKStages; ++s) last_k[s] = -1;
+    for (int s = 0; s < kVStages; ++s) last_v[s] = -1;
+    for (int j = 0; j < nb; ++j) {
+      const int ks = j % kKStages, kn = j / kKStages;
+      if (kn > 0 && !wait_bar(bar(kBarKEmpty + ks), (uint32_t)((kn - 1) & 1), abort, a.err)) break;
+      mbar_arrive_expect_tx(bar(kBarKFull + ks), C::kKVBytes);
       for (int ch = 0; ch < C::kNch; ++ch)
-        tma_load_2d(sK + s * C::kKVBytes + ch * C::kKVChunk, &tmk, bar(kBarKFull + s), ch * 64,
+        tma_load_2d(sK + ks * C::kKVBytes + ch * C::kKVChunk, &tmk, bar(kBarKFull + ks), ch * 64,
                     row0 + j * kBN);
-      mbar_arrive_expect_tx(bar(kBarVFull + s), C::kKVBytes);
+      last_k[ks] = kn;
+      const int vs = j % kVStages, vn = j / kVStages;
+      if (vn > 0 && !wait_bar(bar(kBarVEmpty + vs), (uint32_t)((vn - 1) & 1), abort, a.err)) break;
+      mbar_arrive_expect_tx(bar(kBarVFull + vs), C::kKVBytes);
       for (int ch = 0; ch < C::kNch; ++ch)
-        tma_load_2d(sV + s * C::kKVBytes + ch * C::kKVChunk, &tmv, bar(kBarVFull + s), ch * 64,
+        tma_load_2d(sV + vs * C::kKVBytes + ch * C::kKVChunk, &tmv, bar(kBarVFull + vs), ch * 64,
                     row0 + j * kBN);
-      last_fill[s] = n;
+      last_v[vs] = vn;
     }
     // Drain (bounded, whatever the abort state): no copy may still be landing in shared memory
     // when the CTA exits.
     volatile int no_abort = 0;
     wait_bar(bar(kBarQ), 0, &no_abort, a.err);
-    for (int s = 0; s < kStages; ++s) {
-      if (last_fill[s] < 0) continue;
-      wait_bar(bar(kBarKFull + s), (uint32_t)(last_fill[s] & 1), &no_abort, a.err);
-      wait_bar(bar(kBarVFull + s), (uint32_t)(last_fill[s] & 1), &no_abort, a.err);
-    }
+    for (int s = 0; s < kKStages; ++s)
+      if (last_k[s] >= 0) wait_bar(bar(kBarKFull + s), (uint32_t)(last_k[s] & 1), &no_abort, a.err);
+    for (int s = 0; s < kVStages; ++s)
+      if (last_v[s] >= 0) wait_bar(bar(kBarVFull + s), (uint32_t)(last_v[s] & 1), &no_abort, a.err);
   } else if (warp == 1 && lane == 0 && nb > 0) {
     // ------------------------------ MMA issuer ---------------------------------------------
     constexpr uint32_t idesc_qk = tc::idesc_bf16(kBM, kBN, false);
     constexpr uint32_t idesc_pv = tc::idesc_bf16(kBM, D, true);
-    const uint32_t colS[2] = {C::kColS0, C::kColS1};
-    const uint32_t colO[2] = {C::kColO0, C::kColO1};
-    auto qk = [&](int t, int s) {  // S_t = Q_t K_s^T, K-major operands, 16 columns per MMA
+    auto colS = [](int buf) { return buf ? C::kColS1 : C::kColS0; };
+    auto qk = [&](int j, int buf) {  // S_buf = Q K_j^T; Q (A) from TMEM, 8 columns per 16 of d_h
+      const int ks = j % kKStages;
 #pragma unroll
-      for (int ks = 0; ks < D / 16; ++ks) {
-        const uint32_t off = (uint32_t)((ks >> 2) * C::kQChunk + (ks & 3) * 32);
-        const uint32_t koff = (uint32_t)((ks >> 2) * C::kKVChunk + (ks & 3) * 32);
-        const uint64_t ad = tc::smem_desc(sQ + t * C::kQBytes + off, 16, 1024);
-        const uint64_t bd = tc::smem_desc(sK + s * C::kKVBytes + koff, 16, 1024);
-        tc::mma_ss(tmem + colS[t], ad, bd, idesc_qk, ks > 0 ? 1u : 0u);
+      for (int k = 0; k < D / 16; ++k) {
+        const uint32_t koff = (uint32_t)((k >> 2) * C::kKVChunk + (k & 3) * 32);
+        const uint64_t bd = tc::smem_desc(sK + ks * C::kKVBytes + koff, 16, 1024);
+        tc::mma_ts(tmem + colS(buf), tmem + C::kColQ + k * 8, bd, idesc_qk, k > 0 ? 1u : 0u);
       }
     };
-    auto pv = [&](int t, int s, bool acc) {  // O_t += P_t V_s; P in TMEM (8 columns per 16 keys)
+    auto pv = [&](int j, int buf) {  // O += P_buf V_j; P (A) from TMEM, 8 columns per 16 keys
+      const int vs = j % kVStages;
 #pragma unroll
       for (int kk = 0; kk < kBN / 16; ++kk) {
-        const uint64_t bd = tc::smem_desc(sV + s * C::kKVBytes + kk * 2048, C::kKVChunk, 1024);
-        tc::mma_ts(tmem + colO[t], tmem + colS[t] + kk * 8, bd, idesc_pv,
-                   (acc || kk > 0) ? 1u : 0u);
+        const uint64_t bd = tc::smem_desc(sV + vs * C::kKVBytes + kk * 2048, C::kKVChunk, 1024);
+        tc::mma_ts(tmem + C::kColO, tmem + colS(buf) + kk * 8, bd, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
       }
     };
-    bool ok = wait_bar(bar(kBarQ), 0, abort, a.err);
-    if (ok) ok = wait_bar(bar(kBarKFull + 0), 0, abort, a.err);
-    if (ok) {
+    bool ok = wait_bar(bar(kBarQT), 0, abort, a.err);
+    for (int j = 0; j < 2 && j < nb && ok; ++j) {
+      ok = wait_bar(bar(kBarKFull + j % kKStages), (uint32_t)((j / kKStages) & 1), abort, a.err);
+      if (!ok) break;
       tc::fence_after_sync();
-      qk(0, 0);
-      tc::commit(bar(kBarS + 0));
-      qk(1, 0);
-      tc::commit(bar(kBarS + 1));
+      qk(j, j & 1);
+      tc::commit(bar(kBarS + (j & 1)));
+      tc::commit(bar(kBarKEmpty + j % kKStages));
     }
     for (int j = 0; j < nb && ok; ++j) {
-      const int s = j & 1;
-      const uint32_t ph = (uint32_t)((j >> 1) & 1);
-      const int s1 = (j + 1) & 1;
-      const uint32_t ph1 = (uint32_t)(((j + 1) >> 1) & 1);
-      if (!wait_bar(bar(kBarVFull + s), ph, abort, a.err)) break;
-      // sub-tile 0
-      if (!wait_bar(bar(kBarP + 0), (uint32_t)(j & 1), abort, a.err)) break;
+      const int buf = j & 1;
+      if (!wait_bar(bar(kBarVFull + j % kVStages), (uint32_t)((j / kVStages) & 1), abort, a.err)) break;
+      if (!wait_bar(bar(kBarP + buf), (uint32_t)((j >> 1) & 1), abort, a.err)) break;
       tc::fence_after_sync();
-      pv(0, s, j > 0);
-      tc::commit(bar(kBarO + 0));
-      if (j + 1 < nb) {
-        if (!wait_bar(bar(kBarKFull + s1), ph1, abort, a.err)) break;
+      pv(j, buf);
+      tc::commit(bar(kBarO));
+      tc::commit(bar(kBarVEmpty + j % kVStages));
+      const int jn = j + 2;
+      if (jn < nb) {
+        if (!wait_bar(bar(kBarKFull + jn % kKStages), (uint32_t)((jn / kKStages) & 1), abort, a.err)) break;
         tc::fence_after_sync();
-        qk(0, s1);
-        tc::commit(bar(kBarS + 0));
-      }
-      // sub-tile 1
-      if (!wait_bar(bar(kBarP + 1), (uint32_t)(j & 1), abort, a.err)) break;
-      tc::fence_after_sync();
-      pv(1, s, j > 0);
-      tc::commit(bar(kBarO + 1));
-      tc::commit(bar(kBarKVEmpty + s));  // K_j and V_j are no longer read
-      if (j + 1 < nb) {
-        qk(1, s1);
-        tc::commit(bar(kBarS + 1));
+        qk(jn, buf);
+        tc::commit(bar(kBarS + buf));
+        tc::commit(bar(kBarKEmpty + jn % kKStages));
       }
     }
     // every MMA issued above has completed before TMEM is released
@@ -454,7 +523,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     volatile int no_abort = 0;
     wait_bar(bar(kBarDone), 0, &no_abort, a.err);
   } else if (warp >= 4) {
-    softmax_role<D>(a, tile, warp, lane, tmem, sV, bars, abort);
+    softmax_role<D>(a, tile, warp, lane, tmem, sQ, sV, bars, xbuf, abort);
   }
 
   tc::fence_before_sync();
@@ -484,7 +553,7 @@ cudaError_t launch_prefill_bf16(const PrefillArgs& a, const CUtensorMap* tmaps, 
   p.H = prefill_heads_per_tile(a.h_q, a.h_kv);
   p.P = pf::kBM / p.H;
   p.hblocks = (p.r + p.H - 1) / p.H;
-  p.n_qt = (a.S_q + 2 * p.P - 1) / (2 * p.P);
+  p.n_qt = (a.S_q + p.P - 1) / p.P;
   p.scale_log2 = a.scale * pf::kLog2e;
   p.causal = a.causal;
   p.err = a.err;

@@ -242,38 +242,45 @@ __device__ __forceinline__ void softmax_role(const PArgs& a, const Tile& tile, i
   mbar_arrive(bar(kBarQT));
 
   float m = -INFINITY, l = 0.f;
-  for (int j = 0; j < nb && ok; ++j) {
+  for (int j = 0; j < nb; ++j) {
     const int buf = j & 1;
     const uint32_t colS = buf ? C::kColS1 : C::kColS0;
-    if (!wait_bar(bar(kBarS + buf), (uint32_t)((j >> 1) & 1), abort, a.err)) { ok = false; break; }
-    tc::fence_after_sync();
-    uint32_t su[2][32];
-    tc::ld32(lane_addr + colS + half * 64, su[0]);
-    tc::ld32(lane_addr + colS + half * 64 + 32, su[1]);
-    tc::wait_ld();
+    // After a failed wait the loop keeps running (without touching TMEM or other barriers) so
+    // that every softmax thread takes the per-block named barrier the same number of times.
+    if (ok) ok = wait_bar(bar(kBarS + buf), (uint32_t)((j >> 1) & 1), abort, a.err);
     float sr[64];
-#pragma unroll
-    for (int i = 0; i < 64; ++i) sr[i] = __uint_as_float(su[i >> 5][i & 31]);
+    float lmx = 0.f;
     const int key0 = j * kBN + half * 64;     // first key of this half
     const bool need_mask =
         (a.causal && (long long)key0 + 63 > pos_min) || key0 + 64 > tile.kv;
-    if (need_mask) {
+    if (ok) {
+      tc::fence_after_sync();
+      uint32_t su[2][32];
+      tc::ld32(lane_addr + colS + half * 64, su[0]);
+      tc::ld32(lane_addr + colS + half * 64 + 32, su[1]);
+      tc::wait_ld();
 #pragma unroll
-      for (int i = 0; i < 64; ++i) {
-        const int key = key0 + i;
-        const bool vis = key < tile.kv && (!a.causal || key <= pos);
-        sr[i] = vis ? sr[i] : -INFINITY;
+      for (int i = 0; i < 64; ++i) sr[i] = __uint_as_float(su[i >> 5][i & 31]);
+      if (need_mask) {
+#pragma unroll
+        for (int i = 0; i < 64; ++i) {
+          const int key = key0 + i;
+          const bool vis = key < tile.kv && (!a.causal || key <= pos);
+          sr[i] = vis ? sr[i] : -INFINITY;
+        }
       }
-    }
-    float mx0 = sr[0], mx1 = sr[1];
+      float mx0 = sr[0], mx1 = sr[1];
 #pragma unroll
-    for (int i = 2; i < 64; i += 2) {
-      mx0 = fmaxf(mx0, sr[i]);
-      mx1 = fmaxf(mx1, sr[i + 1]);
+      for (int i = 2; i < 64; i += 2) {
+        mx0 = fmaxf(mx0, sr[i]);
+        mx1 = fmaxf(mx1, sr[i + 1]);
+      }
+      lmx = fmaxf(mx0, mx1);
     }
-    // block maximum over both halves of the row
-    xmax[(buf * 2 + half) * 128 + row] = fmaxf(mx0, mx1);
+    // block maximum over both halves of the row (double-buffered exchange slot per S buffer)
+    xmax[(buf * 2 + half) * 128 + row] = lmx;
     named_barrier_sync(1, 256);
+    if (!ok) continue;
     const float mx = fmaxf(xmax[(buf * 2 + half) * 128 + row], xmax[(buf * 2 + (half ^ 1)) * 128 + row]) * c;
     // running maximum with lazy rescaling (both halves take the same decision)
     const float m_new = fmaxf(m, mx);

@@ -28,6 +28,7 @@ from .attention_ref import (
 )
 from .online_softmax import online_softmax_row, merge_states, blockwise_attention_row
 from .kv_append_ref import kv_append_ref
+from .paged import gather_pages, paged_append_ref, paged_decode_ref
 from . import ledgers
 
 __all__ = [
@@ -40,5 +41,8 @@ __all__ = [
     "merge_states",
     "blockwise_attention_row",
     "kv_append_ref",
+    "gather_pages",
+    "paged_decode_ref",
+    "paged_append_ref",
     "ledgers",
 ]

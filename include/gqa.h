@@ -65,7 +65,8 @@ enum {
   GQA_DEVERR_POSITION = 2,    /* q_start/q_pos < 0, or an append that does not fit in T_max       */
   GQA_DEVERR_NO_VISIBLE = 3,  /* a query row that sees no key (e.g. q_start + i < 0 is impossible,
                                  but kv_len = 0 with a valid position is)                          */
-  GQA_DEVERR_TIMEOUT = 4      /* a bounded pipeline wait ran out (the kernel returned early)      */
+  GQA_DEVERR_TIMEOUT = 4,     /* a bounded pipeline wait ran out (the kernel returned early)      */
+  GQA_DEVERR_PAGE = 5         /* a block-table entry outside [0, num_pages) (paged cache)          */
 };
 
 /*
@@ -169,6 +170,49 @@ gqa_status gqa_decode_noalloc(const void* q, const void* k_cache, const void* v_
 gqa_status kv_append(void* k_cache, void* v_cache, const void* k_new, const void* v_new,
                      const int32_t* pos, int B, int h_kv, int S_new, int T_max, int d_h,
                      gqa_dtype dtype, void* stream);
+
+/*
+ * Paged KV cache. The pages name page metadata and fragmentation as the deployment cost of a
+ * cache that grows token by token [第三章, section 3.6; MHA/MQA/GQA walkthrough, section 8, the
+ * ledger's note on page metadata]. A paged cache keeps K and V in pools of fixed-size pages
+ *   k_pages, v_pages (num_pages, h_kv, page_size, d_h)
+ * and a block table (B, max_pages) of int32 page indices: logical position t of sequence b is row
+ * t % page_size of page block_table[b * max_pages + t / page_size]. Pages may be shared or in any
+ * order; entries for positions a call does not touch are never read. Attention over a paged
+ * cache is, by definition, attention over the contiguous cache the pages spell out, so the
+ * results equal gqa_decode's on that cache (to floating-point rounding; chunk boundaries fall on
+ * multiples of 16 keys here).
+ *
+ * gqa_decode_paged - gqa_decode over a paged cache. T_max is max_pages * page_size.
+ *   page_size  a multiple of 16 (every 16-key sub-tile the kernel loads lies inside one page).
+ *   num_pages * h_kv * page_size must stay below 2^31 (pool rows are addressed with 32 bits).
+ *   block_table device int32 (B, max_pages), row-major. An entry outside [0, num_pages) that a
+ *            call needs is replaced by page 0 and sets GQA_DEVERR_PAGE (the output is then wrong).
+ *   workspace  as gqa_decode, sized by gqa_decode_workspace_size(B, h_q, h_kv,
+ *            max_pages * page_size, d_h, dtype, num_splits).
+ * Other arguments and errors as gqa_decode.
+ */
+gqa_status gqa_decode_paged(const void* q, const void* k_pages, const void* v_pages, void* o,
+                            float* lse, const int32_t* kv_len, const int32_t* q_pos,
+                            const int32_t* block_table, int B, int h_q, int h_kv, int num_pages,
+                            int page_size, int max_pages, int d_h, float scale, gqa_dtype dtype,
+                            void* workspace, size_t workspace_bytes, int num_splits, void* stream);
+
+/*
+ * kv_append_paged - kv_append into a paged cache: new[b, g, t, :] goes to logical position
+ * pos[b] + t, i.e. row (pos[b] + t) % page_size of page block_table[b, (pos[b] + t) / page_size].
+ * Bit-exact; no other byte of the pools is written.
+ *   k_pages, v_pages (num_pages, h_kv, page_size, d_h), written in place; page_size >= 1.
+ *   k_new, v_new     (B, h_kv, S_new, d_h).
+ *   pos      device int32[B]. Sequences whose rows would leave [0, max_pages * page_size) are not
+ *            written (GQA_DEVERR_POSITION); rows whose page entry is outside [0, num_pages) are
+ *            not written (GQA_DEVERR_PAGE).
+ * Errors: INVALID_ARG, CUDA.
+ */
+gqa_status kv_append_paged(void* k_pages, void* v_pages, const void* k_new, const void* v_new,
+                           const int32_t* pos, const int32_t* block_table, int B, int h_kv,
+                           int S_new, int num_pages, int page_size, int max_pages, int d_h,
+                           gqa_dtype dtype, void* stream);
 
 /*
  * gqa_get_device_error - synchronise `stream`, then read and clear the sticky device error word

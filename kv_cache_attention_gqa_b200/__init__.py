@@ -1,4 +1,5 @@
-"""Causal grouped-query attention on B200 (sm_100a): prefill, split-KV decode and KV append.
+"""Causal grouped-query attention on B200 (sm_100a): prefill, split-KV decode and KV append,
+over a contiguous or a paged KV cache.
 
 The computation lives in the CUDA library ``libgqa_b200.so`` behind the C ABI of
 ``include/gqa.h``; this package is a thin ctypes binding over it (``_lib``) plus the build script
@@ -10,9 +11,11 @@ from ._lib import (  # noqa: F401
     LIB_PATH,
     decode,
     decode_noalloc,
+    decode_paged,
     decode_workspace_size,
     get_device_error,
     kv_append,
+    kv_append_paged,
     prefill,
     status_string,
     version,

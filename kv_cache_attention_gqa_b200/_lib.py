@@ -29,7 +29,8 @@ STATUS_NAMES = {
 }
 GQA_BF16, GQA_FP32 = 0, 1
 DEVERR_NAMES = {0: "none", 1: "kv_len out of range", 2: "position out of range",
-                3: "query with no visible key", 4: "pipeline wait timed out"}
+                3: "query with no visible key", 4: "pipeline wait timed out",
+                5: "block-table entry out of range"}
 
 # name -> (restype, argtypes), mirroring include/gqa.h
 _P, _I, _F, _Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
@@ -39,6 +40,9 @@ SIGNATURES = {
     "gqa_decode": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _P, _Z, _I, _P]),
     "gqa_decode_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _I, _P]),
     "kv_append": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P]),
+    "gqa_decode_paged": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I,
+                              _P, _Z, _I, _P]),
+    "kv_append_paged": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P]),
     "gqa_get_device_error": (_I, [ctypes.POINTER(_I), _P]),
     "gqa_status_string": (ctypes.c_char_p, [_I]),
     "gqa_version": (ctypes.c_char_p, []),
@@ -256,3 +260,72 @@ def decode_noalloc(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor
                                                          _ptr(lse), _ptr(kl), _ptr(qp), B, h_q, h_kv, T_max,
                                                          d_h, scale, dt, num_splits, _stream()))
     return (out, lse) if return_lse else out
+
+
+def _block_table(block_table, B: int, device) -> torch.Tensor:
+    t = block_table
+    if not (isinstance(t, torch.Tensor) and t.is_cuda and t.dtype == torch.int32 and t.is_contiguous()):
+        t = torch.as_tensor(block_table, dtype=torch.int32, device=device).contiguous()
+    if t.dim() != 2 or t.shape[0] != B:
+        raise ValueError("block_table must be (B, max_pages)")
+    return t
+
+
+def _pool_shape(k_pages: torch.Tensor, v_pages: torch.Tensor):
+    if k_pages.dim() != 4 or v_pages.shape != k_pages.shape:
+        raise ValueError("k_pages / v_pages must both be (num_pages, h_kv, page_size, d_h)")
+    return k_pages.shape
+
+
+def decode_paged(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.Tensor, block_table, *,
+                 kv_len=None, q_pos=None, scale: float | None = None, num_splits: int = 0,
+                 out=None, return_lse: bool = False, ws: torch.Tensor | None = None):
+    """Split-KV decode of q (B, h_q, d_h) over a paged cache: pools (num_pages, h_kv, page_size,
+    d_h) and block_table (B, max_pages) int32; position t of sequence b is row t % page_size of
+    page block_table[b, t // page_size]."""
+    _need_cuda(q, k_pages, v_pages, out)
+    B, h_q, d_h = q.shape
+    num_pages, h_kv, page_size, dk = _pool_shape(k_pages, v_pages)
+    if dk != d_h:
+        raise ValueError("q and the page pools disagree on d_h")
+    dt = _dtype_code(q)
+    if k_pages.dtype != q.dtype or v_pages.dtype != q.dtype:
+        raise TypeError("q, k_pages and v_pages must share one dtype")
+    bt = _block_table(block_table, B, q.device)
+    max_pages = bt.shape[1]
+    if out is None:
+        out = torch.empty_like(q)
+    lse = torch.empty((B, h_q), dtype=torch.float32, device=q.device) if return_lse else None
+    kl = _int_vec(kv_len, B, q.device, "kv_len")
+    qp = _int_vec(q_pos, B, q.device, "q_pos")
+    scale = 1.0 / math.sqrt(d_h) if scale is None else float(scale)
+    T_max = max_pages * page_size
+    key = (B, h_q, h_kv, T_max, d_h, dt, num_splits, q.device.index)
+    need = _ws_sizes.get(key)
+    if need is None:
+        need = _ws_sizes[key] = decode_workspace_size(B, h_q, h_kv, T_max, d_h, q.dtype, num_splits)
+    if ws is None:
+        ws = workspace(need, q.device)
+    _check("gqa_decode_paged", _lib.gqa_decode_paged(
+        _ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(out), _ptr(lse), _ptr(kl), _ptr(qp), _ptr(bt),
+        B, h_q, h_kv, num_pages, page_size, max_pages, d_h, scale, dt, _ptr(ws), ws.numel(),
+        num_splits, _stream()))
+    return (out, lse) if return_lse else out
+
+
+def kv_append_paged(k_pages: torch.Tensor, v_pages: torch.Tensor, k_new: torch.Tensor,
+                    v_new: torch.Tensor, pos, block_table) -> None:
+    """Write new[b, g, t] at logical position pos[b] + t of a paged cache (in place, bit-exact)."""
+    _need_cuda(k_pages, v_pages, k_new, v_new)
+    num_pages, h_kv, page_size, d_h = _pool_shape(k_pages, v_pages)
+    if k_new.dim() != 4 or k_new.shape != v_new.shape or k_new.shape[1] != h_kv or k_new.shape[3] != d_h:
+        raise ValueError("k_new / v_new must be (B, h_kv, S_new, d_h)")
+    B = k_new.shape[0]
+    dt = _dtype_code(k_pages)
+    if any(t.dtype != k_pages.dtype for t in (v_pages, k_new, v_new)):
+        raise TypeError("all four tensors must share one dtype")
+    bt = _block_table(block_table, B, k_pages.device)
+    pos_t = _int_vec(pos, B, k_pages.device, "pos")
+    _check("kv_append_paged", _lib.kv_append_paged(
+        _ptr(k_pages), _ptr(v_pages), _ptr(k_new), _ptr(v_new), _ptr(pos_t), _ptr(bt), B, h_kv,
+        k_new.shape[2], num_pages, page_size, bt.shape[1], d_h, dt, _stream()))

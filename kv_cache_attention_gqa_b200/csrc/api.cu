@@ -80,6 +80,78 @@ gqa_status from_cuda(cudaError_t e) { return e == cudaSuccess ? GQA_OK : GQA_ERR
 
 using namespace gqa;
 
+namespace {
+// Shared body of gqa_decode and gqa_decode_paged. A paged call passes block_table != nullptr and
+// T_max = max_pages * page_size; k_cache / v_cache are then the page pools.
+gqa_status decode_impl(const void* q, const void* k_cache, const void* v_cache, void* o, float* lse,
+                       const int32_t* kv_len, const int32_t* q_pos, int B, int h_q, int h_kv,
+                       int T_max, int d_h, float scale, gqa_dtype dtype, void* workspace,
+                       size_t workspace_bytes, int num_splits, void* stream,
+                       const int32_t* block_table, int max_pages, int page_size, int num_pages) {
+  using namespace gqa;
+  if (!q || !k_cache || !v_cache || !o) return GQA_ERR_INVALID_ARG;
+  if (B <= 0 || h_q <= 0 || h_kv <= 0 || T_max <= 0 || d_h <= 0 || num_splits < 0)
+    return GQA_ERR_INVALID_ARG;
+  if (h_q % h_kv != 0 || !valid_scale(scale)) return GQA_ERR_INVALID_ARG;
+  if (dtype != GQA_BF16 && dtype != GQA_FP32) return GQA_ERR_INVALID_ARG;
+  if (B > decode_max_batch()) return GQA_ERR_UNSUPPORTED;
+  if (dtype == GQA_FP32 && d_h > 256) return GQA_ERR_UNSUPPORTED;
+  if (dtype == GQA_BF16 && d_h != 64 && d_h != 128) return GQA_ERR_UNSUPPORTED;
+  const long long cache_rows =
+      block_table ? (long long)num_pages * h_kv * page_size : (long long)B * h_kv * T_max;
+  if (cache_rows >= (1ll << 31) || (long long)B * h_q >= (1ll << 31)) return GQA_ERR_UNSUPPORTED;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return GQA_ERR_WORKSPACE;
+  // the workspace check needs no device query when num_splits is given
+  if (num_splits > 0 && workspace_bytes < decode_workspace_bytes(B, h_q, h_kv, T_max, d_h, num_splits, 1))
+    return GQA_ERR_WORKSPACE;
+  const int sms = sm_count();
+  if (sms <= 0) return GQA_ERR_CUDA;
+  if (workspace_bytes < decode_workspace_bytes(B, h_q, h_kv, T_max, d_h, num_splits, sms))
+    return GQA_ERR_WORKSPACE;
+  DecodeArgs a;
+  a.q = q;
+  a.k = k_cache;
+  a.v = v_cache;
+  a.o = o;
+  a.lse = lse;
+  a.kv_len = kv_len;
+  a.q_pos = q_pos;
+  a.B = B;
+  a.h_q = h_q;
+  a.h_kv = h_kv;
+  a.T_max = T_max;
+  a.d_h = d_h;
+  a.scale = scale;
+  a.workspace = workspace;
+  a.workspace_bytes = workspace_bytes;
+  a.num_splits = num_splits;
+  a.num_sms = sms;
+  a.block_table = block_table;
+  a.max_pages = max_pages;
+  a.page_size = page_size;
+  a.num_pages = num_pages;
+  a.err = device_error_ptr();
+  if (!a.err) return GQA_ERR_CUDA;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (dtype == GQA_FP32) return from_cuda(launch_decode_fp32(a, s));
+  const int r = h_q / h_kv;
+  const uint32_t qrows = r > 16 ? 32 : 16;
+  CUtensorMap maps[3];
+  // K/V: rows of d_h elements; a paged pool is (num_pages * h_kv * page_size) rows loaded in
+  // 16-row boxes (one per 16-key sub-tile), a contiguous cache (B * h_kv * T_max) in 64-row boxes
+  const uint64_t kdims[2] = {(uint64_t)d_h, (uint64_t)cache_rows};
+  const uint64_t qdims[2] = {(uint64_t)d_h, (uint64_t)B * h_q};
+  const uint64_t strides[1] = {(uint64_t)d_h * 2};
+  const uint32_t box[2] = {64, block_table ? 16u : 64u};
+  const uint32_t qbox[2] = {64, qrows};
+  if (!encode_bf16(&maps[0], k_cache, 2, kdims, strides, box) ||
+      !encode_bf16(&maps[1], v_cache, 2, kdims, strides, box) ||
+      !encode_bf16(&maps[2], q, 2, qdims, strides, qbox))
+    return GQA_ERR_CUDA;
+  return from_cuda(launch_decode_bf16(a, maps, s));
+}
+}  // namespace
+
 extern "C" {
 
 const char* gqa_status_string(gqa_status s) {
@@ -203,59 +275,55 @@ gqa_status gqa_decode(const void* q, const void* k_cache, const void* v_cache, v
                       const int32_t* kv_len, const int32_t* q_pos,
                       int B, int h_q, int h_kv, int T_max, int d_h, float scale, gqa_dtype dtype,
                       void* workspace, size_t workspace_bytes, int num_splits, void* stream) {
-  if (!q || !k_cache || !v_cache || !o) return GQA_ERR_INVALID_ARG;
-  if (B <= 0 || h_q <= 0 || h_kv <= 0 || T_max <= 0 || d_h <= 0 || num_splits < 0)
-    return GQA_ERR_INVALID_ARG;
-  if (h_q % h_kv != 0 || !valid_scale(scale)) return GQA_ERR_INVALID_ARG;
+  return decode_impl(q, k_cache, v_cache, o, lse, kv_len, q_pos, B, h_q, h_kv, T_max, d_h, scale,
+                     dtype, workspace, workspace_bytes, num_splits, stream, nullptr, 0, 0, 0);
+}
+
+gqa_status gqa_decode_paged(const void* q, const void* k_pages, const void* v_pages, void* o,
+                            float* lse, const int32_t* kv_len, const int32_t* q_pos,
+                            const int32_t* block_table, int B, int h_q, int h_kv, int num_pages,
+                            int page_size, int max_pages, int d_h, float scale, gqa_dtype dtype,
+                            void* workspace, size_t workspace_bytes, int num_splits, void* stream) {
+  if (!block_table || num_pages <= 0 || page_size <= 0 || max_pages <= 0) return GQA_ERR_INVALID_ARG;
+  if (page_size % 16 != 0) return GQA_ERR_UNSUPPORTED;
+  const long long T_max = (long long)max_pages * page_size;
+  if (T_max >= (1ll << 31)) return GQA_ERR_UNSUPPORTED;
+  return decode_impl(q, k_pages, v_pages, o, lse, kv_len, q_pos, B, h_q, h_kv, (int)T_max, d_h,
+                     scale, dtype, workspace, workspace_bytes, num_splits, stream, block_table,
+                     max_pages, page_size, num_pages);
+}
+
+gqa_status kv_append_paged(void* k_pages, void* v_pages, const void* k_new, const void* v_new,
+                           const int32_t* pos, const int32_t* block_table, int B, int h_kv,
+                           int S_new, int num_pages, int page_size, int max_pages, int d_h,
+                           gqa_dtype dtype, void* stream) {
+  using namespace gqa;
+  if (!k_pages || !v_pages || !k_new || !v_new || !pos || !block_table) return GQA_ERR_INVALID_ARG;
+  if (B <= 0 || h_kv <= 0 || S_new < 0 || d_h <= 0) return GQA_ERR_INVALID_ARG;
+  if (num_pages <= 0 || page_size <= 0 || max_pages <= 0) return GQA_ERR_INVALID_ARG;
   if (dtype != GQA_BF16 && dtype != GQA_FP32) return GQA_ERR_INVALID_ARG;
-  if (B > decode_max_batch()) return GQA_ERR_UNSUPPORTED;
-  if (dtype == GQA_FP32 && d_h > 256) return GQA_ERR_UNSUPPORTED;
-  if (dtype == GQA_BF16 && d_h != 64 && d_h != 128) return GQA_ERR_UNSUPPORTED;
-  if ((long long)B * h_kv * T_max >= (1ll << 31) || (long long)B * h_q >= (1ll << 31))
-    return GQA_ERR_UNSUPPORTED;
-  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return GQA_ERR_WORKSPACE;
-  // the workspace check needs no device query when num_splits is given
-  if (num_splits > 0 && workspace_bytes < decode_workspace_bytes(B, h_q, h_kv, T_max, d_h, num_splits, 1))
-    return GQA_ERR_WORKSPACE;
-  const int sms = sm_count();
-  if (sms <= 0) return GQA_ERR_CUDA;
-  if (workspace_bytes < decode_workspace_bytes(B, h_q, h_kv, T_max, d_h, num_splits, sms))
-    return GQA_ERR_WORKSPACE;
-  DecodeArgs a;
-  a.q = q;
-  a.k = k_cache;
-  a.v = v_cache;
-  a.o = o;
-  a.lse = lse;
-  a.kv_len = kv_len;
-  a.q_pos = q_pos;
+  const long long T_max = (long long)max_pages * page_size;
+  if (T_max >= (1ll << 31)) return GQA_ERR_UNSUPPORTED;
+  if (S_new > T_max) return GQA_ERR_INVALID_ARG;
+  AppendArgs a;
+  a.k_cache = k_pages;
+  a.v_cache = v_pages;
+  a.k_new = k_new;
+  a.v_new = v_new;
+  a.pos = pos;
   a.B = B;
-  a.h_q = h_q;
   a.h_kv = h_kv;
-  a.T_max = T_max;
+  a.S_new = S_new;
+  a.T_max = (int)T_max;
   a.d_h = d_h;
-  a.scale = scale;
-  a.workspace = workspace;
-  a.workspace_bytes = workspace_bytes;
-  a.num_splits = num_splits;
-  a.num_sms = sms;
+  a.elem_bytes = dtype == GQA_BF16 ? 2 : 4;
+  a.block_table = block_table;
+  a.max_pages = max_pages;
+  a.page_size = page_size;
+  a.num_pages = num_pages;
   a.err = device_error_ptr();
   if (!a.err) return GQA_ERR_CUDA;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (dtype == GQA_FP32) return from_cuda(launch_decode_fp32(a, s));
-  const int r = h_q / h_kv;
-  const uint32_t qrows = r > 16 ? 32 : 16;
-  CUtensorMap maps[3];
-  const uint64_t kdims[2] = {(uint64_t)d_h, (uint64_t)B * h_kv * T_max};
-  const uint64_t qdims[2] = {(uint64_t)d_h, (uint64_t)B * h_q};
-  const uint64_t strides[1] = {(uint64_t)d_h * 2};
-  const uint32_t box[2] = {64, 64};
-  const uint32_t qbox[2] = {64, qrows};
-  if (!encode_bf16(&maps[0], k_cache, 2, kdims, strides, box) ||
-      !encode_bf16(&maps[1], v_cache, 2, kdims, strides, box) ||
-      !encode_bf16(&maps[2], q, 2, qdims, strides, qbox))
-    return GQA_ERR_CUDA;
-  return from_cuda(launch_decode_bf16(a, maps, s));
+  return from_cuda(launch_kv_append(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 }  // extern "C"

@@ -108,12 +108,18 @@ struct KArgs {
   float* part_lse;
   float* part_o;
   unsigned* err;
+  // paged cache (block_table != nullptr): K/V live in a pool (num_pages, h_kv, page_size, d_h);
+  // position t of sequence b is row t % page_size of page block_table[b * max_pages + t / page_size]
+  const int32_t* block_table;
+  int max_pages, page_size, num_pages;
+  int gran;  // partition granule in keys: 16 for a paged cache (sub-tiles never straddle a page), else 1
 };
 
 // Partition view built in shared memory by every CTA.
 struct Plan {
-  const long long* pre;  // pre[b] = sum_{b' < b} n_b'
+  const long long* pre;  // pre[b] = sum_{b' < b} ceil(n_b' / gran): positions count granules
   const int* nlen;
+  int gran;
   int UPB;               // units per sequence = h_kv * hblocks
   long long K;           // total keys over all units
   long long C;           // chunk size
@@ -126,7 +132,8 @@ struct Piece {
   int k0, k1;    // key range inside the unit
   int n;         // unit length
   int n_pieces;  // pieces of this unit over all chunks
-  long long unit_start;
+  long long unit_start;  // in granules
+  long long end;         // global position (granules) just past this piece
 };
 
 // The piece that starts at global key position x, inside a chunk ending at x_end.
@@ -142,16 +149,18 @@ __device__ __forceinline__ Piece locate(const Plan& p, int B, int hblocks, long 
   Piece pc;
   pc.b = b;
   pc.n = p.nlen[b];
+  const long long ng = (pc.n + p.gran - 1) / p.gran;  // unit length in granules
   const long long rel = x - p.pre[b] * p.UPB;
-  const int ui = (int)(rel / pc.n);  // g * hblocks + hb
+  const int ui = (int)(rel / ng);  // g * hblocks + hb
   pc.g = ui / hblocks;
   pc.hb = ui - pc.g * hblocks;
   pc.unit = b * p.UPB + ui;
-  pc.unit_start = p.pre[b] * p.UPB + (long long)ui * pc.n;
-  pc.k0 = (int)(x - pc.unit_start);
-  const long long e = x_end - pc.unit_start;
-  pc.k1 = e < pc.n ? (int)e : pc.n;
-  pc.n_pieces = (int)((pc.unit_start + pc.n - 1) / p.C - pc.unit_start / p.C) + 1;
+  pc.unit_start = p.pre[b] * p.UPB + (long long)ui * ng;
+  pc.k0 = (int)((x - pc.unit_start) * p.gran);
+  const long long e = x_end - pc.unit_start;  // granules
+  pc.end = e < ng ? x_end : pc.unit_start + ng;
+  pc.k1 = e < ng ? (int)(e * p.gran) : pc.n;
+  pc.n_pieces = (int)((pc.unit_start + ng - 1) / p.C - pc.unit_start / p.C) + 1;
   return pc;
 }
 
@@ -178,13 +187,14 @@ __device__ void build_plan(const KArgs& a, Plan& p, long long* pre, int* nlen, i
         }
         nlen[b] = n;
       }
-      long long s = n;  // inclusive warp scan
+      const long long ngr = (n + a.gran - 1) / a.gran;  // granules
+      long long s = ngr;  // inclusive warp scan
 #pragma unroll
       for (int off = 1; off < 32; off <<= 1) {
         const long long t = __shfl_up_sync(0xffffffffu, s, off);
         if (lane >= off) s += t;
       }
-      if (b < a.B) pre[b] = run + s - n;
+      if (b < a.B) pre[b] = run + s - ngr;
       run += __shfl_sync(0xffffffffu, s, 31);
     }
     if (lane == 0) pre[a.B] = run;
@@ -192,13 +202,15 @@ __device__ void build_plan(const KArgs& a, Plan& p, long long* pre, int* nlen, i
   __syncthreads();
   p.pre = pre;
   p.nlen = nlen;
+  p.gran = a.gran;
   p.UPB = a.h_kv * a.hblocks;
   p.K = pre[a.B] * p.UPB;
   long long C = (p.K + a.n_max - 1) / a.n_max;
   if (a.auto_chunk) {
     // at least kMinChunkAuto keys, and at least 16 keys per query row, so the partial written per
     // chunk (hpu x d_h fp32) stays small against the chunk's K/V bytes (2 x C x d_h bf16)
-    const long long lo = 16LL * a.hpu > kMinChunkAuto ? 16LL * a.hpu : kMinChunkAuto;
+    const long long lo_keys = 16LL * a.hpu > kMinChunkAuto ? 16LL * a.hpu : kMinChunkAuto;
+    const long long lo = (lo_keys + a.gran - 1) / a.gran;
     if (C < lo) C = lo;
   }
   if (C < 1) C = 1;
@@ -329,8 +341,9 @@ __global__ void __launch_bounds__(256) merge_kernel(KArgs a) {
   if (h >= nh) return;
   const int n = a.nlen[b];
   if (n == 0) return;
-  const long long P = a.pre[b] * UPB + (long long)ui * n;
-  const long long c0 = P / C, c1 = (P + n - 1) / C;
+  const long long ng = (n + a.gran - 1) / a.gran;
+  const long long P = a.pre[b] * UPB + (long long)ui * ng;
+  const long long c0 = P / C, c1 = (P + ng - 1) / C;
   if (c0 == c1) return;  // written directly by the decode kernel
   const int head = g * a.r + hb * a.hpu + h;
   const long long ob = ((long long)b * a.h_q + head) * a.D;
@@ -406,7 +419,7 @@ struct Bf16Cfg {
   static_assert(kSmem <= 227 * 1024, "shared memory budget");
 };
 
-template <int D, int MT>
+template <int D, int MT, bool kPaged>
 __global__ void __launch_bounds__(Bf16Cfg<D, MT>::kThreads, 1)
     decode_bf16_kernel(const __grid_constant__ CUtensorMap tmk,
                        const __grid_constant__ CUtensorMap tmv,
@@ -463,6 +476,24 @@ __global__ void __launch_bounds__(Bf16Cfg<D, MT>::kThreads, 1)
           const int row0 = (pc.b * a.h_kv + pc.g) * a.T_max;
           const int qrow = pc.b * a.h_q + pc.g * a.r + pc.hb * a.hpu;
           for (int t = pc.k0; t < pc.k1; t += kTile) {
+            // paged cache: pool rows of the (up to) four 16-key sub-tiles, looked up before the
+            // wait for a free stage so the block-table reads overlap it
+            int prow[kPaged ? 4 : 1];
+            int nsub = 4;
+            if constexpr (kPaged) {
+              nsub = (min(kTile, pc.k1 - t) + 15) >> 4;
+              const int32_t* bt = a.block_table + (long long)pc.b * a.max_pages;
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                const int key = t + 16 * j;
+                int page = j < nsub ? __ldg(bt + key / a.page_size) : 0;
+                if (page < 0 || page >= a.num_pages) {
+                  set_device_error(a.err, GQA_DEVERR_PAGE);
+                  page = 0;
+                }
+                prow[j] = (page * a.h_kv + pc.g) * a.page_size + key % a.page_size;
+              }
+            }
             if (!mbar_wait(smem_u32(&bars[C::kStages + stage]), phase ^ 1u, a.err)) { ok = false; break; }
             const bool first = t == pc.k0;
             TileMeta m;
@@ -476,13 +507,30 @@ __global__ void __launch_bounds__(Bf16Cfg<D, MT>::kThreads, 1)
             m.pad = 0;
             meta[stage] = m;
             const uint32_t full = smem_u32(&bars[stage]);
-            mbar_arrive_expect_tx(full, C::kStageBytes + (first ? C::kQBytes : 0));
+            // sub-tiles past the tile's valid keys are not loaded on a paged cache (the consumer
+            // warp that owns such a 16-key slice skips it)
+            const uint32_t kv_bytes = kPaged ? (uint32_t)nsub * (C::kStageBytes / 4) : C::kStageBytes;
+            mbar_arrive_expect_tx(full, kv_bytes + (first ? C::kQBytes : 0));
             const uint32_t kdst = smem_u32(stage_base + stage * C::kStageBytes);
             const uint32_t vdst = kdst + C::kTileBytes;
+            if constexpr (kPaged) {
+              // one 16-row box per sub-tile; 16 rows x 128 B = 2 KiB keeps the 128-byte swizzle
+              // atoms (1 KiB) aligned, so the stage has the same layout as one 64-row box
 #pragma unroll
-            for (int ch = 0; ch < C::kNch; ++ch) {
-              tma_load_2d(kdst + ch * C::kChunkBytes, &tmk, full, ch * 64, row0 + t);
-              tma_load_2d(vdst + ch * C::kChunkBytes, &tmv, full, ch * 64, row0 + t);
+              for (int j = 0; j < 4; ++j) {
+                if (j >= nsub) break;
+#pragma unroll
+                for (int ch = 0; ch < C::kNch; ++ch) {
+                  tma_load_2d(kdst + ch * C::kChunkBytes + j * 2048, &tmk, full, ch * 64, prow[j]);
+                  tma_load_2d(vdst + ch * C::kChunkBytes + j * 2048, &tmv, full, ch * 64, prow[j]);
+                }
+              }
+            } else {
+#pragma unroll
+              for (int ch = 0; ch < C::kNch; ++ch) {
+                tma_load_2d(kdst + ch * C::kChunkBytes, &tmk, full, ch * 64, row0 + t);
+                tma_load_2d(vdst + ch * C::kChunkBytes, &tmv, full, ch * 64, row0 + t);
+              }
             }
             if (first) {
               const uint32_t qdst = smem_u32(q_base + stage * C::kQBytes);
@@ -493,7 +541,7 @@ __global__ void __launch_bounds__(Bf16Cfg<D, MT>::kThreads, 1)
             ++issued;
             if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
           }
-          x = pc.unit_start + pc.k1;
+          x = pc.end;
         }
         chunk = next;
         if (chunk < plan.n_chunks) next = G + atomicAdd(&a.hdr->ticket, 1);
@@ -749,6 +797,16 @@ __global__ void __launch_bounds__(32 * kF32Warps, 1) decode_fp32_kernel(KArgs a)
         for (int j = pc.k0; j < pc.k1; ++j) {
           const float* kj = kp + (long long)j * D;
           const float* vj = vp + (long long)j * D;
+          if (a.block_table) {
+            int page = a.block_table[(long long)pc.b * a.max_pages + j / a.page_size];
+            if (page < 0 || page >= a.num_pages) {
+              if (lane == 0) set_device_error(a.err, GQA_DEVERR_PAGE);
+              page = 0;
+            }
+            const long long row = ((long long)page * a.h_kv + pc.g) * a.page_size + j % a.page_size;
+            kj = reinterpret_cast<const float*>(a.k) + row * D;
+            vj = reinterpret_cast<const float*>(a.v) + row * D;
+          }
           float part = 0.f;
 #pragma unroll
           for (int e = 0; e < kF32MaxPerLane; ++e) {
@@ -777,7 +835,7 @@ __global__ void __launch_bounds__(32 * kF32Warps, 1) decode_fp32_kernel(KArgs a)
           if (col < D) emit<float>(a, pc.b, pc.g, pc.hb, slot, hl, col, accv[e] * inv, lse2);
         }
       }
-      x = pc.unit_start + pc.k1;
+      x = pc.end;
     }
   }
 }
@@ -810,10 +868,10 @@ cudaError_t launch_merge(const KArgs& ka, cudaStream_t s) {
   return e;
 }
 
-template <int D, int MT>
+template <int D, int MT, bool kPaged>
 cudaError_t launch_bf16_typed(const KArgs& ka, const CUtensorMap* tm, int grid, cudaStream_t s) {
   using C = Bf16Cfg<D, MT>;
-  auto kern = decode_bf16_kernel<D, MT>;
+  auto kern = decode_bf16_kernel<D, MT, kPaged>;
   static bool attr_set[64] = {false};  // per device: the shared-memory opt-in is set once
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -869,6 +927,11 @@ KArgs make_kargs(const DecodeArgs& a) {
   k.part_lse = reinterpret_cast<float*>(ws + L.lse_off);
   k.part_o = reinterpret_cast<float*>(ws + L.o_off);
   k.err = a.err;
+  k.block_table = a.block_table;
+  k.max_pages = a.max_pages;
+  k.page_size = a.page_size;
+  k.num_pages = a.num_pages;
+  k.gran = a.block_table ? 16 : 1;
   return k;
 }
 
@@ -893,18 +956,26 @@ cudaError_t launch_decode_fp32(const DecodeArgs& a, cudaStream_t s) {
   return dec::launch_merge<float, false>(k, s);
 }
 
-cudaError_t launch_decode_bf16(const DecodeArgs& a, const CUtensorMap* tmaps, cudaStream_t s) {
-  const dec::KArgs k = dec::make_kargs(a);
+namespace dec {
+template <bool kPaged>
+cudaError_t launch_bf16_dispatch(const KArgs& k, const CUtensorMap* tmaps, int grid, cudaStream_t s) {
   const bool two = k.hpu > 16;
-  if (a.d_h == 128) {
-    return two ? dec::launch_bf16_typed<128, 2>(k, tmaps, a.num_sms, s)
-               : dec::launch_bf16_typed<128, 1>(k, tmaps, a.num_sms, s);
+  if (k.D == 128) {
+    return two ? launch_bf16_typed<128, 2, kPaged>(k, tmaps, grid, s)
+               : launch_bf16_typed<128, 1, kPaged>(k, tmaps, grid, s);
   }
-  if (a.d_h == 64) {
-    return two ? dec::launch_bf16_typed<64, 2>(k, tmaps, a.num_sms, s)
-               : dec::launch_bf16_typed<64, 1>(k, tmaps, a.num_sms, s);
+  if (k.D == 64) {
+    return two ? launch_bf16_typed<64, 2, kPaged>(k, tmaps, grid, s)
+               : launch_bf16_typed<64, 1, kPaged>(k, tmaps, grid, s);
   }
   return cudaErrorInvalidValue;
+}
+}  // namespace dec
+
+cudaError_t launch_decode_bf16(const DecodeArgs& a, const CUtensorMap* tmaps, cudaStream_t s) {
+  const dec::KArgs k = dec::make_kargs(a);
+  return a.block_table ? dec::launch_bf16_dispatch<true>(k, tmaps, a.num_sms, s)
+                       : dec::launch_bf16_dispatch<false>(k, tmaps, a.num_sms, s);
 }
 
 }  // namespace gqa

@@ -19,6 +19,9 @@ struct AppendArgs {
   int B, h_kv, S_new, T_max, d_h;
   int elem_bytes;
   unsigned* err;
+  // paged cache (see DecodeArgs); T_max = max_pages * page_size
+  const int32_t* block_table = nullptr;
+  int max_pages = 0, page_size = 0, num_pages = 0;
 };
 cudaError_t launch_kv_append(const AppendArgs& a, cudaStream_t s);
 
@@ -59,6 +62,10 @@ struct DecodeArgs {
   int num_splits;  // 0 = automatic chunking, else the number of chunks to cut the keys into
   int num_sms;     // persistent grid size
   unsigned* err;
+  // paged cache, or block_table == nullptr for the contiguous (B, h_kv, T_max, d_h) layout:
+  // k/v are pools (num_pages, h_kv, page_size, d_h), T_max = max_pages * page_size
+  const int32_t* block_table = nullptr;
+  int max_pages = 0, page_size = 0, num_pages = 0;
 };
 
 // Workspace bytes for a decode of this shape (layout in decode.cu).
@@ -67,7 +74,8 @@ size_t decode_workspace_bytes(int B, int h_q, int h_kv, int T_max, int d_h, int 
 int decode_max_batch();
 
 cudaError_t launch_decode_fp32(const DecodeArgs& a, cudaStream_t s);
-// tmaps: [0] = K cache, [1] = V cache as 2-D views (d_h, B*h_kv*T_max) with box (64, 64);
+// tmaps: [0] = K cache, [1] = V cache as 2-D views (d_h, B*h_kv*T_max) with box (64, 64), or for
+// a paged cache (d_h, num_pages*h_kv*page_size) with box (64, 16);
 // [2] = queries as (d_h, B*h_q) with box (64, 16 or 32 rows: 32 when r > 16); SWIZZLE_128B.
 cudaError_t launch_decode_bf16(const DecodeArgs& a, const CUtensorMap* tmaps, cudaStream_t s);
 

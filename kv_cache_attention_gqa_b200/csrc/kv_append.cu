@@ -3,7 +3,8 @@
 // A decode (or chunked-prefill) step appends the new tokens' K/V to the cache before attending
 // [第三章：MHA 的局限与 MQA、GQA、Flash Attention, section 3.1; MHA/MQA/GQA walkthrough,
 // section 4]. The copy is bit-exact and memory-bound: every byte moves once, in 16-byte vectors
-// when the row size allows, else in 4- or 2-byte words.
+// when the row size allows, else in 4- or 2-byte words. On a paged cache each row goes to the
+// page the block table names for its logical position.
 
 #include "common.cuh"
 #include "internal.h"
@@ -27,7 +28,20 @@ __global__ void __launch_bounds__(256) kv_append_kernel(AppendArgs a, int vecs_p
       if (t == 0 && c == 0) set_device_error(a.err, GQA_DEVERR_POSITION);
       continue;
     }
-    const long long dst_row = bg * a.T_max + p + t;
+    long long dst_row;
+    if (a.block_table) {
+      // paged: logical position p + t is row (p + t) % page_size of page table[b][(p + t) / page_size]
+      const int pt = p + t;
+      const int page = a.block_table[(long long)b * a.max_pages + pt / a.page_size];
+      if (page < 0 || page >= a.num_pages) {
+        if (c == 0) set_device_error(a.err, GQA_DEVERR_PAGE);
+        continue;
+      }
+      const int g = (int)(bg - (long long)b * a.h_kv);
+      dst_row = ((long long)page * a.h_kv + g) * a.page_size + pt % a.page_size;
+    } else {
+      dst_row = bg * a.T_max + p + t;
+    }
     const Vec* ks = reinterpret_cast<const Vec*>(a.k_new) + row * vecs_per_row + c;
     const Vec* vs = reinterpret_cast<const Vec*>(a.v_new) + row * vecs_per_row + c;
     Vec* kd = reinterpret_cast<Vec*>(a.k_cache) + dst_row * vecs_per_row + c;

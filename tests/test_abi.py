@@ -93,3 +93,38 @@ def test_workspace_size(lib):
     assert 0 < a < b
     # partials: (splits + units) slots of r heads x (d_h + 1) floats, plus one counter per unit
     assert a >= (148 + 64) * 4 * 129 * 4 + 64 * 4
+
+
+def test_paged_host_side_argument_errors(lib):
+    """gqa_decode_paged / kv_append_paged reject bad page geometry before any CUDA call."""
+    P = ctypes.c_void_p
+    fake = P(0x1000)
+    null = None
+    s = None
+    # args: q, k_pages, v_pages, o, lse, kv_len, q_pos, block_table,
+    #       B, h_q, h_kv, num_pages, page_size, max_pages, d_h, scale, dtype, ws, ws_bytes, splits, stream
+    ok = [fake, fake, fake, fake, null, null, null, fake, 1, 4, 2, 8, 16, 4, 64, 0.1, 0, fake, 1 << 20, 1, s]
+
+    def dec(**kw):
+        a = list(ok)
+        idx = {"bt": 7, "num_pages": 11, "page_size": 12, "max_pages": 13, "d_h": 14, "ws": 17}
+        for k, v in kw.items():
+            a[idx[k]] = v
+        return lib.gqa_decode_paged(*a)
+
+    assert dec(bt=null) == 1
+    assert dec(num_pages=0) == 1
+    assert dec(page_size=0) == 1
+    assert dec(max_pages=0) == 1
+    assert dec(page_size=24) == 2          # not a multiple of 16
+    assert dec(d_h=96) == 2                # bf16 head dims are 64 / 128
+    assert dec(page_size=1 << 16, max_pages=1 << 16) == 2  # T_max beyond 2^31
+    assert dec(page_size=1 << 12, num_pages=1 << 18) == 2  # pool rows beyond 2^31
+    assert dec(ws=null) == 5
+    # kv_append_paged: k, v, k_new, v_new, pos, block_table, B, h_kv, S_new, num_pages, page_size,
+    #                  max_pages, d_h, dtype, stream
+    assert lib.kv_append_paged(fake, fake, fake, fake, fake, null, 1, 2, 1, 8, 16, 4, 64, 0, s) == 1
+    assert lib.kv_append_paged(fake, fake, fake, fake, null, fake, 1, 2, 1, 8, 16, 4, 64, 0, s) == 1
+    assert lib.kv_append_paged(fake, fake, fake, fake, fake, fake, 1, 2, 1, 0, 16, 4, 64, 0, s) == 1
+    assert lib.kv_append_paged(fake, fake, fake, fake, fake, fake, 1, 2, 65, 8, 16, 4, 64, 0, s) == 1
+    assert lib.kv_append_paged(fake, fake, fake, fake, fake, fake, 1, 2, 1, 8, 16, 4, 64, 7, s) == 1

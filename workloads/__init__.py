@@ -17,6 +17,8 @@ the MHA/MQA/GQA walkthrough's parameter table; 64 query / 8 KV heads from 第三
                       [1024, 32768] (inclusive), cache allocated at 32768, tail filled with NaN.
 * ``chunked_prefill`` B=1, h_q=32, h_kv=8, d_h=128: 32256 cached positions, then 512 new
                       queries at positions 32256..32767 over T=32768 after appending their K/V.
+* paged variants of the decode workloads: the same q and lengths over K/V pools of fixed-size
+  pages, assigned to sequences in a seeded random order (``paged_decode_inputs``).
 """
 
 from __future__ import annotations
@@ -140,3 +142,54 @@ def decode_inputs(shape: DecodeShape, seed: int = DEFAULT_SEED, device="cpu",
 def to_f64(t: torch.Tensor) -> np.ndarray:
     """Exact upcast of a (bf16 or fp32) tensor to a float64 NumPy array on the host."""
     return t.detach().to("cpu").to(torch.float64).numpy()
+
+
+def paged_block_table(lengths, page_size: int, seed: int, spare_pages: int = 3,
+                      max_pages: int | None = None):
+    """A shuffled page assignment for sequences of the given lengths.
+
+    Returns (block_table (B, max_pages) int32, num_pages). Sequence b owns ceil(len_b / page_size)
+    distinct pages drawn in a seeded random order from a pool that also holds ``spare_pages``
+    unused pages; table entries past a sequence's last page are -1 (never read).
+    """
+    lengths = np.asarray(lengths, np.int64)
+    need = [(int(n) + page_size - 1) // page_size for n in lengths]
+    num_pages = int(sum(need)) + spare_pages
+    perm = np.random.default_rng(seed).permutation(num_pages).astype(np.int32)
+    mp = max(need) if max_pages is None else max_pages
+    table = np.full((len(lengths), max(mp, 1)), -1, np.int32)
+    at = 0
+    for b, n in enumerate(need):
+        table[b, :n] = perm[at:at + n]
+        at += n
+    return table, num_pages
+
+
+def paged_decode_inputs(shape: DecodeShape, page_size: int, seed: int = DEFAULT_SEED, device="cpu",
+                        dtype=torch.bfloat16, lengths=None, spare_pages: int = 3):
+    """q (B,h_q,d_h), K/V page pools (num_pages, h_kv, page_size, d_h), block_table (B, max_pages)
+    int32, kv_len (B,) int32.
+
+    Draw order: q, K pool, V pool (the pool is drawn whole, then every row that holds no visible
+    position -- spare pages and the tail of each sequence's last page -- is set to NaN). Lengths
+    are ``lengths`` if given, else ragged_lengths for ragged shapes, else T_max.
+    """
+    if lengths is None:
+        lengths = (ragged_lengths(seed, shape.B, shape.len_lo, shape.len_hi) if shape.ragged
+                   else np.full(shape.B, shape.T_max, np.int32))
+    lengths = np.asarray(lengths, np.int32)
+    table, num_pages = paged_block_table(lengths, page_size, seed + 1, spare_pages,
+                                         max_pages=(shape.T_max + page_size - 1) // page_size)
+    g = _generator(seed, device)
+    q = randn_bf16((shape.B, shape.h_q, shape.d_h), g, shape.std, device, dtype)
+    pool = (num_pages, shape.h_kv, page_size, shape.d_h)
+    k = randn_bf16(pool, g, shape.std, device, dtype)
+    v = randn_bf16(pool, g, shape.std, device, dtype)
+    used = np.zeros((num_pages, page_size), bool)
+    for b, n in enumerate(lengths):
+        for t0 in range(0, int(n), page_size):
+            used[table[b, t0 // page_size], :min(page_size, int(n) - t0)] = True
+    unused = torch.from_numpy(~used).to(device)
+    k.transpose(1, 2)[unused] = float("nan")  # (num_pages, page_size) rows, every KV head
+    v.transpose(1, 2)[unused] = float("nan")
+    return q, k, v, torch.from_numpy(table).to(device), torch.from_numpy(lengths).to(device)

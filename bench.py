@@ -7,6 +7,9 @@ the decodes must read (2 * B * h_kv * T * d_h * 2 per variant) divided by the de
 whole step, in GB/s. L2 is flushed (a 256 MiB write, then a 256 MiB read) between steps, outside
 the timed events.
 
+A ``paged`` object repeats the decode_8k step over a paged cache (16-token pages in a shuffled
+pool: ``kv_append_paged`` + ``gqa_decode_paged``), timed the same way.
+
 ``--impl reference`` times the fp64 CPU oracle on a bounded sample of the same workload.
 Run with no flags for N=1; under torchrun every rank runs an independent replica (the path needs
 no exchange between GPUs) and rank 0 prints one JSON line with the max-over-ranks time.
@@ -185,24 +188,23 @@ def job_throughput(unit_per_step, steps, world, total_ms):
 # our implementation
 # ---------------------------------------------------------------------------------------------
 
-def run_ours(args, rank, world, dist):
+def build_variants(args, rank, dev, page_size=0):
+    """decode_8k inputs per h_kv: contiguous caches, or (page_size > 0) K/V pools of that page
+    size with a shuffled block table, plus the new token's K/V appended at position T-1."""
     import torch
 
     import kv_cache_attention_gqa_b200 as gqa
     import workloads
 
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    dev = torch.device("cuda", local)
-    torch.cuda.set_device(dev)
-    stream = torch.cuda.current_stream(dev)
-    hbm_peak, tf_peak, tf_sust, peak_kind = load_peaks()
-    if args.prefill_only:  # profiling aid: the prefill_4k line alone
-        return {"prefill": run_prefill(args, dev, stream, tf_peak, peak_kind)}
-
     variants = []
     for h_kv in args.h_kv:
         shape = workloads.DECODE_8K[h_kv]
-        q, k, v, kv_len = workloads.decode_inputs(shape, seed=args.seed + rank, device=dev)
+        bt = None
+        if page_size:
+            q, k, v, bt, kv_len = workloads.paged_decode_inputs(shape, page_size, seed=args.seed + rank,
+                                                                device=dev)
+        else:
+            q, k, v, kv_len = workloads.decode_inputs(shape, seed=args.seed + rank, device=dev)
         # the new token: its K/V row is appended at position T-1, then the query attends
         g = torch.Generator(device=dev)
         g.manual_seed(10_000 + args.seed + rank + h_kv)
@@ -213,19 +215,43 @@ def run_ours(args, rank, world, dist):
         ws = torch.zeros(gqa.decode_workspace_size(shape.B, shape.h_q, h_kv, shape.T_max, shape.d_h),
                          dtype=torch.uint8, device=dev)
         variants.append(dict(h_kv=h_kv, shape=shape, q=q, k=k, v=v, kv_len=kv_len, k_new=k_new,
-                             v_new=v_new, pos=pos, out=out, ws=ws,
+                             v_new=v_new, pos=pos, out=out, ws=ws, bt=bt,
                              bytes=decode_kv_bytes(shape.B, h_kv, [shape.T_max] * shape.B, shape.d_h)))
-    flush = L2Flush(dev)
+    return variants
+
+
+def decode_step(variants):
+    """One decode step per variant: kv_append of the new token, then gqa_decode (paged variants
+    use kv_append_paged / gqa_decode_paged). `record[i]` = (start, end) events around decode i."""
+    import kv_cache_attention_gqa_b200 as gqa
 
     def step(record=None):
         for i, var in enumerate(variants):
-            gqa.kv_append(var["k"], var["v"], var["k_new"], var["v_new"], var["pos"])
+            if var["bt"] is None:
+                gqa.kv_append(var["k"], var["v"], var["k_new"], var["v_new"], var["pos"])
+            else:
+                gqa.kv_append_paged(var["k"], var["v"], var["k_new"], var["v_new"], var["pos"], var["bt"])
             if record is not None:
                 record[i][0].record()
-            gqa.decode(var["q"], var["k"], var["v"], kv_len=var["kv_len"], out=var["out"], ws=var["ws"])
+            if var["bt"] is None:
+                gqa.decode(var["q"], var["k"], var["v"], kv_len=var["kv_len"], out=var["out"], ws=var["ws"])
+            else:
+                gqa.decode_paged(var["q"], var["k"], var["v"], var["bt"], kv_len=var["kv_len"],
+                                 out=var["out"], ws=var["ws"])
             if record is not None:
                 record[i][1].record()
+    return step
 
+
+def time_decode(args, variants, flush, stream, local, dist, dev):
+    """Warm up, capture the step in a CUDA graph (events inside it around each decode), then time
+    `args.steps` replays, each after an L2 flush outside the events. Returns the max-over-ranks
+    total, per-step per-variant decode times (ms), the launch mode, clocks and wall time."""
+    import torch
+
+    import kv_cache_attention_gqa_b200 as gqa
+
+    step = decode_step(variants)
     for _ in range(args.warmup):
         flush(1)
         step()
@@ -280,16 +306,59 @@ def run_ours(args, rank, world, dist):
     if gqa.get_device_error() != 0:
         raise RuntimeError("device error during the timed steps")
     del graph
+    return {"total_ms": total_ms, "dec_ms": dec_ms, "mode": mode, "clocks": clocks, "wall": wall}
+
+
+def per_variant_rates(variants, dec_ms, hbm_peak):
+    out = {}
+    for i, var in enumerate(variants):
+        ms = statistics.mean(row[i] for row in dec_ms)
+        out[f"h_kv={var['h_kv']}"] = {"decode_us": round(ms * 1e3, 2), "kv_bytes": var["bytes"],
+                                      "GB_s": round(var["bytes"] / (ms / 1e3) / 1e9, 1),
+                                      "frac_of_hbm_peak": round(var["bytes"] / (ms / 1e3) / 1e9 / hbm_peak, 4)}
+    return out
+
+
+def run_paged(args, rank, dev, stream, local, hbm_peak, peak_kind):
+    """decode_8k over a paged cache (16-token pages, shuffled pool): same metric, on one rank."""
+    page = args.page_size
+    variants = build_variants(args, rank, dev, page_size=page)
+    t = time_decode(args, variants, L2Flush(dev), stream, local, None, dev)
+    step_bytes = sum(var["bytes"] for var in variants)
+    dec_total_ms = sum(sum(row) for row in t["dec_ms"]) / args.steps
+    achieved = step_bytes / (dec_total_ms / 1e3) / 1e9
+    return {"workload": f"decode_8k over a paged cache: {page}-token pages in a shuffled pool (3 spare "
+                        "pages), block table per sequence; per step and variant one kv_append_paged + "
+                        "one gqa_decode_paged",
+            "page_size": page, "launch": t["mode"],
+            "value": round(step_bytes * args.steps / (t["total_ms"] / 1e3) / 1e9, 1), "unit": "GB/s",
+            "decode_GB_s": round(achieved, 1), "frac_of_hbm_peak": round(achieved / hbm_peak, 4),
+            "peak_kind": f"hbm_gbs of {peak_kind}",
+            "per_variant": per_variant_rates(variants, t["dec_ms"], hbm_peak),
+            "clocks": t["clocks"]}
+
+
+def run_ours(args, rank, world, dist):
+    import torch
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    hbm_peak, tf_peak, tf_sust, peak_kind = load_peaks()
+    if args.prefill_only:  # profiling aid: the prefill_4k line alone
+        return {"prefill": run_prefill(args, dev, stream, tf_peak, peak_kind)}
+    if args.paged_only:  # profiling aid: the paged decode_8k line alone
+        return {"paged": run_paged(args, rank, dev, stream, local, hbm_peak, peak_kind)}
+
+    variants = build_variants(args, rank, dev)
+    flush = L2Flush(dev)
+    t = time_decode(args, variants, flush, stream, local, dist, dev)
+    total_ms, dec_ms, mode, clocks, wall = t["total_ms"], t["dec_ms"], t["mode"], t["clocks"], t["wall"]
 
     step_bytes = sum(var["bytes"] for var in variants)
     value = job_throughput(step_bytes, args.steps, world, total_ms) / 1e9
-    per_variant = {}
-    for i, var in enumerate(variants):
-        ms = statistics.mean(row[i] for row in dec_ms)
-        per_variant[f"h_kv={var['h_kv']}"] = {"decode_us": round(ms * 1e3, 2),
-                                              "kv_bytes": var["bytes"],
-                                              "GB_s": round(var["bytes"] / (ms / 1e3) / 1e9, 1),
-                                              "frac_of_hbm_peak": round(var["bytes"] / (ms / 1e3) / 1e9 / hbm_peak, 4)}
+    per_variant = per_variant_rates(variants, dec_ms, hbm_peak)
     dec_total_ms = sum(sum(row) for row in dec_ms) / args.steps
     achieved = step_bytes / (dec_total_ms / 1e3) / 1e9
     digest = source_digest(["kv_cache_attention_gqa_b200/csrc/decode.cu", "kv_cache_attention_gqa_b200/csrc/common.cuh"])
@@ -306,6 +375,12 @@ def run_ours(args, rank, world, dist):
 
     e2e = run_e2e(args, variants, dev, stream, dist, world) if not args.skip_e2e else None
     prefill = run_prefill(args, dev, stream, tf_peak, peak_kind) if not args.skip_prefill else None
+    n_variants = len(variants)
+    del variants
+    paged = None
+    if not args.skip_paged:
+        paged = run_paged(args, rank, dev, stream, local, hbm_peak, peak_kind)
+        paged["gpu_launches"] = args.steps * 3 * len(args.h_kv)
 
     result = {
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
@@ -315,13 +390,15 @@ def run_ours(args, rank, world, dist):
         "config": decode_config(world, mode),
         "roofline": roofline,
         "per_variant": per_variant,
-        "gpu_launches": args.steps * 3 * len(variants),  # kv_append, decode, merge per variant
+        "gpu_launches": args.steps * 3 * n_variants,  # kv_append, decode, merge per variant
         "clocks": clocks,
         "e2e": e2e,
         "wall_s_timed_region": round(wall, 3),
     }
     if prefill is not None:
         result["prefill"] = prefill
+    if paged is not None:
+        result["paged"] = paged
     if rank == 0 and world == 1 and not args.skip_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(args)
     return result
@@ -492,6 +569,10 @@ def main():
     ap.add_argument("--skip-e2e", action="store_true")
     ap.add_argument("--eager", action="store_true", help="time eager launches instead of a CUDA graph")
     ap.add_argument("--prefill-only", action="store_true", help="only the prefill_4k line (profiling aid)")
+    ap.add_argument("--skip-paged", action="store_true")
+    ap.add_argument("--paged-only", action="store_true", help="only the paged decode_8k line (profiling aid)")
+    ap.add_argument("--page-size", dest="page_size", type=int, default=16,
+                    help="page size of the paged decode_8k line (a multiple of 16)")
     ap.add_argument("--h-kv", dest="h_kv", type=int, nargs="+", default=[32, 8, 1],
                     help="decode_8k variants to run (default: all three); fewer only for profiling")
     args = ap.parse_args()

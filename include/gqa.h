@@ -181,10 +181,11 @@ gqa_status kv_append(void* k_cache, void* v_cache, const void* k_new, const void
  * order; entries for positions a call does not touch are never read. Attention over a paged
  * cache is, by definition, attention over the contiguous cache the pages spell out, so the
  * results equal gqa_decode's on that cache (to floating-point rounding; chunk boundaries fall on
- * multiples of 16 keys here).
+ * multiples of 16 keys here, of 64 when page_size is a multiple of 64).
  *
  * gqa_decode_paged - gqa_decode over a paged cache. T_max is max_pages * page_size.
- *   page_size  a multiple of 16 (every 16-key sub-tile the kernel loads lies inside one page).
+ *   page_size  a multiple of 16 (every 16-key sub-tile the kernel loads lies inside one page);
+ *            a multiple of 64 lets every 64-key tile load as one block (fewer, larger copies).
  *   num_pages * h_kv * page_size must stay below 2^31 (pool rows are addressed with 32 bits).
  *   block_table device int32 (B, max_pages), row-major. An entry outside [0, num_pages) that a
  *            call needs is replaced by page 0 and sets GQA_DEVERR_PAGE (the output is then wrong).

@@ -138,15 +138,29 @@ gqa_status decode_impl(const void* q, const void* k_cache, const void* v_cache, 
   const uint32_t qrows = r > 16 ? 32 : 16;
   CUtensorMap maps[3];
   // K/V: rows of d_h elements; a paged pool is (num_pages * h_kv * page_size) rows loaded in
-  // 16-row boxes (one per 16-key sub-tile), a contiguous cache (B * h_kv * T_max) in 64-row boxes
+  // 64-row boxes when pages hold a multiple of 64 keys, else in 16-row boxes (one per 16-key
+  // sub-tile); a contiguous cache (B * h_kv * T_max) in 64-row boxes
   const uint64_t kdims[2] = {(uint64_t)d_h, (uint64_t)cache_rows};
   const uint64_t qdims[2] = {(uint64_t)d_h, (uint64_t)B * h_q};
   const uint64_t strides[1] = {(uint64_t)d_h * 2};
-  const uint32_t box[2] = {64, block_table ? 16u : 64u};
+  const uint32_t box[2] = {64, (block_table && page_size % 64 != 0) ? 16u : 64u};
   const uint32_t qbox[2] = {64, qrows};
+  if (!encode_bf16(&maps[2], q, 2, qdims, strides, qbox)) return GQA_ERR_CUDA;
+  if (block_table && page_size % 64 != 0 && d_h == 128) {
+    // 16-row sub-tiles at d_h = 128: a 3-D view whose third dimension steps over the two 128-byte
+    // column chunks of a row, so one box carries a whole 16 x 128 sub-tile (half the copies of
+    // two 2-D boxes). Falls back to the 2-D boxes if the driver declines the view.
+    const uint64_t dims3[3] = {64, (uint64_t)cache_rows, 2};
+    const uint64_t strides3[2] = {(uint64_t)d_h * 2, 128};
+    const uint32_t box3[3] = {64, 16, 2};
+    if (encode_bf16(&maps[0], k_cache, 3, dims3, strides3, box3) &&
+        encode_bf16(&maps[1], v_cache, 3, dims3, strides3, box3)) {
+      a.paged_3d = 1;
+      return from_cuda(launch_decode_bf16(a, maps, s));
+    }
+  }
   if (!encode_bf16(&maps[0], k_cache, 2, kdims, strides, box) ||
-      !encode_bf16(&maps[1], v_cache, 2, kdims, strides, box) ||
-      !encode_bf16(&maps[2], q, 2, qdims, strides, qbox))
+      !encode_bf16(&maps[1], v_cache, 2, kdims, strides, box))
     return GQA_ERR_CUDA;
   return from_cuda(launch_decode_bf16(a, maps, s));
 }

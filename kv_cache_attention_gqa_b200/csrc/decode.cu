@@ -112,7 +112,9 @@ struct KArgs {
   // position t of sequence b is row t % page_size of page block_table[b * max_pages + t / page_size]
   const int32_t* block_table;
   int max_pages, page_size, num_pages;
-  int gran;  // partition granule in keys: 16 for a paged cache (sub-tiles never straddle a page), else 1
+  // partition granule in keys: 1 for a contiguous cache; on a paged cache 64 when pages hold a
+  // multiple of 64 keys (every tile lies in one page), else 16 (every 16-key sub-tile does)
+  int gran;
 };
 
 // Partition view built in shared memory by every CTA.
@@ -404,6 +406,7 @@ struct Bf16Cfg {
   static constexpr int kNch = D / 64;                    // 64-column (128-byte) chunks
   static constexpr int kChunkBytes = kTile * 128;        // one column chunk of one K/V tile
   static constexpr int kTileBytes = kNch * kChunkBytes;  // K (or V) tile
+  static constexpr int kSubBytes = kNch * 16 * 128;       // one 16-key sub-tile, all chunks
   static constexpr int kQRows = 16 * MT;
   static constexpr int kQChunkBytes = kQRows * 128;
   static constexpr int kQBytes = kNch * kQChunkBytes;
@@ -419,7 +422,17 @@ struct Bf16Cfg {
   static_assert(kSmem <= 227 * 1024, "shared memory budget");
 };
 
-template <int D, int MT, bool kPaged>
+// Cache layouts the bf16 kernel reads (template parameter kMode):
+//   kContig    (B, h_kv, T_max, d_h), one 64-row box per column chunk and tile
+//   kPaged2d   page pools, 2-D boxes: 64 rows when pages hold a multiple of 64 keys, else 16 rows
+//              (one box per 16-key sub-tile and column chunk)
+//   kPaged3d   page pools with d_h = 128 and 16-row sub-tiles: a 3-D view (64 columns, rows,
+//              2 column chunks) loads both chunks of a sub-tile in one box, so a stage takes half
+//              as many copies; a sub-tile then sits in shared memory as its own 4 KiB block
+//              (chunk-major, 16 rows each) instead of inside 64-row chunk planes
+constexpr int kContig = 0, kPaged2d = 1, kPaged3d = 2;
+
+template <int D, int MT, int kMode>
 __global__ void __launch_bounds__(Bf16Cfg<D, MT>::kThreads, 1)
     decode_bf16_kernel(const __grid_constant__ CUtensorMap tmk,
                        const __grid_constant__ CUtensorMap tmv,
@@ -454,106 +467,182 @@ __global__ void __launch_bounds__(Bf16Cfg<D, MT>::kThreads, 1)
   pdl_launch_dependents();
 
   if (warp == producer_warp) {
-    if (lane == 0) {
-      tma_prefetch_desc(&tmk);
-      tma_prefetch_desc(&tmv);
-      tma_prefetch_desc(&tmq);
-      int stage = 0;
-      uint32_t phase = 0;
-      int issued = 0;
-      bool ok = true;
-      // Chunk tickets: CTA c starts with chunk c; later chunks come from an atomic counter whose
-      // value is fetched one chunk ahead, so its latency overlaps the current chunk's loads.
-      const int G = gridDim.x;
+    // Stage bookkeeping of the producer: fill f uses stage f % kStages; its consumption completes
+    // phase f / kStages of that stage's empty barrier.
+    int stage = 0;
+    uint32_t phase = 0;
+    int issued = 0;
+    bool ok = true;
+    const int G = gridDim.x;
+    // Writes the stage's descriptor and arms its full barrier for `kv_bytes` of K/V (+ the query
+    // rows on a piece's first tile). Lane 0 only.
+    auto arm = [&](const Piece& pc, int t, int slot, int nh, uint32_t kv_bytes) -> uint32_t {
+      const bool first = t == pc.k0;
+      TileMeta m;
+      m.b = pc.b;
+      m.g = pc.g;
+      m.hb = pc.hb;
+      m.nvalid = min(kTile, pc.k1 - t);
+      m.flags = (first ? kFirst : 0) | (t + kTile >= pc.k1 ? kLast : 0);
+      m.slot = slot;
+      m.nh = nh;
+      m.pad = 0;
+      meta[stage] = m;
+      const uint32_t full = smem_u32(&bars[stage]);
+      mbar_arrive_expect_tx(full, kv_bytes + (first ? C::kQBytes : 0));
+      if (first) {
+        const uint32_t qdst = smem_u32(q_base + stage * C::kQBytes);
+        const int qrow = pc.b * a.h_q + pc.g * a.r + pc.hb * a.hpu;
+#pragma unroll
+        for (int ch = 0; ch < C::kNch; ++ch)
+          tma_load_2d(qdst + ch * C::kQChunkBytes, &tmq, full, ch * 64, qrow);
+      }
+      return full;
+    };
+    auto advance = [&]() {
+      ++issued;
+      if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
+    };
+
+    if constexpr (kMode == kContig) {
+      if (lane == 0) {
+        tma_prefetch_desc(&tmk);
+        tma_prefetch_desc(&tmv);
+        tma_prefetch_desc(&tmq);
+        // Chunk tickets: CTA c starts with chunk c; later chunks come from an atomic counter whose
+        // value is fetched one chunk ahead, so its latency overlaps the current chunk's loads.
+        int chunk = blockIdx.x;
+        int next = chunk < plan.n_chunks ? G + atomicAdd(&a.hdr->ticket, 1) : plan.n_chunks;
+        for (; ok && chunk < plan.n_chunks;) {
+          const long long x1 = min((long long)(chunk + 1) * plan.C, plan.K);
+          for (long long x = (long long)chunk * plan.C; x < x1 && ok;) {
+            const Piece pc = locate(plan, a.B, a.hblocks, x, x1);
+            const int slot = pc.n_pieces == 1 ? -1 : chunk + pc.unit;
+            const int nh = min(a.hpu, a.r - pc.hb * a.hpu);
+            const int row0 = (pc.b * a.h_kv + pc.g) * a.T_max;
+            for (int t = pc.k0; t < pc.k1; t += kTile) {
+              if (!mbar_wait(smem_u32(&bars[C::kStages + stage]), phase ^ 1u, a.err)) { ok = false; break; }
+              const uint32_t full = arm(pc, t, slot, nh, C::kStageBytes);
+              const uint32_t kdst = smem_u32(stage_base + stage * C::kStageBytes);
+              const uint32_t vdst = kdst + C::kTileBytes;
+#pragma unroll
+              for (int ch = 0; ch < C::kNch; ++ch) {
+                tma_load_2d(kdst + ch * C::kChunkBytes, &tmk, full, ch * 64, row0 + t);
+                tma_load_2d(vdst + ch * C::kChunkBytes, &tmv, full, ch * 64, row0 + t);
+              }
+              advance();
+            }
+            x = pc.end;
+          }
+          chunk = next;
+          if (chunk < plan.n_chunks) next = G + atomicAdd(&a.hdr->ticket, 1);
+        }
+      }
+    } else {
+      // Paged cache: the whole warp runs the loop. Each lane holds the block-table entry of one
+      // 16-key sub-tile of a 32-sub-tile window (8 tiles); the next window's entries are loaded
+      // when a window starts, so the table's latency is hidden behind 8 tiles of copies instead of
+      // sitting between consecutive tiles. Lane 0 takes each tile's four rows by shuffle and
+      // issues the copies: one 16-row box per sub-tile (16 rows x 128 B = 2 KiB keeps the 1 KiB
+      // swizzle atoms aligned, so the stage has the layout of one 64-row box). Sub-tiles past the
+      // tile's valid keys are not loaded (the consumer warp owning such a slice skips it).
+      if (lane == 0) {
+        tma_prefetch_desc(&tmk);
+        tma_prefetch_desc(&tmv);
+        tma_prefetch_desc(&tmq);
+      }
       int chunk = blockIdx.x;
-      int next = chunk < plan.n_chunks ? G + atomicAdd(&a.hdr->ticket, 1) : plan.n_chunks;
+      int next = 0;
+      if (lane == 0) next = chunk < plan.n_chunks ? G + atomicAdd(&a.hdr->ticket, 1) : plan.n_chunks;
+      next = __shfl_sync(0xffffffffu, next, 0);
       for (; ok && chunk < plan.n_chunks;) {
         const long long x1 = min((long long)(chunk + 1) * plan.C, plan.K);
         for (long long x = (long long)chunk * plan.C; x < x1 && ok;) {
           const Piece pc = locate(plan, a.B, a.hblocks, x, x1);
           const int slot = pc.n_pieces == 1 ? -1 : chunk + pc.unit;
           const int nh = min(a.hpu, a.r - pc.hb * a.hpu);
-          const int row0 = (pc.b * a.h_kv + pc.g) * a.T_max;
-          const int qrow = pc.b * a.h_q + pc.g * a.r + pc.hb * a.hpu;
-          for (int t = pc.k0; t < pc.k1; t += kTile) {
-            // paged cache: pool rows of the (up to) four 16-key sub-tiles, looked up before the
-            // wait for a free stage so the block-table reads overlap it
-            int prow[kPaged ? 4 : 1];
-            int nsub = 4;
-            if constexpr (kPaged) {
-              nsub = (min(kTile, pc.k1 - t) + 15) >> 4;
-              const int32_t* bt = a.block_table + (long long)pc.b * a.max_pages;
-#pragma unroll
-              for (int j = 0; j < 4; ++j) {
-                const int key = t + 16 * j;
-                int page = j < nsub ? __ldg(bt + key / a.page_size) : 0;
-                if (page < 0 || page >= a.num_pages) {
-                  set_device_error(a.err, GQA_DEVERR_PAGE);
-                  page = 0;
-                }
-                prow[j] = (page * a.h_kv + pc.g) * a.page_size + key % a.page_size;
-              }
+          const int32_t* bt = a.block_table + (long long)pc.b * a.max_pages;
+          const int s_end = (pc.k1 + 15) >> 4;  // sub-tiles of this piece: [k0 / 16, s_end)
+          // raw table entry of sub-tile s (-1 past the piece: never used)
+          auto fetch = [&](int s) -> int { return s < s_end ? __ldg(bt + (s << 4) / a.page_size) : -1; };
+          // pool row of sub-tile s from its table entry; an entry outside the pool is flagged and
+          // replaced by page 0
+          auto to_row = [&](int page, int s) -> int {
+            if (s >= s_end) return 0;
+            if (page < 0 || page >= a.num_pages) {
+              set_device_error(a.err, GQA_DEVERR_PAGE);
+              page = 0;
             }
-            if (!mbar_wait(smem_u32(&bars[C::kStages + stage]), phase ^ 1u, a.err)) { ok = false; break; }
-            const bool first = t == pc.k0;
-            TileMeta m;
-            m.b = pc.b;
-            m.g = pc.g;
-            m.hb = pc.hb;
-            m.nvalid = min(kTile, pc.k1 - t);
-            m.flags = (first ? kFirst : 0) | (t + kTile >= pc.k1 ? kLast : 0);
-            m.slot = slot;
-            m.nh = nh;
-            m.pad = 0;
-            meta[stage] = m;
-            const uint32_t full = smem_u32(&bars[stage]);
-            // sub-tiles past the tile's valid keys are not loaded on a paged cache (the consumer
-            // warp that owns such a 16-key slice skips it)
-            const uint32_t kv_bytes = kPaged ? (uint32_t)nsub * (C::kStageBytes / 4) : C::kStageBytes;
-            mbar_arrive_expect_tx(full, kv_bytes + (first ? C::kQBytes : 0));
-            const uint32_t kdst = smem_u32(stage_base + stage * C::kStageBytes);
-            const uint32_t vdst = kdst + C::kTileBytes;
-            if constexpr (kPaged) {
-              // one 16-row box per sub-tile; 16 rows x 128 B = 2 KiB keeps the 128-byte swizzle
-              // atoms (1 KiB) aligned, so the stage has the same layout as one 64-row box
+            return (page * a.h_kv + pc.g) * a.page_size + (s << 4) % a.page_size;
+          };
+          int wbase = pc.k0 >> 4;  // first sub-tile of the current window
+          int cur = to_row(fetch(wbase + lane), wbase + lane);
+          int nxt = fetch(wbase + 32 + lane);
+          for (int t = pc.k0; t < pc.k1; t += kTile) {
+            const int s = t >> 4;
+            if (s >= wbase + 32) {
+              wbase += 32;
+              cur = to_row(nxt, wbase + lane);
+              nxt = fetch(wbase + 32 + lane);
+            }
+            int prow[4];
 #pragma unroll
-              for (int j = 0; j < 4; ++j) {
-                if (j >= nsub) break;
+            for (int j = 0; j < 4; ++j) prow[j] = __shfl_sync(0xffffffffu, cur, (s - wbase + j) & 31);
+            int good = 1;
+            if (lane == 0) good = mbar_wait(smem_u32(&bars[C::kStages + stage]), phase ^ 1u, a.err) ? 1 : 0;
+            if (!__shfl_sync(0xffffffffu, good, 0)) { ok = false; break; }
+            if (lane == 0) {
+              const uint32_t kdst = smem_u32(stage_base + stage * C::kStageBytes);
+              const uint32_t vdst = kdst + C::kTileBytes;
+              if (kMode == kPaged2d && a.gran == kTile) {
+                // pages hold a multiple of 64 keys and tiles start on multiples of 64: the whole
+                // tile lies in one page and loads as one 64-row box per column chunk
+                const uint32_t full = arm(pc, t, slot, nh, C::kStageBytes);
 #pragma unroll
                 for (int ch = 0; ch < C::kNch; ++ch) {
-                  tma_load_2d(kdst + ch * C::kChunkBytes + j * 2048, &tmk, full, ch * 64, prow[j]);
-                  tma_load_2d(vdst + ch * C::kChunkBytes + j * 2048, &tmv, full, ch * 64, prow[j]);
+                  tma_load_2d(kdst + ch * C::kChunkBytes, &tmk, full, ch * 64, prow[0]);
+                  tma_load_2d(vdst + ch * C::kChunkBytes, &tmv, full, ch * 64, prow[0]);
+                }
+              } else {
+                const int nsub = (min(kTile, pc.k1 - t) + 15) >> 4;
+                const uint32_t full = arm(pc, t, slot, nh, (uint32_t)nsub * (C::kStageBytes / 4));
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                  if (j >= nsub) break;
+                  if constexpr (kMode == kPaged3d) {
+                    tma_load_3d(kdst + j * C::kSubBytes, &tmk, full, 0, prow[j], 0);
+                    tma_load_3d(vdst + j * C::kSubBytes, &tmv, full, 0, prow[j], 0);
+                  } else {
+#pragma unroll
+                    for (int ch = 0; ch < C::kNch; ++ch) {
+                      tma_load_2d(kdst + ch * C::kChunkBytes + j * 2048, &tmk, full, ch * 64, prow[j]);
+                      tma_load_2d(vdst + ch * C::kChunkBytes + j * 2048, &tmv, full, ch * 64, prow[j]);
+                    }
+                  }
                 }
               }
-            } else {
-#pragma unroll
-              for (int ch = 0; ch < C::kNch; ++ch) {
-                tma_load_2d(kdst + ch * C::kChunkBytes, &tmk, full, ch * 64, row0 + t);
-                tma_load_2d(vdst + ch * C::kChunkBytes, &tmv, full, ch * 64, row0 + t);
-              }
             }
-            if (first) {
-              const uint32_t qdst = smem_u32(q_base + stage * C::kQBytes);
-#pragma unroll
-              for (int ch = 0; ch < C::kNch; ++ch)
-                tma_load_2d(qdst + ch * C::kQChunkBytes, &tmq, full, ch * 64, qrow);
-            }
-            ++issued;
-            if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
+            __syncwarp();
+            advance();
           }
           x = pc.end;
         }
         chunk = next;
-        if (chunk < plan.n_chunks) next = G + atomicAdd(&a.hdr->ticket, 1);
+        if (chunk < plan.n_chunks) {
+          if (lane == 0) next = G + atomicAdd(&a.hdr->ticket, 1);
+          next = __shfl_sync(0xffffffffu, next, 0);
+        }
       }
+    }
+
+    if (lane == 0) {
       if (ok && mbar_wait(smem_u32(&bars[C::kStages + stage]), phase ^ 1u, a.err)) {
         meta[stage].flags = kEnd;  // tells the consumers to stop
         mbar_arrive(smem_u32(&bars[stage]));
         ++issued;
       }
-      // Drain (bounded): wait until the last C::kStages fills were consumed, so no copy is in flight
-      // into shared memory when the CTA exits. Fill f used stage f % C::kStages; its consumption
-      // completes phase f / C::kStages of that stage's empty barrier.
+      // Drain (bounded): wait until the last kStages fills were consumed, so no copy is in flight
+      // into shared memory when the CTA exits.
       for (int f = issued > C::kStages ? issued - C::kStages : 0; f < issued; ++f) {
         if (!mbar_wait(smem_u32(&bars[C::kStages + f % C::kStages]), (uint32_t)(f / C::kStages) & 1u, a.err))
           break;
@@ -570,6 +659,13 @@ __global__ void __launch_bounds__(Bf16Cfg<D, MT>::kThreads, 1)
   const float sl2 = a.scale * kLog2e;
   constexpr int NK = D / 16;  // k-steps of Q K^T
   constexpr int NN = D / 8;   // n-tiles of P V
+
+  // K/V addressing in a stage: chunk planes of 64 rows, or (kPaged3d) one block per 16-key
+  // sub-tile, which is this warp's own slice ws
+  constexpr bool kSub = kMode == kPaged3d;
+  constexpr int kKvChunkStride = kSub ? 16 * 128 : C::kChunkBytes;
+  const uint32_t kv_warp_off = kSub ? ws * C::kSubBytes : 0;
+  const int kv_row_mask = kSub ? 15 : 63;
 
   int stage = 0;
   uint32_t phase = 0;
@@ -613,7 +709,8 @@ __global__ void __launch_bounds__(Bf16Cfg<D, MT>::kThreads, 1)
         for (int ks = 0; ks < NK; ++ks) {
           const int d8 = ks * 2 + ((lane >> 3) & 1);
           uint32_t b0, b1, b2, b3;
-          ldsm_x4(swz128(kb + (d8 >> 3) * C::kChunkBytes, krow, d8 & 7), b0, b1, b2, b3);
+          ldsm_x4(swz128(kb + kv_warp_off + (d8 >> 3) * kKvChunkStride, krow & kv_row_mask, d8 & 7),
+                  b0, b1, b2, b3);
           mma_bf16(sc[0], qf[ks], b0, b1);
           mma_bf16(sc[1], qf[ks], b2, b3);
         }
@@ -673,7 +770,8 @@ __global__ void __launch_bounds__(Bf16Cfg<D, MT>::kThreads, 1)
       for (int n2 = 0; n2 < NN / 2; ++n2) {
         const int d8 = n2 * 2 + (lane >> 4);
         uint32_t b0, b1, b2, b3;
-        ldsm_x4_t(swz128(vb + (d8 >> 3) * C::kChunkBytes, vrow, d8 & 7), b0, b1, b2, b3);
+        ldsm_x4_t(swz128(vb + kv_warp_off + (d8 >> 3) * kKvChunkStride, vrow & kv_row_mask, d8 & 7),
+                  b0, b1, b2, b3);
         if (partial) {
           b0 = mask_pair(b0, key_a, nvalid);
           b1 = mask_pair(b1, key_b, nvalid);
@@ -868,10 +966,10 @@ cudaError_t launch_merge(const KArgs& ka, cudaStream_t s) {
   return e;
 }
 
-template <int D, int MT, bool kPaged>
+template <int D, int MT, int kMode>
 cudaError_t launch_bf16_typed(const KArgs& ka, const CUtensorMap* tm, int grid, cudaStream_t s) {
   using C = Bf16Cfg<D, MT>;
-  auto kern = decode_bf16_kernel<D, MT, kPaged>;
+  auto kern = decode_bf16_kernel<D, MT, kMode>;
   static bool attr_set[64] = {false};  // per device: the shared-memory opt-in is set once
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -931,7 +1029,7 @@ KArgs make_kargs(const DecodeArgs& a) {
   k.max_pages = a.max_pages;
   k.page_size = a.page_size;
   k.num_pages = a.num_pages;
-  k.gran = a.block_table ? 16 : 1;
+  k.gran = a.block_table ? (a.page_size % kTile == 0 ? kTile : 16) : 1;
   return k;
 }
 
@@ -957,16 +1055,18 @@ cudaError_t launch_decode_fp32(const DecodeArgs& a, cudaStream_t s) {
 }
 
 namespace dec {
-template <bool kPaged>
+template <int kMode>
 cudaError_t launch_bf16_dispatch(const KArgs& k, const CUtensorMap* tmaps, int grid, cudaStream_t s) {
   const bool two = k.hpu > 16;
   if (k.D == 128) {
-    return two ? launch_bf16_typed<128, 2, kPaged>(k, tmaps, grid, s)
-               : launch_bf16_typed<128, 1, kPaged>(k, tmaps, grid, s);
+    return two ? launch_bf16_typed<128, 2, kMode>(k, tmaps, grid, s)
+               : launch_bf16_typed<128, 1, kMode>(k, tmaps, grid, s);
   }
-  if (k.D == 64) {
-    return two ? launch_bf16_typed<64, 2, kPaged>(k, tmaps, grid, s)
-               : launch_bf16_typed<64, 1, kPaged>(k, tmaps, grid, s);
+  if constexpr (kMode != kPaged3d) {
+    if (k.D == 64) {
+      return two ? launch_bf16_typed<64, 2, kMode>(k, tmaps, grid, s)
+                 : launch_bf16_typed<64, 1, kMode>(k, tmaps, grid, s);
+    }
   }
   return cudaErrorInvalidValue;
 }
@@ -974,8 +1074,9 @@ cudaError_t launch_bf16_dispatch(const KArgs& k, const CUtensorMap* tmaps, int g
 
 cudaError_t launch_decode_bf16(const DecodeArgs& a, const CUtensorMap* tmaps, cudaStream_t s) {
   const dec::KArgs k = dec::make_kargs(a);
-  return a.block_table ? dec::launch_bf16_dispatch<true>(k, tmaps, a.num_sms, s)
-                       : dec::launch_bf16_dispatch<false>(k, tmaps, a.num_sms, s);
+  if (!a.block_table) return dec::launch_bf16_dispatch<dec::kContig>(k, tmaps, a.num_sms, s);
+  return a.paged_3d ? dec::launch_bf16_dispatch<dec::kPaged3d>(k, tmaps, a.num_sms, s)
+                    : dec::launch_bf16_dispatch<dec::kPaged2d>(k, tmaps, a.num_sms, s);
 }
 
 }  // namespace gqa

@@ -66,6 +66,10 @@ struct DecodeArgs {
   // k/v are pools (num_pages, h_kv, page_size, d_h), T_max = max_pages * page_size
   const int32_t* block_table = nullptr;
   int max_pages = 0, page_size = 0, num_pages = 0;
+  // paged, d_h = 128, page_size not a multiple of 64: K/V maps are 3-D views (64 columns,
+  // num_pages*h_kv*page_size rows with a 256-byte stride, 2 column chunks with a 128-byte stride)
+  // with box (64, 16, 2)
+  int paged_3d = 0;
 };
 
 // Workspace bytes for a decode of this shape (layout in decode.cu).

@@ -28,7 +28,7 @@ def _ref(q, k, v, bt, kl, q_pos=None):
                                    q_pos=q_pos)
 
 
-@pytest.mark.parametrize("page_size", [16, 64, 256])
+@pytest.mark.parametrize("page_size", [16, 48, 64, 256])
 @pytest.mark.parametrize("h_q,h_kv", [(32, 8), (32, 32), (32, 1), (40, 5), (64, 2)])
 @pytest.mark.parametrize("d", [64, 128])
 def test_paged_decode_bf16(page_size, h_q, h_kv, d):

@@ -397,7 +397,7 @@ struct TileMeta {
 constexpr int kFirst = 1, kLast = 2, kEnd = 4;
 
 #ifndef GQA_DECODE_STAGES_1
-#define GQA_DECODE_STAGES_1 4
+#define GQA_DECODE_STAGES_1 5
 #endif
 template <int D, int MT>
 struct Bf16Cfg {

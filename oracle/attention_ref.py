@@ -17,6 +17,10 @@ Definition followed, in the pages' notation:
   is_causal only fits equal-length Q and K]. So query row i of batch b sits at position
   q_start[b] + i and sees key j iff j <= q_start[b] + i (causal) and j < kv_len[b] (padding).
 * A query with no visible key is an error [序列计算与存储 §两块算例, the error the listing raises].
+* Sliding window (optional): each query reads only a local window of the history [第三章 §3.7,
+  the Sliding Window Attention row]. The page gives no formula; the reading taken here is that a
+  window of W keeps the W most recent positions up to and including the query's own, i.e. key j is
+  visible iff q_pos - W < j <= q_pos (and j < kv_len). W = None means no window.
 
 The score matrix S and the weights P are materialised in full; K/V are read through g(a) and
 never expanded.  ``scale`` defaults to 1/sqrt(d_h) and may be given explicitly, because the
@@ -41,17 +45,19 @@ def group_of(a: int, h_q: int, h_kv: int) -> int:
     return a // r
 
 
-def visible_count(q_pos: int, kv_len: int, causal: bool = True) -> int:
+def visible_count(q_pos: int, kv_len: int, causal: bool = True, window=None) -> int:
     """Number of keys a query at absolute position ``q_pos`` sees in a sequence of ``kv_len`` keys.
 
-    The visible keys are the prefix j < min(kv_len, q_pos + 1) (causal) or j < kv_len (not causal).
+    The visible keys are j < min(kv_len, q_pos + 1) (causal) or j < kv_len (not causal); a window
+    of W further requires j > q_pos - W.
     """
-    if causal:
-        return max(0, min(kv_len, q_pos + 1))
-    return max(0, kv_len)
+    hi = min(kv_len, q_pos + 1) if causal else kv_len
+    lo = 0 if window is None else max(0, q_pos - window + 1)
+    return max(0, hi - lo)
 
 
-def head_attention(q_rows, k, v, q_pos, kv_len: int, scale: float, causal: bool = True):
+def head_attention(q_rows, k, v, q_pos, kv_len: int, scale: float, causal: bool = True,
+                   window=None):
     """One query head against the K/V head it reads.
 
     q_rows: (n, d_h) queries; k, v: (T, d_h) with T >= kv_len; q_pos: (n,) absolute positions.
@@ -73,6 +79,10 @@ def head_attention(q_rows, k, v, q_pos, kv_len: int, scale: float, causal: bool 
         visible = j[None, :] <= q_pos[:, None]
     else:
         visible = np.ones((n, kv_len), dtype=bool)
+    if window is not None:
+        if window < 1:
+            raise ValueError("a window holds at least one key")
+        visible &= j[None, :] > q_pos[:, None] - window
     if n and not visible.any(axis=1).all():
         raise ValueError("query has no visible key")
     # M: 0 where visible, -inf elsewhere.
@@ -89,12 +99,14 @@ def head_attention(q_rows, k, v, q_pos, kv_len: int, scale: float, causal: bool 
     return O, lse
 
 
-def attention_ref(q, k_cache, v_cache, q_start=None, kv_len=None, scale=None, causal=True):
+def attention_ref(q, k_cache, v_cache, q_start=None, kv_len=None, scale=None, causal=True,
+                  window=None):
     """Grouped-query attention for a batch.
 
     q: (B, h_q, S_q, d_h); k_cache, v_cache: (B, h_kv, T_max, d_h).
     q_start: (B,) absolute position of query row 0 (default 0).
     kv_len: (B,) number of keys present (default T_max).
+    window: None, or W >= 1: row i also needs key j > q_start + i - W.
     Returns (O (B, h_q, S_q, d_h) float64, lse (B, h_q, S_q) float64).
     """
     q = np.asarray(q, dtype=np.float64)
@@ -121,12 +133,12 @@ def attention_ref(q, k_cache, v_cache, q_start=None, kv_len=None, scale=None, ca
         for a in range(h_q):
             g = group_of(a, h_q, h_kv)
             O[b, a], L[b, a] = head_attention(
-                q[b, a], k_cache[b, g], v_cache[b, g], pos, n_keys, scale, causal
+                q[b, a], k_cache[b, g], v_cache[b, g], pos, n_keys, scale, causal, window
             )
     return O, L
 
 
-def decode_ref(q, k_cache, v_cache, kv_len=None, q_pos=None, scale=None):
+def decode_ref(q, k_cache, v_cache, kv_len=None, q_pos=None, scale=None, window=None):
     """Single-token decode: one query per sequence at absolute position q_pos[b].
 
     q: (B, h_q, d_h). q_pos defaults to kv_len[b] - 1: the current token's K/V is already in the
@@ -139,5 +151,5 @@ def decode_ref(q, k_cache, v_cache, kv_len=None, q_pos=None, scale=None):
     kv_len = np.full(B, T_max, np.int64) if kv_len is None else np.asarray(kv_len, np.int64)
     q_pos = kv_len - 1 if q_pos is None else np.asarray(q_pos, np.int64)
     O, L = attention_ref(q[:, :, None, :], k_cache, v_cache, q_start=q_pos, kv_len=kv_len,
-                         scale=scale, causal=True)
+                         scale=scale, causal=True, window=window)
     return O[:, :, 0, :], L[:, :, 0]

@@ -43,11 +43,11 @@ def gather_pages(pages, block_table, lengths, T_max=None):
     return out
 
 
-def paged_decode_ref(q, k_pages, v_pages, block_table, kv_len, q_pos=None, scale=None):
+def paged_decode_ref(q, k_pages, v_pages, block_table, kv_len, q_pos=None, scale=None, window=None):
     """Decode over a paged cache = decode over the gathered contiguous cache."""
     k = gather_pages(k_pages, block_table, kv_len)
     v = gather_pages(v_pages, block_table, kv_len)
-    return decode_ref(q, k, v, kv_len=kv_len, q_pos=q_pos, scale=scale)
+    return decode_ref(q, k, v, kv_len=kv_len, q_pos=q_pos, scale=scale, window=window)
 
 
 def paged_append_ref(k_pages, v_pages, k_new, v_new, block_table, pos):

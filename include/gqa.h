@@ -83,17 +83,24 @@ enum {
  *   scale    finite, > 0; pass 1/sqrt(d_h) for the standard scaling.
  *   causal   1: key j visible to row i iff j <= q_start[b] + i and j < kv_len[b];
  *            0: iff j < kv_len[b].
+ *   window   0: no window. W > 0 (requires causal = 1): sliding-window attention, each row reads
+ *            only its local window [第三章, section 3.7, the Sliding Window Attention row]: key j
+ *            is visible to row i only if also j > q_start[b] + i - W (the W most recent
+ *            positions, the row's own included). K/V blocks below a tile's window are not read.
+ *            A row whose window holds no cached key is written as zeros, lse = -inf, and sets
+ *            GQA_DEVERR_NO_VISIBLE.
  *   dtype    GQA_BF16: d_h in {64, 128}, tcgen05 tensor-core kernel (sm_100a);
  *            GQA_FP32: 1 <= d_h <= 256, scalar check-mode kernel.
  *
  * A chunked prefill over an existing cache is kv_append(...) of the chunk's K/V at position p,
  * then gqa_prefill with q_start[b] = p and kv_len[b] = p + S_q.
- * Errors: INVALID_ARG (nulls, sizes <= 0, h_q % h_kv, scale), UNSUPPORTED (bf16 d_h), CUDA.
+ * Errors: INVALID_ARG (nulls, sizes <= 0, h_q % h_kv, scale, window < 0 or a window without the
+ * causal mask), UNSUPPORTED (bf16 d_h), CUDA.
  */
 gqa_status gqa_prefill(const void* q, const void* k_cache, const void* v_cache, void* o,
                        float* lse, const int32_t* q_start, const int32_t* kv_len,
                        int B, int h_q, int h_kv, int S_q, int T_max, int d_h,
-                       float scale, int causal, gqa_dtype dtype, void* stream);
+                       float scale, int causal, int window, gqa_dtype dtype, void* stream);
 
 /*
  * gqa_decode_workspace_size - bytes of device workspace gqa_decode needs for this shape with
@@ -116,6 +123,8 @@ size_t gqa_decode_workspace_size(int B, int h_q, int h_kv, int T_max, int d_h, g
  *   kv_len   device int32[B] or NULL (= all T_max).
  *   q_pos    device int32[B] or NULL (= kv_len[b] - 1: the token's own K/V was appended first,
  *            so it sees every cached key [MHA/MQA/GQA walkthrough, section 4]).
+ *   window   0: none; W > 0: sliding window as in gqa_prefill, only keys q_pos[b] - W < j are
+ *            visible, and only those are read (the visible keys of a unit start at the window).
  *   workspace, workspace_bytes: caller-owned device memory, >= gqa_decode_workspace_size(...),
  *            256-byte aligned, zero-filled before first use (see above). Calls that share one
  *            workspace must not overlap in time (use one stream, or one workspace per stream).
@@ -129,8 +138,9 @@ size_t gqa_decode_workspace_size(int B, int h_q, int h_kv, int T_max, int d_h, g
  */
 gqa_status gqa_decode(const void* q, const void* k_cache, const void* v_cache, void* o, float* lse,
                       const int32_t* kv_len, const int32_t* q_pos,
-                      int B, int h_q, int h_kv, int T_max, int d_h, float scale, gqa_dtype dtype,
-                      void* workspace, size_t workspace_bytes, int num_splits, void* stream);
+                      int B, int h_q, int h_kv, int T_max, int d_h, float scale, int window,
+                      gqa_dtype dtype, void* workspace, size_t workspace_bytes, int num_splits,
+                      void* stream);
 
 /*
  * gqa_decode_noalloc - gqa_decode for callers that cannot allocate device memory. (The source
@@ -152,7 +162,7 @@ gqa_status gqa_decode(const void* q, const void* k_cache, const void* v_cache, v
 gqa_status gqa_decode_noalloc(const void* q, const void* k_cache, const void* v_cache, void* o,
                               float* lse, const int32_t* kv_len, const int32_t* q_pos,
                               int B, int h_q, int h_kv, int T_max, int d_h, float scale,
-                              gqa_dtype dtype, int num_splits, void* stream);
+                              int window, gqa_dtype dtype, int num_splits, void* stream);
 
 /*
  * kv_append - copy new K/V rows into the cache: cache[b, g, pos[b] + t, :] = new[b, g, t, :]
@@ -196,8 +206,9 @@ gqa_status kv_append(void* k_cache, void* v_cache, const void* k_new, const void
 gqa_status gqa_decode_paged(const void* q, const void* k_pages, const void* v_pages, void* o,
                             float* lse, const int32_t* kv_len, const int32_t* q_pos,
                             const int32_t* block_table, int B, int h_q, int h_kv, int num_pages,
-                            int page_size, int max_pages, int d_h, float scale, gqa_dtype dtype,
-                            void* workspace, size_t workspace_bytes, int num_splits, void* stream);
+                            int page_size, int max_pages, int d_h, float scale, int window,
+                            gqa_dtype dtype, void* workspace, size_t workspace_bytes,
+                            int num_splits, void* stream);
 
 /*
  * kv_append_paged - kv_append into a paged cache: new[b, g, t, :] goes to logical position

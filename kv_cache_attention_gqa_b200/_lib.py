@@ -35,13 +35,13 @@ DEVERR_NAMES = {0: "none", 1: "kv_len out of range", 2: "position out of range",
 # name -> (restype, argtypes), mirroring include/gqa.h
 _P, _I, _F, _Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
 SIGNATURES = {
-    "gqa_prefill": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _I, _P]),
+    "gqa_prefill": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _I, _I, _P]),
     "gqa_decode_workspace_size": (_Z, [_I, _I, _I, _I, _I, _I, _I]),
-    "gqa_decode": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _P, _Z, _I, _P]),
-    "gqa_decode_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _I, _P]),
+    "gqa_decode": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _I, _P, _Z, _I, _P]),
+    "gqa_decode_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _I, _I, _P]),
     "kv_append": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P]),
     "gqa_decode_paged": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I,
-                              _P, _Z, _I, _P]),
+                              _I, _P, _Z, _I, _P]),
     "kv_append_paged": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P]),
     "gqa_get_device_error": (_I, [ctypes.POINTER(_I), _P]),
     "gqa_status_string": (ctypes.c_char_p, [_I]),
@@ -156,9 +156,10 @@ def kv_append(k_cache: torch.Tensor, v_cache: torch.Tensor, k_new: torch.Tensor,
 
 
 def prefill(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, *, q_start=None,
-            kv_len=None, scale: float | None = None, causal: bool = True, out=None,
-            return_lse: bool = False):
-    """Grouped-query attention of q (B, h_q, S_q, d_h) over the cache (B, h_kv, T_max, d_h)."""
+            kv_len=None, scale: float | None = None, causal: bool = True, window: int = 0,
+            out=None, return_lse: bool = False):
+    """Grouped-query attention of q (B, h_q, S_q, d_h) over the cache (B, h_kv, T_max, d_h).
+    ``window`` > 0: sliding window, row at position p sees keys p - window < j <= p."""
     _need_cuda(q, k_cache, v_cache, out)
     B, h_q, S_q, d_h = q.shape
     Bk, h_kv, T_max, dk = k_cache.shape
@@ -175,7 +176,7 @@ def prefill(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, *, q_
     scale = 1.0 / math.sqrt(d_h) if scale is None else float(scale)
     _check("gqa_prefill", _lib.gqa_prefill(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(out), _ptr(lse),
                                            _ptr(qs), _ptr(kl), B, h_q, h_kv, S_q, T_max, d_h, scale,
-                                           1 if causal else 0, dt, _stream()))
+                                           1 if causal else 0, int(window), dt, _stream()))
     return (out, lse) if return_lse else out
 
 
@@ -207,9 +208,10 @@ def workspace(nbytes: int, device) -> torch.Tensor:
 
 
 def decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, *, kv_len=None,
-           q_pos=None, scale: float | None = None, num_splits: int = 0, out=None,
+           q_pos=None, scale: float | None = None, window: int = 0, num_splits: int = 0, out=None,
            return_lse: bool = False, ws: torch.Tensor | None = None):
-    """Split-KV decode of q (B, h_q, d_h) over the cache (B, h_kv, T_max, d_h)."""
+    """Split-KV decode of q (B, h_q, d_h) over the cache (B, h_kv, T_max, d_h).
+    ``window`` > 0: sliding window, the query at q_pos sees keys q_pos - window < j <= q_pos."""
     _need_cuda(q, k_cache, v_cache, out)
     B, h_q, d_h = q.shape
     Bk, h_kv, T_max, dk = k_cache.shape
@@ -231,14 +233,14 @@ def decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, *, kv_
     if ws is None:
         ws = workspace(need, q.device)
     _check("gqa_decode", _lib.gqa_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(out), _ptr(lse),
-                                         _ptr(kl), _ptr(qp), B, h_q, h_kv, T_max, d_h, scale, dt,
-                                         _ptr(ws), ws.numel(), num_splits, _stream()))
+                                         _ptr(kl), _ptr(qp), B, h_q, h_kv, T_max, d_h, scale,
+                                         int(window), dt, _ptr(ws), ws.numel(), num_splits, _stream()))
     return (out, lse) if return_lse else out
 
 
 def decode_noalloc(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, *, kv_len=None,
-                   q_pos=None, scale: float | None = None, num_splits: int = 0, out=None,
-                   return_lse: bool = False):
+                   q_pos=None, scale: float | None = None, window: int = 0, num_splits: int = 0,
+                   out=None, return_lse: bool = False):
     """gqa_decode_noalloc: the decode with the library's fixed device scratch array instead of a
     caller workspace, for callers that cannot allocate device memory (the output buffer may be
     passed in as ``out``). Overlapping calls on different streams race on that array."""
@@ -258,7 +260,7 @@ def decode_noalloc(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor
     scale = 1.0 / math.sqrt(d_h) if scale is None else float(scale)
     _check("gqa_decode_noalloc", _lib.gqa_decode_noalloc(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(out),
                                                          _ptr(lse), _ptr(kl), _ptr(qp), B, h_q, h_kv, T_max,
-                                                         d_h, scale, dt, num_splits, _stream()))
+                                                         d_h, scale, int(window), dt, num_splits, _stream()))
     return (out, lse) if return_lse else out
 
 
@@ -278,8 +280,9 @@ def _pool_shape(k_pages: torch.Tensor, v_pages: torch.Tensor):
 
 
 def decode_paged(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.Tensor, block_table, *,
-                 kv_len=None, q_pos=None, scale: float | None = None, num_splits: int = 0,
-                 out=None, return_lse: bool = False, ws: torch.Tensor | None = None):
+                 kv_len=None, q_pos=None, scale: float | None = None, window: int = 0,
+                 num_splits: int = 0, out=None, return_lse: bool = False,
+                 ws: torch.Tensor | None = None):
     """Split-KV decode of q (B, h_q, d_h) over a paged cache: pools (num_pages, h_kv, page_size,
     d_h) and block_table (B, max_pages) int32; position t of sequence b is row t % page_size of
     page block_table[b, t // page_size]."""
@@ -308,7 +311,7 @@ def decode_paged(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.Tensor, 
         ws = workspace(need, q.device)
     _check("gqa_decode_paged", _lib.gqa_decode_paged(
         _ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(out), _ptr(lse), _ptr(kl), _ptr(qp), _ptr(bt),
-        B, h_q, h_kv, num_pages, page_size, max_pages, d_h, scale, dt, _ptr(ws), ws.numel(),
+        B, h_q, h_kv, num_pages, page_size, max_pages, d_h, scale, int(window), dt, _ptr(ws), ws.numel(),
         num_splits, _stream()))
     return (out, lse) if return_lse else out
 

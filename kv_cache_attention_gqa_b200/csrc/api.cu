@@ -85,11 +85,12 @@ namespace {
 // T_max = max_pages * page_size; k_cache / v_cache are then the page pools.
 gqa_status decode_impl(const void* q, const void* k_cache, const void* v_cache, void* o, float* lse,
                        const int32_t* kv_len, const int32_t* q_pos, int B, int h_q, int h_kv,
-                       int T_max, int d_h, float scale, gqa_dtype dtype, void* workspace,
+                       int T_max, int d_h, float scale, int window, gqa_dtype dtype, void* workspace,
                        size_t workspace_bytes, int num_splits, void* stream,
                        const int32_t* block_table, int max_pages, int page_size, int num_pages) {
   using namespace gqa;
   if (!q || !k_cache || !v_cache || !o) return GQA_ERR_INVALID_ARG;
+  if (window < 0) return GQA_ERR_INVALID_ARG;
   if (B <= 0 || h_q <= 0 || h_kv <= 0 || T_max <= 0 || d_h <= 0 || num_splits < 0)
     return GQA_ERR_INVALID_ARG;
   if (h_q % h_kv != 0 || !valid_scale(scale)) return GQA_ERR_INVALID_ARG;
@@ -122,6 +123,7 @@ gqa_status decode_impl(const void* q, const void* k_cache, const void* v_cache, 
   a.T_max = T_max;
   a.d_h = d_h;
   a.scale = scale;
+  a.window = window;
   a.workspace = workspace;
   a.workspace_bytes = workspace_bytes;
   a.num_splits = num_splits;
@@ -225,8 +227,10 @@ gqa_status kv_append(void* k_cache, void* v_cache, const void* k_new, const void
 gqa_status gqa_prefill(const void* q, const void* k_cache, const void* v_cache, void* o,
                        float* lse, const int32_t* q_start, const int32_t* kv_len,
                        int B, int h_q, int h_kv, int S_q, int T_max, int d_h,
-                       float scale, int causal, gqa_dtype dtype, void* stream) {
+                       float scale, int causal, int window, gqa_dtype dtype, void* stream) {
   if (!q || !k_cache || !v_cache || !o) return GQA_ERR_INVALID_ARG;
+  // a window is measured back from each row's own position, so it needs the causal mask
+  if (window < 0 || (window > 0 && causal != 1)) return GQA_ERR_INVALID_ARG;
   if (B <= 0 || h_q <= 0 || h_kv <= 0 || S_q <= 0 || T_max <= 0 || d_h <= 0)
     return GQA_ERR_INVALID_ARG;
   if (h_q % h_kv != 0 || !valid_scale(scale)) return GQA_ERR_INVALID_ARG;
@@ -247,6 +251,7 @@ gqa_status gqa_prefill(const void* q, const void* k_cache, const void* v_cache, 
   a.d_h = d_h;
   a.scale = scale;
   a.causal = causal;
+  a.window = window;
   a.err = device_error_ptr();
   if (!a.err) return GQA_ERR_CUDA;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -287,23 +292,25 @@ size_t gqa_decode_workspace_size(int B, int h_q, int h_kv, int T_max, int d_h, g
 
 gqa_status gqa_decode(const void* q, const void* k_cache, const void* v_cache, void* o, float* lse,
                       const int32_t* kv_len, const int32_t* q_pos,
-                      int B, int h_q, int h_kv, int T_max, int d_h, float scale, gqa_dtype dtype,
-                      void* workspace, size_t workspace_bytes, int num_splits, void* stream) {
+                      int B, int h_q, int h_kv, int T_max, int d_h, float scale, int window,
+                      gqa_dtype dtype, void* workspace, size_t workspace_bytes, int num_splits,
+                      void* stream) {
   return decode_impl(q, k_cache, v_cache, o, lse, kv_len, q_pos, B, h_q, h_kv, T_max, d_h, scale,
-                     dtype, workspace, workspace_bytes, num_splits, stream, nullptr, 0, 0, 0);
+                     window, dtype, workspace, workspace_bytes, num_splits, stream, nullptr, 0, 0, 0);
 }
 
 gqa_status gqa_decode_paged(const void* q, const void* k_pages, const void* v_pages, void* o,
                             float* lse, const int32_t* kv_len, const int32_t* q_pos,
                             const int32_t* block_table, int B, int h_q, int h_kv, int num_pages,
-                            int page_size, int max_pages, int d_h, float scale, gqa_dtype dtype,
-                            void* workspace, size_t workspace_bytes, int num_splits, void* stream) {
+                            int page_size, int max_pages, int d_h, float scale, int window,
+                            gqa_dtype dtype, void* workspace, size_t workspace_bytes,
+                            int num_splits, void* stream) {
   if (!block_table || num_pages <= 0 || page_size <= 0 || max_pages <= 0) return GQA_ERR_INVALID_ARG;
   if (page_size % 16 != 0) return GQA_ERR_UNSUPPORTED;
   const long long T_max = (long long)max_pages * page_size;
   if (T_max >= (1ll << 31)) return GQA_ERR_UNSUPPORTED;
   return decode_impl(q, k_pages, v_pages, o, lse, kv_len, q_pos, B, h_q, h_kv, (int)T_max, d_h,
-                     scale, dtype, workspace, workspace_bytes, num_splits, stream, block_table,
+                     scale, window, dtype, workspace, workspace_bytes, num_splits, stream, block_table,
                      max_pages, page_size, num_pages);
 }
 

@@ -102,6 +102,7 @@ struct KArgs {
   float scale;     // natural-log scale; the bf16 core folds log2(e) in
   int n_max;       // upper bound on the number of chunks (workspace slots)
   int auto_chunk;  // 1: chunks hold at least kMinChunkAuto keys
+  int window;      // 0: none; W > 0: the query at q_pos sees keys q_pos - W < j <= q_pos
   Header* hdr;
   long long* pre;
   int* nlen;
@@ -120,7 +121,8 @@ struct KArgs {
 // Partition view built in shared memory by every CTA.
 struct Plan {
   const long long* pre;  // pre[b] = sum_{b' < b} ceil(n_b' / gran): positions count granules
-  const int* nlen;
+  const int* nlen;       // unit length: visible keys from the granule-aligned window start
+  const int* wlo;        // first visible key (0 without a sliding window)
   int gran;
   int UPB;               // units per sequence = h_kv * hblocks
   long long K;           // total keys over all units
@@ -170,8 +172,8 @@ __device__ __forceinline__ Piece locate(const Plan& p, int B, int hblocks, long 
 // the chunk size. CTA 0 also publishes them to the workspace for the merge kernel and writes zero
 // rows (lse = -inf) for sequences with no visible key.
 template <typename OutT>
-__device__ void build_plan(const KArgs& a, Plan& p, long long* pre, int* nlen, int warp, int lane,
-                           int w0) {
+__device__ void build_plan(const KArgs& a, Plan& p, long long* pre, int* nlen, int* wlo, int warp,
+                           int lane, int w0) {
   if (warp == w0) {
     long long run = 0;
     for (int base = 0; base < a.B; base += 32) {
@@ -180,14 +182,25 @@ __device__ void build_plan(const KArgs& a, Plan& p, long long* pre, int* nlen, i
       if (b < a.B) {
         const int kv = a.kv_len ? a.kv_len[b] : a.T_max;
         const int qp = a.q_pos ? a.q_pos[b] : kv - 1;
+        int lo = 0;
         if (kv < 1 || kv > a.T_max) {
           if (blockIdx.x == 0) set_device_error(a.err, GQA_DEVERR_KV_LEN);
         } else if (qp < 0) {
           if (blockIdx.x == 0) set_device_error(a.err, GQA_DEVERR_POSITION);
         } else {
           n = qp + 1 < kv ? qp + 1 : kv;
+          if (a.window > 0 && qp - a.window + 1 > 0) lo = qp - a.window + 1;
+          if (lo >= n) {  // the window starts at or past the last cached key
+            if (blockIdx.x == 0) set_device_error(a.err, GQA_DEVERR_NO_VISIBLE);
+            n = 0;
+            lo = 0;
+          }
         }
+        // the unit starts at the window start rounded down to the granule; the keys before the
+        // window inside that first granule are masked (only on a paged cache, gran > 1)
+        if (n > 0) n -= lo / a.gran * a.gran;
         nlen[b] = n;
+        wlo[b] = lo;
       }
       const long long ngr = (n + a.gran - 1) / a.gran;  // granules
       long long s = ngr;  // inclusive warp scan
@@ -204,6 +217,7 @@ __device__ void build_plan(const KArgs& a, Plan& p, long long* pre, int* nlen, i
   __syncthreads();
   p.pre = pre;
   p.nlen = nlen;
+  p.wlo = wlo;
   p.gran = a.gran;
   p.UPB = a.h_kv * a.hblocks;
   p.K = pre[a.B] * p.UPB;
@@ -379,9 +393,9 @@ __device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], 
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 // zero the bf16 halves of a packed pair whose key index is >= nvalid
-__device__ __forceinline__ uint32_t mask_pair(uint32_t v, int key_lo, int nvalid) {
-  const uint32_t lo = key_lo < nvalid ? 0x0000ffffu : 0u;
-  const uint32_t hi = key_lo + 1 < nvalid ? 0xffff0000u : 0u;
+__device__ __forceinline__ uint32_t mask_pair(uint32_t v, int key_lo, int first, int nvalid) {
+  const uint32_t lo = key_lo < nvalid && key_lo >= first ? 0x0000ffffu : 0u;
+  const uint32_t hi = key_lo + 1 < nvalid && key_lo + 1 >= first ? 0xffff0000u : 0u;
   return v & (lo | hi);
 }
 
@@ -392,7 +406,7 @@ struct TileMeta {
   int flags;   // kFirst | kLast | kEnd
   int slot;    // partial slot, or -1: write the output directly
   int nh;      // query heads in the unit
-  int pad;
+  int nskip;   // leading keys of the tile before the sliding window (masked), else 0
 };
 constexpr int kFirst = 1, kLast = 2, kEnd = 4;
 
@@ -417,7 +431,7 @@ struct Bf16Cfg {
   static constexpr int kRedBytes = MT * 4 * 16 * kRedStride * 4;
   static constexpr int kStatBytes = MT * 4 * 16 * 4;
   static constexpr size_t kSmem = (size_t)kStages * (kStageBytes + kQBytes) + kRedBytes +
-                                  2 * kStatBytes + (kMaxBatch + 1) * 8 + kMaxBatch * 4 +
+                                  2 * kStatBytes + (kMaxBatch + 1) * 8 + 2 * kMaxBatch * 4 +
                                   kStages * sizeof(TileMeta) + 2 * kStages * 8 + 1024;
   static_assert(kSmem <= 227 * 1024, "shared memory budget");
 };
@@ -448,7 +462,8 @@ __global__ void __launch_bounds__(Bf16Cfg<D, MT>::kThreads, 1)
   float* st_l = st_m + MT * 64;
   long long* pre = reinterpret_cast<long long*>(st_l + MT * 64);
   int* nlen = reinterpret_cast<int*>(pre + kMaxBatch + 1);
-  TileMeta* meta = reinterpret_cast<TileMeta*>(nlen + kMaxBatch);
+  int* wlo = nlen + kMaxBatch;
+  TileMeta* meta = reinterpret_cast<TileMeta*>(wlo + kMaxBatch);
   uint64_t* bars = reinterpret_cast<uint64_t*>(meta + C::kStages);
 
   const int warp = threadIdx.x >> 5;
@@ -463,7 +478,7 @@ __global__ void __launch_bounds__(Bf16Cfg<D, MT>::kThreads, 1)
     fence_barrier_init();
   }
   Plan plan;
-  build_plan<__nv_bfloat16>(a, plan, pre, nlen, warp, lane, producer_warp);
+  build_plan<__nv_bfloat16>(a, plan, pre, nlen, wlo, warp, lane, producer_warp);
   pdl_launch_dependents();
 
   if (warp == producer_warp) {
@@ -476,7 +491,7 @@ __global__ void __launch_bounds__(Bf16Cfg<D, MT>::kThreads, 1)
     const int G = gridDim.x;
     // Writes the stage's descriptor and arms its full barrier for `kv_bytes` of K/V (+ the query
     // rows on a piece's first tile). Lane 0 only.
-    auto arm = [&](const Piece& pc, int t, int slot, int nh, uint32_t kv_bytes) -> uint32_t {
+    auto arm = [&](const Piece& pc, int t, int slot, int nh, uint32_t kv_bytes, int nskip) -> uint32_t {
       const bool first = t == pc.k0;
       TileMeta m;
       m.b = pc.b;
@@ -486,7 +501,7 @@ __global__ void __launch_bounds__(Bf16Cfg<D, MT>::kThreads, 1)
       m.flags = (first ? kFirst : 0) | (t + kTile >= pc.k1 ? kLast : 0);
       m.slot = slot;
       m.nh = nh;
-      m.pad = 0;
+      m.nskip = t == 0 ? nskip : 0;  // only a unit's first tile starts before the window
       meta[stage] = m;
       const uint32_t full = smem_u32(&bars[stage]);
       mbar_arrive_expect_tx(full, kv_bytes + (first ? C::kQBytes : 0));
@@ -519,10 +534,11 @@ __global__ void __launch_bounds__(Bf16Cfg<D, MT>::kThreads, 1)
             const Piece pc = locate(plan, a.B, a.hblocks, x, x1);
             const int slot = pc.n_pieces == 1 ? -1 : chunk + pc.unit;
             const int nh = min(a.hpu, a.r - pc.hb * a.hpu);
-            const int row0 = (pc.b * a.h_kv + pc.g) * a.T_max;
+            const int lo = plan.wlo[pc.b];  // contiguous cache: granule 1, the unit starts at lo
+            const int row0 = (pc.b * a.h_kv + pc.g) * a.T_max + lo;
             for (int t = pc.k0; t < pc.k1; t += kTile) {
               if (!mbar_wait(smem_u32(&bars[C::kStages + stage]), phase ^ 1u, a.err)) { ok = false; break; }
-              const uint32_t full = arm(pc, t, slot, nh, C::kStageBytes);
+              const uint32_t full = arm(pc, t, slot, nh, C::kStageBytes, 0);
               const uint32_t kdst = smem_u32(stage_base + stage * C::kStageBytes);
               const uint32_t vdst = kdst + C::kTileBytes;
 #pragma unroll
@@ -562,7 +578,12 @@ __global__ void __launch_bounds__(Bf16Cfg<D, MT>::kThreads, 1)
           const int slot = pc.n_pieces == 1 ? -1 : chunk + pc.unit;
           const int nh = min(a.hpu, a.r - pc.hb * a.hpu);
           const int32_t* bt = a.block_table + (long long)pc.b * a.max_pages;
-          const int s_end = (pc.k1 + 15) >> 4;  // sub-tiles of this piece: [k0 / 16, s_end)
+          // keys are absolute positions koff + t: the unit starts at the window start rounded
+          // down to the granule (a multiple of 16), and its first nskip keys are masked
+          const int lo = plan.wlo[pc.b];
+          const int koff = lo / a.gran * a.gran;
+          const int nskip = lo - koff;
+          const int s_end = (koff + pc.k1 + 15) >> 4;  // sub-tiles: [(koff + k0) / 16, s_end)
           // raw table entry of sub-tile s (-1 past the piece: never used)
           auto fetch = [&](int s) -> int { return s < s_end ? __ldg(bt + (s << 4) / a.page_size) : -1; };
           // pool row of sub-tile s from its table entry; an entry outside the pool is flagged and
@@ -575,11 +596,11 @@ __global__ void __launch_bounds__(Bf16Cfg<D, MT>::kThreads, 1)
             }
             return (page * a.h_kv + pc.g) * a.page_size + (s << 4) % a.page_size;
           };
-          int wbase = pc.k0 >> 4;  // first sub-tile of the current window
+          int wbase = (koff + pc.k0) >> 4;  // first sub-tile of the current window
           int cur = to_row(fetch(wbase + lane), wbase + lane);
           int nxt = fetch(wbase + 32 + lane);
           for (int t = pc.k0; t < pc.k1; t += kTile) {
-            const int s = t >> 4;
+            const int s = (koff + t) >> 4;
             if (s >= wbase + 32) {
               wbase += 32;
               cur = to_row(nxt, wbase + lane);
@@ -597,7 +618,7 @@ __global__ void __launch_bounds__(Bf16Cfg<D, MT>::kThreads, 1)
               if (kMode == kPaged2d && a.gran == kTile) {
                 // pages hold a multiple of 64 keys and tiles start on multiples of 64: the whole
                 // tile lies in one page and loads as one 64-row box per column chunk
-                const uint32_t full = arm(pc, t, slot, nh, C::kStageBytes);
+                const uint32_t full = arm(pc, t, slot, nh, C::kStageBytes, nskip);
 #pragma unroll
                 for (int ch = 0; ch < C::kNch; ++ch) {
                   tma_load_2d(kdst + ch * C::kChunkBytes, &tmk, full, ch * 64, prow[0]);
@@ -605,7 +626,7 @@ __global__ void __launch_bounds__(Bf16Cfg<D, MT>::kThreads, 1)
                 }
               } else {
                 const int nsub = (min(kTile, pc.k1 - t) + 15) >> 4;
-                const uint32_t full = arm(pc, t, slot, nh, (uint32_t)nsub * (C::kStageBytes / 4));
+                const uint32_t full = arm(pc, t, slot, nh, (uint32_t)nsub * (C::kStageBytes / 4), nskip);
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
                   if (j >= nsub) break;
@@ -673,7 +694,8 @@ __global__ void __launch_bounds__(Bf16Cfg<D, MT>::kThreads, 1)
   float acc[NN][4];
   float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
   while (true) {
-    if (!mbar_wait(smem_u32(&bars[stage]), phase, a.err)) return;
+    // ldmatrix / mma.sync below need the whole warp: leave together if the wait ran out
+    if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&bars[stage]), phase, a.err))) return;
     const TileMeta m = meta[stage];
     if (m.flags & kEnd) {
       __syncwarp();
@@ -699,8 +721,9 @@ __global__ void __launch_bounds__(Bf16Cfg<D, MT>::kThreads, 1)
       l0 = l1 = 0.f;
     }
     const int nvalid = m.nvalid;
+    const int nskip = m.nskip;
     const int klo = ws * 16;
-    if (klo < nvalid) {
+    if (klo < nvalid && klo + 16 > nskip) {
       // ---- S = Q K^T for keys klo .. klo+15 (two n-tiles of 8 keys)
       float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
       {
@@ -722,7 +745,7 @@ __global__ void __launch_bounds__(Bf16Cfg<D, MT>::kThreads, 1)
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
           const int key = klo + 8 * j + 2 * tq + e;
-          const bool vis = key < nvalid;
+          const bool vis = key < nvalid && key >= nskip;
           sc[j][e] = vis ? sc[j][e] * sl2 : -INFINITY;
           sc[j][2 + e] = vis ? sc[j][2 + e] * sl2 : -INFINITY;
           mx0 = fmaxf(mx0, sc[j][e]);
@@ -763,7 +786,7 @@ __global__ void __launch_bounds__(Bf16Cfg<D, MT>::kThreads, 1)
       pa[2] = pack_bf16x2(sc[1][0], sc[1][1]);
       pa[3] = pack_bf16x2(sc[1][2], sc[1][3]);
       // ---- O += P V (keys klo..klo+15, all d_h columns)
-      const bool partial = klo + 16 > nvalid;
+      const bool partial = klo + 16 > nvalid || klo < nskip;
       const int vrow = klo + ((lane >> 3) & 1) * 8 + (lane & 7);
       const int key_a = klo + 2 * tq, key_b = klo + 8 + 2 * tq;
 #pragma unroll
@@ -773,10 +796,10 @@ __global__ void __launch_bounds__(Bf16Cfg<D, MT>::kThreads, 1)
         ldsm_x4_t(swz128(vb + kv_warp_off + (d8 >> 3) * kKvChunkStride, vrow & kv_row_mask, d8 & 7),
                   b0, b1, b2, b3);
         if (partial) {
-          b0 = mask_pair(b0, key_a, nvalid);
-          b1 = mask_pair(b1, key_b, nvalid);
-          b2 = mask_pair(b2, key_a, nvalid);
-          b3 = mask_pair(b3, key_b, nvalid);
+          b0 = mask_pair(b0, key_a, nskip, nvalid);
+          b1 = mask_pair(b1, key_b, nskip, nvalid);
+          b2 = mask_pair(b2, key_a, nskip, nvalid);
+          b3 = mask_pair(b3, key_b, nskip, nvalid);
         }
         mma_bf16(acc[2 * n2], pa, b0, b1);
         mma_bf16(acc[2 * n2 + 1], pa, b2, b3);
@@ -860,10 +883,11 @@ constexpr int kF32MaxPerLane = 8;  // d_h <= 256
 __global__ void __launch_bounds__(32 * kF32Warps, 1) decode_fp32_kernel(KArgs a) {
   __shared__ long long pre[kMaxBatch + 1];
   __shared__ int nlen[kMaxBatch];
+  __shared__ int wlo[kMaxBatch];
   __shared__ int chunk_s;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   Plan plan;
-  build_plan<float>(a, plan, pre, nlen, warp, lane, 0);
+  build_plan<float>(a, plan, pre, nlen, wlo, warp, lane, 0);
   pdl_launch_dependents();
   const int D = a.D;
   for (int iter = 0;; ++iter) {
@@ -878,6 +902,9 @@ __global__ void __launch_bounds__(32 * kF32Warps, 1) decode_fp32_kernel(KArgs a)
       const Piece pc = locate(plan, a.B, a.hblocks, x, x1);
       const int slot = pc.n_pieces == 1 ? -1 : chunk + pc.unit;
       const int nh = min(a.hpu, a.r - pc.hb * a.hpu);
+      const int lo = wlo[pc.b];
+      const int koff = lo / a.gran * a.gran;  // absolute position of the unit's key 0
+      const int jskip = lo - koff;            // keys of the first granule before the window
       const long long kv_base = ((long long)pc.b * a.h_kv + pc.g) * a.T_max * D;
       const float* kp = reinterpret_cast<const float*>(a.k) + kv_base;
       const float* vp = reinterpret_cast<const float*>(a.v) + kv_base;
@@ -892,7 +919,8 @@ __global__ void __launch_bounds__(32 * kF32Warps, 1) decode_fp32_kernel(KArgs a)
           accv[e] = 0.f;
         }
         float m = -INFINITY, l = 0.f;
-        for (int j = pc.k0; j < pc.k1; ++j) {
+        for (int jr = max(pc.k0, jskip); jr < pc.k1; ++jr) {
+          const int j = koff + jr;  // absolute key position
           const float* kj = kp + (long long)j * D;
           const float* vj = vp + (long long)j * D;
           if (a.block_table) {
@@ -1018,6 +1046,7 @@ KArgs make_kargs(const DecodeArgs& a) {
   k.scale = a.scale;
   k.n_max = n_max;
   k.auto_chunk = auto_chunk ? 1 : 0;
+  k.window = a.window;
   uint8_t* ws = reinterpret_cast<uint8_t*>(a.workspace);
   k.hdr = reinterpret_cast<Header*>(ws);
   k.pre = reinterpret_cast<long long*>(ws + L.pre_off);

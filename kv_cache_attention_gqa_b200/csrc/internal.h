@@ -36,6 +36,7 @@ struct PrefillArgs {
   int B, h_q, h_kv, S_q, T_max, d_h;
   float scale;
   int causal;
+  int window;  // 0: none; W > 0 (causal only): row at position p sees keys p - W < j <= p
   unsigned* err;
 };
 // fp32 check mode (scalar FFMA)
@@ -61,6 +62,7 @@ struct DecodeArgs {
   size_t workspace_bytes;
   int num_splits;  // 0 = automatic chunking, else the number of chunks to cut the keys into
   int num_sms;     // persistent grid size
+  int window = 0;  // 0: none; W > 0: the query at q_pos sees keys q_pos - W < j <= q_pos
   unsigned* err;
   // paged cache, or block_table == nullptr for the contiguous (B, h_kv, T_max, d_h) layout:
   // k/v are pools (num_pages, h_kv, page_size, d_h), T_max = max_pages * page_size

@@ -53,10 +53,10 @@ cudaError_t scratch_address(void** out) {
 extern "C" gqa_status gqa_decode_noalloc(const void* q, const void* k_cache, const void* v_cache,
                                          void* o, float* lse, const int32_t* kv_len,
                                          const int32_t* q_pos, int B, int h_q, int h_kv,
-                                         int T_max, int d_h, float scale, gqa_dtype dtype,
-                                         int num_splits, void* stream) {
+                                         int T_max, int d_h, float scale, int window,
+                                         gqa_dtype dtype, int num_splits, void* stream) {
   using namespace gqa;
-  if (B <= 0 || h_q <= 0 || h_kv <= 0 || T_max <= 0 || d_h <= 0 || num_splits < 0 ||
+  if (B <= 0 || h_q <= 0 || h_kv <= 0 || T_max <= 0 || d_h <= 0 || num_splits < 0 || window < 0 ||
       h_q % h_kv != 0)
     return GQA_ERR_INVALID_ARG;
   const size_t need = gqa_decode_workspace_size(B, h_q, h_kv, T_max, d_h, dtype, num_splits);
@@ -68,5 +68,5 @@ extern "C" gqa_status gqa_decode_noalloc(const void* q, const void* k_cache, con
   // the work ticket (first 256 bytes of the workspace) must be zero when the decode starts
   if (cudaMemsetAsync(scratch, 0, 256, s) != cudaSuccess) return GQA_ERR_CUDA;
   return gqa_decode(q, k_cache, v_cache, o, lse, kv_len, q_pos, B, h_q, h_kv, T_max, d_h, scale,
-                    dtype, scratch, kNoAllocScratchBytes, num_splits, stream);
+                    window, dtype, scratch, kNoAllocScratchBytes, num_splits, stream);
 }

@@ -5,8 +5,8 @@
 // the fp64 oracle at a 1e-5 relative tolerance independently of bf16 rounding.
 //
 // One warp owns one query row (b, a, i). Lane l holds the d_h elements c = l + 32 e of the query
-// and of the running output. For each visible key j (a prefix: j < min(kv_len[b], q_start[b]+i+1)
-// under the causal mask), the warp forms s_j = scale * q . k_j with a shuffle reduction and applies
+// and of the running output. For each visible key j (j < min(kv_len[b], q_start[b]+i+1) under the
+// causal mask, and j > q_start[b]+i - W under a sliding window of W), the warp forms s_j = scale * q . k_j with a shuffle reduction and applies
 // the online-softmax update with a block of one key:
 //   m' = max(m, s_j),  l' = e^{m - m'} l + e^{s_j - m'},  u' = e^{m - m'} u + e^{s_j - m'} v_j
 // [序列计算与存储, section 在线 softmax], starting from m = -inf, l = 0, u = 0; o = u / l.
@@ -40,7 +40,7 @@ __global__ void __launch_bounds__(256) prefill_fp32_kernel(PrefillArgs a) {
 
   const int kv_len = a.kv_len ? a.kv_len[b] : a.T_max;
   const int q0 = a.q_start ? a.q_start[b] : 0;
-  int n_vis = -1;
+  int n_vis = -1, j_lo = 0;
   if (kv_len < 1 || kv_len > a.T_max) {
     if (lane == 0) set_device_error(a.err, GQA_DEVERR_KV_LEN);
   } else if (q0 < 0) {
@@ -48,6 +48,11 @@ __global__ void __launch_bounds__(256) prefill_fp32_kernel(PrefillArgs a) {
   } else {
     const long long lim = (long long)q0 + i + 1;
     n_vis = a.causal ? (int)(lim < kv_len ? lim : kv_len) : kv_len;
+    if (a.window > 0) {
+      const long long lo = lim - a.window;  // first key inside the window
+      if (lo > 0) j_lo = lo < n_vis ? (int)lo : n_vis;
+      n_vis -= j_lo;
+    }
   }
   if (n_vis <= 0) {  // invalid request or no visible key: zero row, flagged
     if (n_vis == 0 && lane == 0) set_device_error(a.err, GQA_DEVERR_NO_VISIBLE);
@@ -64,7 +69,7 @@ __global__ void __launch_bounds__(256) prefill_fp32_kernel(PrefillArgs a) {
     acc[e] = 0.f;
   }
   float m = -INFINITY, l = 0.f;
-  for (int j = 0; j < n_vis; ++j) {
+  for (int j = j_lo; j < j_lo + n_vis; ++j) {
     const float* kj = kp + (long long)j * D;
     const float* vj = vp + (long long)j * D;
     float part = 0.f;

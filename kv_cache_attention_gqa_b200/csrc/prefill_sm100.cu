@@ -4,7 +4,9 @@
 // [序列计算与存储, section 分组查询注意力], the causal/length mask by absolute position
 // [第 09 章 GQA、MLA 与跨层 KV 共享, section 09.2], evaluated block by block with the online
 // softmax state (m, l, u) so the score matrix never reaches memory [序列计算与存储, sections
-// 分块注意力 and 在线 softmax].
+// 分块注意力 and 在线 softmax]. An optional sliding window W limits row p to keys p - W < j <= p
+// [第三章：MHA 的局限与 MQA、GQA、Flash Attention, section 3.7]: K/V blocks below the tile's
+// earliest window are never loaded, and the boundary blocks are masked per row.
 //
 // Work tile. Rows of one tile are (query position, query head) pairs of ONE KV group: H heads
 // (H = min(r, 128)) times P = floor(128 / H) consecutive positions, head-major, so every K/V block
@@ -81,6 +83,7 @@ struct PArgs {
   int H, P, hblocks, n_qt;
   float scale_log2;
   int causal;
+  int window;  // 0: none; W > 0: row at position p also needs key j > p - W (causal only)
   unsigned* err;
 };
 
@@ -121,7 +124,8 @@ struct Tile {
   int b, g, hb, q0;  // q0: first query position (index into S_q) of the tile
   int nh;            // heads of this head block
   int qs, kv;        // q_start[b], kv_len[b]
-  int nb;            // K/V blocks to visit
+  int j0;            // first K/V block visited (> 0 only under a sliding window)
+  int nb;            // K/V blocks to visit: j0 .. j0 + nb - 1
   bool valid;
 };
 
@@ -141,12 +145,20 @@ __device__ __forceinline__ Tile make_tile(const PArgs& a) {
   t.qs = a.q_start ? a.q_start[t.b] : 0;
   t.valid = t.kv >= 1 && t.kv <= a.T_max && t.qs >= 0;
   t.nb = 0;
+  t.j0 = 0;
   if (t.valid) {
     if (a.causal) {
       const int last_row = min(t.q0 + a.P, a.S_q) - 1;
       const long long pos_max = (long long)t.qs + last_row;
       const long long last_key = pos_max < t.kv - 1 ? pos_max : (long long)(t.kv - 1);
-      t.nb = (int)(last_key / kBN) + 1;
+      const int end = (int)(last_key / kBN) + 1;
+      if (a.window > 0) {
+        // blocks wholly below the earliest row's window are skipped [第三章 §3.7: each query
+        // reads only its local window]
+        const long long lo = (long long)t.qs + t.q0 - a.window + 1;
+        if (lo > 0) t.j0 = (int)(lo / kBN);
+      }
+      t.nb = end > t.j0 ? end - t.j0 : 0;
     } else {
       t.nb = (t.kv + kBN - 1) / kBN;
     }
@@ -214,6 +226,7 @@ __device__ __forceinline__ void softmax_role(const PArgs& a, const Tile& tile, i
   const bool store_row = h < tile.nh && row < a.H * a.P && qi < a.S_q;
   const long long pos = (long long)tile.qs + qi;
   const long long pos_min = (long long)tile.qs + tile.q0;  // smallest position in the tile
+  const long long pos_max = (long long)tile.qs + min(tile.q0 + a.P, a.S_q) - 1;  // largest
   const int nb = tile.nb;
   const float c = a.scale_log2;
   const long long orow = ((long long)tile.b * a.h_q + tile.g * a.r + tile.hb * a.H + h) * a.S_q + qi;
@@ -221,7 +234,10 @@ __device__ __forceinline__ void softmax_role(const PArgs& a, const Tile& tile, i
   float* xmax = xbuf;                         // [2 buffers][2 halves][128 rows]
 
   // ---- this half of this row of Q: shared memory (128-byte swizzled) -> TMEM (A of Q K^T)
+  // tcgen05.ld / st / wait are .sync.aligned: every lane of a warp must execute each of them, so
+  // every condition in front of one is made warp-uniform (__all_sync / __any_sync) first.
   bool ok = nb > 0 && wait_bar(bar(kBarQ), 0, abort, a.err);
+  ok = __all_sync(0xffffffffu, ok);
   if (ok) {
 #pragma unroll
     for (int ch = 0; ch < C::kNch; ++ch) {
@@ -248,11 +264,12 @@ __device__ __forceinline__ void softmax_role(const PArgs& a, const Tile& tile, i
     // After a failed wait the loop keeps running (without touching TMEM or other barriers) so
     // that every softmax thread takes the per-block named barrier the same number of times.
     if (ok) ok = wait_bar(bar(kBarS + buf), (uint32_t)((j >> 1) & 1), abort, a.err);
+    ok = __all_sync(0xffffffffu, ok);
     float sr[64];
     float lmx = 0.f;
-    const int key0 = j * kBN + half * 64;     // first key of this half
-    const bool need_mask =
-        (a.causal && (long long)key0 + 63 > pos_min) || key0 + 64 > tile.kv;
+    const int key0 = (tile.j0 + j) * kBN + half * 64;  // first key of this half
+    const bool need_mask = (a.causal && (long long)key0 + 63 > pos_min) || key0 + 64 > tile.kv ||
+                           (a.window > 0 && (long long)key0 <= pos_max - a.window);
     if (ok) {
       tc::fence_after_sync();
       uint32_t su[2][32];
@@ -265,7 +282,8 @@ __device__ __forceinline__ void softmax_role(const PArgs& a, const Tile& tile, i
 #pragma unroll
         for (int i = 0; i < 64; ++i) {
           const int key = key0 + i;
-          const bool vis = key < tile.kv && (!a.causal || key <= pos);
+          const bool vis = key < tile.kv && (!a.causal || key <= pos) &&
+                           (a.window == 0 || (long long)key > pos - a.window);
           sr[i] = vis ? sr[i] : -INFINITY;
         }
       }
@@ -293,7 +311,10 @@ __device__ __forceinline__ void softmax_role(const PArgs& a, const Tile& tile, i
       alpha = fast_exp2(m - m_new);
       rescale_o = true;
     }
-    // P = 2^(s c - m_use) as bf16 pairs: this half's keys go to 32 of the first 64 S columns
+    // P = 2^(s c - m_use) as bf16 pairs: this half's keys go to 32 of the first 64 S columns.
+    // A row that has seen no visible key yet (only possible under a sliding window) keeps
+    // m = -inf; its P is 0, computed against 0 instead of -inf.
+    const float m_sub = m_use == -INFINITY ? 0.f : m_use;
     float sum0 = 0.f, sum1 = 0.f;
 #pragma unroll
     for (int cc = 0; cc < 2; ++cc) {
@@ -301,7 +322,7 @@ __device__ __forceinline__ void softmax_role(const PArgs& a, const Tile& tile, i
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
         float x0, x1;
-        ffma2(x0, x1, sr[cc * 32 + 2 * i], sr[cc * 32 + 2 * i + 1], c, -m_use);
+        ffma2(x0, x1, sr[cc * 32 + 2 * i], sr[cc * 32 + 2 * i + 1], c, -m_sub);
         const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
         fadd2(sum0, sum1, p0, p1);
         pk[i] = pack_bf16x2(p0, p1);
@@ -310,9 +331,12 @@ __device__ __forceinline__ void softmax_role(const PArgs& a, const Tile& tile, i
     }
     l = l * alpha + (sum0 + sum1);
     m = m_use;
-    if (rescale_o && j > 0) {
+    // the warp rescales its O rows together when any of its rows needs it (rows that do not
+    // need it multiply by alpha = 1)
+    if (__any_sync(0xffffffffu, rescale_o && j > 0)) {
       // O must hold every earlier block's contribution before it is rescaled
       if (!wait_bar(bar(kBarO), (uint32_t)((j - 1) & 1), abort, a.err)) ok = false;
+      ok = __all_sync(0xffffffffu, ok);
       if (ok) {
         tc::fence_after_sync();
 #pragma unroll
@@ -327,14 +351,18 @@ __device__ __forceinline__ void softmax_role(const PArgs& a, const Tile& tile, i
       }
     }
     tc::wait_st();
-    const int bkey0 = j * kBN;
-    if (ok && j == nb - 1 && bkey0 + kBN > tile.kv && (C::kNch == 2 || half == 0)) {
-      // V rows at or past kv_len get weight 0 but may hold anything (NaN included): zero them in
-      // shared memory so 0 * V stays 0 (each half zeroes its own 64-column chunk). The block's V
-      // must have landed first.
+    const int bkey0 = (tile.j0 + j) * kBN;
+    // V rows at or past kv_len, and (sliding window) rows below the earliest row's window, get
+    // weight 0 for every row of the tile but may hold anything (NaN included): zero them in shared
+    // memory so 0 * V stays 0 (each half zeroes its own 64-column chunk). The block's V must have
+    // landed first.
+    const bool zero_tail = j == nb - 1 && bkey0 + kBN > tile.kv;
+    const bool zero_head = j == 0 && a.window > 0 && (long long)bkey0 < pos_min - a.window + 1;
+    if (ok && (zero_tail || zero_head) && (C::kNch == 2 || half == 0)) {
       const int vs = j % kVStages;
       if (wait_bar(bar(kBarVFull + vs), (uint32_t)((j / kVStages) & 1), abort, a.err)) {
-        if (row >= tile.kv - bkey0) {
+        const long long key = (long long)bkey0 + row;
+        if ((zero_tail && key >= tile.kv) || (zero_head && key <= pos_min - a.window)) {
 #pragma unroll
           for (int k = 0; k < 8; ++k) {
             const uint32_t addr = sV + vs * C::kKVBytes + (C::kNch == 2 ? half : 0) * C::kKVChunk + row * 128 + k * 16;
@@ -363,11 +391,16 @@ __device__ __forceinline__ void softmax_role(const PArgs& a, const Tile& tile, i
   named_barrier_sync(1, 256);
   l += xsum[(half ^ 1) * 128 + row];
   (void)sm_tid;
-  if (!ok) return;
+  if (!__all_sync(0xffffffffu, ok)) return;
   // epilogue: this half of O / l -> bf16 -> global; lse = (m + log2 l) * ln 2
-  if (!wait_bar(bar(kBarO), (uint32_t)((nb - 1) & 1), abort, a.err)) return;
+  bool ok_o = wait_bar(bar(kBarO), (uint32_t)((nb - 1) & 1), abort, a.err);
+  if (!__all_sync(0xffffffffu, ok_o)) return;
   tc::fence_after_sync();
-  const float inv = 1.f / l;
+  // A row with no visible key (a sliding window that starts at or past kv_len, or a padding row
+  // of the tile) has l = 0: it still takes part in the warp's TMEM loads, and writes zeros.
+  const bool empty = l == 0.f;
+  if (empty && store_row && half == 0) set_device_error(a.err, GQA_DEVERR_NO_VISIBLE);
+  const float inv = empty ? 0.f : 1.f / l;
   uint4* out = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.o) + orow * D + half * kOHalf);
 #pragma unroll
   for (int cc = 0; cc < kOHalf / 32; ++cc) {
@@ -377,14 +410,14 @@ __device__ __forceinline__ void softmax_role(const PArgs& a, const Tile& tile, i
     uint32_t pk[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i)
-      pk[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
+      pk[i] = empty ? 0u : pack_bf16x2(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
     if (store_row) {
 #pragma unroll
       for (int v = 0; v < 4; ++v)
         out[cc * 4 + v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
     }
   }
-  if (store_row && a.lse && half == 0) a.lse[orow] = (m + __log2f(l)) * kLn2;
+  if (store_row && a.lse && half == 0) a.lse[orow] = empty ? -INFINITY : (m + __log2f(l)) * kLn2;
 }
 
 template <int D>
@@ -429,6 +462,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_barrier_init();
     if (!tile.valid) set_device_error(a.err, tile.kv < 1 || tile.kv > a.T_max ? GQA_DEVERR_KV_LEN
                                                                                : GQA_DEVERR_POSITION);
+    else if (tile.nb == 0) set_device_error(a.err, GQA_DEVERR_NO_VISIBLE);
   }
   if (warp == 1) {
     tc::tmem_alloc(smem_u32(tmem_slot), kTmemCols);
@@ -459,14 +493,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive_expect_tx(bar(kBarKFull + ks), C::kKVBytes);
       for (int ch = 0; ch < C::kNch; ++ch)
         tma_load_2d(sK + ks * C::kKVBytes + ch * C::kKVChunk, &tmk, bar(kBarKFull + ks), ch * 64,
-                    row0 + j * kBN);
+                    row0 + (tile.j0 + j) * kBN);
       last_k[ks] = kn;
       const int vs = j % kVStages, vn = j / kVStages;
       if (vn > 0 && !wait_bar(bar(kBarVEmpty + vs), (uint32_t)((vn - 1) & 1), abort, a.err)) break;
       mbar_arrive_expect_tx(bar(kBarVFull + vs), C::kKVBytes);
       for (int ch = 0; ch < C::kNch; ++ch)
         tma_load_2d(sV + vs * C::kKVBytes + ch * C::kKVChunk, &tmv, bar(kBarVFull + vs), ch * 64,
-                    row0 + j * kBN);
+                    row0 + (tile.j0 + j) * kBN);
       last_v[vs] = vn;
     }
     // Drain (bounded, whatever the abort state): no copy may still be landing in shared memory
@@ -563,6 +597,7 @@ cudaError_t launch_prefill_bf16(const PrefillArgs& a, const CUtensorMap* tmaps, 
   p.n_qt = (a.S_q + p.P - 1) / p.P;
   p.scale_log2 = a.scale * pf::kLog2e;
   p.causal = a.causal;
+  p.window = a.window;
   p.err = a.err;
   const long long tiles = (long long)p.n_qt * a.B * a.h_kv * p.hblocks;
   if (tiles <= 0) return cudaSuccess;

@@ -58,26 +58,31 @@ def test_host_side_argument_errors(lib):
     null = None
     s = None
     # null pointers
-    assert lib.gqa_prefill(null, fake, fake, fake, null, null, null, 1, 4, 2, 8, 8, 64, 0.125, 1, 0, s) == 1
+    assert lib.gqa_prefill(null, fake, fake, fake, null, null, null, 1, 4, 2, 8, 8, 64, 0.125, 1, 0, 0, s) == 1
     # h_q not a multiple of h_kv
-    assert lib.gqa_prefill(fake, fake, fake, fake, null, null, null, 1, 6, 4, 8, 8, 64, 0.125, 1, 0, s) == 1
+    assert lib.gqa_prefill(fake, fake, fake, fake, null, null, null, 1, 6, 4, 8, 8, 64, 0.125, 1, 0, 0, s) == 1
     # non-positive sizes, bad scale, bad causal flag
-    assert lib.gqa_prefill(fake, fake, fake, fake, null, null, null, 0, 4, 2, 8, 8, 64, 0.125, 1, 0, s) == 1
-    assert lib.gqa_prefill(fake, fake, fake, fake, null, null, null, 1, 4, 2, 8, 8, 64, float("nan"), 1, 0, s) == 1
-    assert lib.gqa_prefill(fake, fake, fake, fake, null, null, null, 1, 4, 2, 8, 8, 64, -1.0, 1, 0, s) == 1
-    assert lib.gqa_prefill(fake, fake, fake, fake, null, null, null, 1, 4, 2, 8, 8, 64, 0.1, 2, 0, s) == 1
+    assert lib.gqa_prefill(fake, fake, fake, fake, null, null, null, 0, 4, 2, 8, 8, 64, 0.125, 1, 0, 0, s) == 1
+    assert lib.gqa_prefill(fake, fake, fake, fake, null, null, null, 1, 4, 2, 8, 8, 64, float("nan"), 1, 0, 0, s) == 1
+    assert lib.gqa_prefill(fake, fake, fake, fake, null, null, null, 1, 4, 2, 8, 8, 64, -1.0, 1, 0, 0, s) == 1
+    assert lib.gqa_prefill(fake, fake, fake, fake, null, null, null, 1, 4, 2, 8, 8, 64, 0.1, 2, 0, 0, s) == 1
+    # sliding window: negative, or without the causal mask
+    assert lib.gqa_prefill(fake, fake, fake, fake, null, null, null, 1, 4, 2, 8, 8, 64, 0.1, 1, -1, 0, s) == 1
+    assert lib.gqa_prefill(fake, fake, fake, fake, null, null, null, 1, 4, 2, 8, 8, 64, 0.1, 0, 4, 0, s) == 1
+    assert lib.gqa_decode(fake, fake, fake, fake, null, null, null, 1, 4, 2, 8, 64, 0.1, -1, 0, fake, 1 << 20, 1, s) == 1
+    assert lib.gqa_decode_noalloc(fake, fake, fake, fake, null, null, null, 1, 4, 2, 8, 64, 0.1, -1, 0, 1, s) == 1
     # decode
-    assert lib.gqa_decode(null, fake, fake, fake, null, null, null, 1, 4, 2, 8, 64, 0.1, 0, fake, 1 << 20, 1, s) == 1
-    assert lib.gqa_decode(fake, fake, fake, fake, null, null, null, 1, 4, 3, 8, 64, 0.1, 0, fake, 1 << 20, 1, s) == 1
-    assert lib.gqa_decode(fake, fake, fake, fake, null, null, null, 1, 4, 2, 8, 64, 0.1, 0, fake, 1 << 20, -1, s) == 1
-    assert lib.gqa_decode(fake, fake, fake, fake, null, null, null, 1, 4, 2, 8, 64, 0.1, 7, fake, 1 << 20, 1, s) == 1
+    assert lib.gqa_decode(null, fake, fake, fake, null, null, null, 1, 4, 2, 8, 64, 0.1, 0, 0, fake, 1 << 20, 1, s) == 1
+    assert lib.gqa_decode(fake, fake, fake, fake, null, null, null, 1, 4, 3, 8, 64, 0.1, 0, 0, fake, 1 << 20, 1, s) == 1
+    assert lib.gqa_decode(fake, fake, fake, fake, null, null, null, 1, 4, 2, 8, 64, 0.1, 0, 0, fake, 1 << 20, -1, s) == 1
+    assert lib.gqa_decode(fake, fake, fake, fake, null, null, null, 1, 4, 2, 8, 64, 0.1, 0, 7, fake, 1 << 20, 1, s) == 1
     # unsupported: bf16 with d_h = 96; batch beyond the decode limit
-    assert lib.gqa_decode(fake, fake, fake, fake, null, null, null, 1, 4, 2, 8, 96, 0.1, 0, fake, 1 << 20, 1, s) == 2
-    assert lib.gqa_decode(fake, fake, fake, fake, null, null, null, 5000, 4, 2, 8, 64, 0.1, 0, fake, 1 << 20, 1, s) == 2
+    assert lib.gqa_decode(fake, fake, fake, fake, null, null, null, 1, 4, 2, 8, 96, 0.1, 0, 0, fake, 1 << 20, 1, s) == 2
+    assert lib.gqa_decode(fake, fake, fake, fake, null, null, null, 5000, 4, 2, 8, 64, 0.1, 0, 0, fake, 1 << 20, 1, s) == 2
     # workspace: missing, too small, misaligned (num_splits given, so no device query is needed)
-    assert lib.gqa_decode(fake, fake, fake, fake, null, null, null, 1, 4, 2, 8, 64, 0.1, 0, null, 1 << 20, 1, s) == 5
-    assert lib.gqa_decode(fake, fake, fake, fake, null, null, null, 1, 4, 2, 8, 64, 0.1, 0, fake, 16, 1, s) == 5
-    assert lib.gqa_decode(fake, fake, fake, fake, null, null, null, 1, 4, 2, 8, 64, 0.1, 0, P(0x1004), 1 << 20, 1, s) == 5
+    assert lib.gqa_decode(fake, fake, fake, fake, null, null, null, 1, 4, 2, 8, 64, 0.1, 0, 0, null, 1 << 20, 1, s) == 5
+    assert lib.gqa_decode(fake, fake, fake, fake, null, null, null, 1, 4, 2, 8, 64, 0.1, 0, 0, fake, 16, 1, s) == 5
+    assert lib.gqa_decode(fake, fake, fake, fake, null, null, null, 1, 4, 2, 8, 64, 0.1, 0, 0, P(0x1004), 1 << 20, 1, s) == 5
     # kv_append
     assert lib.kv_append(fake, fake, fake, fake, null, 1, 2, 1, 8, 64, 0, s) == 1
     assert lib.kv_append(fake, fake, fake, fake, fake, 1, 2, 9, 8, 64, 0, s) == 1
@@ -102,12 +107,13 @@ def test_paged_host_side_argument_errors(lib):
     null = None
     s = None
     # args: q, k_pages, v_pages, o, lse, kv_len, q_pos, block_table,
-    #       B, h_q, h_kv, num_pages, page_size, max_pages, d_h, scale, dtype, ws, ws_bytes, splits, stream
-    ok = [fake, fake, fake, fake, null, null, null, fake, 1, 4, 2, 8, 16, 4, 64, 0.1, 0, fake, 1 << 20, 1, s]
+    #       B, h_q, h_kv, num_pages, page_size, max_pages, d_h, scale, window, dtype, ws, ws_bytes,
+    #       splits, stream
+    ok = [fake, fake, fake, fake, null, null, null, fake, 1, 4, 2, 8, 16, 4, 64, 0.1, 0, 0, fake, 1 << 20, 1, s]
 
     def dec(**kw):
         a = list(ok)
-        idx = {"bt": 7, "num_pages": 11, "page_size": 12, "max_pages": 13, "d_h": 14, "ws": 17}
+        idx = {"bt": 7, "num_pages": 11, "page_size": 12, "max_pages": 13, "d_h": 14, "window": 16, "ws": 18}
         for k, v in kw.items():
             a[idx[k]] = v
         return lib.gqa_decode_paged(*a)
@@ -121,6 +127,7 @@ def test_paged_host_side_argument_errors(lib):
     assert dec(page_size=1 << 16, max_pages=1 << 16) == 2  # T_max beyond 2^31
     assert dec(page_size=1 << 12, num_pages=1 << 18) == 2  # pool rows beyond 2^31
     assert dec(ws=null) == 5
+    assert dec(window=-1) == 1
     # kv_append_paged: k, v, k_new, v_new, pos, block_table, B, h_kv, S_new, num_pages, page_size,
     #                  max_pages, d_h, dtype, stream
     assert lib.kv_append_paged(fake, fake, fake, fake, fake, null, 1, 2, 1, 8, 16, 4, 64, 0, s) == 1

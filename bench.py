@@ -8,7 +8,8 @@ whole step, in GB/s. L2 is flushed (a 256 MiB write, then a 256 MiB read) betwee
 the timed events.
 
 A ``paged`` object repeats the decode_8k step over a paged cache (16-token pages in a shuffled
-pool: ``kv_append_paged`` + ``gqa_decode_paged``), timed the same way.
+pool: ``kv_append_paged`` + ``gqa_decode_paged``), timed the same way; a ``window`` object runs
+decode_8k and prefill_4k with a 1024-key sliding window (work counted inside the window only).
 
 ``--impl reference`` times the fp64 CPU oracle on a bounded sample of the same workload.
 Run with no flags for N=1; under torchrun every rank runs an independent replica (the path needs
@@ -57,11 +58,15 @@ def decode_kv_bytes(B, h_kv, lengths, d_h, s=2):
     return sum(2 * h_kv * int(n) * d_h * s for n in lengths)
 
 
-def prefill_flops(B, h_q, d_h, S_q, q_start, kv_len):
-    """Algorithmic causal prefill FLOPs: 4 * d_h per visible (query, key) pair per head."""
+def prefill_flops(B, h_q, d_h, S_q, q_start, kv_len, window=0):
+    """Algorithmic causal prefill FLOPs: 4 * d_h per visible (query, key) pair per head (with a
+    sliding window of W, row at position p sees keys max(0, p - W + 1) .. p)."""
     pairs = 0
     for i in range(S_q):
-        pairs += min(kv_len, q_start + i + 1)
+        p = q_start + i
+        hi = min(kv_len, p + 1)
+        lo = max(0, p - window + 1) if window else 0
+        pairs += max(0, hi - lo)
     return 4 * d_h * B * h_q * pairs
 
 
@@ -188,7 +193,7 @@ def job_throughput(unit_per_step, steps, world, total_ms):
 # our implementation
 # ---------------------------------------------------------------------------------------------
 
-def build_variants(args, rank, dev, page_size=0):
+def build_variants(args, rank, dev, page_size=0, window=0):
     """decode_8k inputs per h_kv: contiguous caches, or (page_size > 0) K/V pools of that page
     size with a shuffled block table, plus the new token's K/V appended at position T-1."""
     import torch
@@ -214,9 +219,10 @@ def build_variants(args, rank, dev, page_size=0):
         out = torch.empty_like(q)
         ws = torch.zeros(gqa.decode_workspace_size(shape.B, shape.h_q, h_kv, shape.T_max, shape.d_h),
                          dtype=torch.uint8, device=dev)
+        n_read = min(window, shape.T_max) if window else shape.T_max  # keys each query reads
         variants.append(dict(h_kv=h_kv, shape=shape, q=q, k=k, v=v, kv_len=kv_len, k_new=k_new,
-                             v_new=v_new, pos=pos, out=out, ws=ws, bt=bt,
-                             bytes=decode_kv_bytes(shape.B, h_kv, [shape.T_max] * shape.B, shape.d_h)))
+                             v_new=v_new, pos=pos, out=out, ws=ws, bt=bt, window=window,
+                             bytes=decode_kv_bytes(shape.B, h_kv, [n_read] * shape.B, shape.d_h)))
     return variants
 
 
@@ -234,10 +240,11 @@ def decode_step(variants):
             if record is not None:
                 record[i][0].record()
             if var["bt"] is None:
-                gqa.decode(var["q"], var["k"], var["v"], kv_len=var["kv_len"], out=var["out"], ws=var["ws"])
+                gqa.decode(var["q"], var["k"], var["v"], kv_len=var["kv_len"], out=var["out"], ws=var["ws"],
+                           window=var["window"])
             else:
                 gqa.decode_paged(var["q"], var["k"], var["v"], var["bt"], kv_len=var["kv_len"],
-                                 out=var["out"], ws=var["ws"])
+                                 out=var["out"], ws=var["ws"], window=var["window"])
             if record is not None:
                 record[i][1].record()
     return step
@@ -338,6 +345,27 @@ def run_paged(args, rank, dev, stream, local, hbm_peak, peak_kind):
             "clocks": t["clocks"]}
 
 
+def run_window(args, rank, dev, stream, local, hbm_peak, tf_peak, peak_kind):
+    """Sliding window of 1024 keys [第三章 §3.7]: decode_8k (each query reads its 1024 most recent
+    keys) and prefill_4k; the work counted is only what lies inside the windows."""
+    W = args.window
+    variants = build_variants(args, rank, dev, window=W)
+    t = time_decode(args, variants, L2Flush(dev), stream, local, None, dev)
+    step_bytes = sum(var["bytes"] for var in variants)
+    dec_total_ms = sum(sum(row) for row in t["dec_ms"]) / args.steps
+    achieved = step_bytes / (dec_total_ms / 1e3) / 1e9
+    per_variant = per_variant_rates(variants, t["dec_ms"], hbm_peak)
+    del variants
+    return {"window": W,
+            "decode": {"workload": f"decode_8k with a {W}-key sliding window: per step and variant one "
+                                   "kv_append + one gqa_decode reading the window's keys", "launch": t["mode"],
+                       "value": round(step_bytes * args.steps / (t["total_ms"] / 1e3) / 1e9, 1), "unit": "GB/s",
+                       "decode_GB_s": round(achieved, 1), "frac_of_hbm_peak": round(achieved / hbm_peak, 4),
+                       "peak_kind": f"hbm_gbs of {peak_kind}", "per_variant": per_variant,
+                       "gpu_launches": args.steps * 3 * len(args.h_kv)},
+            "prefill": run_prefill(args, dev, stream, tf_peak, peak_kind, window=W)}
+
+
 def run_ours(args, rank, world, dist):
     import torch
 
@@ -350,6 +378,8 @@ def run_ours(args, rank, world, dist):
         return {"prefill": run_prefill(args, dev, stream, tf_peak, peak_kind)}
     if args.paged_only:  # profiling aid: the paged decode_8k line alone
         return {"paged": run_paged(args, rank, dev, stream, local, hbm_peak, peak_kind)}
+    if args.window_only:  # profiling aid: the sliding-window lines alone
+        return {"window": run_window(args, rank, dev, stream, local, hbm_peak, tf_peak, peak_kind)}
 
     variants = build_variants(args, rank, dev)
     flush = L2Flush(dev)
@@ -381,6 +411,9 @@ def run_ours(args, rank, world, dist):
     if not args.skip_paged:
         paged = run_paged(args, rank, dev, stream, local, hbm_peak, peak_kind)
         paged["gpu_launches"] = args.steps * 3 * len(args.h_kv)
+    window = None
+    if not args.skip_window:
+        window = run_window(args, rank, dev, stream, local, hbm_peak, tf_peak, peak_kind)
 
     result = {
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
@@ -399,6 +432,8 @@ def run_ours(args, rank, world, dist):
         result["prefill"] = prefill
     if paged is not None:
         result["paged"] = paged
+    if window is not None:
+        result["window"] = window
     if rank == 0 and world == 1 and not args.skip_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(args)
     return result
@@ -447,8 +482,9 @@ def run_e2e(args, variants, dev, stream, dist, world):
             "ms_per_step": round(total / args.steps, 4)}
 
 
-def run_prefill(args, dev, stream, tf_peak, peak_kind):
-    """Secondary line: causal prefill prefill_4k (B=1, h_q=32, h_kv=8, T=4096, d_h=128), TFLOPS."""
+def run_prefill(args, dev, stream, tf_peak, peak_kind, window=0):
+    """Secondary line: causal prefill prefill_4k (B=1, h_q=32, h_kv=8, T=4096, d_h=128), TFLOPS
+    (optionally with a sliding window: only the pairs inside the window count as work)."""
     import torch
 
     import kv_cache_attention_gqa_b200 as gqa
@@ -458,25 +494,28 @@ def run_prefill(args, dev, stream, tf_peak, peak_kind):
     q, k, v = workloads.prefill_inputs(shape, seed=args.seed, device=dev)
     out = torch.empty_like(q)
     try:
-        gqa.prefill(q, k, v, out=out)
+        gqa.prefill(q, k, v, out=out, window=window)
     except gqa.GQAError as e:
         return {"unavailable": str(e)}
     flush = L2Flush(dev)
     for _ in range(max(3, args.warmup)):
-        gqa.prefill(q, k, v, out=out)
+        gqa.prefill(q, k, v, out=out, window=window)
     torch.cuda.synchronize()
     n = max(5, args.steps)
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
     for i in range(n):
         flush(i)
         evs[i][0].record(stream)
-        gqa.prefill(q, k, v, out=out)
+        gqa.prefill(q, k, v, out=out, window=window)
         evs[i][1].record(stream)
     torch.cuda.synchronize()
+    if gqa.get_device_error() != 0:
+        raise RuntimeError("device error in the prefill line")
     ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
-    flops = prefill_flops(1, 32, 128, 4096, 0, 4096)
+    flops = prefill_flops(1, 32, 128, 4096, 0, 4096, window)
     tflops = flops / (ms / 1e3) / 1e12
-    return {"workload": "prefill_4k: B=1, h_q=32, h_kv=8, S_q=T=4096, d_h=128, causal",
+    wtxt = f", sliding window {window}" if window else ""
+    return {"workload": f"prefill_4k: B=1, h_q=32, h_kv=8, S_q=T=4096, d_h=128, causal{wtxt}",
             "value": round(tflops, 1), "unit": "TFLOP/s", "ms": round(ms, 4),
             "roofline": {"bound": "tensor", "achieved": round(tflops, 1), "peak": tf_peak, "unit": "TFLOP/s",
                          "frac": round(tflops / tf_peak, 4), "peak_kind": f"bf16_tflops of {peak_kind}",
@@ -573,6 +612,9 @@ def main():
     ap.add_argument("--paged-only", action="store_true", help="only the paged decode_8k line (profiling aid)")
     ap.add_argument("--page-size", dest="page_size", type=int, default=16,
                     help="page size of the paged decode_8k line (a multiple of 16)")
+    ap.add_argument("--skip-window", action="store_true")
+    ap.add_argument("--window-only", action="store_true", help="only the sliding-window lines (profiling aid)")
+    ap.add_argument("--window", type=int, default=1024, help="sliding window of the window lines")
     ap.add_argument("--h-kv", dest="h_kv", type=int, nargs="+", default=[32, 8, 1],
                     help="decode_8k variants to run (default: all three); fewer only for profiling")
     args = ap.parse_args()

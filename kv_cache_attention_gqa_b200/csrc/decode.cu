@@ -489,6 +489,9 @@ __global__ void __launch_bounds__(Bf16Cfg<D, MT>::kThreads, 1)
     int issued = 0;
     bool ok = true;
     const int G = gridDim.x;
+    // chunks past the grid are handed out by the atomic ticket; with no more chunks than CTAs
+    // (the automatic choice) every CTA has its one chunk and takes no ticket
+    const bool dyn = plan.n_chunks > G;
     // Writes the stage's descriptor and arms its full barrier for `kv_bytes` of K/V (+ the query
     // rows on a piece's first tile). Lane 0 only.
     auto arm = [&](const Piece& pc, int t, int slot, int nh, uint32_t kv_bytes, int nskip) -> uint32_t {
@@ -527,7 +530,7 @@ __global__ void __launch_bounds__(Bf16Cfg<D, MT>::kThreads, 1)
         // Chunk tickets: CTA c starts with chunk c; later chunks come from an atomic counter whose
         // value is fetched one chunk ahead, so its latency overlaps the current chunk's loads.
         int chunk = blockIdx.x;
-        int next = chunk < plan.n_chunks ? G + atomicAdd(&a.hdr->ticket, 1) : plan.n_chunks;
+        int next = dyn && chunk < plan.n_chunks ? G + atomicAdd(&a.hdr->ticket, 1) : plan.n_chunks;
         for (; ok && chunk < plan.n_chunks;) {
           const long long x1 = min((long long)(chunk + 1) * plan.C, plan.K);
           for (long long x = (long long)chunk * plan.C; x < x1 && ok;) {
@@ -569,7 +572,7 @@ __global__ void __launch_bounds__(Bf16Cfg<D, MT>::kThreads, 1)
       }
       int chunk = blockIdx.x;
       int next = 0;
-      if (lane == 0) next = chunk < plan.n_chunks ? G + atomicAdd(&a.hdr->ticket, 1) : plan.n_chunks;
+      if (lane == 0) next = dyn && chunk < plan.n_chunks ? G + atomicAdd(&a.hdr->ticket, 1) : plan.n_chunks;
       next = __shfl_sync(0xffffffffu, next, 0);
       for (; ok && chunk < plan.n_chunks;) {
         const long long x1 = min((long long)(chunk + 1) * plan.C, plan.K);

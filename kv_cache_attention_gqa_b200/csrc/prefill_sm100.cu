@@ -210,7 +210,9 @@ __device__ __forceinline__ void fadd2(float& s0, float& s1, float a0, float a1) 
 // independent softmax warps. A thread owns one row (its TMEM lane, warp % 4 selects the lane
 // quarter) and half of the row's columns; the two halves of a row exchange their block maximum
 // through shared memory once per block, and their partial sums at the end.
-template <int D>
+// kWin: the launch has a sliding window (a.window > 0). Without one, the window code is compiled
+// out (its per-element compare in the mask loop costs ~9% of the causal kernel's time).
+template <int D, bool kWin>
 __device__ __forceinline__ void softmax_role(const PArgs& a, const Tile& tile, int warp, int lane,
                                              uint32_t tmem, uint32_t sQ, uint32_t sV, uint64_t* bars,
                                              float* xbuf, volatile int* abort) {
@@ -229,6 +231,10 @@ __device__ __forceinline__ void softmax_role(const PArgs& a, const Tile& tile, i
   const long long pos_max = (long long)tile.qs + min(tile.q0 + a.P, a.S_q) - 1;  // largest
   const int nb = tile.nb;
   const float c = a.scale_log2;
+  const int win = kWin ? a.window : 0;
+  // last key below this row's window, clamped to the int range (keys are ints)
+  const long long wl = pos - win;
+  const int win_last = kWin ? (int)(wl < -1 ? -1 : (wl > 0x7fffffffLL ? 0x7fffffffLL : wl)) : -1;
   const long long orow = ((long long)tile.b * a.h_q + tile.g * a.r + tile.hb * a.H + h) * a.S_q + qi;
   constexpr int kOHalf = D / 2;               // O columns (and Q columns) of this half
   float* xmax = xbuf;                         // [2 buffers][2 halves][128 rows]
@@ -269,7 +275,7 @@ __device__ __forceinline__ void softmax_role(const PArgs& a, const Tile& tile, i
     float lmx = 0.f;
     const int key0 = (tile.j0 + j) * kBN + half * 64;  // first key of this half
     const bool need_mask = (a.causal && (long long)key0 + 63 > pos_min) || key0 + 64 > tile.kv ||
-                           (a.window > 0 && (long long)key0 <= pos_max - a.window);
+                           (kWin && (long long)key0 <= pos_max - win);
     if (ok) {
       tc::fence_after_sync();
       uint32_t su[2][32];
@@ -283,7 +289,7 @@ __device__ __forceinline__ void softmax_role(const PArgs& a, const Tile& tile, i
         for (int i = 0; i < 64; ++i) {
           const int key = key0 + i;
           const bool vis = key < tile.kv && (!a.causal || key <= pos) &&
-                           (a.window == 0 || (long long)key > pos - a.window);
+                           (!kWin || key > win_last);
           sr[i] = vis ? sr[i] : -INFINITY;
         }
       }
@@ -314,7 +320,7 @@ __device__ __forceinline__ void softmax_role(const PArgs& a, const Tile& tile, i
     // P = 2^(s c - m_use) as bf16 pairs: this half's keys go to 32 of the first 64 S columns.
     // A row that has seen no visible key yet (only possible under a sliding window) keeps
     // m = -inf; its P is 0, computed against 0 instead of -inf.
-    const float m_sub = m_use == -INFINITY ? 0.f : m_use;
+    const float m_sub = kWin && m_use == -INFINITY ? 0.f : m_use;
     float sum0 = 0.f, sum1 = 0.f;
 #pragma unroll
     for (int cc = 0; cc < 2; ++cc) {
@@ -357,12 +363,12 @@ __device__ __forceinline__ void softmax_role(const PArgs& a, const Tile& tile, i
     // memory so 0 * V stays 0 (each half zeroes its own 64-column chunk). The block's V must have
     // landed first.
     const bool zero_tail = j == nb - 1 && bkey0 + kBN > tile.kv;
-    const bool zero_head = j == 0 && a.window > 0 && (long long)bkey0 < pos_min - a.window + 1;
+    const bool zero_head = kWin && j == 0 && (long long)bkey0 < pos_min - win + 1;
     if (ok && (zero_tail || zero_head) && (C::kNch == 2 || half == 0)) {
       const int vs = j % kVStages;
       if (wait_bar(bar(kBarVFull + vs), (uint32_t)((j / kVStages) & 1), abort, a.err)) {
         const long long key = (long long)bkey0 + row;
-        if ((zero_tail && key >= tile.kv) || (zero_head && key <= pos_min - a.window)) {
+        if ((zero_tail && key >= tile.kv) || (zero_head && key <= pos_min - win)) {
 #pragma unroll
           for (int k = 0; k < 8; ++k) {
             const uint32_t addr = sV + vs * C::kKVBytes + (C::kNch == 2 ? half : 0) * C::kKVChunk + row * 128 + k * 16;
@@ -398,7 +404,7 @@ __device__ __forceinline__ void softmax_role(const PArgs& a, const Tile& tile, i
   tc::fence_after_sync();
   // A row with no visible key (a sliding window that starts at or past kv_len, or a padding row
   // of the tile) has l = 0: it still takes part in the warp's TMEM loads, and writes zeros.
-  const bool empty = l == 0.f;
+  const bool empty = kWin && l == 0.f;
   if (empty && store_row && half == 0) set_device_error(a.err, GQA_DEVERR_NO_VISIBLE);
   const float inv = empty ? 0.f : 1.f / l;
   uint4* out = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.o) + orow * D + half * kOHalf);
@@ -420,7 +426,7 @@ __device__ __forceinline__ void softmax_role(const PArgs& a, const Tile& tile, i
   if (store_row && a.lse && half == 0) a.lse[orow] = empty ? -INFINITY : (m + __log2f(l)) * kLn2;
 }
 
-template <int D>
+template <int D, bool kWin>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_bf16_kernel(const __grid_constant__ CUtensorMap tmq,
                         const __grid_constant__ CUtensorMap tmk,
@@ -564,7 +570,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     volatile int no_abort = 0;
     wait_bar(bar(kBarDone), 0, &no_abort, a.err);
   } else if (warp >= 4) {
-    softmax_role<D>(a, tile, warp, lane, tmem, sQ, sV, bars, xbuf, abort);
+    softmax_role<D, kWin>(a, tile, warp, lane, tmem, sQ, sV, bars, xbuf, abort);
   }
 
   tc::fence_before_sync();
@@ -573,6 +579,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc::fence_after_sync();
     tc::tmem_dealloc(tmem, kTmemCols);
   }
+}
+
+template <int D, bool kWin>
+cudaError_t launch_typed(const PArgs& p, const CUtensorMap* tmaps, long long tiles, cudaStream_t s) {
+  auto kern = prefill_bf16_kernel<D, kWin>;
+  static bool attr_set[64] = {false};  // per device: the shared-memory opt-in is set once
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<D>::kSmem);
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < 64) attr_set[dev] = true;
+  }
+  kern<<<(unsigned)tiles, kThreads, Cfg<D>::kSmem, s>>>(tmaps[0], tmaps[1], tmaps[2], p);
+  return cudaGetLastError();
 }
 
 }  // namespace pf
@@ -602,33 +624,15 @@ cudaError_t launch_prefill_bf16(const PrefillArgs& a, const CUtensorMap* tmaps, 
   const long long tiles = (long long)p.n_qt * a.B * a.h_kv * p.hblocks;
   if (tiles <= 0) return cudaSuccess;
   if (tiles > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-  cudaError_t e;
-  int dev = 0;
-  e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  static bool set128[64] = {false}, set64[64] = {false};
   if (a.d_h == 128) {
-    if (dev < 0 || dev >= 64 || !set128[dev]) {
-      e = cudaFuncSetAttribute(pf::prefill_bf16_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               pf::Cfg<128>::kSmem);
-      if (e != cudaSuccess) return e;
-      if (dev >= 0 && dev < 64) set128[dev] = true;
-    }
-    pf::prefill_bf16_kernel<128><<<(unsigned)tiles, pf::kThreads, pf::Cfg<128>::kSmem, s>>>(
-        tmaps[0], tmaps[1], tmaps[2], p);
-  } else if (a.d_h == 64) {
-    if (dev < 0 || dev >= 64 || !set64[dev]) {
-      e = cudaFuncSetAttribute(pf::prefill_bf16_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               pf::Cfg<64>::kSmem);
-      if (e != cudaSuccess) return e;
-      if (dev >= 0 && dev < 64) set64[dev] = true;
-    }
-    pf::prefill_bf16_kernel<64><<<(unsigned)tiles, pf::kThreads, pf::Cfg<64>::kSmem, s>>>(
-        tmaps[0], tmaps[1], tmaps[2], p);
-  } else {
-    return cudaErrorInvalidValue;
+    return a.window > 0 ? pf::launch_typed<128, true>(p, tmaps, tiles, s)
+                        : pf::launch_typed<128, false>(p, tmaps, tiles, s);
   }
-  return cudaGetLastError();
+  if (a.d_h == 64) {
+    return a.window > 0 ? pf::launch_typed<64, true>(p, tmaps, tiles, s)
+                        : pf::launch_typed<64, false>(p, tmaps, tiles, s);
+  }
+  return cudaErrorInvalidValue;
 }
 
 int prefill_heads_per_tile(int h_q, int h_kv) {

@@ -29,6 +29,7 @@ from .attention_ref import (
 from .online_softmax import online_softmax_row, merge_states, blockwise_attention_row
 from .kv_append_ref import kv_append_ref
 from .paged import gather_pages, paged_append_ref, paged_decode_ref
+from .backward import attention_backward_ref, softmax_backward_rowterm
 from . import ledgers
 
 __all__ = [
@@ -44,5 +45,7 @@ __all__ = [
     "gather_pages",
     "paged_decode_ref",
     "paged_append_ref",
+    "attention_backward_ref",
+    "softmax_backward_rowterm",
     "ledgers",
 ]

@@ -103,6 +103,38 @@ gqa_status gqa_prefill(const void* q, const void* k_cache, const void* v_cache, 
                        float scale, int causal, int window, gqa_dtype dtype, void* stream);
 
 /*
+ * gqa_prefill_backward - gradients of gqa_prefill for an upstream gradient dO (training).
+ * The pages describe the backward pass as recomputing the local scores from statistics saved in
+ * the forward pass, so the probability matrix is never stored [序列计算与存储, the paragraph
+ * after the 两块算例 listing; 第三章, section 3.5]. With P = exp(S - lse) recomputed per block:
+ *   dV_g = sum over the heads a of group g of P_a^T dO_a,
+ *   dS_a = P_a * (dO_a V_g^T - D_a),  D_a = rowsum(dO_a * O_a),
+ *   dQ_a = scale * dS_a K_g,  dK_g = scale * sum_a dS_a^T Q_a.
+ *
+ *   q, o, d_o   (B, h_q, S_q, d_h): the forward's queries and output, and dL/dO.
+ *   k_cache, v_cache (B, h_kv, T_max, d_h): the forward's keys and values.
+ *   lse         (B, h_q, S_q) fp32: the natural-log lse gqa_prefill returned (required). A row
+ *               with lse = -inf (no visible key) gets dQ = 0 and contributes nothing.
+ *   dq          (B, h_q, S_q, d_h) written.
+ *   dk, dv      (B, h_kv, T_max, d_h) written in full; rows j >= kv_len[b] are zero.
+ *   q_start, kv_len, scale, causal, window: exactly as passed to gqa_prefill.
+ *   dtype       GQA_BF16 (d_h 64 or 128; tcgen05 kernels, bf16 gradients) or GQA_FP32 (d_h <= 256;
+ *               scalar check mode, fp32 gradients). All tensors share the dtype; lse is fp32.
+ *   workspace   device memory of at least gqa_prefill_backward_workspace_size(B, h_q, S_q) bytes,
+ *               256-byte aligned, no initial contents required (two fp32 values per query row).
+ * Three kernels run in order on `stream`: the row term D, the key-stationary dK/dV pass (the heads
+ * of a group add up in one CTA, no atomics), and the query-stationary dQ pass.
+ * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA.
+ */
+size_t gqa_prefill_backward_workspace_size(int B, int h_q, int S_q);
+gqa_status gqa_prefill_backward(const void* q, const void* k_cache, const void* v_cache,
+                                const void* o, const void* d_o, const float* lse, void* dq,
+                                void* dk, void* dv, const int32_t* q_start, const int32_t* kv_len,
+                                int B, int h_q, int h_kv, int S_q, int T_max, int d_h, float scale,
+                                int causal, int window, gqa_dtype dtype, void* workspace,
+                                size_t workspace_bytes, void* stream);
+
+/*
  * gqa_decode_workspace_size - bytes of device workspace gqa_decode needs for this shape with
  * `num_splits` (0 = the automatic choice gqa_decode makes on the current device).
  * The workspace holds a small header (a work ticket), the per-sequence visible lengths and their

@@ -43,6 +43,9 @@ SIGNATURES = {
     "gqa_decode_paged": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I,
                               _I, _P, _Z, _I, _P]),
     "kv_append_paged": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P]),
+    "gqa_prefill_backward_workspace_size": (_Z, [_I, _I, _I]),
+    "gqa_prefill_backward": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I,
+                                  _F, _I, _I, _I, _P, _Z, _P]),
     "gqa_get_device_error": (_I, [ctypes.POINTER(_I), _P]),
     "gqa_status_string": (ctypes.c_char_p, [_I]),
     "gqa_version": (ctypes.c_char_p, []),
@@ -332,3 +335,36 @@ def kv_append_paged(k_pages: torch.Tensor, v_pages: torch.Tensor, k_new: torch.T
     _check("kv_append_paged", _lib.kv_append_paged(
         _ptr(k_pages), _ptr(v_pages), _ptr(k_new), _ptr(v_new), _ptr(pos_t), _ptr(bt), B, h_kv,
         k_new.shape[2], num_pages, page_size, bt.shape[1], d_h, dt, _stream()))
+
+
+def prefill_backward(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, o: torch.Tensor,
+                     d_o: torch.Tensor, lse: torch.Tensor, *, q_start=None, kv_len=None,
+                     scale: float | None = None, causal: bool = True, window: int = 0,
+                     ws: torch.Tensor | None = None):
+    """Gradients (dq, dk, dv) of ``prefill`` for the upstream gradient ``d_o``; ``o`` and ``lse``
+    are the forward's outputs (``prefill(..., return_lse=True)``). dk, dv have the cache's shape,
+    zero past each kv_len."""
+    _need_cuda(q, k_cache, v_cache, o, d_o, lse)
+    B, h_q, S_q, d_h = q.shape
+    Bk, h_kv, T_max, dk_ = k_cache.shape
+    if (Bk, dk_) != (B, d_h) or v_cache.shape != k_cache.shape or o.shape != q.shape or d_o.shape != q.shape:
+        raise ValueError("q / k_cache / v_cache / o / d_o shapes disagree")
+    if lse.shape != (B, h_q, S_q) or lse.dtype != torch.float32:
+        raise ValueError("lse must be fp32 (B, h_q, S_q)")
+    dt = _dtype_code(q)
+    if any(t.dtype != q.dtype for t in (k_cache, v_cache, o, d_o)):
+        raise TypeError("q, k_cache, v_cache, o and d_o must share one dtype")
+    dq = torch.empty_like(q)
+    dk = torch.empty_like(k_cache)
+    dv = torch.empty_like(v_cache)
+    qs = _int_vec(q_start, B, q.device, "q_start")
+    kl = _int_vec(kv_len, B, q.device, "kv_len")
+    scale = 1.0 / math.sqrt(d_h) if scale is None else float(scale)
+    need = _lib.gqa_prefill_backward_workspace_size(B, h_q, S_q)
+    if ws is None or ws.numel() < need:
+        ws = torch.empty(need, dtype=torch.uint8, device=q.device)
+    _check("gqa_prefill_backward", _lib.gqa_prefill_backward(
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(o), _ptr(d_o), _ptr(lse), _ptr(dq), _ptr(dk),
+        _ptr(dv), _ptr(qs), _ptr(kl), B, h_q, h_kv, S_q, T_max, d_h, scale, 1 if causal else 0,
+        int(window), dt, _ptr(ws), ws.numel(), _stream()))
+    return dq, dk, dv

@@ -281,6 +281,80 @@ gqa_status gqa_prefill(const void* q, const void* k_cache, const void* v_cache, 
   return from_cuda(launch_prefill_bf16(a, maps, sm_count(), s));
 }
 
+size_t gqa_prefill_backward_workspace_size(int B, int h_q, int S_q) {
+  if (B <= 0 || h_q <= 0 || S_q <= 0) return 0;
+  const size_t rows = (size_t)B * h_q * S_q;
+  return 2 * ((rows * 4 + 255) / 256 * 256);
+}
+
+gqa_status gqa_prefill_backward(const void* q, const void* k_cache, const void* v_cache,
+                                const void* o, const void* d_o, const float* lse, void* dq,
+                                void* dk, void* dv, const int32_t* q_start, const int32_t* kv_len,
+                                int B, int h_q, int h_kv, int S_q, int T_max, int d_h, float scale,
+                                int causal, int window, gqa_dtype dtype, void* workspace,
+                                size_t workspace_bytes, void* stream) {
+  if (!q || !k_cache || !v_cache || !o || !d_o || !lse || !dq || !dk || !dv) return GQA_ERR_INVALID_ARG;
+  if (B <= 0 || h_q <= 0 || h_kv <= 0 || S_q <= 0 || T_max <= 0 || d_h <= 0) return GQA_ERR_INVALID_ARG;
+  if (h_q % h_kv != 0 || !valid_scale(scale)) return GQA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return GQA_ERR_INVALID_ARG;
+  if (window < 0 || (window > 0 && causal != 1)) return GQA_ERR_INVALID_ARG;
+  if (dtype != GQA_BF16 && dtype != GQA_FP32) return GQA_ERR_INVALID_ARG;
+  if (dtype == GQA_FP32 && d_h > 256) return GQA_ERR_UNSUPPORTED;
+  if (dtype == GQA_BF16 && d_h != 64 && d_h != 128) return GQA_ERR_UNSUPPORTED;
+  if ((long long)B * h_kv * T_max >= (1ll << 31) || (long long)B * h_q * S_q >= (1ll << 31))
+    return GQA_ERR_UNSUPPORTED;
+  const size_t need = gqa_prefill_backward_workspace_size(B, h_q, S_q);
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < need)
+    return GQA_ERR_WORKSPACE;
+  BackwardArgs a;
+  a.q = q;
+  a.k = k_cache;
+  a.v = v_cache;
+  a.o = o;
+  a.d_o = d_o;
+  a.lse = lse;
+  a.dq = dq;
+  a.dk = dk;
+  a.dv = dv;
+  a.q_start = q_start;
+  a.kv_len = kv_len;
+  a.B = B;
+  a.h_q = h_q;
+  a.h_kv = h_kv;
+  a.S_q = S_q;
+  a.T_max = T_max;
+  a.d_h = d_h;
+  a.scale = scale;
+  a.causal = causal;
+  a.window = window;
+  a.lse2 = reinterpret_cast<float*>(workspace);
+  a.drow = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(workspace) + need / 2);
+  a.err = device_error_ptr();
+  if (!a.err) return GQA_ERR_CUDA;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (dtype == GQA_FP32) return from_cuda(launch_backward_fp32(a, s));
+  // TMA views: Q and dO as (d_h, S_q, B*h_q) with box (64, 128, 1) for the key-stationary dK/dV
+  // kernel and (64, P, H) for the query-stationary dQ kernel; K, V as rows with box (64, 128).
+  const int H = prefill_heads_per_tile(h_q, h_kv);
+  const uint32_t P = (uint32_t)(128 / H);
+  CUtensorMap maps[6];
+  const uint64_t qdims[3] = {(uint64_t)d_h, (uint64_t)S_q, (uint64_t)B * h_q};
+  const uint64_t qstrides[2] = {(uint64_t)d_h * 2, (uint64_t)S_q * d_h * 2};
+  const uint32_t qbox_rows[3] = {64, 128, 1};
+  const uint32_t qbox_tile[3] = {64, P, (uint32_t)H};
+  const uint64_t kdims[2] = {(uint64_t)d_h, (uint64_t)B * h_kv * T_max};
+  const uint64_t strides[1] = {(uint64_t)d_h * 2};
+  const uint32_t box[2] = {64, 128};
+  if (!encode_bf16(&maps[0], q, 3, qdims, qstrides, qbox_rows) ||
+      !encode_bf16(&maps[1], d_o, 3, qdims, qstrides, qbox_rows) ||
+      !encode_bf16(&maps[2], k_cache, 2, kdims, strides, box) ||
+      !encode_bf16(&maps[3], v_cache, 2, kdims, strides, box) ||
+      !encode_bf16(&maps[4], q, 3, qdims, qstrides, qbox_tile) ||
+      !encode_bf16(&maps[5], d_o, 3, qdims, qstrides, qbox_tile))
+    return GQA_ERR_CUDA;
+  return from_cuda(launch_backward_bf16(a, maps, s));
+}
+
 size_t gqa_decode_workspace_size(int B, int h_q, int h_kv, int T_max, int d_h, gqa_dtype dtype,
                                  int num_splits) {
   if (B <= 0 || h_q <= 0 || h_kv <= 0 || T_max <= 0 || d_h <= 0 || h_q % h_kv != 0) return 0;

@@ -48,6 +48,31 @@ cudaError_t launch_prefill_bf16(const PrefillArgs& a, const CUtensorMap* tmaps, 
 // query heads per prefill tile (H); a tile holds H heads x floor(128 / H) positions
 int prefill_heads_per_tile(int h_q, int h_kv);
 
+struct BackwardArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  const void* o;
+  const void* d_o;
+  const float* lse;  // natural-log lse from the forward pass (B, h_q, S_q)
+  void* dq;
+  void* dk;
+  void* dv;
+  const int32_t* q_start;
+  const int32_t* kv_len;
+  int B, h_q, h_kv, S_q, T_max, d_h;
+  float scale;
+  int causal, window;
+  float* lse2;  // workspace: (B*h_q*S_q) base-2 lse
+  float* drow;  // workspace: (B*h_q*S_q) rowsum(dO * O)
+  unsigned* err;
+};
+// bf16 tcgen05 path. tmaps: [0] Q, [1] dO as 3-D views (d_h, S_q, B*h_q) with box (64, 128, 1);
+// [2] K, [3] V as 2-D views (d_h, B*h_kv*T_max) with box (64, 128); [4] Q, [5] dO as 3-D views
+// with the forward's box (64, 128 / H, H).
+cudaError_t launch_backward_bf16(const BackwardArgs& a, const CUtensorMap* tmaps, cudaStream_t s);
+cudaError_t launch_backward_fp32(const BackwardArgs& a, cudaStream_t s);
+
 struct DecodeArgs {
   const void* q;
   const void* k;

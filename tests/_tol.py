@@ -31,3 +31,27 @@ def assert_fp32_close(out, ref, what=""):
     scale = max(float(np.abs(ref).max()), 1e-30)
     mx = float(np.abs(out - ref).max())
     assert mx <= FP32_REL * scale, f"{what}: max {mx:.3e} > {FP32_REL} * {scale:.3e}"
+
+
+# Gradients (backward pass) are not O(1) like attention outputs, so their bounds scale with the
+# tensor's largest reference entry. bf16: P and dS are rounded to bf16 before the tensor-core sums
+# over up to S_q (or r * S_q) terms; fp32 check mode: scalar sums over as many terms.
+GRAD_BF16_MAX = 2e-2
+GRAD_BF16_MEAN = 2e-3
+GRAD_FP32_REL = 1e-4
+
+
+GRAD_SCALE_FLOOR = 1e-3  # where the exact gradient vanishes (e.g. a window of one key: P = 1, dS = 0)
+
+
+def assert_grad_close(out, ref, what="", fp32=False):
+    out = np.asarray(out, np.float64)
+    ref = np.asarray(ref, np.float64)
+    assert np.isfinite(out).all(), f"{what}: non-finite gradient"
+    scale = max(float(np.abs(ref).max()), GRAD_SCALE_FLOOR)
+    d = np.abs(out - ref)
+    if fp32:
+        assert d.max() <= GRAD_FP32_REL * scale, f"{what}: max {d.max():.3e} > {GRAD_FP32_REL} * {scale:.3e}"
+    else:
+        assert d.max() <= GRAD_BF16_MAX * scale and d.mean() <= GRAD_BF16_MEAN * scale, \
+            f"{what}: max {d.max():.3e} mean {d.mean():.3e} (scale {scale:.3e})"

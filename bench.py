@@ -9,7 +9,8 @@ the timed events.
 
 A ``paged`` object repeats the decode_8k step over a paged cache (16-token pages in a shuffled
 pool: ``kv_append_paged`` + ``gqa_decode_paged``), timed the same way; a ``window`` object runs
-decode_8k and prefill_4k with a 1024-key sliding window (work counted inside the window only).
+decode_8k and prefill_4k with a 1024-key sliding window (work counted inside the window only); a
+``backward`` object times gqa_prefill_backward on prefill_4k.
 
 ``--impl reference`` times the fp64 CPU oracle on a bounded sample of the same workload.
 Run with no flags for N=1; under torchrun every rank runs an independent replica (the path needs
@@ -345,6 +346,47 @@ def run_paged(args, rank, dev, stream, local, hbm_peak, peak_kind):
             "clocks": t["clocks"]}
 
 
+def run_backward(args, dev, stream, tf_peak, peak_kind):
+    """Backward pass of prefill_4k (B=1, h_q=32, h_kv=8, S=T=4096, d_h=128, causal): dQ, dK, dV from
+    the forward's O and lse. Algorithmic work: five GEMMs per visible (query, key) pair (S, dP, dV,
+    dK, dQ), 10 * d_h FLOPs, i.e. 2.5 times the forward's."""
+    import torch
+
+    import kv_cache_attention_gqa_b200 as gqa
+    import workloads
+
+    shape = workloads.PREFILL_4K
+    q, k, v = workloads.prefill_inputs(shape, seed=args.seed, device=dev)
+    g = torch.Generator(device=dev)
+    g.manual_seed(20_000 + args.seed)
+    d_o = torch.randn(q.shape, generator=g, device=dev).to(torch.bfloat16)
+    o, lse = gqa.prefill(q, k, v, return_lse=True)
+    ws = torch.empty(2 * 32 * 4096 * 4 + 1024, dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
+    for _ in range(max(3, args.warmup)):
+        gqa.prefill_backward(q, k, v, o, d_o, lse, ws=ws)
+    torch.cuda.synchronize()
+    n = max(5, args.steps)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    for i in range(n):
+        flush(i)
+        evs[i][0].record(stream)
+        gqa.prefill_backward(q, k, v, o, d_o, lse, ws=ws)
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    if gqa.get_device_error() != 0:
+        raise RuntimeError("device error in the backward line")
+    ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
+    flops = prefill_flops(1, 32, 128, 4096, 0, 4096) * 5 // 2
+    tflops = flops / (ms / 1e3) / 1e12
+    return {"workload": "prefill_4k backward: dQ, dK, dV (B=1, h_q=32, h_kv=8, S_q=T=4096, d_h=128, causal)",
+            "value": round(tflops, 1), "unit": "TFLOP/s", "ms": round(ms, 4),
+            "launches": "rowterm + dkdv + dq (three kernels), eager, L2 flushed between runs",
+            "roofline": {"bound": "tensor", "achieved": round(tflops, 1), "peak": tf_peak, "unit": "TFLOP/s",
+                         "frac": round(tflops / tf_peak, 4), "peak_kind": f"bf16_tflops of {peak_kind}",
+                         "algorithmic_flops_per_launch": flops}}
+
+
 def run_window(args, rank, dev, stream, local, hbm_peak, tf_peak, peak_kind):
     """Sliding window of 1024 keys [第三章 §3.7]: decode_8k (each query reads its 1024 most recent
     keys) and prefill_4k; the work counted is only what lies inside the windows."""
@@ -378,6 +420,8 @@ def run_ours(args, rank, world, dist):
         return {"prefill": run_prefill(args, dev, stream, tf_peak, peak_kind)}
     if args.paged_only:  # profiling aid: the paged decode_8k line alone
         return {"paged": run_paged(args, rank, dev, stream, local, hbm_peak, peak_kind)}
+    if args.backward_only:  # profiling aid: the backward line alone
+        return {"backward": run_backward(args, dev, stream, tf_peak, peak_kind)}
     if args.window_only:  # profiling aid: the sliding-window lines alone
         return {"window": run_window(args, rank, dev, stream, local, hbm_peak, tf_peak, peak_kind)}
 
@@ -411,6 +455,7 @@ def run_ours(args, rank, world, dist):
     if not args.skip_paged:
         paged = run_paged(args, rank, dev, stream, local, hbm_peak, peak_kind)
         paged["gpu_launches"] = args.steps * 3 * len(args.h_kv)
+    backward = run_backward(args, dev, stream, tf_peak, peak_kind) if not args.skip_backward else None
     window = None
     if not args.skip_window:
         window = run_window(args, rank, dev, stream, local, hbm_peak, tf_peak, peak_kind)
@@ -434,6 +479,8 @@ def run_ours(args, rank, world, dist):
         result["paged"] = paged
     if window is not None:
         result["window"] = window
+    if backward is not None:
+        result["backward"] = backward
     if rank == 0 and world == 1 and not args.skip_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(args)
     return result
@@ -613,6 +660,8 @@ def main():
     ap.add_argument("--page-size", dest="page_size", type=int, default=16,
                     help="page size of the paged decode_8k line (a multiple of 16)")
     ap.add_argument("--skip-window", action="store_true")
+    ap.add_argument("--skip-backward", action="store_true")
+    ap.add_argument("--backward-only", action="store_true", help="only the backward line (profiling aid)")
     ap.add_argument("--window-only", action="store_true", help="only the sliding-window lines (profiling aid)")
     ap.add_argument("--window", type=int, default=1024, help="sliding window of the window lines")
     ap.add_argument("--h-kv", dest="h_kv", type=int, nargs="+", default=[32, 8, 1],

@@ -30,6 +30,7 @@ from .online_softmax import online_softmax_row, merge_states, blockwise_attentio
 from .kv_append_ref import kv_append_ref
 from .paged import gather_pages, paged_append_ref, paged_decode_ref
 from .backward import attention_backward_ref, softmax_backward_rowterm
+from .mla import mla_decode_ref, mla_explicit_ref
 from . import ledgers
 
 __all__ = [
@@ -47,5 +48,7 @@ __all__ = [
     "paged_append_ref",
     "attention_backward_ref",
     "softmax_backward_rowterm",
+    "mla_decode_ref",
+    "mla_explicit_ref",
     "ledgers",
 ]

@@ -103,6 +103,36 @@ gqa_status gqa_prefill(const void* q, const void* k_cache, const void* v_cache, 
                        float scale, int causal, int window, gqa_dtype dtype, void* stream);
 
 /*
+ * gqa_mla_decode - multi-head latent attention decode over a latent cache (absorbed form).
+ * MLA caches one low-dimensional latent per token, C = X W_D, and K = C W_UK, V = C W_UV; for one
+ * head Q (C U_K)^T = (Q U_K^T) C^T and P (C U_V) = (P C) U_V exactly, so a decode step scores
+ * the latent cache directly with the absorbed query and up-projects the latent output afterwards
+ * [第 09 章, section 09.3]. The full MLA keeps a decoupled position key beside the latent
+ * [第三章, section 3.4]; it is the tail of each cache row here. This call computes the attention
+ * core: for every head h of sequence b and visible token j,
+ *   s_hj = scale * q[b, h, :] . cache[b, j, :],   o[b, h, :] = sum_j softmax_j(s_hj) cache[b, j, :d_v]
+ * The projections (q_nope U_K^T, o U_V) are ordinary matrix products left to the caller.
+ *
+ *   q      (B, h_q, d_qk): [absorbed latent query (d_v) | rotary query part], already rotated.
+ *   cache  (B, T_max, d_qk): [latent (d_v) | rotary key part], shared by all heads.
+ *   o      (B, h_q, d_v) written (latent output). lse: (B, h_q) fp32 or NULL (natural log).
+ *   kv_len, q_pos: as gqa_decode. scale: the model's softmax scale (for absorbed MLA this is
+ *          1/sqrt(d_nope + d_rope) of the original heads, not 1/sqrt(d_qk)).
+ *   dtype  GQA_BF16: d_qk = 576 and d_v = 512 (the DeepSeek-V2/V3 latent and rotary widths);
+ *          GQA_FP32: d_qk <= 768, d_v <= min(d_qk, 512) (check mode).
+ *   workspace: >= gqa_mla_decode_workspace_size(B, h_q, T_max, d_v, dtype, num_splits) bytes,
+ *          256-byte aligned, zero-filled before first use, as for gqa_decode (same reuse rules).
+ *   num_splits: as gqa_decode. A unit is 16 heads of one sequence.
+ * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA.
+ */
+size_t gqa_mla_decode_workspace_size(int B, int h_q, int T_max, int d_v, gqa_dtype dtype,
+                                     int num_splits);
+gqa_status gqa_mla_decode(const void* q, const void* cache, void* o, float* lse,
+                          const int32_t* kv_len, const int32_t* q_pos, int B, int h_q, int T_max,
+                          int d_qk, int d_v, float scale, gqa_dtype dtype, void* workspace,
+                          size_t workspace_bytes, int num_splits, void* stream);
+
+/*
  * gqa_prefill_backward - gradients of gqa_prefill for an upstream gradient dO (training).
  * The pages describe the backward pass as recomputing the local scores from statistics saved in
  * the forward pass, so the probability matrix is never stored [序列计算与存储, the paragraph

@@ -1,6 +1,6 @@
 """Causal grouped-query attention on B200 (sm_100a): prefill, split-KV decode and KV append,
-over a contiguous or a paged KV cache, with an optional sliding window, and the prefill's backward
-pass.
+over a contiguous or a paged KV cache, with an optional sliding window, the prefill's backward
+pass, and MLA decode over a latent cache.
 
 The computation lives in the CUDA library ``libgqa_b200.so`` behind the C ABI of
 ``include/gqa.h``; this package is a thin ctypes binding over it (``_lib``) plus the build script
@@ -17,6 +17,7 @@ from ._lib import (  # noqa: F401
     get_device_error,
     kv_append,
     kv_append_paged,
+    mla_decode,
     prefill,
     prefill_backward,
     status_string,

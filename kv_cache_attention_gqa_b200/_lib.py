@@ -44,6 +44,8 @@ SIGNATURES = {
                               _I, _P, _Z, _I, _P]),
     "kv_append_paged": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P]),
     "gqa_prefill_backward_workspace_size": (_Z, [_I, _I, _I]),
+    "gqa_mla_decode_workspace_size": (_Z, [_I, _I, _I, _I, _I, _I]),
+    "gqa_mla_decode": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _P, _Z, _I, _P]),
     "gqa_prefill_backward": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I,
                                   _F, _I, _I, _I, _P, _Z, _P]),
     "gqa_get_device_error": (_I, [ctypes.POINTER(_I), _P]),
@@ -368,3 +370,38 @@ def prefill_backward(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tens
         _ptr(dv), _ptr(qs), _ptr(kl), B, h_q, h_kv, S_q, T_max, d_h, scale, 1 if causal else 0,
         int(window), dt, _ptr(ws), ws.numel(), _stream()))
     return dq, dk, dv
+
+
+def mla_decode(q: torch.Tensor, cache: torch.Tensor, d_v: int = 512, *, kv_len=None, q_pos=None,
+               scale: float | None = None, num_splits: int = 0, out=None, return_lse: bool = False,
+               ws: torch.Tensor | None = None):
+    """MLA decode over a latent cache: q (B, h_q, d_qk) = [absorbed latent query | rotary part],
+    cache (B, T_max, d_qk) = [latent | rotary key]; returns the latent output (B, h_q, d_v) (the
+    value rows are cache[..., :d_v]). ``scale`` should be the model's softmax scale."""
+    _need_cuda(q, cache, out)
+    B, h_q, d_qk = q.shape
+    Bc, T_max, dc = cache.shape
+    if (Bc, dc) != (B, d_qk):
+        raise ValueError("q and cache shapes disagree")
+    dt = _dtype_code(q)
+    if cache.dtype != q.dtype:
+        raise TypeError("q and cache must share one dtype")
+    if out is None:
+        out = torch.empty((B, h_q, d_v), dtype=q.dtype, device=q.device)
+    lse = torch.empty((B, h_q), dtype=torch.float32, device=q.device) if return_lse else None
+    kl = _int_vec(kv_len, B, q.device, "kv_len")
+    qp = _int_vec(q_pos, B, q.device, "q_pos")
+    scale = 1.0 / math.sqrt(d_qk) if scale is None else float(scale)
+    key = ("mla", B, h_q, T_max, d_v, dt, num_splits, q.device.index)
+    need = _ws_sizes.get(key)
+    if need is None:
+        need = _lib.gqa_mla_decode_workspace_size(B, h_q, T_max, d_v, dt, num_splits)
+        if need == 0:
+            raise GQAError("gqa_mla_decode_workspace_size", 1)
+        _ws_sizes[key] = need
+    if ws is None:
+        ws = workspace(need, q.device)
+    _check("gqa_mla_decode", _lib.gqa_mla_decode(
+        _ptr(q), _ptr(cache), _ptr(out), _ptr(lse), _ptr(kl), _ptr(qp), B, h_q, T_max, d_qk, d_v,
+        scale, dt, _ptr(ws), ws.numel(), num_splits, _stream()))
+    return (out, lse) if return_lse else out

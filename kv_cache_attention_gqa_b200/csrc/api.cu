@@ -373,6 +373,72 @@ gqa_status gqa_decode(const void* q, const void* k_cache, const void* v_cache, v
                      window, dtype, workspace, workspace_bytes, num_splits, stream, nullptr, 0, 0, 0);
 }
 
+size_t gqa_mla_decode_workspace_size(int B, int h_q, int T_max, int d_v, gqa_dtype dtype,
+                                     int num_splits) {
+  if (B <= 0 || h_q <= 0 || T_max <= 0 || d_v <= 0 || num_splits < 0) return 0;
+  if (dtype != GQA_BF16 && dtype != GQA_FP32) return 0;
+  const int sms = num_splits > 0 ? 1 : sm_count();
+  if (sms <= 0) return 0;
+  return decode_workspace_bytes(B, h_q, 1, T_max, d_v, num_splits, sms, true);
+}
+
+gqa_status gqa_mla_decode(const void* q, const void* cache, void* o, float* lse,
+                          const int32_t* kv_len, const int32_t* q_pos, int B, int h_q, int T_max,
+                          int d_qk, int d_v, float scale, gqa_dtype dtype, void* workspace,
+                          size_t workspace_bytes, int num_splits, void* stream) {
+  if (!q || !cache || !o) return GQA_ERR_INVALID_ARG;
+  if (B <= 0 || h_q <= 0 || T_max <= 0 || d_qk <= 0 || d_v <= 0 || d_v > d_qk || num_splits < 0)
+    return GQA_ERR_INVALID_ARG;
+  if (!valid_scale(scale)) return GQA_ERR_INVALID_ARG;
+  if (dtype != GQA_BF16 && dtype != GQA_FP32) return GQA_ERR_INVALID_ARG;
+  if (dtype == GQA_BF16 && !mla_dims_supported_bf16(d_qk, d_v)) return GQA_ERR_UNSUPPORTED;
+  if (dtype == GQA_FP32 && (d_qk > 768 || d_v > 512)) return GQA_ERR_UNSUPPORTED;
+  if (B > decode_max_batch()) return GQA_ERR_UNSUPPORTED;
+  if ((long long)B * T_max >= (1ll << 31) || (long long)B * h_q >= (1ll << 31)) return GQA_ERR_UNSUPPORTED;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return GQA_ERR_WORKSPACE;
+  if (num_splits > 0 && workspace_bytes < decode_workspace_bytes(B, h_q, 1, T_max, d_v, num_splits, 1, true))
+    return GQA_ERR_WORKSPACE;
+  const int sms = sm_count();
+  if (sms <= 0) return GQA_ERR_CUDA;
+  if (workspace_bytes < decode_workspace_bytes(B, h_q, 1, T_max, d_v, num_splits, sms, true))
+    return GQA_ERR_WORKSPACE;
+  DecodeArgs a;
+  a.q = q;
+  a.k = cache;
+  a.v = cache;  // values are the first d_v entries of each cache row
+  a.o = o;
+  a.lse = lse;
+  a.kv_len = kv_len;
+  a.q_pos = q_pos;
+  a.B = B;
+  a.h_q = h_q;
+  a.h_kv = 1;
+  a.T_max = T_max;
+  a.d_h = d_qk;
+  a.d_v = d_v;
+  a.mla = 1;
+  a.scale = scale;
+  a.window = 0;
+  a.workspace = workspace;
+  a.workspace_bytes = workspace_bytes;
+  a.num_splits = num_splits;
+  a.num_sms = sms;
+  a.err = device_error_ptr();
+  if (!a.err) return GQA_ERR_CUDA;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (dtype == GQA_FP32) return from_cuda(launch_decode_fp32(a, s));
+  CUtensorMap maps[2];
+  const uint64_t cdims[2] = {(uint64_t)d_qk, (uint64_t)B * T_max};
+  const uint64_t qdims[2] = {(uint64_t)d_qk, (uint64_t)B * h_q};
+  const uint64_t strides[1] = {(uint64_t)d_qk * 2};
+  const uint32_t cbox[2] = {64, 64};
+  const uint32_t qbox[2] = {64, 16};
+  if (!encode_bf16(&maps[0], cache, 2, cdims, strides, cbox) ||
+      !encode_bf16(&maps[1], q, 2, qdims, strides, qbox))
+    return GQA_ERR_CUDA;
+  return from_cuda(launch_mla_bf16(a, maps, s));
+}
+
 gqa_status gqa_decode_paged(const void* q, const void* k_pages, const void* v_pages, void* o,
                             float* lse, const int32_t* kv_len, const int32_t* q_pos,
                             const int32_t* block_table, int B, int h_q, int h_kv, int num_pages,

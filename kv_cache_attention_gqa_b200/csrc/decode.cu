@@ -73,10 +73,13 @@ struct Layout {
   size_t pre_off, nlen_off, lse_off, o_off, total;
 };
 
-__host__ __device__ inline Layout make_layout(int B, int h_q, int h_kv, int d_h, int n_max) {
+// hpu_max: query heads packed into one unit (32 for the GQA kernels, 16 for MLA); d_h: the width
+// of the output and of the partials.
+__host__ __device__ inline Layout make_layout(int B, int h_q, int h_kv, int d_h, int n_max,
+                                              int hpu_max = kHeadsPerUnitMax) {
   Layout L;
   const int r = h_q / h_kv;
-  L.hpu = r < kHeadsPerUnitMax ? r : kHeadsPerUnitMax;
+  L.hpu = r < hpu_max ? r : hpu_max;
   L.hblocks = (r + L.hpu - 1) / L.hpu;
   L.U = B * h_kv * L.hblocks;
   L.n_max = n_max;
@@ -97,7 +100,8 @@ struct KArgs {
   float* lse;
   const int32_t* kv_len;
   const int32_t* q_pos;
-  int B, h_q, h_kv, r, T_max, D;
+  int B, h_q, h_kv, r, T_max, D;  // D: width of the values, the output and the partials
+  int Dqk;                         // width of the query and key rows (= D except for MLA)
   int hpu, hblocks;
   float scale;     // natural-log scale; the bf16 core folds log2(e) in
   int n_max;       // upper bound on the number of chunks (workspace slots)
@@ -292,10 +296,10 @@ __device__ __forceinline__ float ex2(float x) {
 template <typename OutT, bool kFast, int kV>
 __device__ __forceinline__ void merge_row(const KArgs& a, int lane, int unit, int h,
                                           long long c0, long long c1, long long out_base,
-                                          long long lse_index) {
+                                          long long lse_index, int col_base) {
   constexpr int kU = 8;
   const int D = a.D;
-  const int col0 = lane * kV;
+  const int col0 = col_base + lane * kV;
   const bool active = col0 < D;
   float M = -INFINITY, L = 0.f;
   float acc[kV];
@@ -337,7 +341,7 @@ __device__ __forceinline__ void merge_row(const KArgs& a, int lane, int unit, in
     for (int i = 0; i < kV; ++i)
       if (col0 + i < D) store_out(reinterpret_cast<OutT*>(a.o), out_base + col0 + i, acc[i] * inv);
   }
-  if (lane == 0 && a.lse) a.lse[lse_index] = (M + (kFast ? __log2f(L) : log2f(L))) * kLn2;
+  if (lane == 0 && col_base == 0 && a.lse) a.lse[lse_index] = (M + (kFast ? __log2f(L) : log2f(L))) * kLn2;
 }
 
 template <typename OutT, bool kFast>
@@ -364,8 +368,10 @@ __global__ void __launch_bounds__(256) merge_kernel(KArgs a) {
   const int head = g * a.r + hb * a.hpu + h;
   const long long ob = ((long long)b * a.h_q + head) * a.D;
   const long long li = (long long)b * a.h_q + head;
-  if (a.D % 4 == 0 && a.D <= 128) merge_row<OutT, kFast, 4>(a, lane, unit, h, c0, c1, ob, li);
-  else merge_row<OutT, kFast, 8>(a, lane, unit, h, c0, c1, ob, li);  // d_h <= 256, lane-strided
+  if (a.D % 4 == 0 && a.D <= 128) merge_row<OutT, kFast, 4>(a, lane, unit, h, c0, c1, ob, li, 0);
+  else if (a.D <= 256) merge_row<OutT, kFast, 8>(a, lane, unit, h, c0, c1, ob, li, 0);  // lane-strided
+  else  // wide rows (MLA latent, 512): 128 columns per pass, 16-byte loads
+    for (int col = 0; col < a.D; col += 128) merge_row<OutT, kFast, 4>(a, lane, unit, h, c0, c1, ob, li, col);
 }
 
 // =============================================================================================
@@ -878,10 +884,300 @@ __global__ void __launch_bounds__(Bf16Cfg<D, MT>::kThreads, 1)
 }
 
 // =============================================================================================
+// MLA decode (bf16): every head of a sequence against its shared latent cache rows
+// =============================================================================================
+// A cache row is [latent C (512) | decoupled rotary key (64)]; the query row of a head is the
+// absorbed latent query and its rotary part (576); the value is the row's first 512 entries
+// [第 09 章 GQA、MLA 与跨层 KV 共享, section 09.3: Q (C U_K)^T = (Q U_K^T) C^T and
+// P (C U_V) = (P C) U_V; 第三章, section 3.4 on the decoupled position key]. A unit is 16 heads
+// of one sequence; its keys go through the same split-KV chunks, partials and merge as GQA
+// decode. Per 64-key tile (9 column chunks of 64, staged by TMA) eight consumer warps:
+//   S   warp w scores keys [8w, 8w+8) for the 16 heads over all 576 columns (m16n8k16);
+//   max the row maxima of the eight warps meet in shared memory, so all warps share one running
+//       maximum per head; P = 2^(s - m) goes to shared memory as bf16;
+//   PV  warp w accumulates latent columns [64w, 64w+64) of O += P V over the 64 keys, reading V
+//       as the tile's first eight column chunks.
+constexpr int kMlaDqk = 576, kMlaDv = 512, kMlaHeads = 16;
+struct MlaCfg {
+  static constexpr int kStages = 2;  // also the number of query slots (see the producer)
+  static constexpr int kNch = kMlaDqk / 64;              // 9 column chunks of a cache row
+  static constexpr int kChunkBytes = kTile * 128;        // 64 rows x 128 B
+  static constexpr int kTileBytes = kNch * kChunkBytes;  // 72 KiB
+  static constexpr int kQChunkBytes = kMlaHeads * 128;
+  static constexpr int kQBytes = kNch * kQChunkBytes;    // 18 KiB
+  static constexpr int kConsumerWarps = 8;
+  static constexpr int kThreads = 32 * (kConsumerWarps + 1);
+  static constexpr int kPBytes = kMlaHeads * 128;        // 16 heads x 64 keys, bf16, swizzled
+  static constexpr int kRedBytes = 2 * kConsumerWarps * kMlaHeads * 4;
+  static constexpr size_t kSmem = (size_t)kStages * (kTileBytes + kQBytes) + kPBytes + kRedBytes +
+                                  (kMaxBatch + 1) * 8 + 2 * kMaxBatch * 4 + kStages * sizeof(TileMeta) +
+                                  2 * kStages * 8 + 1024;
+  static_assert(kSmem <= 227 * 1024, "shared memory budget");
+};
+
+__global__ void __launch_bounds__(MlaCfg::kThreads, 1)
+    mla_bf16_kernel(const __grid_constant__ CUtensorMap tmc, const __grid_constant__ CUtensorMap tmq,
+                    KArgs a) {
+  using C = MlaCfg;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* stage_base = smem;
+  uint8_t* q_base = smem + C::kStages * C::kTileBytes;
+  uint8_t* p_buf = q_base + C::kStages * C::kQBytes;
+  float* red_m = reinterpret_cast<float*>(p_buf + C::kPBytes);  // [warp][head]
+  float* red_l = red_m + C::kConsumerWarps * kMlaHeads;
+  long long* pre = reinterpret_cast<long long*>(red_l + C::kConsumerWarps * kMlaHeads);
+  int* nlen = reinterpret_cast<int*>(pre + kMaxBatch + 1);
+  int* wlo = nlen + kMaxBatch;
+  TileMeta* meta = reinterpret_cast<TileMeta*>(wlo + kMaxBatch);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(meta + C::kStages);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int producer_warp = C::kConsumerWarps;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(smem_u32(&bars[s]), 1);
+      mbar_init(smem_u32(&bars[C::kStages + s]), C::kConsumerWarps);
+    }
+    fence_barrier_init();
+  }
+  Plan plan;
+  build_plan<__nv_bfloat16>(a, plan, pre, nlen, wlo, warp, lane, producer_warp);
+  pdl_launch_dependents();
+
+  if (warp == producer_warp) {
+    if (lane == 0) {
+      tma_prefetch_desc(&tmc);
+      tma_prefetch_desc(&tmq);
+      int stage = 0;
+      uint32_t phase = 0;
+      int issued = 0;
+      bool ok = true;
+      const int G = gridDim.x;
+      const bool dyn = plan.n_chunks > G;
+      int chunk = blockIdx.x;
+      int next = dyn && chunk < plan.n_chunks ? G + atomicAdd(&a.hdr->ticket, 1) : plan.n_chunks;
+      // the query rows of a piece stay in one of two slots for all of its tiles; pieces alternate
+      // slots, and with two stages the piece two back has been consumed before its slot refills
+      int qslot = 0;
+      for (; ok && chunk < plan.n_chunks;) {
+        const long long x1 = min((long long)(chunk + 1) * plan.C, plan.K);
+        for (long long x = (long long)chunk * plan.C; x < x1 && ok; qslot ^= 1) {
+          const Piece pc = locate(plan, a.B, a.hblocks, x, x1);
+          const int slot = pc.n_pieces == 1 ? -1 : chunk + pc.unit;
+          const int nh = min(a.hpu, a.r - pc.hb * a.hpu);
+          const int row0 = pc.b * a.T_max + plan.wlo[pc.b];
+          const int qrow = pc.b * a.h_q + pc.hb * a.hpu;
+          for (int t = pc.k0; t < pc.k1; t += kTile) {
+            if (!mbar_wait(smem_u32(&bars[C::kStages + stage]), phase ^ 1u, a.err)) { ok = false; break; }
+            const bool first = t == pc.k0;
+            TileMeta m;
+            m.b = pc.b;
+            m.g = qslot;  // MLA has one KV "head": g carries the piece's query slot
+            m.hb = pc.hb;
+            m.nvalid = min(kTile, pc.k1 - t);
+            m.flags = (first ? kFirst : 0) | (t + kTile >= pc.k1 ? kLast : 0);
+            m.slot = slot;
+            m.nh = nh;
+            m.nskip = 0;
+            meta[stage] = m;
+            const uint32_t full = smem_u32(&bars[stage]);
+            mbar_arrive_expect_tx(full, C::kTileBytes + (first ? C::kQBytes : 0));
+            const uint32_t kdst = smem_u32(stage_base + stage * C::kTileBytes);
+#pragma unroll
+            for (int ch = 0; ch < C::kNch; ++ch)
+              tma_load_2d(kdst + ch * C::kChunkBytes, &tmc, full, ch * 64, row0 + t);
+            if (first) {
+              const uint32_t qdst = smem_u32(q_base + qslot * C::kQBytes);
+#pragma unroll
+              for (int ch = 0; ch < C::kNch; ++ch)
+                tma_load_2d(qdst + ch * C::kQChunkBytes, &tmq, full, ch * 64, qrow);
+            }
+            ++issued;
+            if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
+          }
+          x = pc.end;
+        }
+        chunk = next;
+        if (chunk < plan.n_chunks) next = G + atomicAdd(&a.hdr->ticket, 1);
+      }
+      if (ok && mbar_wait(smem_u32(&bars[C::kStages + stage]), phase ^ 1u, a.err)) {
+        meta[stage].flags = kEnd;
+        mbar_arrive(smem_u32(&bars[stage]));
+        ++issued;
+      }
+      for (int f = issued > C::kStages ? issued - C::kStages : 0; f < issued; ++f) {
+        if (!mbar_wait(smem_u32(&bars[C::kStages + f % C::kStages]), (uint32_t)(f / C::kStages) & 1u, a.err))
+          break;
+      }
+    }
+    return;
+  }
+
+  // ------------------------------- consumer warps -------------------------------------------
+  const int w = warp;
+  const int gid = lane >> 2, tq = lane & 3;
+  const float sl2 = a.scale * kLog2e;
+  const uint32_t pb = smem_u32(p_buf);
+  int stage = 0;
+  uint32_t phase = 0;
+  float acc[8][4];
+  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+  while (true) {
+    if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&bars[stage]), phase, a.err))) return;
+    const TileMeta m = meta[stage];
+    if (m.flags & kEnd) {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&bars[C::kStages + stage]));
+      break;
+    }
+    const uint32_t kb = smem_u32(stage_base + stage * C::kTileBytes);
+    const uint32_t qb = smem_u32(q_base + m.g * C::kQBytes);  // the piece's query slot
+    if (m.flags & kFirst) {
+#pragma unroll
+      for (int n = 0; n < 8; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
+      m0 = m1 = -INFINITY;
+      l0 = l1 = 0.f;
+    }
+    const int nvalid = m.nvalid, nskip = m.nskip;
+    // ---- S = Q K^T for keys [8w, 8w + 8), all 576 columns (36 k-steps, two per ldmatrix of K)
+    float sc[4] = {0.f, 0.f, 0.f, 0.f};
+    {
+      const int i = lane >> 3;
+      const int qr = (i & 1) * 8 + (lane & 7);
+#pragma unroll 3
+      for (int kp = 0; kp < kMlaDqk / 32; ++kp) {
+        const int d8 = 4 * kp + (lane >> 3);
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4(swz128(kb + (d8 >> 3) * C::kChunkBytes, 8 * w + (lane & 7), d8 & 7), b0, b1, b2, b3);
+#pragma unroll
+        for (int s2 = 0; s2 < 2; ++s2) {
+          const int d8q = (2 * kp + s2) * 2 + (i >> 1);
+          uint32_t qa[4];
+          ldsm_x4(swz128(qb + (d8q >> 3) * C::kQChunkBytes, qr, d8q & 7), qa[0], qa[1], qa[2], qa[3]);
+          mma_bf16(sc, qa, s2 ? b2 : b0, s2 ? b3 : b1);
+        }
+      }
+    }
+    // ---- mask, base-2 scale, the eight warps' row maxima -> one running maximum per head
+    float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int key = 8 * w + 2 * tq + e;
+      const bool vis = key < nvalid && key >= nskip;
+      sc[e] = vis ? sc[e] * sl2 : -INFINITY;
+      sc[2 + e] = vis ? sc[2 + e] * sl2 : -INFINITY;
+      mx0 = fmaxf(mx0, sc[e]);
+      mx1 = fmaxf(mx1, sc[2 + e]);
+    }
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+    if (tq == 0) {
+      red_m[w * kMlaHeads + gid] = mx0;
+      red_m[w * kMlaHeads + gid + 8] = mx1;
+    }
+    named_barrier_sync(1, 32 * C::kConsumerWarps);
+    float t0 = -INFINITY, t1 = -INFINITY;
+#pragma unroll
+    for (int v = 0; v < C::kConsumerWarps; ++v) {
+      t0 = fmaxf(t0, red_m[v * kMlaHeads + gid]);
+      t1 = fmaxf(t1, red_m[v * kMlaHeads + gid + 8]);
+    }
+    const float mn0 = fmaxf(m0, t0), mn1 = fmaxf(m1, t1);  // finite: every tile has a visible key
+    const float al0 = fast_exp2(m0 - mn0), al1 = fast_exp2(m1 - mn1);
+    m0 = mn0;
+    m1 = mn1;
+    const float p00 = fast_exp2(sc[0] - mn0), p01 = fast_exp2(sc[1] - mn0);
+    const float p10 = fast_exp2(sc[2] - mn1), p11 = fast_exp2(sc[3] - mn1);
+    float ps0 = p00 + p01, ps1 = p10 + p11;
+    ps0 += __shfl_xor_sync(0xffffffffu, ps0, 1);
+    ps0 += __shfl_xor_sync(0xffffffffu, ps0, 2);
+    ps1 += __shfl_xor_sync(0xffffffffu, ps1, 1);
+    ps1 += __shfl_xor_sync(0xffffffffu, ps1, 2);
+    l0 = fmaf(l0, al0, ps0);  // this warp's share of the row sums (its 8 keys), common maximum
+    l1 = fmaf(l1, al1, ps1);
+    // P (bf16) into shared memory: row = head, keys 8w + 2tq, +1 are 4 bytes of 16-byte unit w
+    asm volatile("st.shared.b32 [%0], %1;" ::"r"(swz128(pb, gid, w) + 4 * tq), "r"(pack_bf16x2(p00, p01)) : "memory");
+    asm volatile("st.shared.b32 [%0], %1;" ::"r"(swz128(pb, gid + 8, w) + 4 * tq), "r"(pack_bf16x2(p10, p11)) : "memory");
+    named_barrier_sync(2, 32 * C::kConsumerWarps);
+    // ---- O[:, 64w .. 64w+64) += P V over the tile's 64 keys
+#pragma unroll
+    for (int n = 0; n < 8; ++n) {
+      acc[n][0] *= al0;
+      acc[n][1] *= al0;
+      acc[n][2] *= al1;
+      acc[n][3] *= al1;
+    }
+    const bool partial = nvalid < kTile || nskip > 0;
+#pragma unroll
+    for (int ks = 0; ks < kTile / 16; ++ks) {
+      uint32_t pa[4];
+      {
+        const int i = lane >> 3;
+        const int pr = (i & 1) * 8 + (lane & 7);
+        ldsm_x4(swz128(pb, pr, ks * 2 + (i >> 1)), pa[0], pa[1], pa[2], pa[3]);
+      }
+      const int vrow = 16 * ks + ((lane >> 3) & 1) * 8 + (lane & 7);
+      const int key_a = 16 * ks + 2 * tq, key_b = key_a + 8;
+#pragma unroll
+      for (int n2 = 0; n2 < 4; ++n2) {
+        const int d8 = 8 * w + n2 * 2 + (lane >> 4);
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_t(swz128(kb + (d8 >> 3) * C::kChunkBytes, vrow, d8 & 7), b0, b1, b2, b3);
+        if (partial) {
+          b0 = mask_pair(b0, key_a, nskip, nvalid);
+          b1 = mask_pair(b1, key_b, nskip, nvalid);
+          b2 = mask_pair(b2, key_a, nskip, nvalid);
+          b3 = mask_pair(b3, key_b, nskip, nvalid);
+        }
+        mma_bf16(acc[2 * n2], pa, b0, b1);
+        mma_bf16(acc[2 * n2 + 1], pa, b2, b3);
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(smem_u32(&bars[C::kStages + stage]));
+    if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
+    if (!(m.flags & kLast)) continue;
+
+    // ---- piece end: row sums over the eight warps, normalise, emit latent columns [64w, 64w+64)
+    if (tq == 0) {
+      red_l[w * kMlaHeads + gid] = l0;
+      red_l[w * kMlaHeads + gid + 8] = l1;
+    }
+    named_barrier_sync(3, 32 * C::kConsumerWarps);
+    float L0 = 0.f, L1 = 0.f;
+#pragma unroll
+    for (int v = 0; v < C::kConsumerWarps; ++v) {
+      L0 += red_l[v * kMlaHeads + gid];
+      L1 += red_l[v * kMlaHeads + gid + 8];
+    }
+    const float inv0 = 1.f / L0, inv1 = 1.f / L1;
+    const float lse0 = m0 + __log2f(L0), lse1 = m1 + __log2f(L1);
+#pragma unroll
+    for (int n = 0; n < 8; ++n) {
+      const int col = 64 * w + 8 * n + 2 * tq;
+      if (gid < m.nh) {
+        emit<__nv_bfloat16>(a, m.b, 0, m.hb, m.slot, gid, col, acc[n][0] * inv0, lse0);
+        emit<__nv_bfloat16>(a, m.b, 0, m.hb, m.slot, gid, col + 1, acc[n][1] * inv0, lse0);
+      }
+      if (gid + 8 < m.nh) {
+        emit<__nv_bfloat16>(a, m.b, 0, m.hb, m.slot, gid + 8, col, acc[n][2] * inv1, lse1);
+        emit<__nv_bfloat16>(a, m.b, 0, m.hb, m.slot, gid + 8, col + 1, acc[n][3] * inv1, lse1);
+      }
+    }
+  }
+}
+
+// =============================================================================================
 // fp32 check-mode kernel
 // =============================================================================================
 constexpr int kF32Warps = 4;
-constexpr int kF32MaxPerLane = 8;  // d_h <= 256
+constexpr int kF32MaxPerLane = 16;  // value / output width <= 512 ...
+constexpr int kF32MaxQkPerLane = 24;  // ... query / key width <= 768 (MLA rows: 576)
 
 __global__ void __launch_bounds__(32 * kF32Warps, 1) decode_fp32_kernel(KArgs a) {
   __shared__ long long pre[kMaxBatch + 1];
@@ -908,24 +1204,26 @@ __global__ void __launch_bounds__(32 * kF32Warps, 1) decode_fp32_kernel(KArgs a)
       const int lo = wlo[pc.b];
       const int koff = lo / a.gran * a.gran;  // absolute position of the unit's key 0
       const int jskip = lo - koff;            // keys of the first granule before the window
-      const long long kv_base = ((long long)pc.b * a.h_kv + pc.g) * a.T_max * D;
+      const int Dk = a.Dqk;  // query / key row width; values are the first D entries of V's rows
+      const long long kv_base = ((long long)pc.b * a.h_kv + pc.g) * a.T_max * Dk;
       const float* kp = reinterpret_cast<const float*>(a.k) + kv_base;
       const float* vp = reinterpret_cast<const float*>(a.v) + kv_base;
       for (int hl = warp; hl < nh; hl += kF32Warps) {
         const int head = pc.g * a.r + pc.hb * a.hpu + hl;
-        const float* q = reinterpret_cast<const float*>(a.q) + ((long long)pc.b * a.h_q + head) * D;
-        float qr[kF32MaxPerLane], accv[kF32MaxPerLane];
+        const float* q = reinterpret_cast<const float*>(a.q) + ((long long)pc.b * a.h_q + head) * Dk;
+        float qr[kF32MaxQkPerLane], accv[kF32MaxPerLane];
 #pragma unroll
-        for (int e = 0; e < kF32MaxPerLane; ++e) {
+        for (int e = 0; e < kF32MaxQkPerLane; ++e) {
           const int col = lane + 32 * e;
-          qr[e] = col < D ? q[col] : 0.f;
-          accv[e] = 0.f;
+          qr[e] = col < Dk ? q[col] : 0.f;
         }
+#pragma unroll
+        for (int e = 0; e < kF32MaxPerLane; ++e) accv[e] = 0.f;
         float m = -INFINITY, l = 0.f;
         for (int jr = max(pc.k0, jskip); jr < pc.k1; ++jr) {
           const int j = koff + jr;  // absolute key position
-          const float* kj = kp + (long long)j * D;
-          const float* vj = vp + (long long)j * D;
+          const float* kj = kp + (long long)j * Dk;
+          const float* vj = vp + (long long)j * Dk;
           if (a.block_table) {
             int page = a.block_table[(long long)pc.b * a.max_pages + j / a.page_size];
             if (page < 0 || page >= a.num_pages) {
@@ -933,14 +1231,14 @@ __global__ void __launch_bounds__(32 * kF32Warps, 1) decode_fp32_kernel(KArgs a)
               page = 0;
             }
             const long long row = ((long long)page * a.h_kv + pc.g) * a.page_size + j % a.page_size;
-            kj = reinterpret_cast<const float*>(a.k) + row * D;
-            vj = reinterpret_cast<const float*>(a.v) + row * D;
+            kj = reinterpret_cast<const float*>(a.k) + row * Dk;
+            vj = reinterpret_cast<const float*>(a.v) + row * Dk;
           }
           float part = 0.f;
 #pragma unroll
-          for (int e = 0; e < kF32MaxPerLane; ++e) {
+          for (int e = 0; e < kF32MaxQkPerLane; ++e) {
             const int col = lane + 32 * e;
-            if (col < D) part = fmaf(qr[e], kj[col], part);
+            if (col < Dk) part = fmaf(qr[e], kj[col], part);
           }
 #pragma unroll
           for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
@@ -1026,10 +1324,12 @@ int auto_n_max(long long K_max, int sms) {
 KArgs make_kargs(const DecodeArgs& a) {
   const bool auto_chunk = a.num_splits == 0;
   const int r = a.h_q / a.h_kv;
-  const int hpu = r < kHeadsPerUnitMax ? r : kHeadsPerUnitMax;
+  const int hpu_max = a.mla ? kMlaHeads : kHeadsPerUnitMax;
+  const int hpu = r < hpu_max ? r : hpu_max;
+  const int d_out = a.d_v > 0 ? a.d_v : a.d_h;
   const long long K_max = (long long)a.B * a.h_kv * ((r + hpu - 1) / hpu) * a.T_max;
   const int n_max = auto_chunk ? auto_n_max(K_max, a.num_sms) : a.num_splits;
-  const Layout L = make_layout(a.B, a.h_q, a.h_kv, a.d_h, n_max);
+  const Layout L = make_layout(a.B, a.h_q, a.h_kv, d_out, n_max, hpu_max);
   KArgs k;
   k.q = a.q;
   k.k = a.k;
@@ -1043,7 +1343,8 @@ KArgs make_kargs(const DecodeArgs& a) {
   k.h_kv = a.h_kv;
   k.r = r;
   k.T_max = a.T_max;
-  k.D = a.d_h;
+  k.D = d_out;
+  k.Dqk = a.d_h;
   k.hpu = L.hpu;
   k.hblocks = L.hblocks;
   k.scale = a.scale;
@@ -1068,12 +1369,13 @@ KArgs make_kargs(const DecodeArgs& a) {
 }  // namespace dec
 
 size_t decode_workspace_bytes(int B, int h_q, int h_kv, int T_max, int d_h, int num_splits,
-                              int num_sms) {
+                              int num_sms, bool mla) {
   const int r = h_q / h_kv;
-  const int hpu = r < dec::kHeadsPerUnitMax ? r : dec::kHeadsPerUnitMax;
+  const int hpu_max = mla ? dec::kMlaHeads : dec::kHeadsPerUnitMax;
+  const int hpu = r < hpu_max ? r : hpu_max;
   const long long K_max = (long long)B * h_kv * ((r + hpu - 1) / hpu) * T_max;
   const int n_max = num_splits == 0 ? dec::auto_n_max(K_max, num_sms) : num_splits;
-  return dec::make_layout(B, h_q, h_kv, d_h, n_max).total;
+  return dec::make_layout(B, h_q, h_kv, d_h, n_max, hpu_max).total;
 }
 
 int decode_max_batch() { return dec::kMaxBatch; }
@@ -1110,5 +1412,25 @@ cudaError_t launch_decode_bf16(const DecodeArgs& a, const CUtensorMap* tmaps, cu
   return a.paged_3d ? dec::launch_bf16_dispatch<dec::kPaged3d>(k, tmaps, a.num_sms, s)
                     : dec::launch_bf16_dispatch<dec::kPaged2d>(k, tmaps, a.num_sms, s);
 }
+
+cudaError_t launch_mla_bf16(const DecodeArgs& a, const CUtensorMap* tmaps, cudaStream_t s) {
+  const dec::KArgs k = dec::make_kargs(a);
+  using C = dec::MlaCfg;
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+    e = cudaFuncSetAttribute(dec::mla_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::kSmem);
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < 64) attr_set[dev] = true;
+  }
+  dec::mla_bf16_kernel<<<a.num_sms, C::kThreads, C::kSmem, s>>>(tmaps[0], tmaps[1], k);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  return dec::launch_merge<__nv_bfloat16, true>(k, s);
+}
+
+int mla_dims_supported_bf16(int d_qk, int d_v) { return d_qk == dec::kMlaDqk && d_v == dec::kMlaDv; }
 
 }  // namespace gqa

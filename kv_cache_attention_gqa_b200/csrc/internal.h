@@ -97,11 +97,15 @@ struct DecodeArgs {
   // num_pages*h_kv*page_size rows with a 256-byte stride, 2 column chunks with a 128-byte stride)
   // with box (64, 16, 2)
   int paged_3d = 0;
+  // MLA: one shared cache row per token (k = v = the cache, h_kv = 1), d_h = the query / key row
+  // width (576), d_v = the value / output width (the row's first 512 entries); 16 heads per unit
+  int mla = 0;
+  int d_v = 0;
 };
 
 // Workspace bytes for a decode of this shape (layout in decode.cu).
 size_t decode_workspace_bytes(int B, int h_q, int h_kv, int T_max, int d_h, int num_splits,
-                              int num_sms);
+                              int num_sms, bool mla = false);
 int decode_max_batch();
 
 cudaError_t launch_decode_fp32(const DecodeArgs& a, cudaStream_t s);
@@ -109,5 +113,9 @@ cudaError_t launch_decode_fp32(const DecodeArgs& a, cudaStream_t s);
 // a paged cache (d_h, num_pages*h_kv*page_size) with box (64, 16);
 // [2] = queries as (d_h, B*h_q) with box (64, 16 or 32 rows: 32 when r > 16); SWIZZLE_128B.
 cudaError_t launch_decode_bf16(const DecodeArgs& a, const CUtensorMap* tmaps, cudaStream_t s);
+// MLA (bf16, d_h = 576, d_v = 512): tmaps [0] = the cache as (576, B*T_max) with box (64, 64),
+// [1] = the queries as (576, B*h_q) with box (64, 16); SWIZZLE_128B.
+cudaError_t launch_mla_bf16(const DecodeArgs& a, const CUtensorMap* tmaps, cudaStream_t s);
+int mla_dims_supported_bf16(int d_qk, int d_v);
 
 }  // namespace gqa

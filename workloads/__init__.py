@@ -193,3 +193,38 @@ def paged_decode_inputs(shape: DecodeShape, page_size: int, seed: int = DEFAULT_
     k.transpose(1, 2)[unused] = float("nan")  # (num_pages, page_size) rows, every KV head
     v.transpose(1, 2)[unused] = float("nan")
     return q, k, v, torch.from_numpy(table).to(device), torch.from_numpy(lengths).to(device)
+
+
+@dataclasses.dataclass(frozen=True)
+class MlaShape:
+    B: int
+    h_q: int
+    T_max: int
+    d_qk: int = 576  # latent 512 + decoupled rotary key 64 (DeepSeek-V2/V3 widths)
+    d_v: int = 512
+    d_nope: int = 128  # per-head widths of the original (non-absorbed) heads, for the scale
+    d_rope: int = 64
+
+    @property
+    def scale(self) -> float:
+        return (self.d_nope + self.d_rope) ** -0.5
+
+
+# MLA decode at the decode_8k sizes: B=8, T=8192, 16 heads per GPU (128 heads split 8 ways) and
+# all 128 heads on one GPU.
+MLA_DECODE = {h: MlaShape(B=8, h_q=h, T_max=8192) for h in (16, 128)}
+
+
+def mla_decode_inputs(shape: MlaShape, seed: int = DEFAULT_SEED, device="cpu", dtype=torch.bfloat16,
+                      lengths=None, nan_tail: bool = True):
+    """q (B, h_q, d_qk), cache (B, T_max, d_qk), kv_len (B,) int32. Draw order: q, cache.
+    Rows at or past each length are NaN when ``nan_tail``."""
+    g = _generator(seed, device)
+    q = randn_bf16((shape.B, shape.h_q, shape.d_qk), g, 1.0, device, dtype)
+    cache = randn_bf16((shape.B, shape.T_max, shape.d_qk), g, 1.0, device, dtype)
+    lens = (np.full(shape.B, shape.T_max, np.int32) if lengths is None
+            else np.asarray(lengths, np.int32))
+    if nan_tail:
+        for b in range(shape.B):
+            cache[b, int(lens[b]):] = float("nan")
+    return q, cache, torch.from_numpy(lens).to(device)

@@ -10,7 +10,8 @@ the timed events.
 A ``paged`` object repeats the decode_8k step over a paged cache (16-token pages in a shuffled
 pool: ``kv_append_paged`` + ``gqa_decode_paged``), timed the same way; a ``window`` object runs
 decode_8k and prefill_4k with a 1024-key sliding window (work counted inside the window only); a
-``backward`` object times gqa_prefill_backward on prefill_4k.
+``backward`` object times gqa_prefill_backward on prefill_4k; an ``mla`` object times gqa_mla_decode
+over a latent cache.
 
 ``--impl reference`` times the fp64 CPU oracle on a bounded sample of the same workload.
 Run with no flags for N=1; under torchrun every rank runs an independent replica (the path needs
@@ -387,6 +388,75 @@ def run_backward(args, dev, stream, tf_peak, peak_kind):
                          "algorithmic_flops_per_launch": flops}}
 
 
+def graph_timed(fn, flush, steps, warmup):
+    """Mean device time (ms) of `fn` captured once in a CUDA graph and replayed `steps` times, each
+    replay after an L2 flush outside the events (eager launches if capture fails)."""
+    import torch
+
+    for _ in range(warmup):
+        flush(1)
+        fn()
+    torch.cuda.synchronize()
+    graph = None
+    try:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            fn()
+        graph.replay()
+        torch.cuda.synchronize()
+    except Exception:  # pragma: no cover - depends on the driver/runtime
+        graph = None
+        torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for i in range(steps):
+        flush(i)
+        evs[i][0].record(stream)
+        if graph is not None:
+            graph.replay()
+        else:
+            fn()
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    mode = "cuda_graph" if graph is not None else "eager"
+    del graph
+    return statistics.mean(a.elapsed_time(b) for a, b in evs), mode
+
+
+def run_mla(args, dev, hbm_peak, tf_peak, peak_kind):
+    """MLA decode over a latent cache [第 09 章 §09.3]: B=8, T=8192, rows of 576 (latent 512 +
+    rotary 64), 16 and 128 query heads. Algorithmic bytes: the cache rows once per call
+    (B * T * 576 * 2); FLOPs: 2 * B * h_q * T * (576 + 512)."""
+    import torch
+
+    import kv_cache_attention_gqa_b200 as gqa
+    import workloads
+
+    flush = L2Flush(dev)
+    out = {}
+    for h_q in (16, 128):
+        shape = workloads.MLA_DECODE[h_q]
+        q, cache, kl = workloads.mla_decode_inputs(shape, seed=args.seed, device=dev, nan_tail=False)
+        o = torch.empty((shape.B, h_q, shape.d_v), dtype=torch.bfloat16, device=dev)
+        ws = torch.zeros(gqa._lib._lib.gqa_mla_decode_workspace_size(shape.B, h_q, shape.T_max, shape.d_v, 0, 0),
+                         dtype=torch.uint8, device=dev)
+        fn = lambda: gqa.mla_decode(q, cache, kv_len=kl, scale=shape.scale, out=o, ws=ws)  # noqa: E731
+        ms, mode = graph_timed(fn, flush, max(5, args.steps), max(3, args.warmup))
+        if gqa.get_device_error() != 0:
+            raise RuntimeError("device error in the MLA line")
+        nbytes = shape.B * shape.T_max * shape.d_qk * 2
+        flops = 2 * shape.B * h_q * shape.T_max * (shape.d_qk + shape.d_v)
+        out[f"h_q={h_q}"] = {"decode_us": round(ms * 1e3, 2), "cache_bytes": nbytes,
+                             "GB_s": round(nbytes / (ms / 1e3) / 1e9, 1),
+                             "frac_of_hbm_peak": round(nbytes / (ms / 1e3) / 1e9 / hbm_peak, 4),
+                             "TFLOP_s": round(flops / (ms / 1e3) / 1e12, 1), "launch": mode}
+        del q, cache, o, ws
+    return {"workload": "MLA decode over a latent cache: B=8, T=8192, rows of 576 (latent 512 + rotary 64), "
+                        "h_q in {16, 128}, one gqa_mla_decode per variant",
+            "peak_kind": f"hbm_gbs / bf16_tflops of {peak_kind}", "hbm_peak": hbm_peak, "tensor_peak": tf_peak,
+            "per_variant": out, "gpu_launches_per_call": 2}
+
+
 def run_window(args, rank, dev, stream, local, hbm_peak, tf_peak, peak_kind):
     """Sliding window of 1024 keys [第三章 §3.7]: decode_8k (each query reads its 1024 most recent
     keys) and prefill_4k; the work counted is only what lies inside the windows."""
@@ -420,6 +490,8 @@ def run_ours(args, rank, world, dist):
         return {"prefill": run_prefill(args, dev, stream, tf_peak, peak_kind)}
     if args.paged_only:  # profiling aid: the paged decode_8k line alone
         return {"paged": run_paged(args, rank, dev, stream, local, hbm_peak, peak_kind)}
+    if args.mla_only:  # profiling aid: the MLA line alone
+        return {"mla": run_mla(args, dev, hbm_peak, tf_peak, peak_kind)}
     if args.backward_only:  # profiling aid: the backward line alone
         return {"backward": run_backward(args, dev, stream, tf_peak, peak_kind)}
     if args.window_only:  # profiling aid: the sliding-window lines alone
@@ -456,6 +528,7 @@ def run_ours(args, rank, world, dist):
         paged = run_paged(args, rank, dev, stream, local, hbm_peak, peak_kind)
         paged["gpu_launches"] = args.steps * 3 * len(args.h_kv)
     backward = run_backward(args, dev, stream, tf_peak, peak_kind) if not args.skip_backward else None
+    mla = run_mla(args, dev, hbm_peak, tf_peak, peak_kind) if not args.skip_mla else None
     window = None
     if not args.skip_window:
         window = run_window(args, rank, dev, stream, local, hbm_peak, tf_peak, peak_kind)
@@ -481,6 +554,8 @@ def run_ours(args, rank, world, dist):
         result["window"] = window
     if backward is not None:
         result["backward"] = backward
+    if mla is not None:
+        result["mla"] = mla
     if rank == 0 and world == 1 and not args.skip_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(args)
     return result
@@ -661,6 +736,8 @@ def main():
                     help="page size of the paged decode_8k line (a multiple of 16)")
     ap.add_argument("--skip-window", action="store_true")
     ap.add_argument("--skip-backward", action="store_true")
+    ap.add_argument("--skip-mla", action="store_true")
+    ap.add_argument("--mla-only", action="store_true", help="only the MLA line (profiling aid)")
     ap.add_argument("--backward-only", action="store_true", help="only the backward line (profiling aid)")
     ap.add_argument("--window-only", action="store_true", help="only the sliding-window lines (profiling aid)")
     ap.add_argument("--window", type=int, default=1024, help="sliding window of the window lines")

@@ -344,13 +344,19 @@ __device__ __forceinline__ void merge_row(const KArgs& a, int lane, int unit, in
   if (lane == 0 && col_base == 0 && a.lse) a.lse[lse_index] = (M + (kFast ? __log2f(L) : log2f(L))) * kLn2;
 }
 
+// Rows wider than 256 (the MLA latent) are merged by one warp per 128-column slice.
+__host__ __device__ inline int merge_slices(int D) { return D > 256 ? (D + 127) / 128 : 1; }
+
 template <typename OutT, bool kFast>
 __global__ void __launch_bounds__(256) merge_kernel(KArgs a) {
   pdl_wait();  // the decode grid has completed and its writes are visible
   const long long C = a.hdr->chunk;
   if (blockIdx.x == 0 && threadIdx.x == 0) a.hdr->ticket = 0;  // ready for the next call
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const long long row = (long long)blockIdx.x * 8 + warp;
+  const int slices = merge_slices(a.D);
+  const long long wid = (long long)blockIdx.x * 8 + warp;
+  const long long row = wid / slices;
+  const int slice = (int)(wid - row * slices);
   const int UPB = a.h_kv * a.hblocks;
   const long long U = (long long)a.B * UPB;
   if (row >= U * a.hpu) return;
@@ -370,8 +376,7 @@ __global__ void __launch_bounds__(256) merge_kernel(KArgs a) {
   const long long li = (long long)b * a.h_q + head;
   if (a.D % 4 == 0 && a.D <= 128) merge_row<OutT, kFast, 4>(a, lane, unit, h, c0, c1, ob, li, 0);
   else if (a.D <= 256) merge_row<OutT, kFast, 8>(a, lane, unit, h, c0, c1, ob, li, 0);  // lane-strided
-  else  // wide rows (MLA latent, 512): 128 columns per pass, 16-byte loads
-    for (int col = 0; col < a.D; col += 128) merge_row<OutT, kFast, 4>(a, lane, unit, h, c0, c1, ob, li, col);
+  else merge_row<OutT, kFast, 4>(a, lane, unit, h, c0, c1, ob, li, slice * 128);  // wide rows
 }
 
 // =============================================================================================
@@ -898,6 +903,10 @@ __global__ void __launch_bounds__(Bf16Cfg<D, MT>::kThreads, 1)
 //   PV  warp w accumulates latent columns [64w, 64w+64) of O += P V over the 64 keys, reading V
 //       as the tile's first eight column chunks.
 constexpr int kMlaDqk = 576, kMlaDv = 512, kMlaHeads = 16;
+#ifndef GQA_MLA_QREG
+#define GQA_MLA_QREG 16  // k-steps of the query kept in registers (9 warps: at most 168 regs each; 16 does not spill)
+#endif
+constexpr int kMlaQReg = GQA_MLA_QREG;
 struct MlaCfg {
   static constexpr int kStages = 2;  // also the number of query slots (see the producer)
   static constexpr int kNch = kMlaDqk / 64;              // 9 column chunks of a cache row
@@ -1024,6 +1033,8 @@ __global__ void __launch_bounds__(MlaCfg::kThreads, 1)
   int stage = 0;
   uint32_t phase = 0;
   float acc[8][4];
+  uint32_t qf[kMlaQReg][4];  // the unit's 16 query rows as A fragments, first kMlaQReg k-steps
+  uint32_t qb = 0;           // the piece's query slot (the remaining k-steps are read from it)
   float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
   while (true) {
     if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&bars[stage]), phase, a.err))) return;
@@ -1034,8 +1045,16 @@ __global__ void __launch_bounds__(MlaCfg::kThreads, 1)
       break;
     }
     const uint32_t kb = smem_u32(stage_base + stage * C::kTileBytes);
-    const uint32_t qb = smem_u32(q_base + m.g * C::kQBytes);  // the piece's query slot
     if (m.flags & kFirst) {
+      qb = smem_u32(q_base + m.g * C::kQBytes);
+      const int i = lane >> 3;
+      const int qr = (i & 1) * 8 + (lane & 7);
+#pragma unroll
+      for (int ks = 0; ks < kMlaQReg; ++ks) {
+        const int d8q = ks * 2 + (i >> 1);
+        ldsm_x4(swz128(qb + (d8q >> 3) * C::kQChunkBytes, qr, d8q & 7), qf[ks][0], qf[ks][1], qf[ks][2],
+                qf[ks][3]);
+      }
 #pragma unroll
       for (int n = 0; n < 8; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
       m0 = m1 = -INFINITY;
@@ -1044,19 +1063,22 @@ __global__ void __launch_bounds__(MlaCfg::kThreads, 1)
     const int nvalid = m.nvalid, nskip = m.nskip;
     // ---- S = Q K^T for keys [8w, 8w + 8), all 576 columns (36 k-steps, two per ldmatrix of K)
     float sc[4] = {0.f, 0.f, 0.f, 0.f};
-    {
-      const int i = lane >> 3;
-      const int qr = (i & 1) * 8 + (lane & 7);
-#pragma unroll 3
-      for (int kp = 0; kp < kMlaDqk / 32; ++kp) {
-        const int d8 = 4 * kp + (lane >> 3);
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4(swz128(kb + (d8 >> 3) * C::kChunkBytes, 8 * w + (lane & 7), d8 & 7), b0, b1, b2, b3);
 #pragma unroll
-        for (int s2 = 0; s2 < 2; ++s2) {
-          const int d8q = (2 * kp + s2) * 2 + (i >> 1);
+    for (int kp = 0; kp < kMlaDqk / 32; ++kp) {
+      const int d8 = 4 * kp + (lane >> 3);
+      uint32_t b0, b1, b2, b3;
+      ldsm_x4(swz128(kb + (d8 >> 3) * C::kChunkBytes, 8 * w + (lane & 7), d8 & 7), b0, b1, b2, b3);
+#pragma unroll
+      for (int s2 = 0; s2 < 2; ++s2) {
+        const int ks = 2 * kp + s2;
+        if (ks < kMlaQReg) {
+          mma_bf16(sc, qf[ks < kMlaQReg ? ks : 0], s2 ? b2 : b0, s2 ? b3 : b1);
+        } else {
+          const int i = lane >> 3;
+          const int d8q = ks * 2 + (i >> 1);
           uint32_t qa[4];
-          ldsm_x4(swz128(qb + (d8q >> 3) * C::kQChunkBytes, qr, d8q & 7), qa[0], qa[1], qa[2], qa[3]);
+          ldsm_x4(swz128(qb + (d8q >> 3) * C::kQChunkBytes, (i & 1) * 8 + (lane & 7), d8q & 7), qa[0], qa[1],
+                  qa[2], qa[3]);
           mma_bf16(sc, qa, s2 ? b2 : b0, s2 ? b3 : b1);
         }
       }
@@ -1273,7 +1295,7 @@ __global__ void __launch_bounds__(32 * kF32Warps, 1) decode_fp32_kernel(KArgs a)
 
 template <typename OutT, bool kFast>
 cudaError_t launch_merge(const KArgs& ka, cudaStream_t s) {
-  const long long rows = (long long)ka.B * ka.h_kv * ka.hblocks * ka.hpu;
+  const long long rows = (long long)ka.B * ka.h_kv * ka.hblocks * ka.hpu * merge_slices(ka.D);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)((rows + 7) / 8));
   cfg.blockDim = dim3(256);

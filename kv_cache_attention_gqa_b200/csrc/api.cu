@@ -333,19 +333,23 @@ gqa_status gqa_prefill_backward(const void* q, const void* k_cache, const void* 
   if (!a.err) return GQA_ERR_CUDA;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (dtype == GQA_FP32) return from_cuda(launch_backward_fp32(a, s));
-  // TMA views: Q and dO as (d_h, S_q, B*h_q) with box (64, 128, 1) for the key-stationary dK/dV
-  // kernel and (64, P, H) for the query-stationary dQ kernel; K, V as rows with box (64, 128).
+  // TMA views: Q and dO as (d_h, S_q, B*h_q) with box (64, 64, 1) for the key-stationary dK/dV
+  // kernel and (64, P, H) for the query-stationary dQ kernel; K, V as rows with box (64, 128) for
+  // dK/dV (its 128 stationary keys) and (64, 64) for dQ (its 64-key blocks).
   const int H = prefill_heads_per_tile(h_q, h_kv);
   const uint32_t P = (uint32_t)(128 / H);
-  CUtensorMap maps[6];
+  CUtensorMap maps[8];
   const uint64_t qdims[3] = {(uint64_t)d_h, (uint64_t)S_q, (uint64_t)B * h_q};
   const uint64_t qstrides[2] = {(uint64_t)d_h * 2, (uint64_t)S_q * d_h * 2};
-  const uint32_t qbox_rows[3] = {64, 128, 1};
+  const uint32_t qbox_rows[3] = {64, 64, 1};
   const uint32_t qbox_tile[3] = {64, P, (uint32_t)H};
   const uint64_t kdims[2] = {(uint64_t)d_h, (uint64_t)B * h_kv * T_max};
   const uint64_t strides[1] = {(uint64_t)d_h * 2};
   const uint32_t box[2] = {64, 128};
-  if (!encode_bf16(&maps[0], q, 3, qdims, qstrides, qbox_rows) ||
+  const uint32_t box64[2] = {64, 64};
+  if (!encode_bf16(&maps[6], k_cache, 2, kdims, strides, box64) ||
+      !encode_bf16(&maps[7], v_cache, 2, kdims, strides, box64) ||
+      !encode_bf16(&maps[0], q, 3, qdims, qstrides, qbox_rows) ||
       !encode_bf16(&maps[1], d_o, 3, qdims, qstrides, qbox_rows) ||
       !encode_bf16(&maps[2], k_cache, 2, kdims, strides, box) ||
       !encode_bf16(&maps[3], v_cache, 2, kdims, strides, box) ||

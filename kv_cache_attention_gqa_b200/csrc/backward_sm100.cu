@@ -11,20 +11,22 @@
 // Three launches:
 //   rowterm   one warp per query row: D = rowsum(dO * O) and the base-2 lse (fp32 workspace).
 //   dkdv      one CTA per (sequence, KV head, 128-key block). The keys sit on the 128 TMEM lanes;
-//             the CTA walks every query block of every head of the group, so the r heads' shares
-//             of dK and dV add up in TMEM (no atomics):
+//             the CTA walks every 64-row query block of every head of the group, so the r heads'
+//             shares of dK and dV add up in TMEM (no atomics):
 //               S^T  = K Q^T     tcgen05.mma, A = K and B = Q from shared memory (K-major)
 //               dP^T = V dO^T    A = V, B = dO from shared memory
 //               (4 warps) P^T = 2^(S^T c - lse2), dS^T = P^T (dP^T - D) -> bf16 into TMEM
 //               dV  += P^T dO    A = P^T from TMEM, B = dO (MN-major view of the same tile)
 //               dK  += dS^T Q    A = dS^T from TMEM, B = Q (MN-major)
-//   dq        one CTA per forward tile (H heads x P positions of one group), walking the K/V
-//             blocks the tile sees:
+//   dq        one CTA per forward tile (H heads x P positions of one group), walking the 64-key
+//             K/V blocks the tile sees:
 //               S = Q K^T, dP = dO V^T (A = Q / dO, B = K / V from shared memory), then dS -> bf16
 //               into TMEM, dQ += dS K (A = dS from TMEM, B = K, MN-major view).
-// TMEM (512 columns): S [0,128), dP [128,256), accumulators from 256; P / dS (bf16 pairs) alias
-// the first 64 columns of S / dP. MMAs issued by one thread execute in order, so the next
-// block's S is written only after the accumulating MMAs have read P / dS.
+// TMEM (512 columns): S double-buffered at [0,64) and [64,128), dP at [128,192) and [192,256),
+// accumulators from 256; P / dS (bf16 pairs) are written over the first columns of the scores
+// they come from. MMAs issued by one thread execute in order, so a buffer is rewritten only
+// after the accumulating MMAs have read its P / dS, and the next block's scores overlap the
+// current block's elementwise pass.
 //
 // Every tcgen05.ld/st/wait sits behind warp-uniform conditions; every mbarrier wait is bounded
 // (2 s of %globaltimer) and sets GQA_DEVERR_TIMEOUT instead of hanging.
@@ -38,12 +40,10 @@
 namespace gqa {
 namespace bw {
 
-constexpr int kBK = 128;  // keys per block (dkdv: the CTA's keys; dq: per K/V block)
-constexpr int kBQ = 128;  // query rows per block
-constexpr int kThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2-5 elementwise (TMEM lanes)
+constexpr int kBK = 128;  // keys of a dkdv CTA (one per TMEM lane)
 constexpr uint32_t kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr uint32_t kColS = 0, kColDP = 128, kColAcc0 = 256;
+constexpr uint32_t kColAcc0 = 256;  // first accumulator column (scores and their bf16 P / dS use [0, 256))
 
 struct BArgs {
   const float* lse2;  // (B*h_q*S_q) base-2 log-sum-exp per row (+inf for a row with no key)
@@ -119,25 +119,51 @@ __global__ void __launch_bounds__(256) rowterm_kernel(const T* o, const T* d_o, 
 }
 
 
-// Shared memory of the dkdv kernel (D = head dim): K and V blocks, a two-stage ring of Q and dO
-// blocks with their rows' lse2 and D, barriers.
+// Descriptors for tiles of any row count: `chunk` is the byte stride between 64-column chunks
+// (rows x 128 B).
+__device__ __forceinline__ uint64_t desc_k(uint32_t tile, int k, uint32_t chunk) {
+  return tc::smem_desc(tile + (uint32_t)((k >> 2) * chunk + (k & 3) * 32), 16, 1024);
+}
+__device__ __forceinline__ uint64_t desc_mn(uint32_t tile, int kk, uint32_t chunk) {
+  return tc::smem_desc(tile + (uint32_t)(kk * 2048), chunk, 1024);
+}
+
+// ---- dkdv: key-stationary dK / dV -------------------------------------------------------------
+// Query blocks of 64 rows, so S^T and dP^T are double-buffered in TMEM next to the dV / dK
+// accumulators: the MMA warp issues block i+1's S^T / dP^T while eight warps (two per TMEM lane
+// quarter, one per 32-query half) turn block i into P^T / dS^T. Each half writes its bf16 pairs
+// over the first 16 columns of its own 32, so the halves never touch each other's columns; the
+// accumulating MMAs address their A operand per 16-query step accordingly.
+// TMEM: S^T[buf] at 64 buf, dP^T[buf] at 128 + 64 buf, dV at 256, dK at 256 + D.
+constexpr int kKvBQ = 64;
+constexpr int kKvStages = 3;
+constexpr int kKvThreads = 320;  // warp 0 TMA + statistics, warp 1 MMA, warps 2-9 elementwise
 template <int D>
 struct KvCfg {
   static constexpr int kNch = D / 64;
-  static constexpr int kTile = kNch * 128 * 128;  // one 128-row bf16 tile
+  static constexpr int kKTile = kNch * 128 * 128;     // K or V: 128 rows
+  static constexpr int kQChunk = kKvBQ * 128;         // 64 rows x 128 B
+  static constexpr int kQTile = kNch * kQChunk;       // Q or dO: 64 rows
   static constexpr int kOffK = 0;
-  static constexpr int kOffV = kTile;
-  static constexpr int kOffQ = 2 * kTile;               // + stage * 2 * kTile
-  static constexpr int kOffDO = 3 * kTile;              // + stage * 2 * kTile
-  static constexpr int kOffStat = 6 * kTile;            // 2 stages x (lse2[128], D[128]) floats
-  static constexpr int kOffBar = kOffStat + 2 * 2 * 128 * 4;
+  static constexpr int kOffV = kKTile;
+  static constexpr int kOffQ = 2 * kKTile;                        // + stage * 2 * kQTile
+  static constexpr int kOffStat = kOffQ + kKvStages * 2 * kQTile;  // stages x (lse2[64], D[64])
+  static constexpr int kOffBar = kOffStat + kKvStages * 2 * kKvBQ * 4;
   static constexpr int kSmem = (kOffBar + 256 + 1024) > 120 * 1024 ? kOffBar + 256 + 1024 : 120 * 1024;
   static_assert(kSmem <= 227 * 1024, "shared memory budget");
 };
-enum { kKvFull = 0, kQFull = 1, kQEmpty = 3, kKvS = 5, kKvP = 6, kKvDone = 7, kKvBars = 8 };
+enum {
+  kKvFull = 0,
+  kQFull = 1,                    // + stage (3): TMA bytes + the producer warp's 32 stat arrivals
+  kQEmpty = kQFull + kKvStages,  // + stage
+  kKvS = kQEmpty + kKvStages,    // + buffer (2): S^T, dP^T of a block are in TMEM
+  kKvP = kKvS + 2,               // + buffer (2): P^T, dS^T of a block are in TMEM (256 arrivals)
+  kKvDone = kKvP + 2,
+  kKvBars = kKvDone + 1
+};
 
 template <int D>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kKvThreads, 1)
     dkdv_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmdo,
                 const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                 BArgs a) {
@@ -148,10 +174,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kKvBars);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  float* stat = reinterpret_cast<float*>(smem + C::kOffStat);  // [stage][lse2 128 | D 128]
+  float* stat = reinterpret_cast<float*>(smem + C::kOffStat);  // [stage][lse2 64 | D 64]
   const uint32_t sK = smem_u32(smem + C::kOffK), sV = smem_u32(smem + C::kOffV);
-  auto sQ = [&](int st) { return smem_u32(smem + C::kOffQ + st * 2 * C::kTile); };
-  auto sDO = [&](int st) { return smem_u32(smem + C::kOffDO + st * 2 * C::kTile); };
+  auto sQ = [&](int st) { return smem_u32(smem + C::kOffQ + st * 2 * C::kQTile); };
+  auto sDO = [&](int st) { return smem_u32(smem + C::kOffQ + st * 2 * C::kQTile + C::kQTile); };
   auto bar = [&](int i) { return smem_u32(&bars[i]); };
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -164,17 +190,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int kv = a.kv_len ? a.kv_len[b] : a.T_max;
   const int qs = a.q_start ? a.q_start[b] : 0;
   const bool valid = kv >= 1 && kv <= a.T_max && qs >= 0;
-  const int n_qb = (a.S_q + kBQ - 1) / kBQ;
+  const int n_qb = (a.S_q + kKvBQ - 1) / kKvBQ;
   int qb_lo = 0, qb_hi = -1;
   if (valid && k0 < kv) {
     qb_hi = n_qb - 1;
     if (a.causal) {
       const long long first_q = (long long)k0 - qs;  // earliest row that can see key k0
-      qb_lo = first_q > 0 ? (int)(first_q / kBQ) : 0;
+      qb_lo = first_q > 0 ? (int)(first_q / kKvBQ) : 0;
       if (a.window > 0) {
         const long long k_last = min(k0 + kBK, kv) - 1;
         const long long last_q = k_last + a.window - 1 - qs;  // latest row that can see k_last
-        qb_hi = last_q < 0 ? -1 : (int)min((long long)qb_hi, last_q / kBQ);
+        qb_hi = last_q < 0 ? -1 : (int)min((long long)qb_hi, last_q / kKvBQ);
       }
     }
   }
@@ -183,12 +209,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(bar(kKvFull), 1);
-    for (int st = 0; st < 2; ++st) {
-      mbar_init(bar(kQFull + st), 1 + 32);  // the TMA arrival plus the producer warp's stat rows
+    for (int st = 0; st < kKvStages; ++st) {
+      mbar_init(bar(kQFull + st), 1 + 32);
       mbar_init(bar(kQEmpty + st), 1);
     }
-    mbar_init(bar(kKvS), 1);
-    mbar_init(bar(kKvP), 128);
+    for (int bf = 0; bf < 2; ++bf) {
+      mbar_init(bar(kKvS + bf), 1);
+      mbar_init(bar(kKvP + bf), 256);
+    }
     mbar_init(bar(kKvDone), 1);
     *abort = 0;
     fence_barrier_init();
@@ -214,35 +242,36 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&tmk);
       tma_prefetch_desc(&tmv);
       const int krow = (b * a.h_kv + g) * a.T_max + k0;
-      mbar_arrive_expect_tx(bar(kKvFull), 2 * C::kTile);
+      mbar_arrive_expect_tx(bar(kKvFull), 2 * C::kKTile);
       for (int ch = 0; ch < C::kNch; ++ch) {
         tma_load_2d(sK + ch * 128 * 128, &tmk, bar(kKvFull), ch * 64, krow);
         tma_load_2d(sV + ch * 128 * 128, &tmv, bar(kKvFull), ch * 64, krow);
       }
     }
-    int last[2] = {-1, -1};
+    int last[kKvStages];
+    for (int st = 0; st < kKvStages; ++st) last[st] = -1;
     for (int it = 0; it < n_it; ++it) {
-      const int st = it & 1, n = it >> 1;
+      const int st = it % kKvStages, n = it / kKvStages;
       int ok = 1;
       if (n > 0 && lane == 0) ok = wait_bar(bar(kQEmpty + st), (uint32_t)((n - 1) & 1), abort, a.err);
       if (!__shfl_sync(0xffffffffu, ok, 0)) break;
       const int h = head_of(it), qb = qblk_of(it);
       const int z = b * a.h_q + h;
       if (lane == 0) {
-        mbar_arrive_expect_tx(bar(kQFull + st), 2 * C::kTile);
+        mbar_arrive_expect_tx(bar(kQFull + st), 2 * C::kQTile);
         for (int ch = 0; ch < C::kNch; ++ch) {
-          tma_load_3d(sQ(st) + ch * 128 * 128, &tmq, bar(kQFull + st), ch * 64, qb * kBQ, z);
-          tma_load_3d(sDO(st) + ch * 128 * 128, &tmdo, bar(kQFull + st), ch * 64, qb * kBQ, z);
+          tma_load_3d(sQ(st) + ch * C::kQChunk, &tmq, bar(kQFull + st), ch * 64, qb * kKvBQ, z);
+          tma_load_3d(sDO(st) + ch * C::kQChunk, &tmdo, bar(kQFull + st), ch * 64, qb * kKvBQ, z);
         }
       }
-      float* sl = stat + st * 256;
+      float* sl = stat + st * 2 * kKvBQ;
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int c = lane * 4 + e;
-        const int qi = qb * kBQ + c;
+      for (int e = 0; e < kKvBQ / 32; ++e) {
+        const int c = lane * (kKvBQ / 32) + e;
+        const int qi = qb * kKvBQ + c;
         const long long row = (long long)z * a.S_q + qi;
         sl[c] = qi < a.S_q ? a.lse2[row] : INFINITY;
-        sl[128 + c] = qi < a.S_q ? a.drow[row] : 0.f;
+        sl[kKvBQ + c] = qi < a.S_q ? a.drow[row] : 0.f;
       }
       mbar_arrive(bar(kQFull + st));
       last[st] = n;
@@ -250,32 +279,47 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {  // drain (bounded): no copy may still land in shared memory at exit
       volatile int no_abort = 0;
       wait_bar(bar(kKvFull), 0, &no_abort, a.err);
-      for (int st = 0; st < 2; ++st)
+      for (int st = 0; st < kKvStages; ++st)
         if (last[st] >= 0) wait_bar(bar(kQFull + st), (uint32_t)(last[st] & 1), &no_abort, a.err);
     }
   } else if (warp == 1 && lane == 0 && n_it > 0) {
     // ------------------------------ MMA issuer ---------------------------------------------
-    constexpr uint32_t idesc_s = tc::idesc_bf16(128, kBQ, false);  // S^T, dP^T: M keys, N queries
-    constexpr uint32_t idesc_acc = tc::idesc_bf16(128, D, true);   // dV, dK: M keys, N = d_h
+    constexpr uint32_t idesc_s = tc::idesc_bf16(128, kKvBQ, false);  // S^T, dP^T: M keys, N queries
+    constexpr uint32_t idesc_acc = tc::idesc_bf16(128, D, true);     // dV, dK: M keys, N = d_h
+    auto issue_s = [&](int it) {  // S^T and dP^T of block `it` into buffer it & 1
+      const int st = it % kKvStages, bf = it & 1;
+#pragma unroll
+      for (int k = 0; k < D / 16; ++k)
+        tc::mma_ss(tmem + 64 * bf, desc_k(sK, k, 128 * 128), desc_k(sQ(st), k, C::kQChunk), idesc_s,
+                   k > 0 ? 1u : 0u);
+#pragma unroll
+      for (int k = 0; k < D / 16; ++k)
+        tc::mma_ss(tmem + 128 + 64 * bf, desc_k(sV, k, 128 * 128), desc_k(sDO(st), k, C::kQChunk), idesc_s,
+                   k > 0 ? 1u : 0u);
+      tc::commit(bar(kKvS + bf));
+    };
     bool ok = wait_bar(bar(kKvFull), 0, abort, a.err);
+    if (ok) ok = wait_bar(bar(kQFull), 0, abort, a.err);
+    if (ok) {
+      tc::fence_after_sync();
+      issue_s(0);
+    }
     for (int it = 0; it < n_it && ok; ++it) {
-      const int st = it & 1;
-      if (!wait_bar(bar(kQFull + st), (uint32_t)((it >> 1) & 1), abort, a.err)) break;
+      const int st = it % kKvStages, bf = it & 1;
+      if (it + 1 < n_it) {  // next block's scores overlap this block's elementwise pass
+        const int st1 = (it + 1) % kKvStages;
+        if (!wait_bar(bar(kQFull + st1), (uint32_t)(((it + 1) / kKvStages) & 1), abort, a.err)) break;
+        tc::fence_after_sync();
+        issue_s(it + 1);
+      }
+      if (!wait_bar(bar(kKvP + bf), (uint32_t)((it >> 1) & 1), abort, a.err)) break;
       tc::fence_after_sync();
 #pragma unroll
-      for (int k = 0; k < D / 16; ++k)
-        tc::mma_ss(tmem + kColS, desc_kmajor(sK, k), desc_kmajor(sQ(st), k), idesc_s, k > 0 ? 1u : 0u);
-#pragma unroll
-      for (int k = 0; k < D / 16; ++k)
-        tc::mma_ss(tmem + kColDP, desc_kmajor(sV, k), desc_kmajor(sDO(st), k), idesc_s, k > 0 ? 1u : 0u);
-      tc::commit(bar(kKvS));
-      if (!wait_bar(bar(kKvP), (uint32_t)(it & 1), abort, a.err)) break;
-      tc::fence_after_sync();
-#pragma unroll
-      for (int kk = 0; kk < kBQ / 16; ++kk) {
+      for (int kk = 0; kk < kKvBQ / 16; ++kk) {
         const uint32_t acc = (it > 0 || kk > 0) ? 1u : 0u;
-        tc::mma_ts(tmem + kColAcc0, tmem + kColS + kk * 8, desc_mnmajor(sDO(st), kk), idesc_acc, acc);
-        tc::mma_ts(tmem + kColAcc0 + D, tmem + kColDP + kk * 8, desc_mnmajor(sQ(st), kk), idesc_acc, acc);
+        const uint32_t acol = (uint32_t)(64 * bf + (kk >> 1) * 32 + (kk & 1) * 8);  // half kk/2
+        tc::mma_ts(tmem + kColAcc0, tmem + acol, desc_mn(sDO(st), kk, C::kQChunk), idesc_acc, acc);
+        tc::mma_ts(tmem + kColAcc0 + D, tmem + 128 + acol, desc_mn(sQ(st), kk, C::kQChunk), idesc_acc, acc);
       }
       tc::commit(bar(kQEmpty + st));
     }
@@ -283,87 +327,76 @@ __global__ void __launch_bounds__(kThreads, 1)
     volatile int no_abort = 0;
     wait_bar(bar(kKvDone), 0, &no_abort, a.err);
   } else if (warp >= 2) {
-    // ------------------------------ elementwise: one key row per thread --------------------
+    // ------------------------------ elementwise: one key row, 32 queries per thread ---------
     const int quarter = warp & 3;
+    const int half = (warp - 2) >> 2;     // which 32 queries of each 64-query block
     const int row = quarter * 32 + lane;  // TMEM lane = key k0 + row
     const int key = k0 + row;
     const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
     bool ok = true;
     for (int it = 0; it < n_it; ++it) {
-      const int st = it & 1;
-      if (ok) ok = wait_bar(bar(kKvS), (uint32_t)(it & 1), abort, a.err);
+      const int st = it % kKvStages, bf = it & 1;
+      if (ok) ok = wait_bar(bar(kKvS + bf), (uint32_t)((it >> 1) & 1), abort, a.err);
+      if (ok) ok = wait_bar(bar(kQFull + st), (uint32_t)((it / kKvStages) & 1), abort, a.err);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
-      // the stage's statistics: written by the producer warp before its arrivals on the stage's
-      // full barrier (already complete here; waiting on it orders the reads after those writes)
-      if (ok) ok = wait_bar(bar(kQFull + st), (uint32_t)((it >> 1) & 1), abort, a.err);
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) break;
-      const float* sl = stat + st * 256;
+      const float* sl = stat + st * 2 * kKvBQ + half * 32;
       const int qb = qblk_of(it);
-      const long long pos0 = (long long)qs + qb * kBQ;  // position of the block's first row
-      const bool need_mask = k0 + kBK > kv || qb * kBQ + kBQ > a.S_q ||
+      const int col0 = qb * kKvBQ + half * 32;        // first query (index into S_q) of this half
+      const long long pos0 = (long long)qs + col0;
+      const bool need_mask = k0 + kBK > kv || col0 + 32 > a.S_q ||
                              (a.causal && (long long)k0 + kBK - 1 > pos0) ||
-                             (a.window > 0 && (long long)k0 <= pos0 + kBQ - 1 - a.window);
+                             (a.window > 0 && (long long)k0 <= pos0 + 31 - a.window);
       tc::fence_after_sync();
-#pragma unroll 1
-      for (int c = 0; c < kBQ / 32; ++c) {
-        uint32_t sv[32], dv[32];
-        tc::ld32(lane_addr + kColS + c * 32, sv);
-        tc::ld32(lane_addr + kColDP + c * 32, dv);
-        tc::wait_ld();
-        uint32_t pp[16], pd[16];
+      uint32_t sv[32], dv[32];
+      tc::ld32(lane_addr + 64 * bf + 32 * half, sv);
+      tc::ld32(lane_addr + 128 + 64 * bf + 32 * half, dv);
+      tc::wait_ld();
+      uint32_t pp[16], pd[16];
 #pragma unroll
-        for (int x = 0; x < 32; x += 2) {
-          float p2[2], d2[2];
+      for (int x = 0; x < 32; x += 2) {
+        float p2[2], d2[2];
 #pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int col = c * 32 + x + e;
-            const float sc = __uint_as_float(sv[x + e]);
-            float p = fast_exp2(fmaf(sc, a.sl2, -sl[col]));
-            float ds = p * (__uint_as_float(dv[x + e]) - sl[128 + col]);
-            if (need_mask && !(qb * kBQ + col < a.S_q && visible(key, pos0 + col, kv, a.causal, a.window))) {
-              p = 0.f;
-              ds = 0.f;
-            }
-            p2[e] = p;
-            d2[e] = ds;
+        for (int e = 0; e < 2; ++e) {
+          const int c = x + e;
+          float p = fast_exp2(fmaf(__uint_as_float(sv[c]), a.sl2, -sl[c]));
+          float ds = p * (__uint_as_float(dv[c]) - sl[kKvBQ + c]);
+          if (need_mask && !(col0 + c < a.S_q && visible(key, pos0 + c, kv, a.causal, a.window))) {
+            p = 0.f;
+            ds = 0.f;
           }
-          pp[x / 2] = pack_bf16x2(p2[0], p2[1]);
-          pd[x / 2] = pack_bf16x2(d2[0], d2[1]);
+          p2[e] = p;
+          d2[e] = ds;
         }
-        tc::st16(lane_addr + kColS + c * 16, pp);   // P^T (bf16 pairs) over S^T's first columns
-        tc::st16(lane_addr + kColDP + c * 16, pd);  // dS^T over dP^T's first columns
+        pp[x / 2] = pack_bf16x2(p2[0], p2[1]);
+        pd[x / 2] = pack_bf16x2(d2[0], d2[1]);
       }
+      tc::st16(lane_addr + 64 * bf + 32 * half, pp);        // P^T over this half's first columns
+      tc::st16(lane_addr + 128 + 64 * bf + 32 * half, pd);  // dS^T likewise in dP^T
       tc::wait_st();
       tc::fence_before_sync();
-      mbar_arrive(bar(kKvP));
+      mbar_arrive(bar(kKvP + bf));
     }
-    // ---- epilogue: dV and scale * dK rows -> bf16 (rows past kv_len hold zeros)
+    // ---- epilogue: dV and scale * dK rows -> bf16; each half writes half of the columns
     bool have = n_it > 0 && ok;
     if (have) {
       have = wait_bar(bar(kKvDone), 0, abort, a.err);
       have = __all_sync(0xffffffffu, have);
       if (have) tc::fence_after_sync();
     }
-    if (key < a.T_max) {
-      const long long orow = ((long long)b * a.h_kv + g) * a.T_max + key;
-      uint4* dvo = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.dv) + orow * D);
-      uint4* dko = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.dk) + orow * D);
-      if (!have) {
-        for (int v = 0; v < D / 8; ++v) {
+    const long long orow = ((long long)b * a.h_kv + g) * a.T_max + key;
+    uint4* dvo = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.dv) + orow * D);
+    uint4* dko = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.dk) + orow * D);
+    const bool store = key < a.T_max;
+    if (!have) {
+      if (store)
+        for (int v = half * (D / 16); v < (half + 1) * (D / 16); ++v) {
           dvo[v] = make_uint4(0u, 0u, 0u, 0u);
           dko[v] = make_uint4(0u, 0u, 0u, 0u);
         }
-      }
-    }
-    if (have) {
-      const bool store = key < a.T_max;
-      const long long orow = ((long long)b * a.h_kv + g) * a.T_max + key;
-      uint4* dvo = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.dv) + orow * D);
-      uint4* dko = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.dk) + orow * D);
+    } else {
 #pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
+      for (int c = half * (D / 64); c < (half + 1) * (D / 64); ++c) {  // 32-column chunks
         uint32_t v[32], k[32];
         tc::ld32(lane_addr + kColAcc0 + c * 32, v);
         tc::ld32(lane_addr + kColAcc0 + D + c * 32, k);
@@ -392,24 +425,38 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-
-// Shared memory of the dq kernel: the tile's Q and dO rows, a two-stage ring of K and V blocks.
+// ---- dq: query-stationary dQ on the forward's tiles -------------------------------------------
+// K/V blocks of 64 keys, so S and dP are double-buffered in TMEM next to the dQ accumulator: the
+// MMA warp issues block j+1's S / dP while eight warps (two per lane quarter, one per 32-key half)
+// turn block j into dS. TMEM: S[buf] at 64 buf, dP[buf] at 128 + 64 buf, dQ at 256.
+constexpr int kQBK = 64;
+constexpr int kQStages = 3;
+constexpr int kQThreads = 320;
 template <int D>
 struct QCfg {
   static constexpr int kNch = D / 64;
-  static constexpr int kTile = kNch * 128 * 128;
+  static constexpr int kQTile = kNch * 128 * 128;  // Q or dO: 128 rows
+  static constexpr int kKChunk = kQBK * 128;       // 64 rows x 128 B
+  static constexpr int kKTile = kNch * kKChunk;    // K or V: 64 rows
   static constexpr int kOffQ = 0;
-  static constexpr int kOffDO = kTile;
-  static constexpr int kOffK = 2 * kTile;  // + stage * 2 * kTile
-  static constexpr int kOffV = 3 * kTile;  // + stage * 2 * kTile
-  static constexpr int kOffBar = 6 * kTile;
+  static constexpr int kOffDO = kQTile;
+  static constexpr int kOffK = 2 * kQTile;  // + stage * 2 * kKTile (K, then V)
+  static constexpr int kOffBar = kOffK + kQStages * 2 * kKTile;
   static constexpr int kSmem = (kOffBar + 256 + 1024) > 120 * 1024 ? kOffBar + 256 + 1024 : 120 * 1024;
   static_assert(kSmem <= 227 * 1024, "shared memory budget");
 };
-enum { kQdQ = 0, kQKvFull = 1, kQKvEmpty = 3, kQS = 5, kQP = 6, kQDone = 7, kQBars = 8 };
+enum {
+  kQdQ = 0,
+  kQKvFull = 1,                        // + stage
+  kQKvEmpty = kQKvFull + kQStages,     // + stage
+  kQS = kQKvEmpty + kQStages,          // + buffer
+  kQP = kQS + 2,                       // + buffer (256 arrivals)
+  kQDone = kQP + 2,
+  kQBars = kQDone + 1
+};
 
 template <int D>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kQThreads, 1)
     dq_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmdo,
               const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
               BArgs a) {
@@ -421,8 +468,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kQBars);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const uint32_t sQ = smem_u32(smem + C::kOffQ), sDO = smem_u32(smem + C::kOffDO);
-  auto sK = [&](int st) { return smem_u32(smem + C::kOffK + st * 2 * C::kTile); };
-  auto sV = [&](int st) { return smem_u32(smem + C::kOffV + st * 2 * C::kTile); };
+  auto sK = [&](int st) { return smem_u32(smem + C::kOffK + st * 2 * C::kKTile); };
+  auto sV = [&](int st) { return smem_u32(smem + C::kOffK + st * 2 * C::kKTile + C::kKTile); };
   auto bar = [&](int i) { return smem_u32(&bars[i]); };
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -440,15 +487,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   const bool valid = kv >= 1 && kv <= a.T_max && qs >= 0;
   const long long pos_min = (long long)qs + q0;
   const long long pos_max = (long long)qs + min(q0 + a.P, a.S_q) - 1;
-  int j0 = 0, nb = 0;
+  int j0 = 0, nb = 0;  // 64-key blocks j0 .. j0 + nb - 1
   if (valid) {
-    int end = (kv + kBK - 1) / kBK;
+    int end = (kv + kQBK - 1) / kQBK;
     if (a.causal) {
       const long long last_key = pos_max < kv - 1 ? pos_max : (long long)(kv - 1);
-      end = (int)(last_key / kBK) + 1;
+      end = (int)(last_key / kQBK) + 1;
       if (a.window > 0) {
         const long long lo = pos_min - a.window + 1;
-        if (lo > 0) j0 = (int)(lo / kBK);
+        if (lo > 0) j0 = (int)(lo / kQBK);
       }
     }
     nb = end > j0 ? end - j0 : 0;
@@ -456,12 +503,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(bar(kQdQ), 1);
-    for (int st = 0; st < 2; ++st) {
+    for (int st = 0; st < kQStages; ++st) {
       mbar_init(bar(kQKvFull + st), 1);
       mbar_init(bar(kQKvEmpty + st), 1);
     }
-    mbar_init(bar(kQS), 1);
-    mbar_init(bar(kQP), 128);
+    for (int bf = 0; bf < 2; ++bf) {
+      mbar_init(bar(kQS + bf), 1);
+      mbar_init(bar(kQP + bf), 256);
+    }
     mbar_init(bar(kQDone), 1);
     *abort = 0;
     fence_barrier_init();
@@ -488,51 +537,66 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_load_3d(sQ + ch * 128 * 128, &tmq, bar(kQdQ), ch * 64, q0, zq);
       tma_load_3d(sDO + ch * 128 * 128, &tmdo, bar(kQdQ), ch * 64, q0, zq);
     }
-    int last[2] = {-1, -1};
+    int last[kQStages];
+    for (int st = 0; st < kQStages; ++st) last[st] = -1;
     for (int j = 0; j < nb; ++j) {
-      const int st = j & 1, n = j >> 1;
+      const int st = j % kQStages, n = j / kQStages;
       if (n > 0 && !wait_bar(bar(kQKvEmpty + st), (uint32_t)((n - 1) & 1), abort, a.err)) break;
-      mbar_arrive_expect_tx(bar(kQKvFull + st), 2 * C::kTile);
+      mbar_arrive_expect_tx(bar(kQKvFull + st), 2 * C::kKTile);
       for (int ch = 0; ch < C::kNch; ++ch) {
-        tma_load_2d(sK(st) + ch * 128 * 128, &tmk, bar(kQKvFull + st), ch * 64, row0 + (j0 + j) * kBK);
-        tma_load_2d(sV(st) + ch * 128 * 128, &tmv, bar(kQKvFull + st), ch * 64, row0 + (j0 + j) * kBK);
+        tma_load_2d(sK(st) + ch * C::kKChunk, &tmk, bar(kQKvFull + st), ch * 64, row0 + (j0 + j) * kQBK);
+        tma_load_2d(sV(st) + ch * C::kKChunk, &tmv, bar(kQKvFull + st), ch * 64, row0 + (j0 + j) * kQBK);
       }
       last[st] = n;
     }
     volatile int no_abort = 0;  // drain (bounded)
     wait_bar(bar(kQdQ), 0, &no_abort, a.err);
-    for (int st = 0; st < 2; ++st)
+    for (int st = 0; st < kQStages; ++st)
       if (last[st] >= 0) wait_bar(bar(kQKvFull + st), (uint32_t)(last[st] & 1), &no_abort, a.err);
   } else if (warp == 1 && lane == 0 && nb > 0) {
     // ------------------------------ MMA issuer ---------------------------------------------
-    constexpr uint32_t idesc_s = tc::idesc_bf16(128, kBK, false);  // S, dP: M rows, N keys
-    constexpr uint32_t idesc_acc = tc::idesc_bf16(128, D, true);   // dQ: M rows, N = d_h
+    constexpr uint32_t idesc_s = tc::idesc_bf16(128, kQBK, false);  // S, dP: M rows, N keys
+    constexpr uint32_t idesc_acc = tc::idesc_bf16(128, D, true);    // dQ: M rows, N = d_h
+    auto issue_s = [&](int j) {
+      const int st = j % kQStages, bf = j & 1;
+#pragma unroll
+      for (int k = 0; k < D / 16; ++k)
+        tc::mma_ss(tmem + 64 * bf, desc_k(sQ, k, 128 * 128), desc_k(sK(st), k, C::kKChunk), idesc_s, k > 0 ? 1u : 0u);
+#pragma unroll
+      for (int k = 0; k < D / 16; ++k)
+        tc::mma_ss(tmem + 128 + 64 * bf, desc_k(sDO, k, 128 * 128), desc_k(sV(st), k, C::kKChunk), idesc_s,
+                   k > 0 ? 1u : 0u);
+      tc::commit(bar(kQS + bf));
+    };
     bool ok = wait_bar(bar(kQdQ), 0, abort, a.err);
+    if (ok) ok = wait_bar(bar(kQKvFull), 0, abort, a.err);
+    if (ok) {
+      tc::fence_after_sync();
+      issue_s(0);
+    }
     for (int j = 0; j < nb && ok; ++j) {
-      const int st = j & 1;
-      if (!wait_bar(bar(kQKvFull + st), (uint32_t)((j >> 1) & 1), abort, a.err)) break;
+      const int st = j % kQStages, bf = j & 1;
+      if (j + 1 < nb) {
+        if (!wait_bar(bar(kQKvFull + (j + 1) % kQStages), (uint32_t)(((j + 1) / kQStages) & 1), abort, a.err)) break;
+        tc::fence_after_sync();
+        issue_s(j + 1);
+      }
+      if (!wait_bar(bar(kQP + bf), (uint32_t)((j >> 1) & 1), abort, a.err)) break;
       tc::fence_after_sync();
 #pragma unroll
-      for (int k = 0; k < D / 16; ++k)
-        tc::mma_ss(tmem + kColS, desc_kmajor(sQ, k), desc_kmajor(sK(st), k), idesc_s, k > 0 ? 1u : 0u);
-#pragma unroll
-      for (int k = 0; k < D / 16; ++k)
-        tc::mma_ss(tmem + kColDP, desc_kmajor(sDO, k), desc_kmajor(sV(st), k), idesc_s, k > 0 ? 1u : 0u);
-      tc::commit(bar(kQS));
-      if (!wait_bar(bar(kQP), (uint32_t)(j & 1), abort, a.err)) break;
-      tc::fence_after_sync();
-#pragma unroll
-      for (int kk = 0; kk < kBK / 16; ++kk)
-        tc::mma_ts(tmem + kColAcc0, tmem + kColS + kk * 8, desc_mnmajor(sK(st), kk), idesc_acc,
-                   (j > 0 || kk > 0) ? 1u : 0u);
+      for (int kk = 0; kk < kQBK / 16; ++kk)
+        tc::mma_ts(tmem + kColAcc0, tmem + (uint32_t)(64 * bf + (kk >> 1) * 32 + (kk & 1) * 8),
+                   desc_mn(sK(st), kk, C::kKChunk), idesc_acc, (j > 0 || kk > 0) ? 1u : 0u);
       tc::commit(bar(kQKvEmpty + st));
     }
     tc::commit(bar(kQDone));
     volatile int no_abort = 0;
     wait_bar(bar(kQDone), 0, &no_abort, a.err);
   } else if (warp >= 2) {
-    // ------------------------------ elementwise: one query row per thread ------------------
+    // ------------------------------ elementwise: one query row, 32 keys per thread ----------
     const int quarter = warp & 3;
+    const int half = (warp - 2) >> 2;     // which 32 keys of each 64-key block
+    const int et = (warp - 2) * 32 + lane;  // 0..255, for the K-row zeroing
     const int row = quarter * 32 + lane;  // TMEM lane = tile row (head h, position p)
     const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
     const int h = row / a.P, p = row - h * a.P;
@@ -545,47 +609,45 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float dr = store_row ? a.drow[srow] : 0.f;
     bool ok = true;
     for (int j = 0; j < nb; ++j) {
-      const int st = j & 1;
-      if (ok) ok = wait_bar(bar(kQS), (uint32_t)(j & 1), abort, a.err);
+      const int st = j % kQStages, bf = j & 1;
+      if (ok) ok = wait_bar(bar(kQS + bf), (uint32_t)((j >> 1) & 1), abort, a.err);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
-      const int key0 = (j0 + j) * kBK;
-      const bool need_mask = (a.causal && (long long)key0 + kBK - 1 > pos_min) || key0 + kBK > kv ||
+      const int blk0 = (j0 + j) * kQBK;
+      const int key0 = blk0 + half * 32;  // first key of this half
+      const bool need_mask = (a.causal && (long long)key0 + 31 > pos_min) || key0 + 32 > kv ||
                              (a.window > 0 && (long long)key0 <= pos_max - a.window);
       tc::fence_after_sync();
-#pragma unroll 1
-      for (int c = 0; c < kBK / 32; ++c) {
-        uint32_t sv[32], dv[32];
-        tc::ld32(lane_addr + kColS + c * 32, sv);
-        tc::ld32(lane_addr + kColDP + c * 32, dv);
-        tc::wait_ld();
-        uint32_t pd[16];
+      uint32_t sv[32], dv[32];
+      tc::ld32(lane_addr + 64 * bf + 32 * half, sv);
+      tc::ld32(lane_addr + 128 + 64 * bf + 32 * half, dv);
+      tc::wait_ld();
+      uint32_t pd[16];
 #pragma unroll
-        for (int x = 0; x < 32; x += 2) {
-          float d2[2];
+      for (int x = 0; x < 32; x += 2) {
+        float d2[2];
 #pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int key = key0 + c * 32 + x + e;
-            const float pr = fast_exp2(fmaf(__uint_as_float(sv[x + e]), a.sl2, -lse2));
-            float ds = pr * (__uint_as_float(dv[x + e]) - dr);
-            if (need_mask && !visible(key, pos, kv, a.causal, a.window)) ds = 0.f;
-            d2[e] = ds;
-          }
-          pd[x / 2] = pack_bf16x2(d2[0], d2[1]);
+        for (int e = 0; e < 2; ++e) {
+          const int key = key0 + x + e;
+          const float pr = fast_exp2(fmaf(__uint_as_float(sv[x + e]), a.sl2, -lse2));
+          float ds = pr * (__uint_as_float(dv[x + e]) - dr);
+          if (need_mask && !visible(key, pos, kv, a.causal, a.window)) ds = 0.f;
+          d2[e] = ds;
         }
-        tc::st16(lane_addr + kColS + c * 16, pd);  // dS (bf16 pairs) over S's first columns
+        pd[x / 2] = pack_bf16x2(d2[0], d2[1]);
       }
-      // K rows that no row of the tile may see -- past kv_len (last block), below every row's
-      // window (first block) -- get dS = 0 but may hold anything: zero them before dQ += dS K
-      const bool zero_tail = j == nb - 1 && key0 + kBK > kv;
-      const bool zero_head = j == 0 && a.window > 0 && (long long)key0 < pos_min - a.window + 1;
-      if (zero_tail || zero_head) {
-        const long long key = (long long)key0 + row;  // this thread's K row in the block
+      tc::st16(lane_addr + 64 * bf + 32 * half, pd);  // dS over this half's first columns of S
+      // K rows no row of the tile may see (past kv_len: last block; below every row's window:
+      // first block) get dS = 0 but may hold anything: zero them before dQ += dS K
+      const bool zero_tail = j == nb - 1 && blk0 + kQBK > kv;
+      const bool zero_head = j == 0 && a.window > 0 && (long long)blk0 < pos_min - a.window + 1;
+      if ((zero_tail || zero_head) && et < kQBK) {
+        const long long key = (long long)blk0 + et;  // this thread's K row of the block
         if ((zero_tail && key >= kv) || (zero_head && key <= pos_min - a.window)) {
           for (int ch = 0; ch < C::kNch; ++ch)
 #pragma unroll
             for (int k = 0; k < 8; ++k) {
-              const uint32_t addr = sK(st) + ch * 128 * 128 + row * 128 + k * 16;
+              const uint32_t addr = sK(st) + ch * C::kKChunk + et * 128 + k * 16;
               asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(addr), "r"(0u) : "memory");
             }
         }
@@ -593,9 +655,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc::wait_st();
       tc::fence_before_sync();
-      mbar_arrive(bar(kQP));
+      mbar_arrive(bar(kQP + bf));
     }
-    // ---- epilogue: scale * dQ -> bf16
+    // ---- epilogue: scale * dQ -> bf16; each half writes half of the columns
     bool have = nb > 0 && ok;
     if (have) {
       have = wait_bar(bar(kQDone), 0, abort, a.err);
@@ -605,7 +667,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint4* out = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.dq) + srow * D);
     if (have) {
 #pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
+      for (int c = half * (D / 64); c < (half + 1) * (D / 64); ++c) {
         uint32_t v[32];
         tc::ld32(lane_addr + kColAcc0 + c * 32, v);
         tc::wait_ld();
@@ -619,7 +681,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     } else if (store_row) {
-      for (int v = 0; v < D / 8; ++v) out[v] = make_uint4(0u, 0u, 0u, 0u);
+      for (int v = half * (D / 16); v < (half + 1) * (D / 16); ++v) out[v] = make_uint4(0u, 0u, 0u, 0u);
     }
   }
   tc::fence_before_sync();
@@ -629,7 +691,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc::tmem_dealloc(tmem, kTmemCols);
   }
 }
-
 
 template <int D>
 cudaError_t launch_typed(const BArgs& p, const CUtensorMap* tm, cudaStream_t s) {
@@ -647,10 +708,10 @@ cudaError_t launch_typed(const BArgs& p, const CUtensorMap* tm, cudaStream_t s) 
   const long long n1 = (long long)p.n_kb * p.B * p.h_kv;
   const long long n2 = (long long)p.n_qt * p.B * p.h_kv * p.hblocks;
   if (n1 > 0x7fffffffLL || n2 > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-  dkdv_kernel<D><<<(unsigned)n1, kThreads, KvCfg<D>::kSmem, s>>>(tm[0], tm[1], tm[2], tm[3], p);
+  dkdv_kernel<D><<<(unsigned)n1, kKvThreads, KvCfg<D>::kSmem, s>>>(tm[0], tm[1], tm[2], tm[3], p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  dq_kernel<D><<<(unsigned)n2, kThreads, QCfg<D>::kSmem, s>>>(tm[4], tm[5], tm[2], tm[3], p);
+  dq_kernel<D><<<(unsigned)n2, kQThreads, QCfg<D>::kSmem, s>>>(tm[4], tm[5], tm[6], tm[7], p);
   return cudaGetLastError();
 }
 

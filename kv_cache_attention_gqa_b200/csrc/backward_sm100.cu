@@ -428,7 +428,9 @@ __global__ void __launch_bounds__(kKvThreads, 1)
 // ---- dq: query-stationary dQ on the forward's tiles -------------------------------------------
 // K/V blocks of 64 keys, so S and dP are double-buffered in TMEM next to the dQ accumulator: the
 // MMA warp issues block j+1's S / dP while eight warps (two per lane quarter, one per 32-key half)
-// turn block j into dS. TMEM: S[buf] at 64 buf, dP[buf] at 128 + 64 buf, dQ at 256.
+// turn block j into dS. The tile's Q and dO rows are copied into TMEM once and are the A operands
+// of S = Q K^T and dP = dO V^T, so those MMAs read only K / V from shared memory.
+// TMEM: S[buf] at 64 buf, dP[buf] at 128 + 64 buf, dQ at 256, Q at 256 + D, dO at 256 + 3D/2.
 constexpr int kQBK = 64;
 constexpr int kQStages = 3;
 constexpr int kQThreads = 320;
@@ -447,7 +449,8 @@ struct QCfg {
 };
 enum {
   kQdQ = 0,
-  kQKvFull = 1,                        // + stage
+  kQT = 1,                             // Q, dO copied into TMEM (256 arrivals)
+  kQKvFull = 2,                        // + stage
   kQKvEmpty = kQKvFull + kQStages,     // + stage
   kQS = kQKvEmpty + kQStages,          // + buffer
   kQP = kQS + 2,                       // + buffer (256 arrivals)
@@ -503,6 +506,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(bar(kQdQ), 1);
+    mbar_init(bar(kQT), 256);
     for (int st = 0; st < kQStages; ++st) {
       mbar_init(bar(kQKvFull + st), 1);
       mbar_init(bar(kQKvEmpty + st), 1);
@@ -557,18 +561,19 @@ __global__ void __launch_bounds__(kQThreads, 1)
     // ------------------------------ MMA issuer ---------------------------------------------
     constexpr uint32_t idesc_s = tc::idesc_bf16(128, kQBK, false);  // S, dP: M rows, N keys
     constexpr uint32_t idesc_acc = tc::idesc_bf16(128, D, true);    // dQ: M rows, N = d_h
+    constexpr uint32_t kColQ = kColAcc0 + D, kColDO = kColAcc0 + D + D / 2;
     auto issue_s = [&](int j) {
       const int st = j % kQStages, bf = j & 1;
 #pragma unroll
       for (int k = 0; k < D / 16; ++k)
-        tc::mma_ss(tmem + 64 * bf, desc_k(sQ, k, 128 * 128), desc_k(sK(st), k, C::kKChunk), idesc_s, k > 0 ? 1u : 0u);
+        tc::mma_ts(tmem + 64 * bf, tmem + kColQ + k * 8, desc_k(sK(st), k, C::kKChunk), idesc_s, k > 0 ? 1u : 0u);
 #pragma unroll
       for (int k = 0; k < D / 16; ++k)
-        tc::mma_ss(tmem + 128 + 64 * bf, desc_k(sDO, k, 128 * 128), desc_k(sV(st), k, C::kKChunk), idesc_s,
+        tc::mma_ts(tmem + 128 + 64 * bf, tmem + kColDO + k * 8, desc_k(sV(st), k, C::kKChunk), idesc_s,
                    k > 0 ? 1u : 0u);
       tc::commit(bar(kQS + bf));
     };
-    bool ok = wait_bar(bar(kQdQ), 0, abort, a.err);
+    bool ok = wait_bar(bar(kQT), 0, abort, a.err);
     if (ok) ok = wait_bar(bar(kQKvFull), 0, abort, a.err);
     if (ok) {
       tc::fence_after_sync();
@@ -607,7 +612,28 @@ __global__ void __launch_bounds__(kQThreads, 1)
     const long long pos = (long long)qs + qi;
     const float lse2 = store_row ? a.lse2[srow] : INFINITY;
     const float dr = store_row ? a.drow[srow] : 0.f;
-    bool ok = true;
+    // this row of Q (half 0) or dO (half 1): shared memory (128-byte swizzled) -> TMEM
+    bool ok = nb > 0 && wait_bar(bar(kQdQ), 0, abort, a.err);
+    ok = __all_sync(0xffffffffu, ok);
+    if (ok) {
+      const uint32_t src = half == 0 ? sQ : sDO;
+      const uint32_t dst = lane_addr + kColAcc0 + D + half * (D / 2);
+#pragma unroll
+      for (int ch = 0; ch < C::kNch; ++ch) {
+        uint32_t r[32];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const uint32_t addr = swz128(src + ch * 128 * 128, row, k);
+          asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                       : "=r"(r[4 * k]), "=r"(r[4 * k + 1]), "=r"(r[4 * k + 2]), "=r"(r[4 * k + 3])
+                       : "r"(addr));
+        }
+        tc::st32(dst + ch * 32, r);
+      }
+      tc::wait_st();
+    }
+    tc::fence_before_sync();
+    if (nb > 0) mbar_arrive(bar(kQT));
     for (int j = 0; j < nb; ++j) {
       const int st = j % kQStages, bf = j & 1;
       if (ok) ok = wait_bar(bar(kQS + bf), (uint32_t)((j >> 1) & 1), abort, a.err);

@@ -135,3 +135,43 @@ def test_paged_host_side_argument_errors(lib):
     assert lib.kv_append_paged(fake, fake, fake, fake, fake, fake, 1, 2, 1, 0, 16, 4, 64, 0, s) == 1
     assert lib.kv_append_paged(fake, fake, fake, fake, fake, fake, 1, 2, 65, 8, 16, 4, 64, 0, s) == 1
     assert lib.kv_append_paged(fake, fake, fake, fake, fake, fake, 1, 2, 1, 8, 16, 4, 64, 7, s) == 1
+
+
+def test_mla_and_backward_host_side_argument_errors(lib):
+    P = ctypes.c_void_p
+    fake = P(0x1000)
+    null = None
+    s = None
+    # gqa_mla_decode(q, cache, o, lse, kv_len, q_pos, B, h_q, T_max, d_qk, d_v, scale, dtype, ws, bytes, splits, stream)
+    mla = lambda *a: lib.gqa_mla_decode(*a)  # noqa: E731
+    assert mla(null, fake, fake, null, null, null, 2, 16, 64, 576, 512, 0.07, 0, fake, 1 << 20, 1, s) == 1
+    assert mla(fake, fake, fake, null, null, null, 2, 16, 64, 512, 576, 0.07, 0, fake, 1 << 20, 1, s) == 1  # d_v > d_qk
+    assert mla(fake, fake, fake, null, null, null, 2, 16, 64, 576, 512, -1.0, 0, fake, 1 << 20, 1, s) == 1
+    assert mla(fake, fake, fake, null, null, null, 2, 16, 64, 576, 256, 0.07, 0, fake, 1 << 20, 1, s) == 2  # bf16 widths
+    assert mla(fake, fake, fake, null, null, null, 2, 16, 64, 800, 512, 0.07, 1, fake, 1 << 20, 1, s) == 2  # fp32 limit
+    assert mla(fake, fake, fake, null, null, null, 2, 16, 64, 576, 512, 0.07, 0, null, 1 << 20, 1, s) == 5
+    assert mla(fake, fake, fake, null, null, null, 2, 16, 64, 576, 512, 0.07, 0, fake, 16, 1, s) == 5
+    assert lib.gqa_mla_decode_workspace_size(0, 16, 64, 512, 0, 1) == 0
+    assert lib.gqa_mla_decode_workspace_size(2, 16, 64, 512, 0, 4) > 0
+    # gqa_prefill_backward(q, k, v, o, dO, lse, dq, dk, dv, q_start, kv_len, B, h_q, h_kv, S_q, T_max, d_h,
+    #                      scale, causal, window, dtype, ws, bytes, stream)
+    ok = [fake] * 9 + [null, null, 1, 4, 2, 8, 8, 64, 0.125, 1, 0, 0, fake, 1 << 20, s]
+
+    def bwd(**kw):
+        a = list(ok)
+        idx = {"lse": 5, "dq": 6, "h_kv": 13, "d_h": 16, "causal": 18, "window": 19, "ws": 21, "bytes": 22}
+        for k, v in kw.items():
+            a[idx[k]] = v
+        return lib.gqa_prefill_backward(*a)
+
+    assert bwd(lse=null) == 1
+    assert bwd(dq=null) == 1
+    assert bwd(h_kv=3) == 1
+    assert bwd(causal=0, window=4) == 1
+    assert bwd(window=-2) == 1
+    assert bwd(d_h=96) == 2
+    assert bwd(ws=null) == 5
+    assert bwd(ws=P(0x1010)) == 5  # misaligned
+    assert bwd(bytes=8) == 5
+    assert lib.gqa_prefill_backward_workspace_size(1, 4, 8) == 2 * 256
+    assert lib.gqa_prefill_backward_workspace_size(0, 4, 8) == 0

@@ -80,6 +80,32 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile
   }
 }
 
+// Packed fp32x2 arithmetic (sm_100): two lanes of work per instruction in the elementwise passes.
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "mov.b64 rc, {%6, %7};\n\tfma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+
 __device__ __forceinline__ bool visible(long long key, long long pos, int kv, int causal, int window) {
   return key < kv && (!causal || key <= pos) && (window == 0 || key > pos - window);
 }
@@ -270,8 +296,8 @@ __global__ void __launch_bounds__(kKvThreads, 1)
         const int c = lane * (kKvBQ / 32) + e;
         const int qi = qb * kKvBQ + c;
         const long long row = (long long)z * a.S_q + qi;
-        sl[c] = qi < a.S_q ? a.lse2[row] : INFINITY;
-        sl[kKvBQ + c] = qi < a.S_q ? a.drow[row] : 0.f;
+        sl[c] = qi < a.S_q ? -a.lse2[row] : -INFINITY;  // stored negated for the fused FMAs
+        sl[kKvBQ + c] = qi < a.S_q ? -a.drow[row] : 0.f;
       }
       mbar_arrive(bar(kQFull + st));
       last[st] = n;
@@ -353,23 +379,20 @@ __global__ void __launch_bounds__(kKvThreads, 1)
       tc::ld32(lane_addr + 128 + 64 * bf + 32 * half, dv);
       tc::wait_ld();
       uint32_t pp[16], pd[16];
+      const float2 c2 = make_float2(a.sl2, a.sl2);
 #pragma unroll
       for (int x = 0; x < 32; x += 2) {
-        float p2[2], d2[2];
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int c = x + e;
-          float p = fast_exp2(fmaf(__uint_as_float(sv[c]), a.sl2, -sl[c]));
-          float ds = p * (__uint_as_float(dv[c]) - sl[kKvBQ + c]);
-          if (need_mask && !(col0 + c < a.S_q && visible(key, pos0 + c, kv, a.causal, a.window))) {
-            p = 0.f;
-            ds = 0.f;
-          }
-          p2[e] = p;
-          d2[e] = ds;
+        const float2 nl = *reinterpret_cast<const float2*>(sl + x);          // -lse2 of the two rows
+        const float2 nd = *reinterpret_cast<const float2*>(sl + kKvBQ + x);  // -D of the two rows
+        const float2 arg = fma2(make_float2(__uint_as_float(sv[x]), __uint_as_float(sv[x + 1])), c2, nl);
+        float2 p = make_float2(fast_exp2(arg.x), fast_exp2(arg.y));
+        float2 ds = mul2(p, add2(make_float2(__uint_as_float(dv[x]), __uint_as_float(dv[x + 1])), nd));
+        if (need_mask) {
+          if (!(col0 + x < a.S_q && visible(key, pos0 + x, kv, a.causal, a.window))) p.x = ds.x = 0.f;
+          if (!(col0 + x + 1 < a.S_q && visible(key, pos0 + x + 1, kv, a.causal, a.window))) p.y = ds.y = 0.f;
         }
-        pp[x / 2] = pack_bf16x2(p2[0], p2[1]);
-        pd[x / 2] = pack_bf16x2(d2[0], d2[1]);
+        pp[x / 2] = pack_bf16x2(p.x, p.y);
+        pd[x / 2] = pack_bf16x2(ds.x, ds.y);
       }
       tc::st16(lane_addr + 64 * bf + 32 * half, pp);        // P^T over this half's first columns
       tc::st16(lane_addr + 128 + 64 * bf + 32 * half, pd);  // dS^T likewise in dP^T
@@ -649,18 +672,17 @@ __global__ void __launch_bounds__(kQThreads, 1)
       tc::ld32(lane_addr + 128 + 64 * bf + 32 * half, dv);
       tc::wait_ld();
       uint32_t pd[16];
+      const float2 c2 = make_float2(a.sl2, a.sl2), nl = make_float2(-lse2, -lse2), nd = make_float2(-dr, -dr);
 #pragma unroll
       for (int x = 0; x < 32; x += 2) {
-        float d2[2];
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int key = key0 + x + e;
-          const float pr = fast_exp2(fmaf(__uint_as_float(sv[x + e]), a.sl2, -lse2));
-          float ds = pr * (__uint_as_float(dv[x + e]) - dr);
-          if (need_mask && !visible(key, pos, kv, a.causal, a.window)) ds = 0.f;
-          d2[e] = ds;
+        const float2 arg = fma2(make_float2(__uint_as_float(sv[x]), __uint_as_float(sv[x + 1])), c2, nl);
+        const float2 pr = make_float2(fast_exp2(arg.x), fast_exp2(arg.y));
+        float2 ds = mul2(pr, add2(make_float2(__uint_as_float(dv[x]), __uint_as_float(dv[x + 1])), nd));
+        if (need_mask) {
+          if (!visible(key0 + x, pos, kv, a.causal, a.window)) ds.x = 0.f;
+          if (!visible(key0 + x + 1, pos, kv, a.causal, a.window)) ds.y = 0.f;
         }
-        pd[x / 2] = pack_bf16x2(d2[0], d2[1]);
+        pd[x / 2] = pack_bf16x2(ds.x, ds.y);
       }
       tc::st16(lane_addr + 64 * bf + 32 * half, pd);  // dS over this half's first columns of S
       // K rows no row of the tile may see (past kv_len: last block; below every row's window:

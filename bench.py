@@ -382,7 +382,7 @@ def run_backward(args, dev, stream, tf_peak, peak_kind):
     tflops = flops / (ms / 1e3) / 1e12
     return {"workload": "prefill_4k backward: dQ, dK, dV (B=1, h_q=32, h_kv=8, S_q=T=4096, d_h=128, causal)",
             "value": round(tflops, 1), "unit": "TFLOP/s", "ms": round(ms, 4),
-            "launches": "rowterm + dkdv + dq (three kernels), eager, L2 flushed between runs",
+            "launches": "rowterm + one grid of dK/dV and dQ CTAs (two kernels), eager, L2 flushed between runs",
             "roofline": {"bound": "tensor", "achieved": round(tflops, 1), "peak": tf_peak, "unit": "TFLOP/s",
                          "frac": round(tflops / tf_peak, 4), "peak_kind": f"bf16_tflops of {peak_kind}",
                          "algorithmic_flops_per_launch": flops}}

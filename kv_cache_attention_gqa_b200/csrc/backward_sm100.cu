@@ -8,7 +8,7 @@
 //   dS = P * (dP - D),  dQ_a = scale dS K_g,  dK_g += scale dS^T Q_a.
 // The mask is the forward's: causal by absolute position, length, and an optional sliding window.
 //
-// Three launches:
+// Two launches: rowterm, then one grid whose first CTAs run dkdv and the rest dq:
 //   rowterm   one warp per query row: D = rowsum(dO * O) and the base-2 lse (fp32 workspace).
 //   dkdv      one CTA per (sequence, KV head, 128-key block). The keys sit on the 128 TMEM lanes;
 //             the CTA walks every 64-row query block of every head of the group, so the r heads'
@@ -188,11 +188,11 @@ enum {
   kKvBars = kKvDone + 1
 };
 
+// One CTA of the dK / dV pass for tile `tile` (sequence, KV head, key block).
 template <int D>
-__global__ void __launch_bounds__(kKvThreads, 1)
-    dkdv_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmdo,
-                const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
-                BArgs a) {
+__device__ __forceinline__ void dkdv_cta(const CUtensorMap& tmq, const CUtensorMap& tmdo,
+                                         const CUtensorMap& tmk, const CUtensorMap& tmv, const BArgs& a,
+                                         int tile) {
   using C = KvCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -209,9 +209,9 @@ __global__ void __launch_bounds__(kKvThreads, 1)
 
   // ---- this CTA's keys and the query blocks that see them
   const int per = a.B * a.h_kv;
-  const int kb = blockIdx.x / per;
-  const int b = (blockIdx.x - kb * per) / a.h_kv;
-  const int g = blockIdx.x - kb * per - b * a.h_kv;
+  const int kb = tile / per;
+  const int b = (tile - kb * per) / a.h_kv;
+  const int g = tile - kb * per - b * a.h_kv;
   const int k0 = kb * kBK;
   const int kv = a.kv_len ? a.kv_len[b] : a.T_max;
   const int qs = a.q_start ? a.q_start[b] : 0;
@@ -481,11 +481,11 @@ enum {
   kQBars = kQDone + 1
 };
 
+// One CTA of the dQ pass for forward tile `tile`.
 template <int D>
-__global__ void __launch_bounds__(kQThreads, 1)
-    dq_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmdo,
-              const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
-              BArgs a) {
+__device__ __forceinline__ void dq_cta(const CUtensorMap& tmq, const CUtensorMap& tmdo,
+                                       const CUtensorMap& tmk, const CUtensorMap& tmv, const BArgs& a,
+                                       int tile) {
   using C = QCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -501,8 +501,8 @@ __global__ void __launch_bounds__(kQThreads, 1)
 
   // ---- the tile (as in the forward): H heads x P positions of one group, heaviest first
   const int per = a.B * a.h_kv * a.hblocks;
-  const int qt = a.n_qt - 1 - (int)(blockIdx.x / per);
-  const int rem = blockIdx.x - (blockIdx.x / per) * per;
+  const int qt = a.n_qt - 1 - tile / per;
+  const int rem = tile - (tile / per) * per;
   const int b = rem / (a.h_kv * a.hblocks);
   const int gh = rem - b * (a.h_kv * a.hblocks);
   const int g = gh / a.hblocks, hb = gh - g * a.hblocks;
@@ -740,26 +740,43 @@ __global__ void __launch_bounds__(kQThreads, 1)
   }
 }
 
+// One launch for both passes: the first n_dkdv CTAs run the key-stationary dK / dV pass
+// (heaviest key blocks first), the rest the query-stationary dQ pass, which fills the SMs the
+// uneven dK / dV CTAs leave idle. Both use 320 threads, the larger of the two shared-memory sizes
+// and their own 512 TMEM columns (one CTA per SM).
+static_assert(kKvThreads == kQThreads, "one block size for both passes");
+template <int D>
+struct BwCfg {
+  static constexpr int kSmem = KvCfg<D>::kSmem > QCfg<D>::kSmem ? KvCfg<D>::kSmem : QCfg<D>::kSmem;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kKvThreads, 1)
+    backward_kernel(const __grid_constant__ CUtensorMap tmq_rows, const __grid_constant__ CUtensorMap tmdo_rows,
+                    const __grid_constant__ CUtensorMap tmk128, const __grid_constant__ CUtensorMap tmv128,
+                    const __grid_constant__ CUtensorMap tmq_tile, const __grid_constant__ CUtensorMap tmdo_tile,
+                    const __grid_constant__ CUtensorMap tmk64, const __grid_constant__ CUtensorMap tmv64,
+                    BArgs a, int n_dkdv) {
+  if ((int)blockIdx.x < n_dkdv) dkdv_cta<D>(tmq_rows, tmdo_rows, tmk128, tmv128, a, (int)blockIdx.x);
+  else dq_cta<D>(tmq_tile, tmdo_tile, tmk64, tmv64, a, (int)blockIdx.x - n_dkdv);
+}
+
 template <int D>
 cudaError_t launch_typed(const BArgs& p, const CUtensorMap* tm, cudaStream_t s) {
-  static bool attr_set[64] = {false};  // per device: the shared-memory opt-ins are set once
+  static bool attr_set[64] = {false};  // per device: the shared-memory opt-in is set once
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64 || !attr_set[dev]) {
-    e = cudaFuncSetAttribute(dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, KvCfg<D>::kSmem);
-    if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, QCfg<D>::kSmem);
+    e = cudaFuncSetAttribute(backward_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, BwCfg<D>::kSmem);
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < 64) attr_set[dev] = true;
   }
   const long long n1 = (long long)p.n_kb * p.B * p.h_kv;
   const long long n2 = (long long)p.n_qt * p.B * p.h_kv * p.hblocks;
-  if (n1 > 0x7fffffffLL || n2 > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-  dkdv_kernel<D><<<(unsigned)n1, kKvThreads, KvCfg<D>::kSmem, s>>>(tm[0], tm[1], tm[2], tm[3], p);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  dq_kernel<D><<<(unsigned)n2, kQThreads, QCfg<D>::kSmem, s>>>(tm[4], tm[5], tm[6], tm[7], p);
+  if (n1 + n2 > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  backward_kernel<D><<<(unsigned)(n1 + n2), kKvThreads, BwCfg<D>::kSmem, s>>>(
+      tm[0], tm[1], tm[2], tm[3], tm[4], tm[5], tm[6], tm[7], p, (int)n1);
   return cudaGetLastError();
 }
 

@@ -114,3 +114,23 @@ def test_one_workspace_shared_by_different_shapes():
             o = gqa.decode(q, k, v, kv_len=kv_len, num_splits=splits, ws=ws)
             assert_bf16_close(_f64(o), ref, f"shared workspace rep={rep}")
             assert ws[:4].view(torch.int32).item() == 0  # the work ticket
+
+
+def test_decode_more_chunks_than_ctas_uses_the_ticket():
+    """num_splits above the CTA count: CTAs take further chunks from the atomic work ticket."""
+    import kv_cache_attention_gqa_b200 as gqa
+
+    shape = workloads.DecodeShape(B=4, h_q=32, h_kv=8, T_max=4096, d_h=128)
+    q, k, v, _ = workloads.decode_inputs(shape, seed=12)
+    lens = np.array([4096, 3000, 77, 1], np.int32)
+    ref, _ = oracle.decode_ref(_f64(q), _f64(k), _f64(v), kv_len=lens)
+    n = gqa.decode_workspace_size(4, 32, 8, 4096, 128, torch.bfloat16, 400)
+    ws = torch.zeros(n, dtype=torch.uint8, device="cuda")
+    for rep in range(2):
+        o = gqa.decode(q.cuda(), k.cuda(), v.cuda(), kv_len=lens.tolist(), num_splits=400, ws=ws)
+        assert_bf16_close(_f64(o), ref, f"400 splits rep {rep}")
+        assert ws[:4].view(torch.int32).item() == 0
+    o32 = gqa.decode(q.float().cuda(), k.float().cuda(), v.float().cuda(), kv_len=lens.tolist(), num_splits=400)
+    from _tol import assert_fp32_close
+    assert_fp32_close(_f64(o32), ref, "fp32 400 splits")
+    assert gqa.get_device_error() == 0

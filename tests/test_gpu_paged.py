@@ -235,3 +235,19 @@ def test_paged_ragged_decode_full_size_sampled():
         ref, _ = oracle.paged_decode_ref(_f64(q[b:b + 1]), _f64(k[idx]), _f64(v[idx]), table,
                                          lens[b:b + 1])
         assert_bf16_close(_f64(o[b:b + 1]), ref, f"paged ragged b={b} len={lens[b]}")
+
+
+def test_paged_and_mla_decode_more_chunks_than_ctas():
+    import kv_cache_attention_gqa_b200 as gqa
+    from oracle import mla as mla_ref
+
+    shape = workloads.DecodeShape(B=3, h_q=16, h_kv=4, T_max=3000, d_h=128)
+    q, k, v, bt, kl = workloads.paged_decode_inputs(shape, 16, seed=30, device="cuda", lengths=[3000, 1234, 9])
+    o = gqa.decode_paged(q, k, v, bt, kv_len=kl, num_splits=400)
+    assert_bf16_close(_f64(o), _ref(q, k, v, bt, kl)[0], "paged 400 splits")
+    mshape = workloads.MlaShape(B=2, h_q=16, T_max=3000)
+    mq, mc, mkl = workloads.mla_decode_inputs(mshape, seed=31, lengths=[3000, 500])
+    om = gqa.mla_decode(mq.cuda(), mc.cuda(), kv_len=[3000, 500], scale=mshape.scale, num_splits=400)
+    mref, _ = mla_ref.mla_decode_ref(_f64(mq), _f64(mc), 512, kv_len=np.array([3000, 500]), scale=mshape.scale)
+    assert_bf16_close(_f64(om), mref, "mla 400 splits")
+    assert gqa.get_device_error() == 0

@@ -233,7 +233,8 @@ gqa_status gqa_decode_noalloc(const void* q, const void* k_cache, const void* v_
  *
  *   k_cache, v_cache (B, h_kv, T_max, d_h), written in place.
  *   k_new, v_new     (B, h_kv, S_new, d_h), read.
- *   pos      device int32[B] (required): first cache row written for sequence b.
+ *   pos      device int32[B] (required when S_new > 0): first cache row written for sequence b.
+ *            S_new = 0 is a no-op; k_new, v_new and pos may then be NULL.
  *            Rows that would fall outside [0, T_max) are not written; the device error word is
  *            set to GQA_DEVERR_POSITION.
  *   dtype    element type of all four tensors (bf16: 2 bytes, fp32: 4 bytes); any d_h >= 1.
@@ -278,7 +279,8 @@ gqa_status gqa_decode_paged(const void* q, const void* k_pages, const void* v_pa
  * Bit-exact; no other byte of the pools is written.
  *   k_pages, v_pages (num_pages, h_kv, page_size, d_h), written in place; page_size >= 1.
  *   k_new, v_new     (B, h_kv, S_new, d_h).
- *   pos      device int32[B]. Sequences whose rows would leave [0, max_pages * page_size) are not
+ *   pos      device int32[B] (with k_new, v_new and block_table, required when S_new > 0; S_new = 0
+ *            is a no-op). Sequences whose rows would leave [0, max_pages * page_size) are not
  *            written (GQA_DEVERR_POSITION); rows whose page entry is outside [0, num_pages) are
  *            not written (GQA_DEVERR_PAGE).
  * Errors: INVALID_ARG, CUDA.

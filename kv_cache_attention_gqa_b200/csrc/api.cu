@@ -203,10 +203,12 @@ gqa_status gqa_get_device_error(int* code, void* stream) {
 gqa_status kv_append(void* k_cache, void* v_cache, const void* k_new, const void* v_new,
                      const int32_t* pos, int B, int h_kv, int S_new, int T_max, int d_h,
                      gqa_dtype dtype, void* stream) {
-  if (!k_cache || !v_cache || !k_new || !v_new || !pos) return GQA_ERR_INVALID_ARG;
+  if (!k_cache || !v_cache) return GQA_ERR_INVALID_ARG;
+  if (S_new > 0 && (!k_new || !v_new || !pos)) return GQA_ERR_INVALID_ARG;  // S_new = 0: no-op
   if (B <= 0 || h_kv <= 0 || S_new < 0 || T_max <= 0 || d_h <= 0) return GQA_ERR_INVALID_ARG;
   if (dtype != GQA_BF16 && dtype != GQA_FP32) return GQA_ERR_INVALID_ARG;
   if (S_new > T_max) return GQA_ERR_INVALID_ARG;
+  if (S_new == 0) return GQA_OK;  // nothing to copy
   AppendArgs a;
   a.k_cache = k_cache;
   a.v_cache = v_cache;
@@ -463,13 +465,15 @@ gqa_status kv_append_paged(void* k_pages, void* v_pages, const void* k_new, cons
                            int S_new, int num_pages, int page_size, int max_pages, int d_h,
                            gqa_dtype dtype, void* stream) {
   using namespace gqa;
-  if (!k_pages || !v_pages || !k_new || !v_new || !pos || !block_table) return GQA_ERR_INVALID_ARG;
+  if (!k_pages || !v_pages) return GQA_ERR_INVALID_ARG;
+  if (S_new > 0 && (!k_new || !v_new || !pos || !block_table)) return GQA_ERR_INVALID_ARG;  // S_new = 0: no-op
   if (B <= 0 || h_kv <= 0 || S_new < 0 || d_h <= 0) return GQA_ERR_INVALID_ARG;
   if (num_pages <= 0 || page_size <= 0 || max_pages <= 0) return GQA_ERR_INVALID_ARG;
   if (dtype != GQA_BF16 && dtype != GQA_FP32) return GQA_ERR_INVALID_ARG;
   const long long T_max = (long long)max_pages * page_size;
   if (T_max >= (1ll << 31)) return GQA_ERR_UNSUPPORTED;
   if (S_new > T_max) return GQA_ERR_INVALID_ARG;
+  if (S_new == 0) return GQA_OK;  // nothing to copy
   AppendArgs a;
   a.k_cache = k_pages;
   a.v_cache = v_pages;

@@ -178,35 +178,38 @@ __device__ __forceinline__ Piece locate(const Plan& p, int B, int hblocks, long 
 template <typename OutT>
 __device__ void build_plan(const KArgs& a, Plan& p, long long* pre, int* nlen, int* wlo, int warp,
                            int lane, int w0) {
+  // Every thread of the CTA reads the lengths of its share of the sequences in one round of loads
+  // (a batch of up to kMaxBatch costs one memory round trip, not one per 32 sequences) ...
+  for (int b = threadIdx.x; b < a.B; b += blockDim.x) {
+    const int kv = a.kv_len ? a.kv_len[b] : a.T_max;
+    const int qp = a.q_pos ? a.q_pos[b] : kv - 1;
+    int n = 0, lo = 0;
+    if (kv < 1 || kv > a.T_max) {
+      if (blockIdx.x == 0) set_device_error(a.err, GQA_DEVERR_KV_LEN);
+    } else if (qp < 0) {
+      if (blockIdx.x == 0) set_device_error(a.err, GQA_DEVERR_POSITION);
+    } else {
+      n = qp + 1 < kv ? qp + 1 : kv;
+      if (a.window > 0 && qp - a.window + 1 > 0) lo = qp - a.window + 1;
+      if (lo >= n) {  // the window starts at or past the last cached key
+        if (blockIdx.x == 0) set_device_error(a.err, GQA_DEVERR_NO_VISIBLE);
+        n = 0;
+        lo = 0;
+      }
+    }
+    // the unit starts at the window start rounded down to the granule; the keys before the
+    // window inside that first granule are masked (only on a paged cache, gran > 1)
+    if (n > 0) n -= lo / a.gran * a.gran;
+    nlen[b] = n;
+    wlo[b] = lo;
+  }
+  __syncthreads();
+  // ... then one warp turns them into prefix sums in granules, from shared memory
   if (warp == w0) {
     long long run = 0;
     for (int base = 0; base < a.B; base += 32) {
       const int b = base + lane;
-      int n = 0;
-      if (b < a.B) {
-        const int kv = a.kv_len ? a.kv_len[b] : a.T_max;
-        const int qp = a.q_pos ? a.q_pos[b] : kv - 1;
-        int lo = 0;
-        if (kv < 1 || kv > a.T_max) {
-          if (blockIdx.x == 0) set_device_error(a.err, GQA_DEVERR_KV_LEN);
-        } else if (qp < 0) {
-          if (blockIdx.x == 0) set_device_error(a.err, GQA_DEVERR_POSITION);
-        } else {
-          n = qp + 1 < kv ? qp + 1 : kv;
-          if (a.window > 0 && qp - a.window + 1 > 0) lo = qp - a.window + 1;
-          if (lo >= n) {  // the window starts at or past the last cached key
-            if (blockIdx.x == 0) set_device_error(a.err, GQA_DEVERR_NO_VISIBLE);
-            n = 0;
-            lo = 0;
-          }
-        }
-        // the unit starts at the window start rounded down to the granule; the keys before the
-        // window inside that first granule are masked (only on a paged cache, gran > 1)
-        if (n > 0) n -= lo / a.gran * a.gran;
-        nlen[b] = n;
-        wlo[b] = lo;
-      }
-      const long long ngr = (n + a.gran - 1) / a.gran;  // granules
+      const long long ngr = b < a.B ? (nlen[b] + a.gran - 1) / a.gran : 0;  // granules
       long long s = ngr;  // inclusive warp scan
 #pragma unroll
       for (int off = 1; off < 32; off <<= 1) {

@@ -85,6 +85,8 @@ def test_host_side_argument_errors(lib):
     assert lib.gqa_decode(fake, fake, fake, fake, null, null, null, 1, 4, 2, 8, 64, 0.1, 0, 0, P(0x1004), 1 << 20, 1, s) == 5
     # kv_append
     assert lib.kv_append(fake, fake, fake, fake, null, 1, 2, 1, 8, 64, 0, s) == 1
+    assert lib.kv_append(null, fake, fake, fake, fake, 1, 2, 1, 8, 64, 0, s) == 1
+    assert lib.kv_append(fake, fake, null, null, null, 1, 2, 0, 8, 64, 0, s) == 0  # zero rows: no-op
     assert lib.kv_append(fake, fake, fake, fake, fake, 1, 2, 9, 8, 64, 0, s) == 1
     assert lib.kv_append(fake, fake, fake, fake, fake, 1, 2, 1, 8, 64, 9, s) == 1
     assert lib.gqa_get_device_error(None, s) == 1
@@ -131,6 +133,7 @@ def test_paged_host_side_argument_errors(lib):
     # kv_append_paged: k, v, k_new, v_new, pos, block_table, B, h_kv, S_new, num_pages, page_size,
     #                  max_pages, d_h, dtype, stream
     assert lib.kv_append_paged(fake, fake, fake, fake, fake, null, 1, 2, 1, 8, 16, 4, 64, 0, s) == 1
+    assert lib.kv_append_paged(fake, fake, null, null, null, null, 1, 2, 0, 8, 16, 4, 64, 0, s) == 0
     assert lib.kv_append_paged(fake, fake, fake, fake, null, fake, 1, 2, 1, 8, 16, 4, 64, 0, s) == 1
     assert lib.kv_append_paged(fake, fake, fake, fake, fake, fake, 1, 2, 1, 0, 16, 4, 64, 0, s) == 1
     assert lib.kv_append_paged(fake, fake, fake, fake, fake, fake, 1, 2, 65, 8, 16, 4, 64, 0, s) == 1

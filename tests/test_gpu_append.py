@@ -45,3 +45,16 @@ def test_append_out_of_range_is_flagged_and_writes_nothing():
     assert k[0].abs().sum().item() == 0  # sequence 0 did not fit: untouched
     assert torch.equal(k[1, :, 0:2], kn[1])  # sequence 1 was written
     assert gqa.get_device_error() == 0  # the word was cleared by the read
+
+
+def test_append_of_zero_rows_is_a_no_op():
+    import kv_cache_attention_gqa_b200 as gqa
+
+    k = torch.randn(2, 2, 8, 64).to(torch.bfloat16).cuda()
+    v = torch.randn(2, 2, 8, 64).to(torch.bfloat16).cuda()
+    k0, v0 = k.clone(), v.clone()
+    empty = torch.empty(2, 2, 0, 64, dtype=torch.bfloat16, device="cuda")
+    gqa.kv_append(k, v, empty, empty, [3, 8])
+    torch.cuda.synchronize()
+    assert torch.equal(k, k0) and torch.equal(v, v0)
+    assert gqa.get_device_error() == 0

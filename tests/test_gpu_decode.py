@@ -134,3 +134,26 @@ def test_decode_more_chunks_than_ctas_uses_the_ticket():
     from _tol import assert_fp32_close
     assert_fp32_close(_f64(o32), ref, "fp32 400 splits")
     assert gqa.get_device_error() == 0
+
+
+def test_decode_maximum_batch():
+    """B = 1024 (the largest batch the decode accepts) with ragged lengths, a few empty-window
+    rows' neighbours and q_pos inside the cache: every output against the oracle."""
+    import kv_cache_attention_gqa_b200 as gqa
+
+    B, h_q, h_kv, T, d = 1024, 8, 2, 96, 64
+    shape = workloads.DecodeShape(B=B, h_q=h_q, h_kv=h_kv, T_max=T, d_h=d)
+    q, k, v, _ = workloads.decode_inputs(shape, seed=21)
+    rng = np.random.default_rng(21)
+    lens = rng.integers(1, T + 1, size=B).astype(np.int32)
+    q_pos = np.minimum(lens - 1, rng.integers(0, T, size=B)).astype(np.int32)
+    ref, lref = oracle.decode_ref(_f64(q), _f64(k), _f64(v), kv_len=lens, q_pos=q_pos)
+    for splits in (0, 300):
+        o, lse = gqa.decode(q.cuda(), k.cuda(), v.cuda(), kv_len=lens.tolist(), q_pos=q_pos.tolist(),
+                            num_splits=splits, return_lse=True)
+        assert_bf16_close(_f64(o), ref, f"B=1024 splits={splits}")
+        assert np.abs(lse.cpu().double().numpy() - lref).max() < 2e-2
+    assert gqa.get_device_error() == 0
+    with pytest.raises(gqa.GQAError):
+        gqa.decode(q[:1].cuda().expand(1025, h_q, d).contiguous(), k[:1].cuda().expand(1025, h_kv, T, d).contiguous(),
+                   v[:1].cuda().expand(1025, h_kv, T, d).contiguous())

@@ -136,6 +136,9 @@ gqa_status decode_impl(const void* q, const void* k_cache, const void* v_cache, 
   if (!a.err) return GQA_ERR_CUDA;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (dtype == GQA_FP32) return from_cuda(launch_decode_fp32(a, s));
+  // Query rows per TMA box = the kernel's m-tiles x 16: units hold min(r, 32) heads (the decode
+  // kernel's heads-per-unit limit), two m-tiles above 16. The box height and the kernel's expected
+  // bytes must agree, or its full barriers never complete (the bounded waits then report a timeout).
   const int r = h_q / h_kv;
   const uint32_t qrows = r > 16 ? 32 : 16;
   CUtensorMap maps[3];

@@ -72,10 +72,19 @@ def prefill_flops(B, h_q, d_h, S_q, q_start, kv_len, window=0):
     return 4 * d_h * B * h_q * pairs
 
 
+def _code_only(text):
+    """Source with // and /* */ comments and trailing blanks removed, so that a comment edit does
+    not count as a kernel change (string literals in these files hold no comment markers)."""
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    return "\n".join(line.rstrip() for line in text.splitlines() if line.strip())
+
+
 def source_digest(paths):
+    """Digest of the kernel sources' code (comments ignored) at the time the counters were taken."""
     h = hashlib.sha256()
     for p in sorted(paths):
-        h.update(open(os.path.join(ROOT, p), "rb").read())
+        h.update(_code_only(open(os.path.join(ROOT, p), encoding="utf-8").read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -8,8 +8,8 @@
 // n_b = min(kv_len[b], q_pos[b] + 1). The visible keys of all units, laid end to end, are cut into
 // equal chunks of C keys ("split along history" [MHA/MQA/GQA walkthrough, section 9]). A chunk
 // may hold the end of one unit and the start of the next; the part of a unit inside a chunk is a
-// "piece". Persistent CTAs take chunks from an atomic ticket, so a CTA that gets more memory
-// bandwidth takes more chunks and all CTAs finish together.
+// "piece". CTA c starts with chunk c; when there are more chunks than CTAs, further chunks come
+// from an atomic ticket, so a CTA that gets more memory bandwidth takes more of them.
 //
 // Per piece the CTA keeps the online-softmax state (m, l, u) of each query row
 // [序列计算与存储, section 在线 softmax] and produces the normalised piece output o_p and its
@@ -22,7 +22,8 @@
 // bf16 kernel, warp-specialised. One producer warp takes chunks, writes one small descriptor per
 // 64-key tile into shared memory, and streams the tile's K and V (and, on the first tile of a
 // piece, the unit's query rows) with TMA (cp.async.bulk.tensor, 128-byte swizzle, no multicast)
-// into a 4-stage ring guarded by mbarriers. Four consumer warps per 16-row m-tile each take 16 keys
+// into a 5-stage (one m-tile) or 4-stage (two) ring guarded by mbarriers. Four consumer warps per
+// 16-row m-tile each take 16 keys
 // of every tile: S = Q K^T and O += P V run on the tensor cores as m16n8k16 bf16 MMAs with fp32
 // accumulators (a unit has at most 32 query rows, too few for a 64/128-row tcgen05 tile, and the
 // kernel is bound by HBM, not by the MMA rate). Scores use base-2 exponents with scale * log2(e)
@@ -30,6 +31,15 @@
 //
 // fp32 kernel (check mode): the same chunks, pieces, partials and merge, with a scalar core (one
 // warp per query head, lanes split d_h, one key per online-softmax step).
+//
+// Also here, on the same plan / pieces / merge:
+//   * a paged cache (pools of fixed-size pages and a block table): the partition counts 16- or
+//     64-key granules so no loaded sub-tile straddles a page, and the whole producer warp
+//     prefetches a window of block-table entries (see the producer);
+//   * a sliding window: a unit starts at its window (rounded down to the granule), leading keys
+//     before the window are masked per tile;
+//   * MLA decode over a latent cache (mla_bf16_kernel): one shared KV "head" whose value is the
+//     first 512 entries of each 576-wide cache row.
 
 #include <math.h>
 

@@ -227,6 +227,9 @@ __device__ __forceinline__ void softmax_role(const PArgs& a, const Tile& tile, i
   const int qi = tile.q0 + p;                 // query index into S_q
   const bool store_row = h < tile.nh && row < a.H * a.P && qi < a.S_q;
   const long long pos = (long long)tile.qs + qi;
+  // last key this row may see (length and causal limits in one 32-bit bound for the mask loop)
+  const long long kl = a.causal && pos < tile.kv - 1 ? pos : (long long)tile.kv - 1;
+  const int key_last = (int)kl;
   const long long pos_min = (long long)tile.qs + tile.q0;  // smallest position in the tile
   const long long pos_max = (long long)tile.qs + min(tile.q0 + a.P, a.S_q) - 1;  // largest
   const int nb = tile.nb;
@@ -288,8 +291,7 @@ __device__ __forceinline__ void softmax_role(const PArgs& a, const Tile& tile, i
 #pragma unroll
         for (int i = 0; i < 64; ++i) {
           const int key = key0 + i;
-          const bool vis = key < tile.kv && (!a.causal || key <= pos) &&
-                           (!kWin || key > win_last);
+          const bool vis = key <= key_last && (!kWin || key > win_last);
           sr[i] = vis ? sr[i] : -INFINITY;
         }
       }

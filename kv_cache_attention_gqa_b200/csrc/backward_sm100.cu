@@ -106,10 +106,6 @@ __device__ __forceinline__ float2 mul2(float2 a, float2 b) {
   return d;
 }
 
-__device__ __forceinline__ bool visible(long long key, long long pos, int kv, int causal, int window) {
-  return key < kv && (!causal || key <= pos) && (window == 0 || key > pos - window);
-}
-
 // ---- K-major / MN-major shared-memory descriptors for a 128-row bf16 tile in 64-column chunks
 // (128-byte swizzle, as written by TMA with a 64 x 128 box per chunk).
 // K-major (the tile's columns are the contraction): k-th 16-wide step.
@@ -378,6 +374,16 @@ __device__ __forceinline__ void dkdv_cta(const CUtensorMap& tmq, const CUtensorM
       tc::ld32(lane_addr + 64 * bf + 32 * half, sv);
       tc::ld32(lane_addr + 128 + 64 * bf + 32 * half, dv);
       tc::wait_ld();
+      // query columns [c_lo, c_hi) of this half that see this key: rows at or past it (causal),
+      // within its window, inside S_q; none when the key is past kv_len
+      int c_lo = 0, c_hi = 32;
+      if (need_mask) {
+        const long long rel = (long long)key - pos0;  // column of the row at the key's position
+        if (a.causal) c_lo = (int)(rel < 0 ? 0 : (rel > 32 ? 32 : rel));
+        long long hi = a.S_q - col0 < 32 ? a.S_q - col0 : 32;
+        if (a.window > 0 && rel + a.window < hi) hi = rel + a.window;
+        c_hi = key < kv ? (int)(hi < 0 ? 0 : hi) : 0;
+      }
       uint32_t pp[16], pd[16];
       const float2 c2 = make_float2(a.sl2, a.sl2);
 #pragma unroll
@@ -388,8 +394,8 @@ __device__ __forceinline__ void dkdv_cta(const CUtensorMap& tmq, const CUtensorM
         float2 p = make_float2(fast_exp2(arg.x), fast_exp2(arg.y));
         float2 ds = mul2(p, add2(make_float2(__uint_as_float(dv[x]), __uint_as_float(dv[x + 1])), nd));
         if (need_mask) {
-          if (!(col0 + x < a.S_q && visible(key, pos0 + x, kv, a.causal, a.window))) p.x = ds.x = 0.f;
-          if (!(col0 + x + 1 < a.S_q && visible(key, pos0 + x + 1, kv, a.causal, a.window))) p.y = ds.y = 0.f;
+          if (x < c_lo || x >= c_hi) p.x = ds.x = 0.f;
+          if (x + 1 < c_lo || x + 1 >= c_hi) p.y = ds.y = 0.f;
         }
         pp[x / 2] = pack_bf16x2(p.x, p.y);
         pd[x / 2] = pack_bf16x2(ds.x, ds.y);
@@ -635,6 +641,11 @@ __device__ __forceinline__ void dq_cta(const CUtensorMap& tmq, const CUtensorMap
     const long long pos = (long long)qs + qi;
     const float lse2 = store_row ? a.lse2[srow] : INFINITY;
     const float dr = store_row ? a.drow[srow] : 0.f;
+    // keys [k_first, k_last] this row sees (length, causal and window limits as 32-bit bounds)
+    const long long kl = a.causal && pos < kv - 1 ? pos : (long long)kv - 1;
+    const int k_last = (int)kl;
+    const long long kf = a.window > 0 ? pos - a.window + 1 : 0;
+    const int k_first = kf < 0 ? 0 : (kf > 0x7fffffffLL ? 0x7fffffff : (int)kf);
     // this row of Q (half 0) or dO (half 1): shared memory (128-byte swizzled) -> TMEM
     bool ok = nb > 0 && wait_bar(bar(kQdQ), 0, abort, a.err);
     ok = __all_sync(0xffffffffu, ok);
@@ -679,8 +690,8 @@ __device__ __forceinline__ void dq_cta(const CUtensorMap& tmq, const CUtensorMap
         const float2 pr = make_float2(fast_exp2(arg.x), fast_exp2(arg.y));
         float2 ds = mul2(pr, add2(make_float2(__uint_as_float(dv[x]), __uint_as_float(dv[x + 1])), nd));
         if (need_mask) {
-          if (!visible(key0 + x, pos, kv, a.causal, a.window)) ds.x = 0.f;
-          if (!visible(key0 + x + 1, pos, kv, a.causal, a.window)) ds.y = 0.f;
+          if (key0 + x < k_first || key0 + x > k_last) ds.x = 0.f;
+          if (key0 + x + 1 < k_first || key0 + x + 1 > k_last) ds.y = 0.f;
         }
         pd[x / 2] = pack_bf16x2(ds.x, ds.y);
       }

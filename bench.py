@@ -11,7 +11,9 @@ A ``paged`` object repeats the decode_8k step over a paged cache (16-token pages
 pool: ``kv_append_paged`` + ``gqa_decode_paged``), timed the same way; a ``window`` object runs
 decode_8k and prefill_4k with a 1024-key sliding window (work counted inside the window only); a
 ``backward`` object times gqa_prefill_backward on prefill_4k; an ``mla`` object times gqa_mla_decode
-over a latent cache.
+over a latent cache; a ``ragged`` object times gqa_decode on ragged_decode (64 sequences with
+seeded lengths on [1024, 32768]); a ``chunked`` object times the chunked prefill (512 new queries
+over 32768 keys) and its kv_append.
 
 ``--impl reference`` times the fp64 CPU oracle on a bounded sample of the same workload.
 Run with no flags for N=1; under torchrun every rank runs an independent replica (the path needs
@@ -466,6 +468,74 @@ def run_mla(args, dev, hbm_peak, tf_peak, peak_kind):
             "per_variant": out, "gpu_launches_per_call": 2}
 
 
+def run_ragged(args, dev, hbm_peak, peak_kind):
+    """ragged_decode: B=64, h_q=64, h_kv=8, d_h=128, cached lengths uniform on [1024, 32768]
+    (seeded), cache allocated at 32768 with NaN past each length. One gqa_decode per call; the
+    algorithmic bytes are the visible K/V rows only (2 * h_kv * d_h * 2 bytes per key)."""
+    import torch
+
+    import kv_cache_attention_gqa_b200 as gqa
+    import workloads
+
+    shape = workloads.RAGGED_DECODE
+    q, k, v, kv_len = workloads.decode_inputs(shape, seed=args.seed, device=dev)
+    out = torch.empty_like(q)
+    ws = torch.zeros(gqa.decode_workspace_size(shape.B, shape.h_q, shape.h_kv, shape.T_max, shape.d_h),
+                     dtype=torch.uint8, device=dev)
+    fn = lambda: gqa.decode(q, k, v, kv_len=kv_len, out=out, ws=ws)  # noqa: E731
+    ms, mode = graph_timed(fn, L2Flush(dev), max(5, args.steps), max(3, args.warmup))
+    if gqa.get_device_error() != 0:
+        raise RuntimeError("device error in the ragged decode line")
+    lens = kv_len.cpu().tolist()
+    nbytes = decode_kv_bytes(shape.B, shape.h_kv, lens, shape.d_h)
+    gbs = nbytes / (ms / 1e3) / 1e9
+    finite = bool(torch.isfinite(out.float()).all())  # the NaN past every length never reaches O
+    del q, k, v, out, ws
+    return {"workload": "ragged_decode: B=64, h_q=64, h_kv=8, d_h=128, lengths uniform on [1024, 32768] "
+                        f"(seed {args.seed}, sum {sum(lens)}), cache allocated at 32768 with NaN past each length; "
+                        "one gqa_decode per call, L2 flushed between calls",
+            "launch": mode, "value": round(gbs, 1), "unit": "GB/s", "us": round(ms * 1e3, 2),
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm_peak, "unit": "GB/s",
+                         "frac": round(gbs / hbm_peak, 4), "peak_kind": f"hbm_gbs of {peak_kind}",
+                         "algorithmic_bytes_per_launch": nbytes},
+            "output_finite": finite, "gpu_launches_per_call": 2}
+
+
+def run_chunked(args, dev, tf_peak, peak_kind):
+    """chunked prefill: 32256 cached positions plus 512 new queries at positions 32256..32767
+    (B=1, h_q=32, h_kv=8, d_h=128). kv_append writes the new K/V rows first; the attention and the
+    append are timed separately."""
+    import torch
+
+    import kv_cache_attention_gqa_b200 as gqa
+    import workloads
+
+    shape = workloads.CHUNKED_PREFILL
+    k, v, k_new, v_new, q = workloads.chunked_prefill_inputs(shape, seed=args.seed, device=dev)
+    pos = torch.full((shape.B,), shape.q_start, dtype=torch.int32, device=dev)
+    kl = torch.full((shape.B,), shape.kv_len, dtype=torch.int32, device=dev)
+    out = torch.empty_like(q)
+    flush = L2Flush(dev)
+    app = lambda: gqa.kv_append(k, v, k_new, v_new, pos)  # noqa: E731
+    att = lambda: gqa.prefill(q, k, v, q_start=pos, kv_len=kl, out=out)  # noqa: E731
+    app_ms, _ = graph_timed(app, flush, max(5, args.steps), max(3, args.warmup))
+    ms, mode = graph_timed(att, flush, max(5, args.steps), max(3, args.warmup))
+    if gqa.get_device_error() != 0:
+        raise RuntimeError("device error in the chunked prefill line")
+    flops = prefill_flops(shape.B, shape.h_q, shape.d_h, shape.S_q, shape.q_start, shape.kv_len)
+    tflops = flops / (ms / 1e3) / 1e12
+    app_bytes = 2 * 2 * k_new.nbytes  # K and V rows read once and written once
+    del k, v, k_new, v_new, q, out
+    return {"workload": "chunked prefill: B=1, h_q=32, h_kv=8, d_h=128, 32256 cached + 512 new queries at "
+                        "positions 32256..32767, T=32768, causal by absolute position; L2 flushed between calls",
+            "launch": mode, "value": round(tflops, 1), "unit": "TFLOP/s", "ms": round(ms, 4),
+            "roofline": {"bound": "tensor", "achieved": round(tflops, 1), "peak": tf_peak, "unit": "TFLOP/s",
+                         "frac": round(tflops / tf_peak, 4), "peak_kind": f"bf16_tflops of {peak_kind}",
+                         "algorithmic_flops_per_launch": flops},
+            "kv_append": {"us": round(app_ms * 1e3, 2), "bytes": app_bytes,
+                          "GB_s": round(app_bytes / (app_ms / 1e3) / 1e9, 1)}}
+
+
 def run_window(args, rank, dev, stream, local, hbm_peak, tf_peak, peak_kind):
     """Sliding window of 1024 keys [第三章 §3.7]: decode_8k (each query reads its 1024 most recent
     keys) and prefill_4k; the work counted is only what lies inside the windows."""
@@ -505,6 +575,10 @@ def run_ours(args, rank, world, dist):
         return {"backward": run_backward(args, dev, stream, tf_peak, peak_kind)}
     if args.window_only:  # profiling aid: the sliding-window lines alone
         return {"window": run_window(args, rank, dev, stream, local, hbm_peak, tf_peak, peak_kind)}
+    if args.ragged_only:  # profiling aid: the ragged decode line alone
+        return {"ragged": run_ragged(args, dev, hbm_peak, peak_kind)}
+    if args.chunked_only:  # profiling aid: the chunked prefill line alone
+        return {"chunked": run_chunked(args, dev, tf_peak, peak_kind)}
 
     variants = build_variants(args, rank, dev)
     flush = L2Flush(dev)
@@ -541,6 +615,8 @@ def run_ours(args, rank, world, dist):
     window = None
     if not args.skip_window:
         window = run_window(args, rank, dev, stream, local, hbm_peak, tf_peak, peak_kind)
+    ragged = run_ragged(args, dev, hbm_peak, peak_kind) if not args.skip_ragged else None
+    chunked = run_chunked(args, dev, tf_peak, peak_kind) if not args.skip_chunked else None
 
     result = {
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
@@ -565,6 +641,10 @@ def run_ours(args, rank, world, dist):
         result["backward"] = backward
     if mla is not None:
         result["mla"] = mla
+    if ragged is not None:
+        result["ragged"] = ragged
+    if chunked is not None:
+        result["chunked"] = chunked
     if rank == 0 and world == 1 and not args.skip_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(args)
     return result
@@ -773,6 +853,10 @@ def main():
     ap.add_argument("--backward-only", action="store_true", help="only the backward line (profiling aid)")
     ap.add_argument("--window-only", action="store_true", help="only the sliding-window lines (profiling aid)")
     ap.add_argument("--window", type=int, default=1024, help="sliding window of the window lines")
+    ap.add_argument("--skip-ragged", action="store_true")
+    ap.add_argument("--ragged-only", action="store_true", help="only the ragged decode line (profiling aid)")
+    ap.add_argument("--skip-chunked", action="store_true")
+    ap.add_argument("--chunked-only", action="store_true", help="only the chunked prefill line (profiling aid)")
     ap.add_argument("--h-kv", dest="h_kv", type=int, nargs="+", default=[32, 8, 1],
                     help="decode_8k variants to run (default: all three); fewer only for profiling")
     args = ap.parse_args()

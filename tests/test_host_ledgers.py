@@ -47,3 +47,24 @@ def test_paged_decode_inputs_spell_out_a_finite_cache():
         assert np.isfinite(kc[b, :, :n]).all() and np.isnan(kc[b, :, n:]).all()
     # every row of the pool that no sequence reads is NaN
     assert np.isnan(workloads.to_f64(k)).sum() == (k.shape[0] * 16 - 134) * 2 * 16
+
+
+def test_bench_ledgers_at_the_five_configs():
+    """The bench's algorithmic work at the five workloads equals the closed forms: causal prefill
+    4 d_h B h_q sum_i (q_start + i + 1) FLOPs; decode 2 B h_kv T d_h 2 KV bytes; the backward's five
+    GEMMs per visible pair are 2.5x the forward's two."""
+    # prefill_small: 4 * 4 * 64 * (256 * 257 / 2)
+    assert bench.prefill_flops(1, 4, 64, 256, 0, 256) == 33_685_504
+    # prefill_4k: 4 * 32 * 128 * (4096 * 4097 / 2)
+    assert bench.prefill_flops(1, 32, 128, 4096, 0, 4096) == 137_472_507_904
+    # chunked prefill: 512 rows at positions 32256..32767, each sees position + 1 keys
+    assert bench.prefill_flops(1, 32, 128, 512, 32256, 32768) == 272_734_617_600
+    # decode_8k: 1 GiB / 256 MiB / 32 MiB of K/V for h_kv = 32 / 8 / 1
+    for h_kv, nbytes in ((32, 1_073_741_824), (8, 268_435_456), (1, 33_554_432)):
+        assert bench.decode_kv_bytes(8, h_kv, [8192] * 8, 128) == nbytes
+    # ragged_decode: 2 * 8 * 128 * 2 = 4096 bytes per visible key
+    lens = workloads.ragged_lengths(0)
+    assert bench.decode_kv_bytes(64, 8, lens.tolist(), 128) == 4096 * int(lens.sum())
+    assert lens.min() >= 1024 and lens.max() <= 32768 and lens.shape == (64,)
+    # backward of prefill_4k, as the bench line states it
+    assert 5 * bench.prefill_flops(1, 32, 128, 4096, 0, 4096) // 2 == 343_681_269_760

@@ -105,6 +105,9 @@ def _ptr(t):
 
 
 def _need_cuda(*ts):
+    """Every tensor given is a contiguous CUDA tensor on the current device (the library launches on
+    the current device and its current stream)."""
+    dev = None
     for t in ts:
         if t is None:
             continue
@@ -112,13 +115,18 @@ def _need_cuda(*ts):
             raise ValueError("tensors must live on a CUDA device")
         if not t.is_contiguous():
             raise ValueError("tensors must be contiguous (row-major)")
+        if dev is None:
+            dev = torch.cuda.current_device()
+        if t.device.index != dev:
+            raise ValueError(f"tensors must live on the current CUDA device (cuda:{dev}), not {t.device}")
 
 
 def _int_vec(x, B: int, device, name: str):
     """Device int32[B] from None / int / sequence / tensor (None stays None = library default)."""
     if x is None:
         return None
-    if isinstance(x, torch.Tensor) and x.is_cuda and x.dtype == torch.int32 and x.is_contiguous():
+    if (isinstance(x, torch.Tensor) and x.is_cuda and x.device == torch.device(device)
+            and x.dtype == torch.int32 and x.is_contiguous()):
         if x.numel() != B:
             raise ValueError(f"{name} must have {B} entries")
         return x
@@ -271,7 +279,8 @@ def decode_noalloc(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor
 
 def _block_table(block_table, B: int, device) -> torch.Tensor:
     t = block_table
-    if not (isinstance(t, torch.Tensor) and t.is_cuda and t.dtype == torch.int32 and t.is_contiguous()):
+    if not (isinstance(t, torch.Tensor) and t.is_cuda and t.device == torch.device(device)
+            and t.dtype == torch.int32 and t.is_contiguous()):
         t = torch.as_tensor(block_table, dtype=torch.int32, device=device).contiguous()
     if t.dim() != 2 or t.shape[0] != B:
         raise ValueError("block_table must be (B, max_pages)")

@@ -178,3 +178,33 @@ def test_mla_and_backward_host_side_argument_errors(lib):
     assert bwd(bytes=8) == 5
     assert lib.gqa_prefill_backward_workspace_size(1, 4, 8) == 2 * 256
     assert lib.gqa_prefill_backward_workspace_size(0, 4, 8) == 0
+
+
+class _FakeCudaTensor:
+    """Stands in for a CUDA tensor on a machine without a GPU (only what the binding's checks read)."""
+
+    def __init__(self, index, contiguous=True):
+        import torch
+
+        self.is_cuda = True
+        self.device = torch.device("cuda", index)
+        self._contiguous = contiguous
+
+    def is_contiguous(self):
+        return self._contiguous
+
+
+def test_binding_rejects_tensors_off_the_current_device(monkeypatch):
+    """The library launches on the current device and stream, so every tensor must live there."""
+    import torch
+
+    from kv_cache_attention_gqa_b200 import _lib
+
+    monkeypatch.setattr(torch.cuda, "current_device", lambda: 1)
+    _lib._need_cuda(_FakeCudaTensor(1), None, _FakeCudaTensor(1))
+    with pytest.raises(ValueError, match="current CUDA device"):
+        _lib._need_cuda(_FakeCudaTensor(1), _FakeCudaTensor(0))
+    with pytest.raises(ValueError, match="contiguous"):
+        _lib._need_cuda(_FakeCudaTensor(1, contiguous=False))
+    with pytest.raises(ValueError, match="CUDA device"):
+        _lib._need_cuda(torch.zeros(2))

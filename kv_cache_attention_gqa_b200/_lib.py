@@ -138,6 +138,22 @@ def _int_vec(x, B: int, device, name: str):
     return t
 
 
+def _out(out, shape, dtype, device):
+    """The output tensor: a new one, or the caller's after checking its shape and dtype (the kernels
+    write every element of ``shape``; a smaller buffer would be overrun)."""
+    if out is None:
+        return torch.empty(shape, dtype=dtype, device=device)
+    if tuple(out.shape) != tuple(shape) or out.dtype != dtype:
+        raise ValueError(f"out must be {dtype} of shape {tuple(shape)}, not {out.dtype} {tuple(out.shape)}")
+    return out
+
+
+def _ws_bytes(ws) -> int:
+    """Byte size of a caller workspace, which must be a contiguous tensor on the current device."""
+    _need_cuda(ws)
+    return ws.numel() * ws.element_size()
+
+
 def _stream():
     return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
 
@@ -181,8 +197,7 @@ def prefill(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, *, q_
     dt = _dtype_code(q)
     if k_cache.dtype != q.dtype or v_cache.dtype != q.dtype:
         raise TypeError("q, k_cache and v_cache must share one dtype")
-    if out is None:
-        out = torch.empty_like(q)
+    out = _out(out, q.shape, q.dtype, q.device)
     lse = torch.empty((B, h_q, S_q), dtype=torch.float32, device=q.device) if return_lse else None
     qs = _int_vec(q_start, B, q.device, "q_start")
     kl = _int_vec(kv_len, B, q.device, "kv_len")
@@ -233,8 +248,7 @@ def decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, *, kv_
     dt = _dtype_code(q)
     if k_cache.dtype != q.dtype or v_cache.dtype != q.dtype:
         raise TypeError("q, k_cache and v_cache must share one dtype")
-    if out is None:
-        out = torch.empty_like(q)
+    out = _out(out, q.shape, q.dtype, q.device)
     lse = torch.empty((B, h_q), dtype=torch.float32, device=q.device) if return_lse else None
     kl = _int_vec(kv_len, B, q.device, "kv_len")
     qp = _int_vec(q_pos, B, q.device, "q_pos")
@@ -247,7 +261,7 @@ def decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, *, kv_
         ws = workspace(need, q.device)
     _check("gqa_decode", _lib.gqa_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(out), _ptr(lse),
                                          _ptr(kl), _ptr(qp), B, h_q, h_kv, T_max, d_h, scale,
-                                         int(window), dt, _ptr(ws), ws.numel(), num_splits, _stream()))
+                                         int(window), dt, _ptr(ws), _ws_bytes(ws), num_splits, _stream()))
     return (out, lse) if return_lse else out
 
 
@@ -265,8 +279,7 @@ def decode_noalloc(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor
     dt = _dtype_code(q)
     if k_cache.dtype != q.dtype or v_cache.dtype != q.dtype:
         raise TypeError("q, k_cache and v_cache must share one dtype")
-    if out is None:
-        out = torch.empty_like(q)
+    out = _out(out, q.shape, q.dtype, q.device)
     lse = torch.empty((B, h_q), dtype=torch.float32, device=q.device) if return_lse else None
     kl = _int_vec(kv_len, B, q.device, "kv_len")
     qp = _int_vec(q_pos, B, q.device, "q_pos")
@@ -310,8 +323,7 @@ def decode_paged(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.Tensor, 
         raise TypeError("q, k_pages and v_pages must share one dtype")
     bt = _block_table(block_table, B, q.device)
     max_pages = bt.shape[1]
-    if out is None:
-        out = torch.empty_like(q)
+    out = _out(out, q.shape, q.dtype, q.device)
     lse = torch.empty((B, h_q), dtype=torch.float32, device=q.device) if return_lse else None
     kl = _int_vec(kv_len, B, q.device, "kv_len")
     qp = _int_vec(q_pos, B, q.device, "q_pos")
@@ -325,7 +337,7 @@ def decode_paged(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.Tensor, 
         ws = workspace(need, q.device)
     _check("gqa_decode_paged", _lib.gqa_decode_paged(
         _ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(out), _ptr(lse), _ptr(kl), _ptr(qp), _ptr(bt),
-        B, h_q, h_kv, num_pages, page_size, max_pages, d_h, scale, int(window), dt, _ptr(ws), ws.numel(),
+        B, h_q, h_kv, num_pages, page_size, max_pages, d_h, scale, int(window), dt, _ptr(ws), _ws_bytes(ws),
         num_splits, _stream()))
     return (out, lse) if return_lse else out
 
@@ -372,12 +384,12 @@ def prefill_backward(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tens
     kl = _int_vec(kv_len, B, q.device, "kv_len")
     scale = 1.0 / math.sqrt(d_h) if scale is None else float(scale)
     need = _lib.gqa_prefill_backward_workspace_size(B, h_q, S_q)
-    if ws is None or ws.numel() < need:
+    if ws is None or _ws_bytes(ws) < need:
         ws = torch.empty(need, dtype=torch.uint8, device=q.device)
     _check("gqa_prefill_backward", _lib.gqa_prefill_backward(
         _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(o), _ptr(d_o), _ptr(lse), _ptr(dq), _ptr(dk),
         _ptr(dv), _ptr(qs), _ptr(kl), B, h_q, h_kv, S_q, T_max, d_h, scale, 1 if causal else 0,
-        int(window), dt, _ptr(ws), ws.numel(), _stream()))
+        int(window), dt, _ptr(ws), _ws_bytes(ws), _stream()))
     return dq, dk, dv
 
 
@@ -395,8 +407,7 @@ def mla_decode(q: torch.Tensor, cache: torch.Tensor, d_v: int = 512, *, kv_len=N
     dt = _dtype_code(q)
     if cache.dtype != q.dtype:
         raise TypeError("q and cache must share one dtype")
-    if out is None:
-        out = torch.empty((B, h_q, d_v), dtype=q.dtype, device=q.device)
+    out = _out(out, (B, h_q, d_v), q.dtype, q.device)
     lse = torch.empty((B, h_q), dtype=torch.float32, device=q.device) if return_lse else None
     kl = _int_vec(kv_len, B, q.device, "kv_len")
     qp = _int_vec(q_pos, B, q.device, "q_pos")
@@ -412,5 +423,5 @@ def mla_decode(q: torch.Tensor, cache: torch.Tensor, d_v: int = 512, *, kv_len=N
         ws = workspace(need, q.device)
     _check("gqa_mla_decode", _lib.gqa_mla_decode(
         _ptr(q), _ptr(cache), _ptr(out), _ptr(lse), _ptr(kl), _ptr(qp), B, h_q, T_max, d_qk, d_v,
-        scale, dt, _ptr(ws), ws.numel(), num_splits, _stream()))
+        scale, dt, _ptr(ws), _ws_bytes(ws), num_splits, _stream()))
     return (out, lse) if return_lse else out

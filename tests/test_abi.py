@@ -208,3 +208,31 @@ def test_binding_rejects_tensors_off_the_current_device(monkeypatch):
         _lib._need_cuda(_FakeCudaTensor(1, contiguous=False))
     with pytest.raises(ValueError, match="CUDA device"):
         _lib._need_cuda(torch.zeros(2))
+
+
+def test_binding_checks_caller_outputs_and_workspaces(monkeypatch):
+    """A caller's output must have the exact shape and dtype the kernel writes; a caller's
+    workspace is sized in bytes whatever its element type, and must be a device tensor."""
+    import torch
+
+    from kv_cache_attention_gqa_b200 import _lib
+
+    out = torch.empty(2, 3, 4, dtype=torch.bfloat16)
+    assert _lib._out(out, (2, 3, 4), torch.bfloat16, "cpu") is out
+    assert _lib._out(None, (2, 3, 4), torch.float32, "cpu").shape == (2, 3, 4)
+    with pytest.raises(ValueError, match="shape"):
+        _lib._out(out, (2, 3, 5), torch.bfloat16, "cpu")
+    with pytest.raises(ValueError, match="shape"):
+        _lib._out(out, (2, 3, 4), torch.float32, "cpu")
+    with pytest.raises(ValueError, match="CUDA device"):
+        _lib._ws_bytes(torch.zeros(16, dtype=torch.uint8))
+
+    class _FakeWs(_FakeCudaTensor):
+        def numel(self):
+            return 10
+
+        def element_size(self):
+            return 4
+
+    monkeypatch.setattr(torch.cuda, "current_device", lambda: 0)
+    assert _lib._ws_bytes(_FakeWs(0)) == 40

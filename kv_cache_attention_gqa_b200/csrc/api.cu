@@ -240,6 +240,14 @@ gqa_status gqa_prefill(const void* q, const void* k_cache, const void* v_cache, 
     return GQA_ERR_INVALID_ARG;
   if (h_q % h_kv != 0 || !valid_scale(scale)) return GQA_ERR_INVALID_ARG;
   if (causal != 0 && causal != 1) return GQA_ERR_INVALID_ARG;
+  // every host-detectable problem is reported before the first CUDA call
+  if (dtype != GQA_BF16 && dtype != GQA_FP32) return GQA_ERR_INVALID_ARG;
+  if (dtype == GQA_FP32 && d_h > 256) return GQA_ERR_UNSUPPORTED;
+  if (dtype == GQA_BF16) {
+    if (d_h != 64 && d_h != 128) return GQA_ERR_UNSUPPORTED;
+    if ((long long)B * h_kv * T_max >= (1ll << 31) || (long long)B * h_q * S_q >= (1ll << 31))
+      return GQA_ERR_UNSUPPORTED;
+  }
   PrefillArgs a;
   a.q = q;
   a.k = k_cache;
@@ -260,14 +268,7 @@ gqa_status gqa_prefill(const void* q, const void* k_cache, const void* v_cache, 
   a.err = device_error_ptr();
   if (!a.err) return GQA_ERR_CUDA;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (dtype == GQA_FP32) {
-    if (d_h > 256) return GQA_ERR_UNSUPPORTED;
-    return from_cuda(launch_prefill_fp32(a, s));
-  }
-  if (dtype != GQA_BF16) return GQA_ERR_INVALID_ARG;
-  if (d_h != 64 && d_h != 128) return GQA_ERR_UNSUPPORTED;
-  if ((long long)B * h_kv * T_max >= (1ll << 31) || (long long)B * h_q * S_q >= (1ll << 31))
-    return GQA_ERR_UNSUPPORTED;
+  if (dtype == GQA_FP32) return from_cuda(launch_prefill_fp32(a, s));
   // TMA views: Q as (d_h, S_q, B*h_q) with box (64, P, H): one box holds the H heads x P
   // positions of a tile, head-major; K, V as rows (B*h_kv*T_max, d_h) with box (64, 128).
   const int H = prefill_heads_per_tile(h_q, h_kv);

@@ -70,6 +70,16 @@ def test_host_side_argument_errors(lib):
     assert lib.gqa_prefill(fake, fake, fake, fake, null, null, null, 1, 4, 2, 8, 8, 64, 0.1, 1, -1, 0, s) == 1
     assert lib.gqa_prefill(fake, fake, fake, fake, null, null, null, 1, 4, 2, 8, 8, 64, 0.1, 0, 4, 0, s) == 1
     assert lib.gqa_decode(fake, fake, fake, fake, null, null, null, 1, 4, 2, 8, 64, 0.1, -1, 0, fake, 1 << 20, 1, s) == 1
+    # prefill: unsupported head dims, an unknown dtype and sizes past 32-bit row indexing, all reported
+    # before any CUDA call
+    assert lib.gqa_prefill(fake, fake, fake, fake, null, null, null, 1, 4, 2, 8, 8, 96, 0.1, 1, 0, 0, s) == 2
+    assert lib.gqa_prefill(fake, fake, fake, fake, null, null, null, 1, 4, 2, 8, 8, 300, 0.1, 1, 0, 1, s) == 2
+    assert lib.gqa_prefill(fake, fake, fake, fake, null, null, null, 1, 4, 2, 8, 8, 64, 0.1, 1, 0, 7, s) == 1
+    assert lib.gqa_prefill(fake, fake, fake, fake, null, null, null, 1024, 32, 32, 8, 65536, 128, 0.1, 1, 0, 0, s) == 2
+    assert lib.gqa_prefill(fake, fake, fake, fake, null, null, null, 1024, 32, 8, 65536, 8, 128, 0.1, 1, 0, 0, s) == 2
+    # decode: cache rows past 32-bit row indexing
+    assert lib.gqa_decode(fake, fake, fake, fake, null, null, null, 1024, 32, 32, 65536, 128, 0.1, 0, 0, fake,
+                          1 << 20, 1, s) == 2
     assert lib.gqa_decode_noalloc(fake, fake, fake, fake, null, null, null, 1, 4, 2, 8, 64, 0.1, -1, 0, 1, s) == 1
     # decode
     assert lib.gqa_decode(null, fake, fake, fake, null, null, null, 1, 4, 2, 8, 64, 0.1, 0, 0, fake, 1 << 20, 1, s) == 1

@@ -1,11 +1,12 @@
-// 2^x on the FMA/ALU pipes, for part of the softmax exponentials (the special-function unit is
-// the prefill softmax's bottleneck).
+// 2^x on the FMA/ALU pipes, to move part of the softmax exponentials off the special-function
+// unit. The prefill kernel measured slower with it (its softmax is bound by latency, not by that
+// unit), so GQA_PREFILL_POLY_EVERY keeps it off by default.
 //
 // Method: Cody-Waite range reduction. x = n + f with n = rint(x), obtained by adding 1.5 * 2^23
 // (which leaves the rounded integer in the low mantissa bits), and f = x - n in [-1/2, 1/2].
 // 2^f is a degree-3 polynomial, a relative-error minimax fit on [-1/2, 1/2] made for this
 // library by Remez exchange (max relative error 7.5e-5 in fp32 coefficients, far below the 2^-9
-// rounding of the bf16 P it feeds). 2^n is added to the exponent field: bits(2^f) + (bits(t) << 23).
+// rounding of the bf16 P it feeds; tests/test_exp2_poly.py re-derives the constants). 2^n is added to the exponent field: bits(2^f) + (bits(t) << 23).
 // Inputs are clamped to >= -126 so the exponent field cannot wrap; callers use this only where
 // every input is finite (blocks without masked keys), so masked weights stay exactly 0.
 #pragma once

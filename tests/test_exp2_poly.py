@@ -41,3 +41,31 @@ def test_range_reduction_in_fp32():
     normal = x >= -125.0
     assert np.all(np.abs(y[normal] / ref[normal] - 1.0) < 1e-4)
     assert np.all(y >= 0) and np.all(np.isfinite(y))
+
+
+def _remez_relative(deg, a=-0.5, b=0.5, iters=30, grid=200001):
+    """Minimax fit of 2^f in relative error by Remez exchange: solve for the coefficients that make
+    the relative error equioscillate at deg + 2 reference points, then move the points to the
+    extrema of the error's sign-constant runs."""
+    n = deg + 2
+    x = 0.5 * (a + b) + 0.5 * (b - a) * np.cos(np.pi * np.arange(n)[::-1] / (n - 1))
+    xs = np.linspace(a, b, grid)
+    for _ in range(iters):
+        A = np.zeros((n, n))
+        A[:, :deg + 1] = x[:, None] ** np.arange(deg + 1)
+        A[:, deg + 1] = (-1.0) ** np.arange(n) * 2.0 ** x
+        c = np.linalg.solve(A, 2.0 ** x)[:deg + 1]
+        err = np.polyval(c[::-1], xs) / 2.0 ** xs - 1.0
+        runs = np.split(np.arange(grid), np.flatnonzero(np.diff(np.sign(err))) + 1)
+        ext = [r[np.argmax(np.abs(err[r]))] for r in runs]
+        if len(ext) > n:
+            ext = sorted(ext, key=lambda i: -abs(err[i]))[:n]
+        if len(ext) == n:
+            x = np.sort(xs[ext])
+    return c
+
+
+def test_coefficients_are_the_minimax_fit():
+    """The header's constants are the degree-3 relative-error minimax fit, rounded to fp32."""
+    fit = _remez_relative(3).astype(np.float32)
+    assert np.array_equal(fit.view(np.uint32), _coeffs().view(np.uint32))

@@ -13,9 +13,9 @@
 // staged in shared memory serves all r heads of the group [MHA/MQA/GQA walkthrough, section 7:
 // e.g. 32 positions x 4 heads = 128 rows; the mask still uses each row's own position].
 //
-// Roles (256 threads, one 128-row tile per CTA):
-//   warp 0      TMA producer: the tile's Q rows once, then 128-key K blocks and V blocks into two
-//               3-deep rings (cp.async.bulk.tensor, 128-byte swizzle, no multicast).
+// Roles (384 threads, one 128-row tile per CTA):
+//   warp 0      TMA producer: the tile's Q rows once, then 128-key K blocks into a 3-deep ring and
+//               V blocks into a 2-deep ring (cp.async.bulk.tensor, 128-byte swizzle, no multicast).
 //   warp 1      allocates 512 TMEM columns and issues every MMA from one thread:
 //               S_j = Q K_j^T  (tcgen05.mma kind::f16, A = Q from TMEM, B = K from shared memory),
 //               O  += P_j V_j  (A = P_j from TMEM, B = V from shared memory, MN-major).
@@ -23,11 +23,16 @@
 //               the next block are ready when the softmax finishes the current one. Both MMAs read
 //               only one operand from shared memory (a 128x128x16 MMA with both operands there
 //               would need the whole shared-memory bandwidth).
-//   warps 4-7   softmax, one thread per row (TMEM lane). Each first copies its Q row from shared
-//               memory into TMEM, then per block reads its score row, masks by absolute position,
-//               updates (m, l), writes P = 2^(s - m) as bf16 into the block's S columns, and
-//               rescales its O row only when the running maximum grew by more than 8 (base 2):
-//               between rescales P and l share the stale maximum, which leaves O = u / l unchanged.
+//   warps 4-11  softmax: two warpgroups serve the same 128 rows (one row per TMEM lane), each
+//               taking 64 of every block's 128 score columns. First each copies its 64-column
+//               chunk of the Q rows from shared memory into TMEM. Per block each thread reads its
+//               half row and masks it by absolute position (one clamped 32-bit bound per row);
+//               the two halves meet at a named barrier to share the block's row maximum. Each
+//               half then writes
+//               P = 2^(s - m) as bf16 into its share of the block's first 64 S columns and
+//               rescales its half of the O row only when the running maximum grew by more than 8
+//               (base 2): between rescales P and l share the stale maximum, which leaves
+//               O = u / l unchanged. The row sums meet once, at the end.
 // TMEM columns: S_0 [0,128), S_1 [128,256), O [256, 256+D), Q [256+D, 256+3D/2); P_b aliases the
 // first 64 columns of S_b. MMAs issued by one thread execute in order, so S_b of block j+2 is
 // written only after O += P_j V_j has read P_j.

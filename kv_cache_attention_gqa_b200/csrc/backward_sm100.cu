@@ -15,13 +15,18 @@
 //             shares of dK and dV add up in TMEM (no atomics):
 //               S^T  = K Q^T     tcgen05.mma, A = K and B = Q from shared memory (K-major)
 //               dP^T = V dO^T    A = V, B = dO from shared memory
-//               (4 warps) P^T = 2^(S^T c - lse2), dS^T = P^T (dP^T - D) -> bf16 into TMEM
+//               (8 warps: two per TMEM lane quarter, one per 32-column half of the block)
+//               P^T = 2^(S^T c - lse2), dS^T = P^T (dP^T - D) -> bf16 into TMEM
 //               dV  += P^T dO    A = P^T from TMEM, B = dO (MN-major view of the same tile)
 //               dK  += dS^T Q    A = dS^T from TMEM, B = Q (MN-major)
 //   dq        one CTA per forward tile (H heads x P positions of one group), walking the 64-key
 //             K/V blocks the tile sees:
-//               S = Q K^T, dP = dO V^T (A = Q / dO, B = K / V from shared memory), then dS -> bf16
-//               into TMEM, dQ += dS K (A = dS from TMEM, B = K, MN-major view).
+//               S = Q K^T, dP = dO V^T (A = the tile's Q / dO rows, copied once into TMEM;
+//               B = K / V from shared memory), then dS -> bf16 into TMEM, dQ += dS K (A = dS from
+//               TMEM, B = K, MN-major view).
+// Masks: on blocks that straddle the diagonal, the window or the length, each elementwise thread
+// compares indices with one pair of 32-bit bounds fixed for the block: the query columns that see
+// its key (dkdv) or the keys its row sees (dq).
 // TMEM (512 columns): S double-buffered at [0,64) and [64,128), dP at [128,192) and [192,256),
 // accumulators from 256; P / dS (bf16 pairs) are written over the first columns of the scores
 // they come from. MMAs issued by one thread execute in order, so a buffer is rewritten only

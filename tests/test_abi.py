@@ -246,3 +246,23 @@ def test_binding_checks_caller_outputs_and_workspaces(monkeypatch):
 
     monkeypatch.setattr(torch.cuda, "current_device", lambda: 0)
     assert _lib._ws_bytes(_FakeWs(0)) == 40
+
+
+def test_plain_c_client_compiles_links_and_runs(tmp_path):
+    """gqa.h is a C header (strict C99, no C++ or CUDA types in the signatures): a C program that
+    includes only it links against the library and makes the host-only calls."""
+    import shutil
+
+    from kv_cache_attention_gqa_b200 import _lib
+
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    exe = str(tmp_path / "client")
+    lib_dir = os.path.dirname(_lib.LIB_PATH)
+    subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic", "-I", os.path.join(ROOT, "include"),
+                    os.path.join(ROOT, "tests", "c_abi_client.c"), "-o", exe, "-L", lib_dir, "-lgqa_b200",
+                    "-Wl,-rpath," + lib_dir], check=True, capture_output=True, text=True)
+    r = subprocess.run([exe], capture_output=True, text=True, timeout=60)
+    assert r.returncode == 0, r.stderr
+    assert "sm_100a" in r.stdout

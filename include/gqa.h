@@ -94,8 +94,10 @@ enum {
  *
  * A chunked prefill over an existing cache is kv_append(...) of the chunk's K/V at position p,
  * then gqa_prefill with q_start[b] = p and kv_len[b] = p + S_q.
- * Errors: INVALID_ARG (nulls, sizes <= 0, h_q % h_kv, scale, window < 0 or a window without the
- * causal mask), UNSUPPORTED (bf16 d_h), CUDA.
+ * Errors: INVALID_ARG (nulls, sizes <= 0, h_q % h_kv, scale, an unknown dtype, window < 0 or a
+ * window without the causal mask), UNSUPPORTED (bf16 d_h outside {64, 128}, fp32 d_h > 256, or in
+ * bf16 B*h_kv*T_max or B*h_q*S_q at or above 2^31 rows), CUDA. Every status but CUDA is decided on
+ * the host before any CUDA call.
  */
 gqa_status gqa_prefill(const void* q, const void* k_cache, const void* v_cache, void* o,
                        float* lse, const int32_t* q_start, const int32_t* kv_len,

@@ -29,6 +29,9 @@
  *     asynchronous on that stream; the library keeps no per-request state and allocates nothing
  *     per call (tensor-map descriptors are encoded on the host and passed by value).
  *   - Buffers are owned by the caller. The library never frees or retains them after the call.
+ *   - The library caches a little per-device state on first use (the device address of its error
+ *     word, kernel attributes). A device reset (cudaDeviceReset) invalidates it: after resetting a
+ *     device, do not call the library on that device again in the same process.
  *   - Host-detectable argument errors return a status without launching anything. Errors that only
  *     the device can see (a length or position out of range, a query with no visible key) never
  *     trap: the kernel writes zeros for the affected output rows, records the first such error in
@@ -46,7 +49,8 @@ extern "C" {
 
 typedef enum {
   GQA_OK = 0,
-  GQA_ERR_INVALID_ARG = 1, /* null pointer, non-positive size, h_q % h_kv != 0, bad scale ...   */
+  GQA_ERR_INVALID_ARG = 1, /* null pointer, non-positive size, h_q % h_kv != 0, a scale that is
+                              negative, NaN or infinite ...                                        */
   GQA_ERR_UNSUPPORTED = 2, /* a valid request this build does not implement (e.g. bf16 d_h 96)  */
   GQA_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed (launch, symbol, tensor map)      */
   GQA_ERR_DEVICE = 4,      /* returned by gqa_get_device_error when the device word was set       */
@@ -80,7 +84,8 @@ enum {
  *            (the softmax normaliser; written when non-NULL).
  *   q_start  device int32[B] or NULL (= all 0): absolute position of query row 0.
  *   kv_len   device int32[B] or NULL (= all T_max): keys present, 1 <= kv_len[b] <= T_max.
- *   scale    finite, > 0; pass 1/sqrt(d_h) for the standard scaling.
+ *   scale    finite and > 0, or 0 for the standard 1/sqrt(d_h) (computed in double precision and
+ *            rounded once to fp32). The same rule holds for every call that takes a scale.
  *   causal   1: key j visible to row i iff j <= q_start[b] + i and j < kv_len[b];
  *            0: iff j < kv_len[b].
  *   window   0: no window. W > 0 (requires causal = 1): sliding-window attention, each row reads
@@ -119,7 +124,8 @@ gqa_status gqa_prefill(const void* q, const void* k_cache, const void* v_cache, 
  *   cache  (B, T_max, d_qk): [latent (d_v) | rotary key part], shared by all heads.
  *   o      (B, h_q, d_v) written (latent output). lse: (B, h_q) fp32 or NULL (natural log).
  *   kv_len, q_pos: as gqa_decode. scale: the model's softmax scale (for absorbed MLA this is
- *          1/sqrt(d_nope + d_rope) of the original heads, not 1/sqrt(d_qk)).
+ *          1/sqrt(d_nope + d_rope) of the original heads, not 1/sqrt(d_qk)); 0 selects
+ *          1/sqrt(d_qk), which is rarely the right value for a real model.
  *   dtype  GQA_BF16: d_qk = 576 and d_v = 512 (the DeepSeek-V2/V3 latent and rotary widths);
  *          GQA_FP32: d_qk <= 768, d_v <= min(d_qk, 512) (check mode).
  *   workspace: >= gqa_mla_decode_workspace_size(B, h_q, T_max, d_v, dtype, num_splits) bytes,
@@ -154,8 +160,9 @@ gqa_status gqa_mla_decode(const void* q, const void* cache, void* o, float* lse,
  *               scalar check mode, fp32 gradients). All tensors share the dtype; lse is fp32.
  *   workspace   device memory of at least gqa_prefill_backward_workspace_size(B, h_q, S_q) bytes,
  *               256-byte aligned, no initial contents required (two fp32 values per query row).
- * Three kernels run in order on `stream`: the row term D, the key-stationary dK/dV pass (the heads
- * of a group add up in one CTA, no atomics), and the query-stationary dQ pass.
+ * Two launches run in order on `stream`: the row term D (with the base-2 lse), then one grid
+ * whose first CTAs run the key-stationary dK/dV pass (the heads of a group add up in one CTA, no
+ * atomics) and whose remaining CTAs run the query-stationary dQ pass.
  * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA.
  */
 size_t gqa_prefill_backward_workspace_size(int B, int h_q, int S_q);
@@ -217,11 +224,13 @@ gqa_status gqa_decode(const void* q, const void* k_cache, const void* v_cache, v
  *   - Shapes whose workspace (gqa_decode_workspace_size) exceeds 16 MiB are rejected with
  *     GQA_ERR_WORKSPACE; use gqa_decode with your own workspace for those.
  *   - The first call on a device looks up the scratch array's device address and caches it; make
- *     that first call before any stream capture.
+ *     that first call before any stream capture. A device reset (cudaDeviceReset) frees the array
+ *     and leaves that address stale: do not call the library on a device after resetting it.
  *   - All calls share the one array, which keeps the previous call's contents; the part that must
  *     start at zero is cleared on `stream` before each launch. Calls that overlap on the GPU (on
  *     different streams or from different host threads) race on the array: serialise them.
- * Errors: as gqa_decode.
+ * Errors: as gqa_decode, checked in the same order (so an unsupported shape is UNSUPPORTED even
+ * when its workspace would also exceed the scratch array), then WORKSPACE for the size limit.
  */
 gqa_status gqa_decode_noalloc(const void* q, const void* k_cache, const void* v_cache, void* o,
                               float* lse, const int32_t* kv_len, const int32_t* q_pos,
@@ -302,8 +311,23 @@ gqa_status gqa_get_device_error(int* code, void* stream);
 /* Human-readable name of a status. Never NULL. */
 const char* gqa_status_string(gqa_status s);
 
-/* Library version string, e.g. "gqa-b200 0.1.0 (sm_100a)". */
+/* Library version string, e.g. "gqa-b200 0.2.0 (sm_100a)". */
 const char* gqa_version(void);
+
+/*
+ * gqa_debug_expire_waits - failure-detection test hook; never needed in normal use.
+ * Every pipeline wait of the kernels is bounded (about 2 s of %globaltimer); when one runs out the
+ * kernel records GQA_DEVERR_TIMEOUT and returns instead of spinning, so the context stays usable.
+ * With enable = 1, every later bf16 gqa_prefill and contiguous bf16 gqa_decode on any device makes
+ * CTA 0 wait on a barrier that nothing signals, so that bound is reached on purpose: the call
+ * takes about 2 s longer, the error word reads GQA_DEVERR_TIMEOUT, prefill writes the rows of the
+ * tile that gave up as zeros (lse = -inf), and decode leaves the rows of CTA 0's first chunk
+ * unspecified. A following call with the hook off is unaffected (a decode workspace stays
+ * reusable). enable = 0 (the default) turns it off. Other calls ignore it. Not thread-safe with
+ * respect to concurrent launches: set it only while no other thread calls the library.
+ * Errors: INVALID_ARG (enable not 0 or 1).
+ */
+gqa_status gqa_debug_expire_waits(int enable);
 
 #ifdef __cplusplus
 }

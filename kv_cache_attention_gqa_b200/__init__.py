@@ -10,6 +10,7 @@ The computation lives in the CUDA library ``libgqa_b200.so`` behind the C ABI of
 from ._lib import (  # noqa: F401
     GQAError,
     LIB_PATH,
+    debug_expire_waits,
     decode,
     decode_noalloc,
     decode_paged,

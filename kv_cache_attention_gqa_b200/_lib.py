@@ -9,7 +9,6 @@ fallback: if the library is missing, importing this module raises.
 from __future__ import annotations
 
 import ctypes
-import math
 import os
 import threading
 
@@ -51,6 +50,7 @@ SIGNATURES = {
     "gqa_get_device_error": (_I, [ctypes.POINTER(_I), _P]),
     "gqa_status_string": (ctypes.c_char_p, [_I]),
     "gqa_version": (ctypes.c_char_p, []),
+    "gqa_debug_expire_waits": (_I, [_I]),
 }
 
 
@@ -154,8 +154,19 @@ def _ws_bytes(ws) -> int:
     return ws.numel() * ws.element_size()
 
 
+def _scale(scale) -> float:
+    """None -> 0.0, which the C ABI reads as its default 1/sqrt(d_h) (MLA: 1/sqrt(d_qk))."""
+    return 0.0 if scale is None else float(scale)
+
+
 def _stream():
     return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def debug_expire_waits(enable: bool) -> None:
+    """Failure-detection test hook (gqa_debug_expire_waits): while enabled, bf16 prefill and
+    contiguous bf16 decode make one bounded wait run out, so the call reports a timeout."""
+    _check("gqa_debug_expire_waits", _lib.gqa_debug_expire_waits(1 if enable else 0))
 
 
 def get_device_error() -> int:
@@ -201,7 +212,7 @@ def prefill(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, *, q_
     lse = torch.empty((B, h_q, S_q), dtype=torch.float32, device=q.device) if return_lse else None
     qs = _int_vec(q_start, B, q.device, "q_start")
     kl = _int_vec(kv_len, B, q.device, "kv_len")
-    scale = 1.0 / math.sqrt(d_h) if scale is None else float(scale)
+    scale = _scale(scale)
     _check("gqa_prefill", _lib.gqa_prefill(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(out), _ptr(lse),
                                            _ptr(qs), _ptr(kl), B, h_q, h_kv, S_q, T_max, d_h, scale,
                                            1 if causal else 0, int(window), dt, _stream()))
@@ -252,7 +263,7 @@ def decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, *, kv_
     lse = torch.empty((B, h_q), dtype=torch.float32, device=q.device) if return_lse else None
     kl = _int_vec(kv_len, B, q.device, "kv_len")
     qp = _int_vec(q_pos, B, q.device, "q_pos")
-    scale = 1.0 / math.sqrt(d_h) if scale is None else float(scale)
+    scale = _scale(scale)
     key = (B, h_q, h_kv, T_max, d_h, dt, num_splits, q.device.index)
     need = _ws_sizes.get(key)
     if need is None:
@@ -283,7 +294,7 @@ def decode_noalloc(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor
     lse = torch.empty((B, h_q), dtype=torch.float32, device=q.device) if return_lse else None
     kl = _int_vec(kv_len, B, q.device, "kv_len")
     qp = _int_vec(q_pos, B, q.device, "q_pos")
-    scale = 1.0 / math.sqrt(d_h) if scale is None else float(scale)
+    scale = _scale(scale)
     _check("gqa_decode_noalloc", _lib.gqa_decode_noalloc(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(out),
                                                          _ptr(lse), _ptr(kl), _ptr(qp), B, h_q, h_kv, T_max,
                                                          d_h, scale, int(window), dt, num_splits, _stream()))
@@ -327,7 +338,7 @@ def decode_paged(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.Tensor, 
     lse = torch.empty((B, h_q), dtype=torch.float32, device=q.device) if return_lse else None
     kl = _int_vec(kv_len, B, q.device, "kv_len")
     qp = _int_vec(q_pos, B, q.device, "q_pos")
-    scale = 1.0 / math.sqrt(d_h) if scale is None else float(scale)
+    scale = _scale(scale)
     T_max = max_pages * page_size
     key = (B, h_q, h_kv, T_max, d_h, dt, num_splits, q.device.index)
     need = _ws_sizes.get(key)
@@ -382,7 +393,7 @@ def prefill_backward(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tens
     dv = torch.empty_like(v_cache)
     qs = _int_vec(q_start, B, q.device, "q_start")
     kl = _int_vec(kv_len, B, q.device, "kv_len")
-    scale = 1.0 / math.sqrt(d_h) if scale is None else float(scale)
+    scale = _scale(scale)
     need = _lib.gqa_prefill_backward_workspace_size(B, h_q, S_q)
     if ws is None or _ws_bytes(ws) < need:
         ws = torch.empty(need, dtype=torch.uint8, device=q.device)
@@ -411,7 +422,7 @@ def mla_decode(q: torch.Tensor, cache: torch.Tensor, d_v: int = 512, *, kv_len=N
     lse = torch.empty((B, h_q), dtype=torch.float32, device=q.device) if return_lse else None
     kl = _int_vec(kv_len, B, q.device, "kv_len")
     qp = _int_vec(q_pos, B, q.device, "q_pos")
-    scale = 1.0 / math.sqrt(d_qk) if scale is None else float(scale)
+    scale = _scale(scale)
     key = ("mla", B, h_q, T_max, d_v, dt, num_splits, q.device.index)
     need = _ws_sizes.get(key)
     if need is None:

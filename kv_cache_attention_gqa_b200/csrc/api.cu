@@ -3,6 +3,7 @@
 
 #include <cudaTypedefs.h>
 #include <math.h>
+#include <atomic>
 #include <mutex>
 #include <string.h>
 
@@ -17,6 +18,10 @@ __device__ unsigned g_device_error_word;
 namespace {
 
 constexpr int kMaxDevices = 64;
+
+// Test hook set by gqa_debug_expire_waits: the bf16 prefill and the contiguous bf16 decode pass
+// it to their kernels, whose CTA 0 then waits on a barrier that nothing signals.
+std::atomic<int> g_expire_waits{0};
 
 unsigned* device_error_ptr() {
   static unsigned* ptrs[kMaxDevices] = {nullptr};
@@ -70,12 +75,33 @@ bool encode_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* d
   return r == CUDA_SUCCESS;
 }
 
-bool valid_scale(float s) { return isfinite(s) && s > 0.f; }
+// scale: finite and > 0, or exactly 0 for the default 1/sqrt(d_h) (computed in double, then
+// rounded once to fp32, so every caller of the C ABI gets the same fp32 value)
+bool valid_scale(float s) { return isfinite(s) && s >= 0.f; }
+float resolve_scale(float s, int d) { return s == 0.f ? (float)(1.0 / sqrt((double)d)) : s; }
 
 gqa_status from_cuda(cudaError_t e) { return e == cudaSuccess ? GQA_OK : GQA_ERR_CUDA; }
 
 }  // namespace
 
+}  // namespace gqa
+
+namespace gqa {
+gqa_status decode_check_args(const void* q, const void* k_cache, const void* v_cache, const void* o,
+                             int B, int h_q, int h_kv, int T_max, int d_h, float scale, int window,
+                             gqa_dtype dtype, int num_splits, long long cache_rows) {
+  if (!q || !k_cache || !v_cache || !o) return GQA_ERR_INVALID_ARG;
+  if (window < 0) return GQA_ERR_INVALID_ARG;
+  if (B <= 0 || h_q <= 0 || h_kv <= 0 || T_max <= 0 || d_h <= 0 || num_splits < 0)
+    return GQA_ERR_INVALID_ARG;
+  if (h_q % h_kv != 0 || !valid_scale(scale)) return GQA_ERR_INVALID_ARG;
+  if (dtype != GQA_BF16 && dtype != GQA_FP32) return GQA_ERR_INVALID_ARG;
+  if (B > decode_max_batch()) return GQA_ERR_UNSUPPORTED;
+  if (dtype == GQA_FP32 && d_h > 256) return GQA_ERR_UNSUPPORTED;
+  if (dtype == GQA_BF16 && d_h != 64 && d_h != 128) return GQA_ERR_UNSUPPORTED;
+  if (cache_rows >= (1ll << 31) || (long long)B * h_q >= (1ll << 31)) return GQA_ERR_UNSUPPORTED;
+  return GQA_OK;
+}
 }  // namespace gqa
 
 using namespace gqa;
@@ -89,18 +115,12 @@ gqa_status decode_impl(const void* q, const void* k_cache, const void* v_cache, 
                        size_t workspace_bytes, int num_splits, void* stream,
                        const int32_t* block_table, int max_pages, int page_size, int num_pages) {
   using namespace gqa;
-  if (!q || !k_cache || !v_cache || !o) return GQA_ERR_INVALID_ARG;
-  if (window < 0) return GQA_ERR_INVALID_ARG;
-  if (B <= 0 || h_q <= 0 || h_kv <= 0 || T_max <= 0 || d_h <= 0 || num_splits < 0)
-    return GQA_ERR_INVALID_ARG;
-  if (h_q % h_kv != 0 || !valid_scale(scale)) return GQA_ERR_INVALID_ARG;
-  if (dtype != GQA_BF16 && dtype != GQA_FP32) return GQA_ERR_INVALID_ARG;
-  if (B > decode_max_batch()) return GQA_ERR_UNSUPPORTED;
-  if (dtype == GQA_FP32 && d_h > 256) return GQA_ERR_UNSUPPORTED;
-  if (dtype == GQA_BF16 && d_h != 64 && d_h != 128) return GQA_ERR_UNSUPPORTED;
   const long long cache_rows =
       block_table ? (long long)num_pages * h_kv * page_size : (long long)B * h_kv * T_max;
-  if (cache_rows >= (1ll << 31) || (long long)B * h_q >= (1ll << 31)) return GQA_ERR_UNSUPPORTED;
+  const gqa_status st = decode_check_args(q, k_cache, v_cache, o, B, h_q, h_kv, T_max, d_h, scale,
+                                          window, dtype, num_splits, cache_rows);
+  if (st != GQA_OK) return st;
+  scale = resolve_scale(scale, d_h);
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return GQA_ERR_WORKSPACE;
   // the workspace check needs no device query when num_splits is given
   if (num_splits > 0 && workspace_bytes < decode_workspace_bytes(B, h_q, h_kv, T_max, d_h, num_splits, 1))
@@ -132,6 +152,7 @@ gqa_status decode_impl(const void* q, const void* k_cache, const void* v_cache, 
   a.max_pages = max_pages;
   a.page_size = page_size;
   a.num_pages = num_pages;
+  a.expire_wait = g_expire_waits.load(std::memory_order_relaxed);
   a.err = device_error_ptr();
   if (!a.err) return GQA_ERR_CUDA;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -185,7 +206,13 @@ const char* gqa_status_string(gqa_status s) {
   return "GQA_ERR_UNKNOWN";
 }
 
-const char* gqa_version(void) { return "gqa-b200 0.1.0 (sm_100a)"; }
+const char* gqa_version(void) { return "gqa-b200 0.2.0 (sm_100a)"; }
+
+gqa_status gqa_debug_expire_waits(int enable) {
+  if (enable != 0 && enable != 1) return GQA_ERR_INVALID_ARG;
+  g_expire_waits.store(enable, std::memory_order_relaxed);
+  return GQA_OK;
+}
 
 gqa_status gqa_get_device_error(int* code, void* stream) {
   if (!code) return GQA_ERR_INVALID_ARG;
@@ -239,6 +266,7 @@ gqa_status gqa_prefill(const void* q, const void* k_cache, const void* v_cache, 
   if (B <= 0 || h_q <= 0 || h_kv <= 0 || S_q <= 0 || T_max <= 0 || d_h <= 0)
     return GQA_ERR_INVALID_ARG;
   if (h_q % h_kv != 0 || !valid_scale(scale)) return GQA_ERR_INVALID_ARG;
+  scale = resolve_scale(scale, d_h);
   if (causal != 0 && causal != 1) return GQA_ERR_INVALID_ARG;
   // every host-detectable problem is reported before the first CUDA call
   if (dtype != GQA_BF16 && dtype != GQA_FP32) return GQA_ERR_INVALID_ARG;
@@ -265,6 +293,7 @@ gqa_status gqa_prefill(const void* q, const void* k_cache, const void* v_cache, 
   a.scale = scale;
   a.causal = causal;
   a.window = window;
+  a.expire_wait = g_expire_waits.load(std::memory_order_relaxed);
   a.err = device_error_ptr();
   if (!a.err) return GQA_ERR_CUDA;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -302,6 +331,7 @@ gqa_status gqa_prefill_backward(const void* q, const void* k_cache, const void* 
   if (!q || !k_cache || !v_cache || !o || !d_o || !lse || !dq || !dk || !dv) return GQA_ERR_INVALID_ARG;
   if (B <= 0 || h_q <= 0 || h_kv <= 0 || S_q <= 0 || T_max <= 0 || d_h <= 0) return GQA_ERR_INVALID_ARG;
   if (h_q % h_kv != 0 || !valid_scale(scale)) return GQA_ERR_INVALID_ARG;
+  scale = resolve_scale(scale, d_h);
   if (causal != 0 && causal != 1) return GQA_ERR_INVALID_ARG;
   if (window < 0 || (window > 0 && causal != 1)) return GQA_ERR_INVALID_ARG;
   if (dtype != GQA_BF16 && dtype != GQA_FP32) return GQA_ERR_INVALID_ARG;
@@ -400,6 +430,7 @@ gqa_status gqa_mla_decode(const void* q, const void* cache, void* o, float* lse,
   if (B <= 0 || h_q <= 0 || T_max <= 0 || d_qk <= 0 || d_v <= 0 || d_v > d_qk || num_splits < 0)
     return GQA_ERR_INVALID_ARG;
   if (!valid_scale(scale)) return GQA_ERR_INVALID_ARG;
+  scale = resolve_scale(scale, d_qk);
   if (dtype != GQA_BF16 && dtype != GQA_FP32) return GQA_ERR_INVALID_ARG;
   if (dtype == GQA_BF16 && !mla_dims_supported_bf16(d_qk, d_v)) return GQA_ERR_UNSUPPORTED;
   if (dtype == GQA_FP32 && (d_qk > 768 || d_v > 512)) return GQA_ERR_UNSUPPORTED;

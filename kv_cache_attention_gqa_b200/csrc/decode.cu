@@ -130,6 +130,7 @@ struct KArgs {
   // partition granule in keys: 1 for a contiguous cache; on a paged cache 64 when pages hold a
   // multiple of 64 keys (every tile lies in one page), else 16 (every 16-key sub-tile does)
   int gran;
+  int expire_wait;  // test hook: CTA 0's producer first waits on a barrier that nothing signals
 };
 
 // Partition view built in shared memory by every CTA.
@@ -456,7 +457,7 @@ struct Bf16Cfg {
   static constexpr int kStatBytes = MT * 4 * 16 * 4;
   static constexpr size_t kSmem = (size_t)kStages * (kStageBytes + kQBytes) + kRedBytes +
                                   2 * kStatBytes + (kMaxBatch + 1) * 8 + 2 * kMaxBatch * 4 +
-                                  kStages * sizeof(TileMeta) + 2 * kStages * 8 + 1024;
+                                  kStages * sizeof(TileMeta) + (2 * kStages + 1) * 8 + 1024;
   static_assert(kSmem <= 227 * 1024, "shared memory budget");
 };
 
@@ -499,6 +500,7 @@ __global__ void __launch_bounds__(Bf16Cfg<D, MT>::kThreads, 1)
       mbar_init(smem_u32(&bars[s]), 1);                            // full: producer + tx bytes
       mbar_init(smem_u32(&bars[C::kStages + s]), C::kConsumerWarps);  // empty: one per consumer warp
     }
+    mbar_init(smem_u32(&bars[2 * C::kStages]), 1);  // never signalled (test hook)
     fence_barrier_init();
   }
   Plan plan;
@@ -551,10 +553,17 @@ __global__ void __launch_bounds__(Bf16Cfg<D, MT>::kThreads, 1)
         tma_prefetch_desc(&tmk);
         tma_prefetch_desc(&tmv);
         tma_prefetch_desc(&tmq);
+        // Test hook (off unless the host enabled it): CTA 0's producer waits on a barrier that
+        // nothing signals; the bounded wait runs out and records GQA_DEVERR_TIMEOUT, no copy is
+        // issued, and the consumers' own bounded waits on the first stage then run out too (all
+        // at their first tile, so no consumer is left at a named barrier). The rows of CTA 0's
+        // chunk are then left unwritten or merged from stale partials.
+        if (a.expire_wait && blockIdx.x == 0 && !mbar_wait(smem_u32(&bars[2 * C::kStages]), 0, a.err))
+          ok = false;
         // Chunk tickets: CTA c starts with chunk c; later chunks come from an atomic counter whose
         // value is fetched one chunk ahead, so its latency overlaps the current chunk's loads.
         int chunk = blockIdx.x;
-        int next = dyn && chunk < plan.n_chunks ? G + atomicAdd(&a.hdr->ticket, 1) : plan.n_chunks;
+        int next = ok && dyn && chunk < plan.n_chunks ? G + atomicAdd(&a.hdr->ticket, 1) : plan.n_chunks;
         for (; ok && chunk < plan.n_chunks;) {
           const long long x1 = min((long long)(chunk + 1) * plan.C, plan.K);
           for (long long x = (long long)chunk * plan.C; x < x1 && ok;) {
@@ -1398,6 +1407,7 @@ KArgs make_kargs(const DecodeArgs& a) {
   k.page_size = a.page_size;
   k.num_pages = a.num_pages;
   k.gran = a.block_table ? (a.page_size % kTile == 0 ? kTile : 16) : 1;
+  k.expire_wait = a.block_table || a.mla ? 0 : a.expire_wait;
   return k;
 }
 

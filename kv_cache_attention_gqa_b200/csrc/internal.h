@@ -37,6 +37,7 @@ struct PrefillArgs {
   float scale;
   int causal;
   int window;  // 0: none; W > 0 (causal only): row at position p sees keys p - W < j <= p
+  int expire_wait = 0;  // test hook (gqa_debug_expire_waits): one bounded wait runs out
   unsigned* err;
 };
 // fp32 check mode (scalar FFMA)
@@ -101,7 +102,14 @@ struct DecodeArgs {
   // width (576), d_v = the value / output width (the row's first 512 entries); 16 heads per unit
   int mla = 0;
   int d_v = 0;
+  int expire_wait = 0;  // test hook (gqa_debug_expire_waits), contiguous bf16 decode only
 };
+
+// The host-side argument checks of gqa_decode (contiguous: cache_rows = B * h_kv * T_max), in
+// the order gqa_decode applies them; GQA_OK when the request may proceed to the workspace checks.
+gqa_status decode_check_args(const void* q, const void* k_cache, const void* v_cache, const void* o,
+                             int B, int h_q, int h_kv, int T_max, int d_h, float scale, int window,
+                             gqa_dtype dtype, int num_splits, long long cache_rows);
 
 // Workspace bytes for a decode of this shape (layout in decode.cu).
 size_t decode_workspace_bytes(int B, int h_q, int h_kv, int T_max, int d_h, int num_splits,

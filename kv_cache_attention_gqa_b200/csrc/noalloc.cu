@@ -10,7 +10,9 @@
 // The array is a file-scope __device__ variable: every GPU that loads the library holds
 // kNoAllocScratchBytes of it until the process exits. In host code its name is only a host-side
 // handle, so the device address is looked up with cudaGetSymbolAddress once per device (with
-// that device current) on the first call and cached. All calls share the array and it keeps the
+// that device current) on the first call and cached. A device reset (cudaDeviceReset) frees the
+// array and leaves the cached address stale, so the library is not to be used on a device after
+// it was reset in the same process (the same holds for its other per-device state). All calls share the array and it keeps the
 // last call's contents; the work ticket that must start at zero is cleared on the stream before
 // every launch. Calls whose execution overlaps on the GPU (different streams, or different host
 // threads on one device) race on the array and must be serialised by the caller.
@@ -56,9 +58,11 @@ extern "C" gqa_status gqa_decode_noalloc(const void* q, const void* k_cache, con
                                          int T_max, int d_h, float scale, int window,
                                          gqa_dtype dtype, int num_splits, void* stream) {
   using namespace gqa;
-  if (B <= 0 || h_q <= 0 || h_kv <= 0 || T_max <= 0 || d_h <= 0 || num_splits < 0 || window < 0 ||
-      h_q % h_kv != 0)
-    return GQA_ERR_INVALID_ARG;
+  // gqa_decode's own checks come first, so a request it would refuse gets the same status here
+  // (an unsupported shape is UNSUPPORTED, not a too-small scratch array)
+  const gqa_status st = decode_check_args(q, k_cache, v_cache, o, B, h_q, h_kv, T_max, d_h, scale,
+                                          window, dtype, num_splits, (long long)B * h_kv * T_max);
+  if (st != GQA_OK) return st;
   const size_t need = gqa_decode_workspace_size(B, h_q, h_kv, T_max, d_h, dtype, num_splits);
   if (need == 0) return GQA_ERR_INVALID_ARG;
   if (need > kNoAllocScratchBytes) return GQA_ERR_WORKSPACE;  // beyond the fixed scratch size

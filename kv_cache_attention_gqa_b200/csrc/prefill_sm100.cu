@@ -40,7 +40,6 @@
 #include <math.h>
 
 #include "common.cuh"
-#include "exp2_poly.cuh"
 #include "internal.h"
 #include "tcgen05.cuh"
 
@@ -54,9 +53,6 @@ constexpr int kVStages = 2;  // V ring depth
 constexpr int kThreads = 384;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // base-2 units: P <= 2^8 between rescales
-#ifndef GQA_PREFILL_POLY_EVERY
-#define GQA_PREFILL_POLY_EVERY 0  // one exponential pair in this many goes to the polynomial (0: none)
-#endif
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -89,6 +85,7 @@ struct PArgs {
   float scale_log2;
   int causal;
   int window;  // 0: none; W > 0: row at position p also needs key j > p - W (causal only)
+  int expire_wait;  // test hook: CTA 0's producer first waits on a barrier that nothing signals
   unsigned* err;
 };
 
@@ -104,7 +101,8 @@ enum {
   kBarP = 16,         // + S buffer (2): P of a block is in TMEM
   kBarO = 18,         // O += P V of a block completed
   kBarDone = 19,
-  kNumBars = 20
+  kBarNever = 20,     // never signalled: the test hook's wait on it always runs out
+  kNumBars = 21
 };
 
 // Bounded wait that also gives up as soon as another thread of the CTA has aborted.
@@ -171,39 +169,14 @@ __device__ __forceinline__ Tile make_tile(const PArgs& a) {
   return t;
 }
 
-#ifndef GQA_PREFILL_EXP_F16X2
-#define GQA_PREFILL_EXP_F16X2 0  // two exponentials per special-function op, in f16
-#endif
-// 2^x0, 2^x1 with one packed f16x2 special-function op: the arguments (<= 8) are rounded to f16,
-// the results widened back to fp32 (they are rounded to bf16 for P in any case).
-__device__ __forceinline__ void exp2_f16x2(float x0, float x1, float& y0, float& y1) {
-  uint32_t h;
-  asm("{\n\t.reg .b32 t;\n\tcvt.rn.f16x2.f32 t, %2, %1;\n\tex2.approx.f16x2 %0, t;\n\t}"
-      : "=r"(h) : "f"(x0), "f"(x1));
-  asm("{\n\t.reg .f16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\tcvt.f32.f16 %0, lo;\n\tcvt.f32.f16 %1, hi;\n\t}"
-      : "=f"(y0), "=f"(y1) : "r"(h));
-}
-#ifndef GQA_PREFILL_PACKED
-#define GQA_PREFILL_PACKED 1  // packed fp32x2 FMA/ADD in the softmax
-#endif
 // packed fp32x2 helpers (sm_100): d = a * b + c and s += a, on register pairs
 __device__ __forceinline__ void ffma2(float& d0, float& d1, float a0, float a1, float b, float c) {
-#if !GQA_PREFILL_PACKED
-  d0 = fmaf(a0, b, c);
-  d1 = fmaf(a1, b, c);
-  return;
-#endif
   asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %4};\n\t"
       "mov.b64 rc, {%5, %5};\n\tfma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
       : "=f"(d0), "=f"(d1)
       : "f"(a0), "f"(a1), "f"(b), "f"(c));
 }
 __device__ __forceinline__ void fadd2(float& s0, float& s1, float a0, float a1) {
-#if !GQA_PREFILL_PACKED
-  s0 += a0;
-  s1 += a1;
-  return;
-#endif
   asm("{\n\t.reg .b64 ra, rs;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rs, {%0, %1};\n\t"
       "add.rn.f32x2 rs, rs, ra;\n\tmov.b64 {%0, %1}, rs;\n\t}"
       : "+f"(s0), "+f"(s1)
@@ -404,10 +377,25 @@ __device__ __forceinline__ void softmax_role(const PArgs& a, const Tile& tile, i
   named_barrier_sync(1, 256);
   l += xsum[(half ^ 1) * 128 + row];
   (void)sm_tid;
-  if (!__all_sync(0xffffffffu, ok)) return;
+  // A tile whose pipeline gave up (a bounded wait ran out; the error word says so) writes zero
+  // rows and lse = -inf, without touching TMEM.
+  auto zero_rows = [&]() {
+    if (!store_row) return;
+    uint4* z = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.o) + orow * D + half * kOHalf);
+#pragma unroll
+    for (int v = 0; v < kOHalf / 8; ++v) z[v] = make_uint4(0u, 0u, 0u, 0u);
+    if (a.lse && half == 0) a.lse[orow] = -INFINITY;
+  };
+  if (!__all_sync(0xffffffffu, ok)) {
+    zero_rows();
+    return;
+  }
   // epilogue: this half of O / l -> bf16 -> global; lse = (m + log2 l) * ln 2
   bool ok_o = wait_bar(bar(kBarO), (uint32_t)((nb - 1) & 1), abort, a.err);
-  if (!__all_sync(0xffffffffu, ok_o)) return;
+  if (!__all_sync(0xffffffffu, ok_o)) {
+    zero_rows();
+    return;
+  }
   tc::fence_after_sync();
   // A row with no visible key (a sliding window that starts at or past kv_len, or a padding row
   // of the tile) has l = 0: it still takes part in the warp's TMEM loads, and writes zeros.
@@ -471,6 +459,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(bar(kBarO), 1);
     mbar_init(bar(kBarDone), 1);
+    mbar_init(bar(kBarNever), 1);
     *abort = 0;
     fence_barrier_init();
     if (!tile.valid) set_device_error(a.err, tile.kv < 1 || tile.kv > a.T_max ? GQA_DEVERR_KV_LEN
@@ -492,15 +481,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&tmq);
     tma_prefetch_desc(&tmk);
     tma_prefetch_desc(&tmv);
-    const int zq = tile.b * a.h_q + tile.g * a.r + tile.hb * a.H;  // first head of the block
-    mbar_arrive_expect_tx(bar(kBarQ), (uint32_t)(C::kNch * a.H * a.P * 128));
-    for (int ch = 0; ch < C::kNch; ++ch)
-      tma_load_3d(sQ + ch * C::kQChunk, &tmq, bar(kBarQ), ch * 64, tile.q0, zq);
-    const int row0 = (tile.b * a.h_kv + tile.g) * a.T_max;
     int last_k[kKStages], last_v[kVStages];
     for (int s = 0; s < kKStages; ++s) last_k[s] = -1;
     for (int s = 0; s < kVStages; ++s) last_v[s] = -1;
-    for (int j = 0; j < nb; ++j) {
+    // Test hook (off unless the host enabled it): CTA 0 first waits on a barrier that nothing
+    // signals, so its bounded wait runs out, records GQA_DEVERR_TIMEOUT and aborts the CTA before
+    // any copy is issued; every other role then gives up through the abort flag.
+    const bool go = !(a.expire_wait && blockIdx.x == 0) || wait_bar(bar(kBarNever), 0, abort, a.err);
+    if (go) {
+      const int zq = tile.b * a.h_q + tile.g * a.r + tile.hb * a.H;  // first head of the block
+      mbar_arrive_expect_tx(bar(kBarQ), (uint32_t)(C::kNch * a.H * a.P * 128));
+      for (int ch = 0; ch < C::kNch; ++ch)
+        tma_load_3d(sQ + ch * C::kQChunk, &tmq, bar(kBarQ), ch * 64, tile.q0, zq);
+    }
+    const int row0 = (tile.b * a.h_kv + tile.g) * a.T_max;
+    for (int j = 0; j < nb && go; ++j) {
       const int ks = j % kKStages, kn = j / kKStages;
       if (kn > 0 && !wait_bar(bar(kBarKEmpty + ks), (uint32_t)((kn - 1) & 1), abort, a.err)) break;
       mbar_arrive_expect_tx(bar(kBarKFull + ks), C::kKVBytes);
@@ -519,7 +514,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Drain (bounded, whatever the abort state): no copy may still be landing in shared memory
     // when the CTA exits.
     volatile int no_abort = 0;
-    wait_bar(bar(kBarQ), 0, &no_abort, a.err);
+    if (go) wait_bar(bar(kBarQ), 0, &no_abort, a.err);
     for (int s = 0; s < kKStages; ++s)
       if (last_k[s] >= 0) wait_bar(bar(kBarKFull + s), (uint32_t)(last_k[s] & 1), &no_abort, a.err);
     for (int s = 0; s < kVStages; ++s)
@@ -627,6 +622,7 @@ cudaError_t launch_prefill_bf16(const PrefillArgs& a, const CUtensorMap* tmaps, 
   p.scale_log2 = a.scale * pf::kLog2e;
   p.causal = a.causal;
   p.window = a.window;
+  p.expire_wait = a.expire_wait;
   p.err = a.err;
   const long long tiles = (long long)p.n_qt * a.B * a.h_kv * p.hblocks;
   if (tiles <= 0) return cudaSuccess;

@@ -52,6 +52,13 @@ def test_status_strings_and_version(lib):
     assert b"sm_100a" in lib.gqa_version()
 
 
+def test_expire_waits_hook_takes_only_zero_or_one(lib):
+    assert lib.gqa_debug_expire_waits(2) == 1
+    assert lib.gqa_debug_expire_waits(-1) == 1
+    assert lib.gqa_debug_expire_waits(1) == 0
+    assert lib.gqa_debug_expire_waits(0) == 0  # left off
+
+
 def test_host_side_argument_errors(lib):
     P = ctypes.c_void_p
     fake = P(0x1000)
@@ -81,6 +88,19 @@ def test_host_side_argument_errors(lib):
     assert lib.gqa_decode(fake, fake, fake, fake, null, null, null, 1024, 32, 32, 65536, 128, 0.1, 0, 0, fake,
                           1 << 20, 1, s) == 2
     assert lib.gqa_decode_noalloc(fake, fake, fake, fake, null, null, null, 1, 4, 2, 8, 64, 0.1, -1, 0, 1, s) == 1
+    # the no-alloc decode applies gqa_decode's checks first: a batch beyond the decode limit and a bf16
+    # d_h outside {64, 128} are UNSUPPORTED (not WORKSPACE, though their workspace would also exceed the
+    # fixed scratch array); a null output is INVALID_ARG
+    assert lib.gqa_decode_noalloc(fake, fake, fake, fake, null, null, null, 2000, 64, 64, 4096, 128, 0.1, 0, 0,
+                                  100000, s) == 2
+    assert lib.gqa_decode_noalloc(fake, fake, fake, fake, null, null, null, 1, 4, 2, 8, 96, 0.1, 0, 0, 1, s) == 2
+    assert lib.gqa_decode_noalloc(fake, fake, fake, null, null, null, null, 1, 4, 2, 8, 64, 0.1, 0, 0, 1, s) == 1
+    # scale: 0 selects the default 1/sqrt(d_h); negative, NaN and infinite scales are refused
+    for bad in (-0.5, float("nan"), float("inf"), float("-inf")):
+        assert lib.gqa_prefill(fake, fake, fake, fake, null, null, null, 1, 4, 2, 8, 8, 64, bad, 1, 0, 0, s) == 1
+        assert lib.gqa_decode_noalloc(fake, fake, fake, fake, null, null, null, 1, 4, 2, 8, 64, bad, 0, 0, 1, s) == 1
+    # scale 0 passes the host checks (the next refusal is the unsupported d_h)
+    assert lib.gqa_prefill(fake, fake, fake, fake, null, null, null, 1, 4, 2, 8, 8, 96, 0.0, 1, 0, 0, s) == 2
     # decode
     assert lib.gqa_decode(null, fake, fake, fake, null, null, null, 1, 4, 2, 8, 64, 0.1, 0, 0, fake, 1 << 20, 1, s) == 1
     assert lib.gqa_decode(fake, fake, fake, fake, null, null, null, 1, 4, 3, 8, 64, 0.1, 0, 0, fake, 1 << 20, 1, s) == 1

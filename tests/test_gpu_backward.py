@@ -2,7 +2,7 @@
 
 The forward runs through the library (gqa_prefill with lse); the backward recomputes P from that
 lse. The oracle differentiates the plain definition on the same inputs. bf16 gradients within
-2e-2 (max) / 2e-3 (mean) of the tensor's largest entry, fp32 check mode within 1e-4 of it; dK and
+2e-2 (max) / 2e-3 (mean) of the tensor's largest entry, fp32 check mode within 1e-5 of it; dK and
 dV rows past kv_len must be exactly zero.
 """
 
@@ -94,9 +94,9 @@ def test_backward_bf16_group_identities():
         assert np.abs(dv[g].sum(axis=0) - want).max() <= 1e-2 * np.abs(dv[g]).sum(axis=0).max()
 
 
-def test_backward_prefill_4k_one_group():
-    """prefill_4k (h_q=32, h_kv=8, S=T=4096, d_h=128): the gradients of group 0 (4 query heads,
-    KV head 0) against the oracle on that group alone (other groups do not touch it)."""
+def test_backward_prefill_4k_full_size():
+    """prefill_4k (h_q=32, h_kv=8, S=T=4096, d_h=128): dQ of all 32 heads and dK, dV of all 8 KV
+    heads against the oracle's gradients."""
     import kv_cache_attention_gqa_b200 as gqa
 
     shape = workloads.PREFILL_4K
@@ -106,7 +106,7 @@ def test_backward_prefill_4k_one_group():
     o, lse = gqa.prefill(q, k, v, return_lse=True)
     dq, dk, dv = gqa.prefill_backward(q, k, v, o, d_o, lse)
     assert gqa.get_device_error() == 0
-    rq, rk, rv = oracle.attention_backward_ref(_f64(q[:, :4]), _f64(k[:, :1]), _f64(v[:, :1]), _f64(d_o[:, :4]))
-    assert_grad_close(_f64(dq[:, :4]), rq, "prefill_4k dQ")
-    assert_grad_close(_f64(dk[:, :1]), rk, "prefill_4k dK")
-    assert_grad_close(_f64(dv[:, :1]), rv, "prefill_4k dV")
+    rq, rk, rv = oracle.attention_backward_ref(_f64(q), _f64(k), _f64(v), _f64(d_o))
+    assert_grad_close(_f64(dq), rq, "prefill_4k dQ")
+    assert_grad_close(_f64(dk), rk, "prefill_4k dK")
+    assert_grad_close(_f64(dv), rv, "prefill_4k dV")

@@ -536,6 +536,32 @@ def run_chunked(args, dev, tf_peak, peak_kind):
                           "GB_s": round(app_bytes / (app_ms / 1e3) / 1e9, 1)}}
 
 
+def run_prefill_small(args, dev, tf_peak, peak_kind):
+    """prefill_small: B=1, h_q=4, h_kv=2 (r=2), S_q=T=256, d_h=64, causal, N(0,1) -- the d_h=64
+    tcgen05 instantiation. 33.7 MFLOP of work is a few microseconds of one launch on 8 CTAs: the
+    line is launch- and latency-bound, so its TFLOPS is reported, not held to the tensor peak."""
+    import torch
+
+    import kv_cache_attention_gqa_b200 as gqa
+    import workloads
+
+    shape = workloads.PREFILL_SMALL
+    q, k, v = workloads.prefill_inputs(shape, seed=args.seed, device=dev)
+    out = torch.empty_like(q)
+    fn = lambda: gqa.prefill(q, k, v, out=out)  # noqa: E731
+    ms, mode = graph_timed(fn, L2Flush(dev), max(20, args.steps), max(3, args.warmup))
+    if gqa.get_device_error() != 0:
+        raise RuntimeError("device error in the prefill_small line")
+    flops = prefill_flops(shape.B, shape.h_q, shape.d_h, shape.S_q, 0, shape.T_max)
+    tflops = flops / (ms / 1e3) / 1e12
+    return {"workload": "prefill_small: B=1, h_q=4, h_kv=2, S_q=T=256, d_h=64, causal; one gqa_prefill per call, "
+                        "L2 flushed between calls",
+            "launch": mode, "value": round(tflops, 2), "unit": "TFLOP/s", "us": round(ms * 1e3, 2),
+            "bound": "launch/latency (8 tiles of 128 rows on 148 SMs)",
+            "frac_of_bf16_peak": round(tflops / tf_peak, 5), "peak_kind": f"bf16_tflops of {peak_kind}",
+            "algorithmic_flops_per_launch": flops, "gpu_launches_per_call": 1}
+
+
 def run_window(args, rank, dev, stream, local, hbm_peak, tf_peak, peak_kind):
     """Sliding window of 1024 keys [第三章 §3.7]: decode_8k (each query reads its 1024 most recent
     keys) and prefill_4k; the work counted is only what lies inside the windows."""
@@ -579,6 +605,8 @@ def run_ours(args, rank, world, dist):
         return {"ragged": run_ragged(args, dev, hbm_peak, peak_kind)}
     if args.chunked_only:  # profiling aid: the chunked prefill line alone
         return {"chunked": run_chunked(args, dev, tf_peak, peak_kind)}
+    if args.small_only:  # profiling aid: the prefill_small line alone
+        return {"prefill_small": run_prefill_small(args, dev, tf_peak, peak_kind)}
 
     variants = build_variants(args, rank, dev)
     flush = L2Flush(dev)
@@ -617,6 +645,7 @@ def run_ours(args, rank, world, dist):
         window = run_window(args, rank, dev, stream, local, hbm_peak, tf_peak, peak_kind)
     ragged = run_ragged(args, dev, hbm_peak, peak_kind) if not args.skip_ragged else None
     chunked = run_chunked(args, dev, tf_peak, peak_kind) if not args.skip_chunked else None
+    small = run_prefill_small(args, dev, tf_peak, peak_kind) if not args.skip_small else None
 
     result = {
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
@@ -645,6 +674,8 @@ def run_ours(args, rank, world, dist):
         result["ragged"] = ragged
     if chunked is not None:
         result["chunked"] = chunked
+    if small is not None:
+        result["prefill_small"] = small
     if rank == 0 and world == 1 and not args.skip_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(args)
     return result
@@ -782,9 +813,73 @@ def _threads():
         return os.cpu_count() or 1
 
 
+def _time_until(fn, budget_s, max_reps=1000):
+    """Run `fn` until about `budget_s` seconds have passed; returns (repetitions, seconds)."""
+    reps, t = 0, 0.0
+    while (t < budget_s or reps == 0) and reps < max_reps:
+        t0 = time.perf_counter()
+        fn()
+        t += time.perf_counter() - t0
+        reps += 1
+    return reps, t
+
+
+def cpu_baseline_per_config(args, budget_s=3.0):
+    """The fp64 oracle on a bounded sample of each of the other workloads, at the same seed and
+    shapes as the GPU lines: prefill_small whole; prefill_4k one query head (4096 x 4096 pairs);
+    chunked prefill one query head (512 queries over 32768 keys); ragged_decode one sequence (the
+    first of the seeded lengths, all 64 query heads). Each sample repeats for about `budget_s`."""
+    import numpy as np
+
+    import oracle
+    import workloads
+
+    f64 = workloads.to_f64
+    out = {}
+    # C1 prefill_small, whole
+    sh = workloads.PREFILL_SMALL
+    q, k, v = (f64(t) for t in workloads.prefill_inputs(sh, seed=args.seed))
+    reps, t = _time_until(lambda: oracle.attention_ref(q, k, v), budget_s)
+    fl = prefill_flops(sh.B, sh.h_q, sh.d_h, sh.S_q, 0, sh.T_max)
+    out["prefill_small"] = {"GFLOP_s": round(fl * reps / t / 1e9, 3), "s_per_call": round(t / reps, 5),
+                            "sample": "the whole workload (4 heads, 256 rows)", "reps": reps}
+    # C3 prefill_4k, one query head
+    sh = workloads.PREFILL_4K
+    q, k, v = workloads.prefill_inputs(sh, seed=args.seed)
+    q0, k0, v0 = f64(q[0, 0]), f64(k[0, 0]), f64(v[0, 0])
+    pos = np.arange(sh.S_q)
+    reps, t = _time_until(lambda: oracle.head_attention(q0, k0, v0, pos, sh.kv_len, sh.d_h ** -0.5), budget_s)
+    fl = prefill_flops(1, 1, sh.d_h, sh.S_q, 0, sh.kv_len)
+    out["prefill_4k"] = {"GFLOP_s": round(fl * reps / t / 1e9, 3), "s_per_head": round(t / reps, 4),
+                         "sample": "query head 0 of 32 (4096 x 4096 causal pairs)", "reps": reps}
+    # C5 chunked prefill, one query head
+    sh = workloads.CHUNKED_PREFILL
+    k, v, k_new, v_new, q = workloads.chunked_prefill_inputs(sh, seed=args.seed)
+    k[:, :, sh.q_start:] = k_new
+    v[:, :, sh.q_start:] = v_new
+    q0, k0, v0 = f64(q[0, 0]), f64(k[0, 0]), f64(v[0, 0])
+    pos = sh.q_start + np.arange(sh.S_q)
+    reps, t = _time_until(lambda: oracle.head_attention(q0, k0, v0, pos, sh.kv_len, sh.d_h ** -0.5), budget_s)
+    fl = prefill_flops(1, 1, sh.d_h, sh.S_q, sh.q_start, sh.kv_len)
+    out["chunked_prefill"] = {"GFLOP_s": round(fl * reps / t / 1e9, 3), "s_per_head": round(t / reps, 4),
+                              "sample": "query head 0 of 32 (512 queries over 32768 keys)", "reps": reps}
+    # C4 ragged decode, one sequence
+    sh = workloads.RAGGED_DECODE
+    n0 = int(workloads.ragged_lengths(args.seed, sh.B, sh.len_lo, sh.len_hi)[0])
+    one = workloads.DecodeShape(B=1, h_q=sh.h_q, h_kv=sh.h_kv, T_max=n0, d_h=sh.d_h)
+    q, k, v, kl = workloads.decode_inputs(one, seed=args.seed)
+    q, k, v, kl = f64(q), f64(k), f64(v), kl.numpy()
+    reps, t = _time_until(lambda: oracle.decode_ref(q, k, v, kv_len=kl), budget_s)
+    nb = decode_kv_bytes(1, sh.h_kv, [n0], sh.d_h)
+    out["ragged_decode"] = {"GB_s": round(nb * reps / t / 1e9, 4), "s_per_sequence": round(t / reps, 4),
+                            "sample": f"one sequence of length {n0} (the first seeded length), 64 query heads",
+                            "reps": reps}
+    return out
+
+
 def cpu_baseline(args, budget_s=10.0):
     """fp64 oracle on a bounded sample of decode_8k: sequence 0 of each h_kv variant, repeated
-    until about `budget_s` seconds of CPU work."""
+    until about `budget_s` seconds of CPU work; plus the other workloads' samples."""
     import oracle
 
     samples = _oracle_sample_inputs(args.seed)
@@ -796,9 +891,12 @@ def cpu_baseline(args, budget_s=10.0):
             t_total += time.perf_counter() - t0
             nbytes += decode_kv_bytes(1, h_kv, kv_len, 128)
         reps += 1
-    return {"value": round(nbytes / t_total / 1e9, 4), "unit": "GB/s", "cores": _threads(), "kind": "oracle",
-            "sample": f"decode_8k, sequence 0 of each h_kv variant (all 32 query heads, 8192 keys), "
-                      f"{reps} repetitions, {t_total:.1f} s of fp64 NumPy"}
+    res = {"value": round(nbytes / t_total / 1e9, 4), "unit": "GB/s", "cores": _threads(), "kind": "oracle",
+           "sample": f"decode_8k, sequence 0 of each h_kv variant (all 32 query heads, 8192 keys), "
+                     f"{reps} repetitions, {t_total:.1f} s of fp64 NumPy"}
+    if not args.skip_oracle_configs:
+        res["per_config"] = cpu_baseline_per_config(args)
+    return res
 
 
 def run_reference(args, rank):
@@ -839,6 +937,8 @@ def main():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--skip-prefill", action="store_true")
     ap.add_argument("--skip-cpu-baseline", action="store_true")
+    ap.add_argument("--skip-oracle-configs", action="store_true",
+                    help="time the oracle on decode_8k only (not on the other workloads' samples)")
     ap.add_argument("--skip-e2e", action="store_true")
     ap.add_argument("--eager", action="store_true", help="time eager launches instead of a CUDA graph")
     ap.add_argument("--prefill-only", action="store_true", help="only the prefill_4k line (profiling aid)")
@@ -857,6 +957,8 @@ def main():
     ap.add_argument("--ragged-only", action="store_true", help="only the ragged decode line (profiling aid)")
     ap.add_argument("--skip-chunked", action="store_true")
     ap.add_argument("--chunked-only", action="store_true", help="only the chunked prefill line (profiling aid)")
+    ap.add_argument("--skip-small", action="store_true")
+    ap.add_argument("--small-only", action="store_true", help="only the prefill_small line (profiling aid)")
     ap.add_argument("--h-kv", dest="h_kv", type=int, nargs="+", default=[32, 8, 1],
                     help="decode_8k variants to run (default: all three); fewer only for profiling")
     args = ap.parse_args()

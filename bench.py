@@ -477,7 +477,11 @@ def run_ragged(args, dev, hbm_peak, peak_kind):
     import kv_cache_attention_gqa_b200 as gqa
     import workloads
 
+    import dataclasses
+
     shape = workloads.RAGGED_DECODE
+    if args.ragged_b != shape.B:  # profiling aid: fewer sequences of the same length distribution
+        shape = dataclasses.replace(shape, B=args.ragged_b)
     q, k, v, kv_len = workloads.decode_inputs(shape, seed=args.seed, device=dev)
     out = torch.empty_like(q)
     ws = torch.zeros(gqa.decode_workspace_size(shape.B, shape.h_q, shape.h_kv, shape.T_max, shape.d_h),
@@ -491,7 +495,7 @@ def run_ragged(args, dev, hbm_peak, peak_kind):
     gbs = nbytes / (ms / 1e3) / 1e9
     finite = bool(torch.isfinite(out.float()).all())  # the NaN past every length never reaches O
     del q, k, v, out, ws
-    return {"workload": "ragged_decode: B=64, h_q=64, h_kv=8, d_h=128, lengths uniform on [1024, 32768] "
+    return {"workload": f"ragged_decode: B={shape.B}, h_q=64, h_kv=8, d_h=128, lengths uniform on [1024, 32768] "
                         f"(seed {args.seed}, sum {sum(lens)}), cache allocated at 32768 with NaN past each length; "
                         "one gqa_decode per call, L2 flushed between calls",
             "launch": mode, "value": round(gbs, 1), "unit": "GB/s", "us": round(ms * 1e3, 2),
@@ -955,6 +959,8 @@ def main():
     ap.add_argument("--window", type=int, default=1024, help="sliding window of the window lines")
     ap.add_argument("--skip-ragged", action="store_true")
     ap.add_argument("--ragged-only", action="store_true", help="only the ragged decode line (profiling aid)")
+    ap.add_argument("--ragged-b", dest="ragged_b", type=int, default=64,
+                    help="sequences of the ragged decode line (profiling aid; the workload has 64)")
     ap.add_argument("--skip-chunked", action="store_true")
     ap.add_argument("--chunked-only", action="store_true", help="only the chunked prefill line (profiling aid)")
     ap.add_argument("--skip-small", action="store_true")

@@ -154,6 +154,20 @@ __device__ __forceinline__ uint64_t desc_k(uint32_t tile, int k, uint32_t chunk)
 __device__ __forceinline__ uint64_t desc_mn(uint32_t tile, int kk, uint32_t chunk) {
   return tc::smem_desc(tile + (uint32_t)(kk * 2048), chunk, 1024);
 }
+// The same descriptors as a base plus a constant: the start address sits in the low 14 bits
+// (address >> 4, below 2^14 for any shared-memory address), so the descriptor of tile + offset is
+// the tile's descriptor plus offset >> 4. The MMA issuers build the bases once per stage and add
+// compile-time offsets inside their unrolled loops.
+__device__ __forceinline__ uint64_t koff(int k, uint32_t chunk) {
+  return (uint64_t)(((k >> 2) * chunk + (k & 3) * 32) >> 4);
+}
+__device__ __forceinline__ uint64_t mnoff(int kk) { return (uint64_t)((kk * 2048) >> 4); }
+
+__device__ __forceinline__ bool elect_one() {
+  uint32_t p;
+  asm volatile("{\n\t.reg .pred q;\n\telect.sync _|q, 0xffffffff;\n\tselp.u32 %0, 1, 0, q;\n\t}" : "=r"(p));
+  return p != 0;
+}
 
 // ---- dkdv: key-stationary dK / dV -------------------------------------------------------------
 // Query blocks of 64 rows, so S^T and dP^T are double-buffered in TMEM next to the dV / dK
@@ -309,24 +323,33 @@ __device__ __forceinline__ void dkdv_cta(const CUtensorMap& tmq, const CUtensorM
       for (int st = 0; st < kKvStages; ++st)
         if (last[st] >= 0) wait_bar(bar(kQFull + st), (uint32_t)(last[st] & 1), &no_abort, a.err);
     }
-  } else if (warp == 1 && lane == 0 && n_it > 0) {
+  } else if (warp == 1 && n_it > 0) {
     // ------------------------------ MMA issuer ---------------------------------------------
+    // The whole warp runs the loop (its state and the descriptors stay warp-uniform) and one
+    // elected lane issues each batch of MMAs together with its commit. (One thread issuing with
+    // descriptors built per MMA spent most of its time between MMAs, not in them.)
     constexpr uint32_t idesc_s = tc::idesc_bf16(128, kKvBQ, false);  // S^T, dP^T: M keys, N queries
     constexpr uint32_t idesc_acc = tc::idesc_bf16(128, D, true);     // dV, dK: M keys, N = d_h
+    const uint64_t dK = tc::smem_desc(sK, 16, 1024), dV = tc::smem_desc(sV, 16, 1024);
+    auto wait = [&](int b_, uint32_t parity) {
+      return __all_sync(0xffffffffu, wait_bar(bar(b_), parity, abort, a.err));
+    };
     auto issue_s = [&](int it) {  // S^T and dP^T of block `it` into buffer it & 1
       const int st = it % kKvStages, bf = it & 1;
+      const uint64_t dq = tc::smem_desc(sQ(st), 16, 1024), ddo = tc::smem_desc(sDO(st), 16, 1024);
+      if (elect_one()) {
 #pragma unroll
-      for (int k = 0; k < D / 16; ++k)
-        tc::mma_ss(tmem + 64 * bf, desc_k(sK, k, 128 * 128), desc_k(sQ(st), k, C::kQChunk), idesc_s,
-                   k > 0 ? 1u : 0u);
+        for (int k = 0; k < D / 16; ++k)
+          tc::mma_ss(tmem + 64 * bf, dK + koff(k, 128 * 128), dq + koff(k, C::kQChunk), idesc_s, k > 0 ? 1u : 0u);
 #pragma unroll
-      for (int k = 0; k < D / 16; ++k)
-        tc::mma_ss(tmem + 128 + 64 * bf, desc_k(sV, k, 128 * 128), desc_k(sDO(st), k, C::kQChunk), idesc_s,
-                   k > 0 ? 1u : 0u);
-      tc::commit(bar(kKvS + bf));
+        for (int k = 0; k < D / 16; ++k)
+          tc::mma_ss(tmem + 128 + 64 * bf, dV + koff(k, 128 * 128), ddo + koff(k, C::kQChunk), idesc_s,
+                     k > 0 ? 1u : 0u);
+        tc::commit(bar(kKvS + bf));
+      }
+      __syncwarp();
     };
-    bool ok = wait_bar(bar(kKvFull), 0, abort, a.err);
-    if (ok) ok = wait_bar(bar(kQFull), 0, abort, a.err);
+    bool ok = wait(kKvFull, 0) && wait(kQFull, 0);
     if (ok) {
       tc::fence_after_sync();
       issue_s(0);
@@ -335,22 +358,28 @@ __device__ __forceinline__ void dkdv_cta(const CUtensorMap& tmq, const CUtensorM
       const int st = it % kKvStages, bf = it & 1;
       if (it + 1 < n_it) {  // next block's scores overlap this block's elementwise pass
         const int st1 = (it + 1) % kKvStages;
-        if (!wait_bar(bar(kQFull + st1), (uint32_t)(((it + 1) / kKvStages) & 1), abort, a.err)) break;
+        if (!(ok = wait(kQFull + st1, (uint32_t)(((it + 1) / kKvStages) & 1)))) break;
         tc::fence_after_sync();
         issue_s(it + 1);
       }
-      if (!wait_bar(bar(kKvP + bf), (uint32_t)((it >> 1) & 1), abort, a.err)) break;
+      if (!(ok = wait(kKvP + bf, (uint32_t)((it >> 1) & 1)))) break;
       tc::fence_after_sync();
+      const uint64_t ddo_mn = tc::smem_desc(sDO(st), C::kQChunk, 1024);
+      const uint64_t dq_mn = tc::smem_desc(sQ(st), C::kQChunk, 1024);
+      if (elect_one()) {
 #pragma unroll
-      for (int kk = 0; kk < kKvBQ / 16; ++kk) {
-        const uint32_t acc = (it > 0 || kk > 0) ? 1u : 0u;
-        const uint32_t acol = (uint32_t)(64 * bf + (kk >> 1) * 32 + (kk & 1) * 8);  // half kk/2
-        tc::mma_ts(tmem + kColAcc0, tmem + acol, desc_mn(sDO(st), kk, C::kQChunk), idesc_acc, acc);
-        tc::mma_ts(tmem + kColAcc0 + D, tmem + 128 + acol, desc_mn(sQ(st), kk, C::kQChunk), idesc_acc, acc);
+        for (int kk = 0; kk < kKvBQ / 16; ++kk) {
+          const uint32_t acc = (it > 0 || kk > 0) ? 1u : 0u;
+          const uint32_t acol = (uint32_t)(64 * bf + (kk >> 1) * 32 + (kk & 1) * 8);  // half kk/2
+          tc::mma_ts(tmem + kColAcc0, tmem + acol, ddo_mn + mnoff(kk), idesc_acc, acc);
+          tc::mma_ts(tmem + kColAcc0 + D, tmem + 128 + acol, dq_mn + mnoff(kk), idesc_acc, acc);
+        }
+        tc::commit(bar(kQEmpty + st));
       }
-      tc::commit(bar(kQEmpty + st));
+      __syncwarp();
     }
-    tc::commit(bar(kKvDone));
+    if (elect_one()) tc::commit(bar(kKvDone));
+    __syncwarp();
     volatile int no_abort = 0;
     wait_bar(bar(kKvDone), 0, &no_abort, a.err);
   } else if (warp >= 2) {
@@ -591,24 +620,30 @@ __device__ __forceinline__ void dq_cta(const CUtensorMap& tmq, const CUtensorMap
     wait_bar(bar(kQdQ), 0, &no_abort, a.err);
     for (int st = 0; st < kQStages; ++st)
       if (last[st] >= 0) wait_bar(bar(kQKvFull + st), (uint32_t)(last[st] & 1), &no_abort, a.err);
-  } else if (warp == 1 && lane == 0 && nb > 0) {
+  } else if (warp == 1 && nb > 0) {
     // ------------------------------ MMA issuer ---------------------------------------------
+    // whole warp, one elected lane per batch of MMAs and its commit (as in the dK / dV pass)
     constexpr uint32_t idesc_s = tc::idesc_bf16(128, kQBK, false);  // S, dP: M rows, N keys
     constexpr uint32_t idesc_acc = tc::idesc_bf16(128, D, true);    // dQ: M rows, N = d_h
     constexpr uint32_t kColQ = kColAcc0 + D, kColDO = kColAcc0 + D + D / 2;
+    auto wait = [&](int b_, uint32_t parity) {
+      return __all_sync(0xffffffffu, wait_bar(bar(b_), parity, abort, a.err));
+    };
     auto issue_s = [&](int j) {
       const int st = j % kQStages, bf = j & 1;
+      const uint64_t dk = tc::smem_desc(sK(st), 16, 1024), dv = tc::smem_desc(sV(st), 16, 1024);
+      if (elect_one()) {
 #pragma unroll
-      for (int k = 0; k < D / 16; ++k)
-        tc::mma_ts(tmem + 64 * bf, tmem + kColQ + k * 8, desc_k(sK(st), k, C::kKChunk), idesc_s, k > 0 ? 1u : 0u);
+        for (int k = 0; k < D / 16; ++k)
+          tc::mma_ts(tmem + 64 * bf, tmem + kColQ + k * 8, dk + koff(k, C::kKChunk), idesc_s, k > 0 ? 1u : 0u);
 #pragma unroll
-      for (int k = 0; k < D / 16; ++k)
-        tc::mma_ts(tmem + 128 + 64 * bf, tmem + kColDO + k * 8, desc_k(sV(st), k, C::kKChunk), idesc_s,
-                   k > 0 ? 1u : 0u);
-      tc::commit(bar(kQS + bf));
+        for (int k = 0; k < D / 16; ++k)
+          tc::mma_ts(tmem + 128 + 64 * bf, tmem + kColDO + k * 8, dv + koff(k, C::kKChunk), idesc_s, k > 0 ? 1u : 0u);
+        tc::commit(bar(kQS + bf));
+      }
+      __syncwarp();
     };
-    bool ok = wait_bar(bar(kQT), 0, abort, a.err);
-    if (ok) ok = wait_bar(bar(kQKvFull), 0, abort, a.err);
+    bool ok = wait(kQT, 0) && wait(kQKvFull, 0);
     if (ok) {
       tc::fence_after_sync();
       issue_s(0);
@@ -616,19 +651,24 @@ __device__ __forceinline__ void dq_cta(const CUtensorMap& tmq, const CUtensorMap
     for (int j = 0; j < nb && ok; ++j) {
       const int st = j % kQStages, bf = j & 1;
       if (j + 1 < nb) {
-        if (!wait_bar(bar(kQKvFull + (j + 1) % kQStages), (uint32_t)(((j + 1) / kQStages) & 1), abort, a.err)) break;
+        if (!(ok = wait(kQKvFull + (j + 1) % kQStages, (uint32_t)(((j + 1) / kQStages) & 1)))) break;
         tc::fence_after_sync();
         issue_s(j + 1);
       }
-      if (!wait_bar(bar(kQP + bf), (uint32_t)((j >> 1) & 1), abort, a.err)) break;
+      if (!(ok = wait(kQP + bf, (uint32_t)((j >> 1) & 1)))) break;
       tc::fence_after_sync();
+      const uint64_t dk_mn = tc::smem_desc(sK(st), C::kKChunk, 1024);
+      if (elect_one()) {
 #pragma unroll
-      for (int kk = 0; kk < kQBK / 16; ++kk)
-        tc::mma_ts(tmem + kColAcc0, tmem + (uint32_t)(64 * bf + (kk >> 1) * 32 + (kk & 1) * 8),
-                   desc_mn(sK(st), kk, C::kKChunk), idesc_acc, (j > 0 || kk > 0) ? 1u : 0u);
-      tc::commit(bar(kQKvEmpty + st));
+        for (int kk = 0; kk < kQBK / 16; ++kk)
+          tc::mma_ts(tmem + kColAcc0, tmem + (uint32_t)(64 * bf + (kk >> 1) * 32 + (kk & 1) * 8),
+                     dk_mn + mnoff(kk), idesc_acc, (j > 0 || kk > 0) ? 1u : 0u);
+        tc::commit(bar(kQKvEmpty + st));
+      }
+      __syncwarp();
     }
-    tc::commit(bar(kQDone));
+    if (elect_one()) tc::commit(bar(kQDone));
+    __syncwarp();
     volatile int no_abort = 0;
     wait_bar(bar(kQDone), 0, &no_abort, a.err);
   } else if (warp >= 2) {

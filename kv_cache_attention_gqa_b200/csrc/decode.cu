@@ -503,6 +503,15 @@ __global__ void __launch_bounds__(Bf16Cfg<D, MT>::kThreads, 1)
     mbar_init(smem_u32(&bars[2 * C::kStages]), 1);  // never signalled (test hook)
     fence_barrier_init();
   }
+  if (warp == producer_warp && lane == 0) {
+    tma_prefetch_desc(&tmk);
+    tma_prefetch_desc(&tmv);
+    tma_prefetch_desc(&tmq);
+  }
+  // The kernel is launched as a programmatic dependent of the previous kernel on the stream (for
+  // example the kv_append that wrote the new token's K/V): everything above overlaps that kernel,
+  // and no input (lengths, positions, queries, cache, block table) is read before it completed.
+  pdl_wait();
   Plan plan;
   build_plan<__nv_bfloat16>(a, plan, pre, nlen, wlo, warp, lane, producer_warp);
   pdl_launch_dependents();
@@ -550,9 +559,6 @@ __global__ void __launch_bounds__(Bf16Cfg<D, MT>::kThreads, 1)
 
     if constexpr (kMode == kContig) {
       if (lane == 0) {
-        tma_prefetch_desc(&tmk);
-        tma_prefetch_desc(&tmv);
-        tma_prefetch_desc(&tmq);
         // Test hook (off unless the host enabled it): CTA 0's producer waits on a barrier that
         // nothing signals; the bounded wait runs out and records GQA_DEVERR_TIMEOUT, no copy is
         // issued, and the consumers' own bounded waits on the first stage then run out too (all
@@ -598,11 +604,6 @@ __global__ void __launch_bounds__(Bf16Cfg<D, MT>::kThreads, 1)
       // issues the copies: one 16-row box per sub-tile (16 rows x 128 B = 2 KiB keeps the 1 KiB
       // swizzle atoms aligned, so the stage has the layout of one 64-row box). Sub-tiles past the
       // tile's valid keys are not loaded (the consumer warp owning such a slice skips it).
-      if (lane == 0) {
-        tma_prefetch_desc(&tmk);
-        tma_prefetch_desc(&tmv);
-        tma_prefetch_desc(&tmq);
-      }
       int chunk = blockIdx.x;
       int next = 0;
       if (lane == 0) next = dyn && chunk < plan.n_chunks ? G + atomicAdd(&a.hdr->ticket, 1) : plan.n_chunks;
@@ -974,14 +975,17 @@ __global__ void __launch_bounds__(MlaCfg::kThreads, 1)
     }
     fence_barrier_init();
   }
+  if (warp == producer_warp && lane == 0) {
+    tma_prefetch_desc(&tmc);
+    tma_prefetch_desc(&tmq);
+  }
+  pdl_wait();  // launched as a programmatic dependent: no input is read before this
   Plan plan;
   build_plan<__nv_bfloat16>(a, plan, pre, nlen, wlo, warp, lane, producer_warp);
   pdl_launch_dependents();
 
   if (warp == producer_warp) {
     if (lane == 0) {
-      tma_prefetch_desc(&tmc);
-      tma_prefetch_desc(&tmq);
       int stage = 0;
       uint32_t phase = 0;
       int issued = 0;
@@ -1339,6 +1343,31 @@ cudaError_t launch_merge(const KArgs& ka, cudaStream_t s) {
   return e;
 }
 
+// Launch `kern` as a programmatic dependent of the previous kernel on the stream (its prologue
+// overlaps that kernel; the kernel waits with griddepcontrol.wait before reading any input), or
+// as an ordinary launch where the stream does not support it.
+template <typename... KParams, typename... Args>
+cudaError_t launch_dependent(void (*kern)(KParams...), int grid, int threads, size_t smem, cudaStream_t s,
+                             Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3((unsigned)threads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, args...);
+  if (e != cudaSuccess) {
+    (void)cudaGetLastError();
+    cfg.numAttrs = 0;
+    e = cudaLaunchKernelEx(&cfg, kern, args...);
+  }
+  return e;
+}
+
 template <int D, int MT, int kMode>
 cudaError_t launch_bf16_typed(const KArgs& ka, const CUtensorMap* tm, int grid, cudaStream_t s) {
   using C = Bf16Cfg<D, MT>;
@@ -1352,8 +1381,7 @@ cudaError_t launch_bf16_typed(const KArgs& ka, const CUtensorMap* tm, int grid, 
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < 64) attr_set[dev] = true;
   }
-  kern<<<grid, C::kThreads, C::kSmem, s>>>(tm[0], tm[1], tm[2], ka);
-  e = cudaGetLastError();
+  e = launch_dependent(kern, grid, C::kThreads, C::kSmem, s, tm[0], tm[1], tm[2], ka);
   if (e != cudaSuccess) return e;
   return launch_merge<__nv_bfloat16, true>(ka, s);
 }
@@ -1470,8 +1498,7 @@ cudaError_t launch_mla_bf16(const DecodeArgs& a, const CUtensorMap* tmaps, cudaS
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < 64) attr_set[dev] = true;
   }
-  dec::mla_bf16_kernel<<<a.num_sms, C::kThreads, C::kSmem, s>>>(tmaps[0], tmaps[1], k);
-  e = cudaGetLastError();
+  e = dec::launch_dependent(dec::mla_bf16_kernel, a.num_sms, C::kThreads, C::kSmem, s, tmaps[0], tmaps[1], k);
   if (e != cudaSuccess) return e;
   return dec::launch_merge<__nv_bfloat16, true>(k, s);
 }

@@ -16,6 +16,9 @@ namespace {
 template <typename Vec>
 __global__ void __launch_bounds__(256) kv_append_kernel(AppendArgs a, int vecs_per_row,
                                                          long long total) {
+  // A decode launched as a programmatic dependent of this copy may start its prologue now; it
+  // reads the cache only after this grid has completed (griddepcontrol.wait).
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const long long stride = (long long)gridDim.x * blockDim.x;
   for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += stride) {
     const long long row = i / vecs_per_row;

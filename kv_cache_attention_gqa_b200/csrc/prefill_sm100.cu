@@ -69,6 +69,7 @@ constexpr int kSoftmaxWarp0 = 4;  // first softmax warp: warps 4-7 serve tile 0,
 constexpr int kRegsControl = 64;  // per thread, first warpgroup (producer, MMA issuer, idle)
 constexpr int kRegsSoftmax = 216; // per thread, softmax warpgroups
 constexpr uint32_t kTmemCols = 512;
+constexpr int kBarBytes = 512;  // barrier block: the mbarriers, the TMEM address and the abort flag
 constexpr float kRescaleThreshold = 8.0f;  // base-2 units: P <= 2^8 between rescales
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -86,7 +87,8 @@ struct Cfg {
   static constexpr int kOffBar = kOffV + kVStages * kKVBytes;
   // barriers + slack for 1024-byte alignment; at least 120 KiB so that only one CTA (which
   // allocates all 512 TMEM columns) is resident per SM
-  static constexpr int kSmem = kOffBar + 256 + 1024 > 120 * 1024 ? kOffBar + 256 + 1024 : 120 * 1024;
+  static constexpr int kSmem =
+      kOffBar + kBarBytes + 1024 > 120 * 1024 ? kOffBar + kBarBytes + 1024 : 120 * 1024;
   static_assert(kSmem <= 227 * 1024, "shared memory budget");
   static constexpr uint32_t colS(int t) { return (uint32_t)(256 * t); }
   static constexpr uint32_t colO(int t) { return (uint32_t)(256 * t + 128); }
@@ -107,21 +109,26 @@ struct PArgs {
   unsigned* err;
 };
 
-// barrier indices inside the barrier block
-enum {
-  kBarQ = 0,          // + tile (2): Q rows landed in shared memory (TMA)
-  kBarKFull = 2,      // + K stage (3)
-  kBarVFull = 5,      // + V stage (2)
-  kBarKEmpty = 7,     // + tile * 3 + K stage: the tile's S = Q K^T on that stage completed
-  kBarVEmpty = 13,    // + tile * 2 + V stage: the tile's O += P V on that stage completed
-  kBarS = 17,         // + tile (2): S_t = Q_t K_j^T of the tile's current block completed
-  kBarP = 19,         // + tile (2): P_t of the current block is in TMEM (128 arrivals)
-  kBarO = 21,         // + tile (2): O_t += P_t V_j of the current block completed
-  kBarDone = 23,      // + tile (2): every MMA of the tile's issuer completed
-  kBarNever = 25,     // never signalled: the test hook's wait on it always runs out
-  kBarTurn = 26,      // + tile (2): the other tile finished its exponentials (128 arrivals)
-  kNumBars = 28
+// barrier indices inside the barrier block (derived from the ring depths, so they never overlap)
+enum : int {
+  kBarQ = 0,                                    // + tile: Q rows landed in shared memory (TMA)
+  kBarKFull = kBarQ + kTiles,                   // + K stage
+  kBarVFull = kBarKFull + kKStages,             // + V stage
+  kBarKEmpty = kBarVFull + kVStages,            // + chain * kKStages + K stage: the chain's
+                                                //   S = Q K^T on that stage completed
+  kBarVEmpty = kBarKEmpty + kTiles * kKStages,  // + chain * kVStages + V stage: its O += P V did
+  kBarS = kBarVEmpty + kTiles * kVStages,       // + chain: S_t of the chain's current block is in
+                                                //   TMEM
+  kBarP = kBarS + kTiles,                       // + chain: P_t of its current block is in TMEM
+                                                //   (128 arrivals)
+  kBarO = kBarP + kTiles,                       // + chain: O_t += P_t V of its current block done
+  kBarDone = kBarO + kTiles,                    // + chain: every MMA of the chain's issuer done
+  kBarNever = kBarDone + kTiles,                // never signalled: the test hook's wait runs out
+  kBarTurn = kBarNever + 1,                     // + chain: the other chain finished its
+                                                //   exponentials (128 arrivals)
+  kNumBars = kBarTurn + kTiles
 };
+static_assert(kNumBars * 8 + 8 <= kBarBytes, "barrier block");
 
 // Bounded wait that also gives up as soon as another thread of the CTA has aborted.
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort,
@@ -332,9 +339,10 @@ __device__ __forceinline__ void softmax_role(const PArgs& a, const Work& w, int 
       }
     }
     // P = 2^(s c - m_use) as bf16 pairs over the first 64 S columns. A row that has seen no
-    // visible key yet (only possible under a sliding window) keeps m = -inf; its P is 0, computed
-    // against 0 instead of -inf.
-    const float m_sub = kWin && m_use == -INFINITY ? 0.f : m_use;
+    // visible key yet keeps m = -inf (under a sliding window, or in split mode when the chain's
+    // first block lies wholly after the row's position); its P is 0, computed against 0 instead
+    // of -inf.
+    const float m_sub = m_use == -INFINITY ? 0.f : m_use;
     float sum0 = 0.f, sum1 = 0.f;
 #pragma unroll
     for (int cc = 0; cc < 4; ++cc) {
@@ -382,8 +390,8 @@ __device__ __forceinline__ void softmax_role(const PArgs& a, const Work& w, int 
     if (ok && (zero_tail || zero_head)) {
       const int vs = j % kVStages;
       if (wait_bar(bar(kBarVFull + vs), (uint32_t)((j / kVStages) & 1), abort, a.err)) {
-        const long long key = (long long)bkey0 + row;
-        if ((zero_tail && key >= w.kv) || (zero_head && key <= cta_pos_min - win)) {
+        const long long key = (long long)bkey0 + row;  // thread `row` owns V row `row` of the block
+        if (row < kBN && ((zero_tail && key >= w.kv) || (zero_head && key <= cta_pos_min - win))) {
 #pragma unroll
           for (int ch = 0; ch < C::kNch; ++ch) {
 #pragma unroll
@@ -659,11 +667,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       if constexpr (kSplit) {
         const int period = stages % 2 ? 2 * stages : stages;
         return wait_bar(bar(empty0 + (b % 2) * stages + s), (uint32_t)((b / period) & 1), abort, a.err);
+      } else {
+        for (int t = 0; t < w.nt; ++t)
+          if (b < w.nb[t] && !wait_bar(bar(empty0 + t * stages + s), (uint32_t)((b / stages) & 1), abort, a.err))
+            return false;
+        return true;
       }
-      for (int t = 0; t < w.nt; ++t)
-        if (b < w.nb[t] && !wait_bar(bar(empty0 + t * stages + s), (uint32_t)((b / stages) & 1), abort, a.err))
-          return false;
-      return true;
     };
     for (int j = 0; j < nbmax && go; ++j) {
       const int ks = j % kKStages, kn = j / kKStages;

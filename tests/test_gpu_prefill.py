@@ -52,6 +52,16 @@ def test_prefill_offset_and_nan_tail(d):
     _run(2, 8, 2, 130, 600, d, [300, 460], [431, 590], seed=7, nan_tail=True)
 
 
+@pytest.mark.parametrize("d", [64, 128])
+def test_prefill_rows_before_a_chains_first_block(d):
+    # Few tiles, so each CTA runs one tile with its K/V blocks alternating between two chains. With
+    # r=1 a tile holds 128 positions; from position 50 it spans key blocks 0 and 1, so the rows
+    # before position 128 see no key of the second chain's first block (their running maximum is
+    # still -inf there) and must take nothing from it.
+    _run(1, 2, 2, 200, 300, d, [50], [250], seed=13)
+    _run(2, 4, 4, 180, 400, d, [100, 0], [280, 180], seed=14)
+
+
 def test_prefill_not_causal():
     _run(1, 8, 2, 100, 300, 128, [0], [260], causal=False, seed=3)
 

@@ -356,8 +356,10 @@ __device__ __forceinline__ void softmax_role(const PArgs& a, const Work& w, int 
         pk[k] = pack_bf16x2(p0, p1);
       }
       tc::st16(lane_addr + colS + cc * 16, pk);
+      // the other chain's turn starts halfway through this one's exponentials (the halves
+      // overlap a little on the unit, which measured faster than strict alternation)
+      if (cc == 1 && w.nt == 2) mbar_arrive(bar(kBarTurn + (t ^ 1)));
     }
-    if (w.nt == 2) mbar_arrive(bar(kBarTurn + (t ^ 1)));  // the other chain's turn
     l = l * alpha + (sum0 + sum1);
     m = m_use;
     // the warp rescales its O rows together when any of its rows needs it (rows that do not need

@@ -103,7 +103,24 @@ def recorded_traffic(summary_name, digest):
     out = {}
     for key, val in re.findall(r"traffic_bytes_per_launch\[([^\]]+)\]:\s*([0-9]+)", text):
         out[key] = int(val)
+    for key, val in re.findall(r"algorithmic_bytes\[([^\]]+)\]:\s*([0-9]+)", text):
+        out["algorithmic:" + key] = int(val)
     return out or None
+
+
+DECODE_SOURCES = ["kv_cache_attention_gqa_b200/csrc/decode.cu", "kv_cache_attention_gqa_b200/csrc/common.cuh"]
+PREFILL_SOURCES = ["kv_cache_attention_gqa_b200/csrc/prefill_sm100.cu", "kv_cache_attention_gqa_b200/csrc/common.cuh",
+                   "kv_cache_attention_gqa_b200/csrc/tcgen05.cuh"]
+
+
+def scaled_traffic(summary_name, sources, key, algorithmic_bytes):
+    """DRAM bytes per launch from an ncu summary taken on a (possibly smaller) case of the same
+    kernel, scaled to `algorithmic_bytes` by the captured case's traffic / algorithmic ratio; None
+    when absent or captured on a different version of the kernel."""
+    rec = recorded_traffic(summary_name, source_digest(sources))
+    if not rec or key not in rec or ("algorithmic:" + key) not in rec:
+        return None
+    return round(rec[key] * algorithmic_bytes / rec["algorithmic:" + key])
 
 
 class L2Flush:
@@ -517,7 +534,10 @@ def run_ragged(args, dev, hbm_peak, peak_kind):
             "launch": mode, "value": round(gbs, 1), "unit": "GB/s", "us": round(ms * 1e3, 2),
             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm_peak, "unit": "GB/s",
                          "frac": round(gbs / hbm_peak, 4), "peak_kind": f"hbm_gbs of {peak_kind}",
-                         "algorithmic_bytes_per_launch": nbytes},
+                         "algorithmic_bytes_per_launch": nbytes,
+                         "traffic": scaled_traffic("decode_ragged_decode_b16.md", DECODE_SOURCES, "ragged_b16", nbytes),
+                         "traffic_note": "ncu DRAM read + write of 16 sequences of the same length distribution, "
+                                         "scaled by algorithmic bytes"},
             "output_finite": finite, "gpu_launches_per_call": 2}
 
 
@@ -551,7 +571,10 @@ def run_chunked(args, dev, tf_peak, peak_kind):
             "launch": mode, "value": round(tflops, 1), "unit": "TFLOP/s", "ms": round(ms, 4),
             "roofline": {"bound": "tensor", "achieved": round(tflops, 1), "peak": tf_peak, "unit": "TFLOP/s",
                          "frac": round(tflops / tf_peak, 4), "peak_kind": f"bf16_tflops of {peak_kind}",
-                         "algorithmic_flops_per_launch": flops},
+                         "algorithmic_flops_per_launch": flops,
+                         "traffic": scaled_traffic("prefill_chunked_prefill.md", PREFILL_SOURCES, "chunked",
+                                                   138412032),
+                         "traffic_note": "ncu DRAM read + write of one launch (K/V + Q: 138,412,032 B)"},
             "kv_append": {"us": round(app_ms * 1e3, 2), "bytes": app_bytes,
                           "GB_s": round(app_bytes / (app_ms / 1e3) / 1e9, 1)}}
 
@@ -638,7 +661,7 @@ def run_ours(args, rank, world, dist):
     per_variant = per_variant_rates(variants, dec_ms, hbm_peak)
     dec_total_ms = sum(sum(row) for row in dec_ms) / args.steps
     achieved = step_bytes / (dec_total_ms / 1e3) / 1e9
-    digest = source_digest(["kv_cache_attention_gqa_b200/csrc/decode.cu", "kv_cache_attention_gqa_b200/csrc/common.cuh"])
+    digest = source_digest(DECODE_SOURCES)
     traffic = recorded_traffic("decode_splitkv_decode_8k.md", digest)
     traffic_per_launch = None
     if traffic and all(f"h_kv={v['h_kv']}" in traffic for v in variants):

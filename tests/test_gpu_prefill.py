@@ -62,6 +62,26 @@ def test_prefill_rows_before_a_chains_first_block(d):
     _run(2, 4, 4, 180, 400, d, [100, 0], [280, 180], seed=14)
 
 
+@pytest.mark.parametrize("h_q,h_kv,S_q,T", [
+    (64, 2, 37, 150),    # r=32: tiles of 4 positions x 32 heads; few CTAs (one tile each)
+    (64, 1, 23, 90),     # r=64: 2 positions per tile
+    (128, 1, 300, 300),  # r=128: 1 position per tile; 150 pairs of tiles (pair mode)
+    (256, 1, 9, 140),    # r=256: two 128-head blocks per group
+    (8, 2, 1, 77),       # a single query row
+])
+def test_prefill_wide_groups_and_tiny_tiles(h_q, h_kv, S_q, T):
+    _run(1, h_q, h_kv, S_q, T, 128, [T - S_q], [T], seed=h_q + S_q)
+
+
+def test_prefill_many_sequences_offsets_and_lengths():
+    """B=6 with per-sequence query offsets and lengths (pair mode: enough tiles for every SM)."""
+    rng = np.random.default_rng(5)
+    kv = rng.integers(200, 600, size=6)
+    qs = np.maximum(kv - 180, 0) - rng.integers(0, 20, size=6).clip(0, None)
+    qs = np.maximum(qs, 0)
+    _run(6, 16, 4, 180, 600, 128, qs.tolist(), kv.tolist(), seed=8, nan_tail=True)
+
+
 def test_prefill_not_causal():
     _run(1, 8, 2, 100, 300, 128, [0], [260], causal=False, seed=3)
 

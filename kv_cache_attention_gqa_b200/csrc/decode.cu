@@ -435,13 +435,10 @@ struct TileMeta {
 };
 constexpr int kFirst = 1, kLast = 2, kEnd = 4;
 
-#ifndef GQA_DECODE_STAGES_1
-#define GQA_DECODE_STAGES_1 5
-#endif
 template <int D, int MT>
 struct Bf16Cfg {
   // pipeline depth: as many 32 KiB stages as shared memory allows next to the other buffers
-  static constexpr int kStages = MT == 1 ? GQA_DECODE_STAGES_1 : 4;
+  static constexpr int kStages = MT == 1 ? 5 : 4;
   static constexpr int kNch = D / 64;                    // 64-column (128-byte) chunks
   static constexpr int kChunkBytes = kTile * 128;        // one column chunk of one K/V tile
   static constexpr int kTileBytes = kNch * kChunkBytes;  // K (or V) tile
@@ -926,10 +923,8 @@ __global__ void __launch_bounds__(Bf16Cfg<D, MT>::kThreads, 1)
 //   PV  warp w accumulates latent columns [64w, 64w+64) of O += P V over the 64 keys, reading V
 //       as the tile's first eight column chunks.
 constexpr int kMlaDqk = 576, kMlaDv = 512, kMlaHeads = 16;
-#ifndef GQA_MLA_QREG
-#define GQA_MLA_QREG 16  // k-steps of the query kept in registers (9 warps: at most 168 regs each; 16 does not spill)
-#endif
-constexpr int kMlaQReg = GQA_MLA_QREG;
+// k-steps of the query kept in registers (9 warps: at most 168 registers each; 16 does not spill)
+constexpr int kMlaQReg = 16;
 struct MlaCfg {
   static constexpr int kStages = 2;  // also the number of query slots (see the producer)
   static constexpr int kNch = kMlaDqk / 64;              // 9 column chunks of a cache row

@@ -63,6 +63,15 @@ constexpr float kLn2 = 0.6931471805599453f;
 
 __host__ __device__ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// Quotient of two non-negative 64-bit integers. When both fit in 32 bits (every workload short of
+// 2^32 keys in all) it takes a 32-bit unsigned division, a fraction of the 64-bit routine's
+// dependent instructions; the plan and the merge sit on the critical path of every call.
+__device__ __forceinline__ long long udiv(long long n, long long d) {
+  if ((((unsigned long long)n | (unsigned long long)d) >> 32) == 0)
+    return (long long)((unsigned)n / (unsigned)d);
+  return n / d;
+}
+
 // Workspace:
 //   [0, 256)       header: chunk ticket (reset to 0 by the merge kernel), chunk size, chunk count
 //   pre_off        int64 pre[B + 1]: prefix sums of the visible lengths (written by CTA 0)
@@ -170,7 +179,7 @@ __device__ __forceinline__ Piece locate(const Plan& p, int B, int hblocks, long 
   pc.n = p.nlen[b];
   const long long ng = (pc.n + p.gran - 1) / p.gran;  // unit length in granules
   const long long rel = x - p.pre[b] * p.UPB;
-  const int ui = (int)(rel / ng);  // g * hblocks + hb
+  const int ui = (int)udiv(rel, ng);  // g * hblocks + hb
   pc.g = ui / hblocks;
   pc.hb = ui - pc.g * hblocks;
   pc.unit = b * p.UPB + ui;
@@ -179,7 +188,7 @@ __device__ __forceinline__ Piece locate(const Plan& p, int B, int hblocks, long 
   const long long e = x_end - pc.unit_start;  // granules
   pc.end = e < ng ? x_end : pc.unit_start + ng;
   pc.k1 = e < ng ? (int)(e * p.gran) : pc.n;
-  pc.n_pieces = (int)((pc.unit_start + ng - 1) / p.C - pc.unit_start / p.C) + 1;
+  pc.n_pieces = (int)(udiv(pc.unit_start + ng - 1, p.C) - udiv(pc.unit_start, p.C)) + 1;
   return pc;
 }
 
@@ -239,17 +248,17 @@ __device__ void build_plan(const KArgs& a, Plan& p, long long* pre, int* nlen, i
   p.gran = a.gran;
   p.UPB = a.h_kv * a.hblocks;
   p.K = pre[a.B] * p.UPB;
-  long long C = (p.K + a.n_max - 1) / a.n_max;
+  long long C = udiv(p.K + a.n_max - 1, a.n_max);
   if (a.auto_chunk) {
     // at least kMinChunkAuto keys, and at least 16 keys per query row, so the partial written per
     // chunk (hpu x d_h fp32) stays small against the chunk's K/V bytes (2 x C x d_h bf16)
     const long long lo_keys = 16LL * a.hpu > kMinChunkAuto ? 16LL * a.hpu : kMinChunkAuto;
-    const long long lo = (lo_keys + a.gran - 1) / a.gran;
+    const long long lo = udiv(lo_keys + a.gran - 1, a.gran);
     if (C < lo) C = lo;
   }
   if (C < 1) C = 1;
   p.C = C;
-  p.n_chunks = (int)((p.K + C - 1) / C);
+  p.n_chunks = (int)udiv(p.K + C - 1, C);
 
   if (blockIdx.x == 0) {
     for (int b = threadIdx.x; b <= a.B; b += blockDim.x) {
@@ -311,7 +320,7 @@ template <typename OutT, bool kFast, int kV>
 __device__ __forceinline__ void merge_row(const KArgs& a, int lane, int unit, int h,
                                           long long c0, long long c1, long long out_base,
                                           long long lse_index, int col_base) {
-  constexpr int kU = 8;
+  constexpr int kU = 16;
   const int D = a.D;
   const int col0 = col_base + lane * kV;
   const bool active = col0 < D;
@@ -363,27 +372,31 @@ __host__ __device__ inline int merge_slices(int D) { return D > 256 ? (D + 127) 
 
 template <typename OutT, bool kFast>
 __global__ void __launch_bounds__(256) merge_kernel(KArgs a) {
-  pdl_wait();  // the decode grid has completed and its writes are visible
-  const long long C = a.hdr->chunk;
-  if (blockIdx.x == 0 && threadIdx.x == 0) a.hdr->ticket = 0;  // ready for the next call
+  // The row's place (unit, head, output offsets) depends only on the arguments, so it is worked
+  // out before the wait (units number fewer than 2^31: B * h_q is below it).
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int slices = merge_slices(a.D);
   const long long wid = (long long)blockIdx.x * 8 + warp;
-  const long long row = wid / slices;
+  const long long row = udiv(wid, slices);
   const int slice = (int)(wid - row * slices);
   const int UPB = a.h_kv * a.hblocks;
-  const long long U = (long long)a.B * UPB;
-  if (row >= U * a.hpu) return;
-  const int unit = (int)(row / a.hpu), h = (int)(row - (long long)unit * a.hpu);
+  const long long rows = (long long)a.B * UPB * a.hpu;
+  const int unit = (int)udiv(row, a.hpu), h = (int)(row - (long long)unit * a.hpu);
   const int b = unit / UPB, ui = unit - b * UPB;
   const int g = ui / a.hblocks, hb = ui - g * a.hblocks;
   const int nh = min(a.hpu, a.r - hb * a.hpu);
-  if (h >= nh) return;
-  const int n = a.nlen[b];
+  pdl_wait();  // the decode grid has completed and its writes are visible
+  if (blockIdx.x == 0 && threadIdx.x == 0) a.hdr->ticket = 0;  // ready for the next call
+  if (row >= rows || h >= nh) return;
+  // the chunk size, the unit's length and its sequence's prefix: three independent loads, one
+  // round trip
+  const long long C = __ldcg(&a.hdr->chunk);
+  const int n = __ldcg(&a.nlen[b]);
+  const long long pre_b = __ldcg(&a.pre[b]);
   if (n == 0) return;
   const long long ng = (n + a.gran - 1) / a.gran;
-  const long long P = a.pre[b] * UPB + (long long)ui * ng;
-  const long long c0 = P / C, c1 = (P + ng - 1) / C;
+  const long long P = pre_b * UPB + (long long)ui * ng;
+  const long long c0 = udiv(P, C), c1 = udiv(P + ng - 1, C);
   if (c0 == c1) return;  // written directly by the decode kernel
   const int head = g * a.r + hb * a.hpu + h;
   const long long ob = ((long long)b * a.h_q + head) * a.D;

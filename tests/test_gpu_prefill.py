@@ -82,6 +82,26 @@ def test_prefill_many_sequences_offsets_and_lengths():
     _run(6, 16, 4, 180, 600, 128, qs.tolist(), kv.tolist(), seed=8, nan_tail=True)
 
 
+@pytest.mark.parametrize("d", [64, 128])
+def test_prefill_persistent_walk_mha_ragged(d):
+    """More pairs than SMs, so each CTA walks several items: r=1 (tiles of 128 positions, so the
+    second tile of a pair sees one more key block than the first and the first chain passes that
+    block over), an odd tile count (items with one tile), per-sequence offsets and lengths, and
+    NaN past every length."""
+    rng = np.random.default_rng(17)
+    kv = rng.integers(650, 900, size=8)
+    qs = (kv - 600 - rng.integers(0, 40, size=8)).clip(0, None)
+    _run(8, 8, 8, 600, 900, d, qs.tolist(), kv.tolist(), seed=21 + d, nan_tail=True)
+
+
+def test_prefill_persistent_walk_many_single_block_items():
+    """256 items of one K/V block each (64 short prompts x 4 groups): consecutive one-block items
+    on every CTA, where the chains' turn-taking has no waits at the start of each item."""
+    rng = np.random.default_rng(19)
+    kv = rng.integers(40, 128, size=64)
+    _run(64, 16, 4, 40, 128, 128, (kv - 40).tolist(), kv.tolist(), seed=23, nan_tail=True)
+
+
 def test_prefill_not_causal():
     _run(1, 8, 2, 100, 300, 128, [0], [260], causal=False, seed=3)
 

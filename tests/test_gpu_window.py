@@ -71,6 +71,32 @@ def test_prefill_window_offset_ragged_nan_outside(W):
     assert gqa.get_device_error() == 0
 
 
+@pytest.mark.parametrize("W", [100, 300])
+def test_prefill_window_persistent_walk(W):
+    """More pairs than SMs (each CTA walks several items) under a sliding window: r=1 tiles of 128
+    positions, per-sequence offsets and lengths, NaN below every sequence's earliest window and
+    past its length."""
+    import kv_cache_attention_gqa_b200 as gqa
+
+    B, h_q, h_kv, S_q, T, d = 8, 8, 8, 600, 1000, 128
+    g = torch.Generator().manual_seed(W + 1)
+    q = torch.randn(B, h_q, S_q, d, generator=g).to(torch.bfloat16)
+    k = torch.randn(B, h_kv, T, d, generator=g).to(torch.bfloat16)
+    v = torch.randn(B, h_kv, T, d, generator=g).to(torch.bfloat16)
+    rng = np.random.default_rng(W)
+    q_start = rng.integers(0, T - S_q + 1, size=B).astype(np.int32)
+    kv_len = np.minimum(q_start + S_q + rng.integers(0, 30, size=B), T).astype(np.int32)
+    lo = np.maximum(0, q_start - W + 1)
+    kp, vp = _poison_below(k, lo), _poison_below(v, lo)
+    for b in range(B):
+        kp[b, :, kv_len[b]:] = float("nan")
+        vp[b, :, kv_len[b]:] = float("nan")
+    o = gqa.prefill(q.cuda(), kp.cuda(), vp.cuda(), q_start=q_start.tolist(), kv_len=kv_len.tolist(), window=W)
+    ref, _ = oracle.attention_ref(_f64(q), _f64(k), _f64(v), q_start=q_start, kv_len=kv_len, window=W)
+    assert_bf16_close(_f64(o), ref, f"persistent walk W={W}")
+    assert gqa.get_device_error() == 0
+
+
 @pytest.mark.parametrize("W", [1, 5, 70])
 def test_prefill_window_fp32_check_mode(W):
     import kv_cache_attention_gqa_b200 as gqa

@@ -159,10 +159,12 @@ gqa_status gqa_mla_decode(const void* q, const void* cache, void* o, float* lse,
  *   dtype       GQA_BF16 (d_h 64 or 128; tcgen05 kernels, bf16 gradients) or GQA_FP32 (d_h <= 256;
  *               scalar check mode, fp32 gradients). All tensors share the dtype; lse is fp32.
  *   workspace   device memory of at least gqa_prefill_backward_workspace_size(B, h_q, S_q) bytes,
- *               256-byte aligned, no initial contents required (two fp32 values per query row).
- * Two launches run in order on `stream`: the row term D (with the base-2 lse), then one grid
- * whose first CTAs run the key-stationary dK/dV pass (the heads of a group add up in one CTA, no
- * atomics) and whose remaining CTAs run the query-stationary dQ pass.
+ *               256-byte aligned, no initial contents required (two fp32 values per query row and
+ *               a work-item counter). Calls that share a workspace must not overlap on the GPU.
+ * Two launches run in order on `stream`: the row term D (with the base-2 lse; it also resets the
+ * counter), then one persistent grid whose CTAs take the key-stationary dK/dV tiles (the heads of
+ * a group add up in one CTA, no atomics) and then the query-stationary dQ tiles, heaviest first,
+ * from the counter.
  * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA.
  */
 size_t gqa_prefill_backward_workspace_size(int B, int h_q, int S_q);

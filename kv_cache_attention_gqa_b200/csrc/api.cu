@@ -319,7 +319,7 @@ gqa_status gqa_prefill(const void* q, const void* k_cache, const void* v_cache, 
 size_t gqa_prefill_backward_workspace_size(int B, int h_q, int S_q) {
   if (B <= 0 || h_q <= 0 || S_q <= 0) return 0;
   const size_t rows = (size_t)B * h_q * S_q;
-  return 2 * ((rows * 4 + 255) / 256 * 256);
+  return 2 * ((rows * 4 + 255) / 256 * 256) + 256;  // lse2, D, the work-item counter
 }
 
 gqa_status gqa_prefill_backward(const void* q, const void* k_cache, const void* v_cache,
@@ -363,8 +363,10 @@ gqa_status gqa_prefill_backward(const void* q, const void* k_cache, const void* 
   a.scale = scale;
   a.causal = causal;
   a.window = window;
+  const size_t half = (need - 256) / 2;
   a.lse2 = reinterpret_cast<float*>(workspace);
-  a.drow = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(workspace) + need / 2);
+  a.drow = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(workspace) + half);
+  a.ticket = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(workspace) + 2 * half);
   a.err = device_error_ptr();
   if (!a.err) return GQA_ERR_CUDA;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -392,7 +394,9 @@ gqa_status gqa_prefill_backward(const void* q, const void* k_cache, const void* 
       !encode_bf16(&maps[4], q, 3, qdims, qstrides, qbox_tile) ||
       !encode_bf16(&maps[5], d_o, 3, qdims, qstrides, qbox_tile))
     return GQA_ERR_CUDA;
-  return from_cuda(launch_backward_bf16(a, maps, s));
+  const int sms = sm_count();
+  if (sms <= 0) return GQA_ERR_CUDA;
+  return from_cuda(launch_backward_bf16(a, maps, sms, s));
 }
 
 size_t gqa_decode_workspace_size(int B, int h_q, int h_kv, int T_max, int d_h, gqa_dtype dtype,

@@ -8,7 +8,12 @@
 //   dS = P * (dP - D),  dQ_a = scale dS K_g,  dK_g += scale dS^T Q_a.
 // The mask is the forward's: causal by absolute position, length, and an optional sliding window.
 //
-// Two launches: rowterm, then one grid whose first CTAs run dkdv and the rest dq:
+// Two launches: rowterm, then one persistent grid (one CTA per SM) whose CTAs take work items in
+// the order dkdv tiles (heaviest first), then dq tiles (heaviest first): item c for CTA c, then
+// items from a ticket counter that rowterm resets, so an SM that finishes early takes the next
+// item, as the hardware's CTA scheduler would, without a CTA exit and launch per item (measured:
+// the 512-column TMEM release of an exiting CTA took 3.5-5 us after these kernels' epilogues).
+// Each item initialises its barriers and invalidates them at its end.
 //   rowterm   one warp per query row: D = rowsum(dO * O) and the base-2 lse (fp32 workspace).
 //   dkdv      one CTA per (sequence, KV head, 128-key block). The keys sit on the 128 TMEM lanes;
 //             the CTA walks every 64-row query block of every head of the group, so the r heads'
@@ -63,6 +68,8 @@ struct BArgs {
   int n_kb;                 // key blocks per (b, g): ceil(T_max / 128)
   float scale, sl2;         // scale and scale * log2(e)
   int causal, window;
+  int n_items;              // dkdv tiles + dq tiles
+  int* ticket;              // items handed out past the first gridDim.x (reset by rowterm)
   unsigned* err;
 };
 
@@ -128,9 +135,11 @@ __device__ __forceinline__ uint64_t desc_mnmajor(uint32_t tile, int kk) {
 // =============================================================================================
 template <typename T>
 __global__ void __launch_bounds__(256) rowterm_kernel(const T* o, const T* d_o, const float* lse,
-                                                      float* lse2, float* drow, long long rows, int D) {
+                                                      float* lse2, float* drow, long long rows, int D,
+                                                      int* ticket) {
   const long long row = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
+  if (ticket && blockIdx.x == 0 && threadIdx.x == 0) *ticket = 0;  // for the next kernel's items
   if (row >= rows) return;
   const T* a = o + row * D;
   const T* b = d_o + row * D;
@@ -207,7 +216,7 @@ enum {
 template <int D>
 __device__ __forceinline__ void dkdv_cta(const CUtensorMap& tmq, const CUtensorMap& tmdo,
                                          const CUtensorMap& tmk, const CUtensorMap& tmv, const BArgs& a,
-                                         int tile) {
+                                         int tile, uint32_t tmem) {
   using C = KvCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -264,14 +273,10 @@ __device__ __forceinline__ void dkdv_cta(const CUtensorMap& tmq, const CUtensorM
     if (!valid && kb == 0 && g == 0)
       set_device_error(a.err, kv < 1 || kv > a.T_max ? GQA_DEVERR_KV_LEN : GQA_DEVERR_POSITION);
   }
-  if (warp == 1) {
-    tc::tmem_alloc(smem_u32(tmem_slot), kTmemCols);
-    tc::tmem_relinquish();
-  }
+  (void)tmem_slot;
   tc::fence_before_sync();
-  __syncthreads();
+  cta_sync();
   tc::fence_after_sync();
-  const uint32_t tmem = *tmem_slot;
   auto head_of = [&](int it) { return g * a.r + it / nq; };
   auto qblk_of = [&](int it) { return qb_lo + it % nq; };
 
@@ -480,12 +485,11 @@ __device__ __forceinline__ void dkdv_cta(const CUtensorMap& tmq, const CUtensorM
       }
     }
   }
+  // every role is done with the item (copies landed, MMAs complete, TMEM read): its barriers go
   tc::fence_before_sync();
-  __syncthreads();
-  if (warp == 1) {
-    tc::fence_after_sync();
-    tc::tmem_dealloc(tmem, kTmemCols);
-  }
+  cta_sync();
+  if (threadIdx.x == 0)
+    for (int i = 0; i < kKvBars; ++i) mbar_inval(bar(i));
 }
 
 // ---- dq: query-stationary dQ on the forward's tiles -------------------------------------------
@@ -525,7 +529,7 @@ enum {
 template <int D>
 __device__ __forceinline__ void dq_cta(const CUtensorMap& tmq, const CUtensorMap& tmdo,
                                        const CUtensorMap& tmk, const CUtensorMap& tmv, const BArgs& a,
-                                       int tile) {
+                                       int tile, uint32_t tmem) {
   using C = QCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -582,14 +586,10 @@ __device__ __forceinline__ void dq_cta(const CUtensorMap& tmq, const CUtensorMap
     *abort = 0;
     fence_barrier_init();
   }
-  if (warp == 1) {
-    tc::tmem_alloc(smem_u32(tmem_slot), kTmemCols);
-    tc::tmem_relinquish();
-  }
+  (void)tmem_slot;
   tc::fence_before_sync();
-  __syncthreads();
+  cta_sync();
   tc::fence_after_sync();
-  const uint32_t tmem = *tmem_slot;
   const int row0 = (b * a.h_kv + g) * a.T_max;
 
   if (warp == 0 && lane == 0 && nb > 0) {
@@ -788,12 +788,11 @@ __device__ __forceinline__ void dq_cta(const CUtensorMap& tmq, const CUtensorMap
       for (int v = half * (D / 16); v < (half + 1) * (D / 16); ++v) out[v] = make_uint4(0u, 0u, 0u, 0u);
     }
   }
+  // every role is done with the item (copies landed, MMAs complete, TMEM read): its barriers go
   tc::fence_before_sync();
-  __syncthreads();
-  if (warp == 1) {
-    tc::fence_after_sync();
-    tc::tmem_dealloc(tmem, kTmemCols);
-  }
+  cta_sync();
+  if (threadIdx.x == 0)
+    for (int i = 0; i < kQBars; ++i) mbar_inval(bar(i));
 }
 
 // One launch for both passes: the first n_dkdv CTAs run the key-stationary dK / dV pass
@@ -813,12 +812,36 @@ __global__ void __launch_bounds__(kKvThreads, 1)
                     const __grid_constant__ CUtensorMap tmq_tile, const __grid_constant__ CUtensorMap tmdo_tile,
                     const __grid_constant__ CUtensorMap tmk64, const __grid_constant__ CUtensorMap tmv64,
                     BArgs a, int n_dkdv) {
-  if ((int)blockIdx.x < n_dkdv) dkdv_cta<D>(tmq_rows, tmdo_rows, tmk128, tmv128, a, (int)blockIdx.x);
-  else dq_cta<D>(tmq_tile, tmdo_tile, tmk64, tmv64, a, (int)blockIdx.x - n_dkdv);
+  __shared__ uint32_t s_tmem;
+  __shared__ int s_next;
+  const int warp = threadIdx.x >> 5;
+  if (warp == 1) {  // all 512 columns, held across the CTA's items
+    tc::tmem_alloc(smem_u32(&s_tmem), kTmemCols);
+    tc::tmem_relinquish();
+  }
+  tc::fence_before_sync();
+  cta_sync();
+  tc::fence_after_sync();
+  const uint32_t tmem = s_tmem;
+  for (int item = blockIdx.x; item < a.n_items;) {
+    // the next item's ticket, fetched while this item runs by a thread of the elementwise warps
+    // (which wait for the first scores anyway); the item's closing barrier publishes it
+    if (threadIdx.x == 64) s_next = (int)gridDim.x + atomicAdd(a.ticket, 1);
+    if (item < n_dkdv) dkdv_cta<D>(tmq_rows, tmdo_rows, tmk128, tmv128, a, item, tmem);
+    else dq_cta<D>(tmq_tile, tmdo_tile, tmk64, tmv64, a, item - n_dkdv, tmem);
+    item = s_next;
+    cta_sync();  // every thread has read s_next before the next item writes it
+  }
+  tc::fence_before_sync();
+  cta_sync();
+  if (warp == 1) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, kTmemCols);
+  }
 }
 
 template <int D>
-cudaError_t launch_typed(const BArgs& p, const CUtensorMap* tm, cudaStream_t s) {
+cudaError_t launch_typed(const BArgs& p, const CUtensorMap* tm, int num_sms, cudaStream_t s) {
   static bool attr_set[64] = {false};  // per device: the shared-memory opt-in is set once
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -831,19 +854,24 @@ cudaError_t launch_typed(const BArgs& p, const CUtensorMap* tm, cudaStream_t s) 
   const long long n1 = (long long)p.n_kb * p.B * p.h_kv;
   const long long n2 = (long long)p.n_qt * p.B * p.h_kv * p.hblocks;
   if (n1 + n2 > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-  backward_kernel<D><<<(unsigned)(n1 + n2), kKvThreads, BwCfg<D>::kSmem, s>>>(
-      tm[0], tm[1], tm[2], tm[3], tm[4], tm[5], tm[6], tm[7], p, (int)n1);
+  if (n1 + n2 <= 0) return cudaSuccess;
+  BArgs q = p;
+  q.n_items = (int)(n1 + n2);
+  const long long ctas = n1 + n2 < num_sms ? n1 + n2 : num_sms;  // one CTA per SM
+  backward_kernel<D><<<(unsigned)ctas, kKvThreads, BwCfg<D>::kSmem, s>>>(
+      tm[0], tm[1], tm[2], tm[3], tm[4], tm[5], tm[6], tm[7], q, (int)n1);
   return cudaGetLastError();
 }
 
 }  // namespace bw
 
-cudaError_t launch_backward_bf16(const BackwardArgs& a, const CUtensorMap* tmaps, cudaStream_t s) {
+cudaError_t launch_backward_bf16(const BackwardArgs& a, const CUtensorMap* tmaps, int num_sms,
+                                 cudaStream_t s) {
   const long long rows = (long long)a.B * a.h_q * a.S_q;
   if (rows <= 0) return cudaSuccess;
   bw::rowterm_kernel<__nv_bfloat16><<<(unsigned)((rows * 32 + 255) / 256), 256, 0, s>>>(
       reinterpret_cast<const __nv_bfloat16*>(a.o), reinterpret_cast<const __nv_bfloat16*>(a.d_o), a.lse,
-      a.lse2, a.drow, rows, a.d_h);
+      a.lse2, a.drow, rows, a.d_h, a.ticket);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   bw::BArgs p;
@@ -869,9 +897,11 @@ cudaError_t launch_backward_bf16(const BackwardArgs& a, const CUtensorMap* tmaps
   p.sl2 = a.scale * bw::kLog2e;
   p.causal = a.causal;
   p.window = a.window;
+  p.ticket = a.ticket;
+  p.n_items = 0;
   p.err = a.err;
-  if (a.d_h == 128) return bw::launch_typed<128>(p, tmaps, s);
-  if (a.d_h == 64) return bw::launch_typed<64>(p, tmaps, s);
+  if (a.d_h == 128) return bw::launch_typed<128>(p, tmaps, num_sms, s);
+  if (a.d_h == 64) return bw::launch_typed<64>(p, tmaps, num_sms, s);
   return cudaErrorInvalidValue;
 }
 

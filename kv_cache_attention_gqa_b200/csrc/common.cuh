@@ -37,6 +37,20 @@ __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
 }
 
+// CTA-wide barrier for code where a warp's lanes may have diverged before it (one lane running a
+// producer loop while the others skip it, a loop over threadIdx). __syncthreads is the aligned
+// form of the barrier, which expects every warp to arrive converged: a warp whose lanes got there
+// at different times counted twice, and the barrier ending an item of the backward kernel let
+// thread 0 through two to five microseconds before the MMA and elementwise warps arrived (a
+// __syncwarp in front did not change that). The unaligned form counts threads one by one.
+__device__ __forceinline__ void cta_sync() {
+  asm volatile("barrier.sync 0;" ::: "memory");
+}
+
+// Invalidates an mbarrier (before its shared memory is initialised again or used for data).
+__device__ __forceinline__ void mbar_inval(uint32_t bar) {
+  asm volatile("mbarrier.inval.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+}
 __device__ __forceinline__ void fence_barrier_init() {
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
@@ -120,6 +134,9 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
+// Barrier among `threads` threads (whole warps) on barrier `id`, aligned form: only where every
+// warp taking part arrives converged (no role or lane-divergent loop right before it; the
+// unaligned form, as in cta_sync, measured 2% slower on the decode_8k step).
 __device__ __forceinline__ void named_barrier_sync(int id, int threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }

@@ -223,7 +223,7 @@ __device__ void build_plan(const KArgs& a, Plan& p, long long* pre, int* nlen, i
     nlen[b] = n;
     wlo[b] = lo;
   }
-  __syncthreads();
+  cta_sync();
   // ... then one warp turns them into prefix sums in granules, from shared memory
   if (warp == w0) {
     long long run = 0;
@@ -241,7 +241,7 @@ __device__ void build_plan(const KArgs& a, Plan& p, long long* pre, int* nlen, i
     }
     if (lane == 0) pre[a.B] = run;
   }
-  __syncthreads();
+  cta_sync();
   p.pre = pre;
   p.nlen = nlen;
   p.wlo = wlo;
@@ -864,12 +864,12 @@ __global__ void __launch_bounds__(Bf16Cfg<D, MT>::kThreads, 1)
     const float l1t = l1s + __shfl_xor_sync(0xffffffffu, l1s, 2);
     float* sm = st_m + mt * 64;
     float* sl = st_l + mt * 64;
-    if (tq == 0) {
-      sm[ws * 16 + gid] = m0;
-      sm[ws * 16 + gid + 8] = m1;
-      sl[ws * 16 + gid] = l0t;
-      sl[ws * 16 + gid + 8] = l1t;
-    }
+    // the four lanes of a row hold the same m and l: all store (the same values), so the warp
+    // reaches the barrier with no lane-divergent code in front of it
+    sm[ws * 16 + gid] = m0;
+    sm[ws * 16 + gid + 8] = m1;
+    sl[ws * 16 + gid] = l0t;
+    sl[ws * 16 + gid + 8] = l1t;
     named_barrier_sync(1 + mt, 128);
     float M0 = -INFINITY, M1 = -INFINITY;
 #pragma unroll
@@ -1246,10 +1246,10 @@ __global__ void __launch_bounds__(32 * kF32Warps, 1) decode_fp32_kernel(KArgs a)
   pdl_launch_dependents();
   const int D = a.D;
   for (int iter = 0;; ++iter) {
-    __syncthreads();
+    cta_sync();
     if (threadIdx.x == 0)
       chunk_s = iter == 0 ? (int)blockIdx.x : (int)gridDim.x + atomicAdd(&a.hdr->ticket, 1);
-    __syncthreads();
+    cta_sync();
     const int chunk = chunk_s;
     if (chunk >= plan.n_chunks) break;
     const long long x1 = min((long long)(chunk + 1) * plan.C, plan.K);

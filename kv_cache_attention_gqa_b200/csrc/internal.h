@@ -66,12 +66,14 @@ struct BackwardArgs {
   int causal, window;
   float* lse2;  // workspace: (B*h_q*S_q) base-2 lse
   float* drow;  // workspace: (B*h_q*S_q) rowsum(dO * O)
+  int* ticket;  // workspace: the bf16 kernel's work-item counter (reset by its row-term kernel)
   unsigned* err;
 };
 // bf16 tcgen05 path. tmaps: [0] Q, [1] dO as 3-D views (d_h, S_q, B*h_q) with box (64, 64, 1);
 // [2] K, [3] V as 2-D views (d_h, B*h_kv*T_max) with box (64, 128); [4] Q, [5] dO as 3-D views
 // with the forward's box (64, 128 / H, H); [6] K, [7] V as 2-D views with box (64, 64).
-cudaError_t launch_backward_bf16(const BackwardArgs& a, const CUtensorMap* tmaps, cudaStream_t s);
+cudaError_t launch_backward_bf16(const BackwardArgs& a, const CUtensorMap* tmaps, int num_sms,
+                                 cudaStream_t s);
 cudaError_t launch_backward_fp32(const BackwardArgs& a, cudaStream_t s);
 
 struct DecodeArgs {

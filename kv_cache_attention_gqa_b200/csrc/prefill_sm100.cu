@@ -776,7 +776,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc::tmem_relinquish();
   }
   tc::fence_before_sync();
-  __syncthreads();
+  cta_sync();
   tc::fence_after_sync();
   const uint32_t tmem = *tmem_slot;
   // Whole warpgroups move registers from the control roles to the softmax; each setmaxnreg sits
@@ -887,7 +887,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   tc::fence_before_sync();
-  __syncthreads();
+  cta_sync();
   if (warp == 1) {
     tc::fence_after_sync();
     tc::tmem_dealloc(tmem, kTmemCols);

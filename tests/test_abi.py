@@ -206,7 +206,7 @@ def test_mla_and_backward_host_side_argument_errors(lib):
     assert bwd(ws=null) == 5
     assert bwd(ws=P(0x1010)) == 5  # misaligned
     assert bwd(bytes=8) == 5
-    assert lib.gqa_prefill_backward_workspace_size(1, 4, 8) == 2 * 256
+    assert lib.gqa_prefill_backward_workspace_size(1, 4, 8) == 3 * 256  # lse2, D, item counter
     assert lib.gqa_prefill_backward_workspace_size(0, 4, 8) == 0
 
 

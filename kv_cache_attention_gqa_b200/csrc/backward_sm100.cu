@@ -154,6 +154,40 @@ __global__ void __launch_bounds__(256) rowterm_kernel(const T* o, const T* d_o, 
   }
 }
 
+// The same for bf16 rows of D = 64 or 128 elements with 16-byte aligned bases: D / 8 lanes per
+// row each load 16 bytes of O and of dO, so a warp covers 32 / (D / 8) rows. (One warp per row
+// with 2-byte loads ran at under half the DRAM bandwidth that reading O and dO needs.)
+template <int D>
+__global__ void __launch_bounds__(256) rowterm_vec_kernel(const __nv_bfloat16* o, const __nv_bfloat16* d_o,
+                                                          const float* lse, float* lse2, float* drow,
+                                                          long long rows, int* ticket) {
+  constexpr int kLpr = D / 8;       // lanes per row
+  constexpr int kRpw = 32 / kLpr;   // rows per warp
+  const int lane = threadIdx.x & 31;
+  if (ticket && blockIdx.x == 0 && threadIdx.x == 0) *ticket = 0;  // for the next kernel's items
+  const long long row = (((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5) * kRpw + lane / kLpr;
+  const int sub = lane % kLpr;
+  float s = 0.f;
+  if (row < rows) {
+    const uint4 av = __ldg(reinterpret_cast<const uint4*>(o + row * D) + sub);
+    const uint4 bv = __ldg(reinterpret_cast<const uint4*>(d_o + row * D) + sub);
+    const uint32_t aw[4] = {av.x, av.y, av.z, av.w}, bw_[4] = {bv.x, bv.y, bv.z, bv.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 fa = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&aw[i]));
+      const float2 fb = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&bw_[i]));
+      s = fmaf(fa.x, fb.x, s);
+      s = fmaf(fa.y, fb.y, s);
+    }
+  }
+#pragma unroll
+  for (int off = kLpr / 2; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+  if (sub == 0 && row < rows) {
+    drow[row] = s;
+    const float l = lse[row];
+    lse2[row] = l == -INFINITY || l != l ? INFINITY : l * kLog2e;
+  }
+}
 
 // Descriptors for tiles of any row count: `chunk` is the byte stride between 64-column chunks
 // (rows x 128 B).
@@ -869,9 +903,19 @@ cudaError_t launch_backward_bf16(const BackwardArgs& a, const CUtensorMap* tmaps
                                  cudaStream_t s) {
   const long long rows = (long long)a.B * a.h_q * a.S_q;
   if (rows <= 0) return cudaSuccess;
-  bw::rowterm_kernel<__nv_bfloat16><<<(unsigned)((rows * 32 + 255) / 256), 256, 0, s>>>(
-      reinterpret_cast<const __nv_bfloat16*>(a.o), reinterpret_cast<const __nv_bfloat16*>(a.d_o), a.lse,
-      a.lse2, a.drow, rows, a.d_h, a.ticket);
+  const auto* ob = reinterpret_cast<const __nv_bfloat16*>(a.o);
+  const auto* dob = reinterpret_cast<const __nv_bfloat16*>(a.d_o);
+  const bool vec = ((reinterpret_cast<uintptr_t>(a.o) | reinterpret_cast<uintptr_t>(a.d_o)) & 15u) == 0;
+  if (vec && a.d_h == 128) {  // 2 rows per warp, 16 per block
+    bw::rowterm_vec_kernel<128><<<(unsigned)((rows + 15) / 16), 256, 0, s>>>(ob, dob, a.lse, a.lse2, a.drow,
+                                                                             rows, a.ticket);
+  } else if (vec && a.d_h == 64) {  // 4 rows per warp, 32 per block
+    bw::rowterm_vec_kernel<64><<<(unsigned)((rows + 31) / 32), 256, 0, s>>>(ob, dob, a.lse, a.lse2, a.drow,
+                                                                            rows, a.ticket);
+  } else {
+    bw::rowterm_kernel<__nv_bfloat16><<<(unsigned)((rows * 32 + 255) / 256), 256, 0, s>>>(
+        ob, dob, a.lse, a.lse2, a.drow, rows, a.d_h, a.ticket);
+  }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   bw::BArgs p;

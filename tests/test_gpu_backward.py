@@ -110,3 +110,30 @@ def test_backward_prefill_4k_full_size():
     assert_grad_close(_f64(dq), rq, "prefill_4k dQ")
     assert_grad_close(_f64(dk), rk, "prefill_4k dK")
     assert_grad_close(_f64(dv), rv, "prefill_4k dV")
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_backward_bf16_unaligned_o(d):
+    """O at an address 2 bytes past a 16-byte boundary (O is read by the row term only; dO goes
+    through TMA and must be 16-byte aligned): the row term then takes its element-by-element path
+    (another summation order for D); both results match the oracle."""
+    import kv_cache_attention_gqa_b200 as gqa
+
+    g = torch.Generator().manual_seed(31 + d)
+    B, h_q, h_kv, S, T = 2, 8, 2, 200, 200
+    q = (torch.randn(B, h_q, S, d, generator=g) * 0.5).to(torch.bfloat16).cuda()
+    k = (torch.randn(B, h_kv, T, d, generator=g) * 0.5).to(torch.bfloat16).cuda()
+    v = torch.randn(B, h_kv, T, d, generator=g).to(torch.bfloat16).cuda()
+    d_o = torch.randn(B, h_q, S, d, generator=g).to(torch.bfloat16).cuda()
+    o, lse = gqa.prefill(q, k, v, return_lse=True)
+    ob = torch.empty(o.numel() + 1, dtype=torch.bfloat16, device="cuda")
+    o_u = ob[1:].view(o.shape)
+    o_u.copy_(o)
+    assert o_u.data_ptr() % 16 == 2
+    rq, rk, rv = oracle.attention_backward_ref(_f64(q), _f64(k), _f64(v), _f64(d_o))
+    for oo, what in ((o, "aligned"), (o_u, "unaligned")):
+        dq, dk, dv = gqa.prefill_backward(q, k, v, oo, d_o, lse)
+        assert gqa.get_device_error() == 0
+        assert_grad_close(_f64(dq), rq, f"dQ {what} d={d}", False)
+        assert_grad_close(_f64(dk), rk, f"dK {what} d={d}", False)
+        assert_grad_close(_f64(dv), rv, f"dV {what} d={d}", False)

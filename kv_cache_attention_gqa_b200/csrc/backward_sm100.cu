@@ -13,7 +13,9 @@
 // items from a ticket counter that rowterm resets, so an SM that finishes early takes the next
 // item, as the hardware's CTA scheduler would, without a CTA exit and launch per item (measured:
 // the 512-column TMEM release of an exiting CTA took 3.5-5 us after these kernels' epilogues).
-// Each item initialises its barriers and invalidates them at its end.
+// Each dkdv item initialises its barriers and invalidates them at its end; once a CTA draws a dq
+// tile, every later ticket is a dq tile too, and it runs them as one pipelined sequence (the next
+// tile's loads and first scores overlap the current tile's dQ write-out).
 //   rowterm   one warp per query row: D = rowsum(dO * O) and the base-2 lse (fp32 workspace).
 //   dkdv      one CTA per (sequence, KV head, 128-key block). The keys sit on the 128 TMEM lanes;
 //             the CTA walks every 64-row query block of every head of the group, so the r heads'
@@ -68,6 +70,7 @@ struct BArgs {
   int n_kb;                 // key blocks per (b, g): ceil(T_max / 128)
   float scale, sl2;         // scale and scale * log2(e)
   int causal, window;
+  FastDiv div_per, div_gh, div_hb;  // by B*h_kv*hblocks, h_kv*hblocks, hblocks (dq tile numbers)
   int n_items;              // dkdv tiles + dq tiles
   int* ticket;              // items handed out past the first gridDim.x (reset by rowterm)
   unsigned* err;
@@ -256,8 +259,8 @@ __device__ __forceinline__ void dkdv_cta(const CUtensorMap& tmq, const CUtensorM
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kKvBars);
-  volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  // the abort flag sits after the barriers (the TMEM address is the kernel's, held across items)
+  volatile int* abort = reinterpret_cast<volatile int*>(bars + kKvBars) + 1;
   float* stat = reinterpret_cast<float*>(smem + C::kOffStat);  // [stage][lse2 64 | D 64]
   const uint32_t sK = smem_u32(smem + C::kOffK), sV = smem_u32(smem + C::kOffV);
   auto sQ = [&](int st) { return smem_u32(smem + C::kOffQ + st * 2 * C::kQTile); };
@@ -307,7 +310,6 @@ __device__ __forceinline__ void dkdv_cta(const CUtensorMap& tmq, const CUtensorM
     if (!valid && kb == 0 && g == 0)
       set_device_error(a.err, kv < 1 || kv > a.T_max ? GQA_DEVERR_KV_LEN : GQA_DEVERR_POSITION);
   }
-  (void)tmem_slot;
   tc::fence_before_sync();
   cta_sync();
   tc::fence_after_sync();
@@ -549,64 +551,87 @@ struct QCfg {
   static_assert(kSmem <= 227 * 1024, "shared memory budget");
 };
 enum {
-  kQdQ = 0,
+  kQdQ = 0,                            // Q / dO of a tile in shared memory (or the end)
   kQT = 1,                             // Q, dO copied into TMEM (256 arrivals)
   kQKvFull = 2,                        // + stage
   kQKvEmpty = kQKvFull + kQStages,     // + stage
   kQS = kQKvEmpty + kQStages,          // + buffer
   kQP = kQS + 2,                       // + buffer (256 arrivals)
-  kQDone = kQP + 2,
-  kQBars = kQDone + 1
+  kQDone = kQP + 2,                    // a tile's dQ MMAs complete
+  kQdQEmpty = kQDone + 1,              // Q / dO copied into TMEM and the tile number read (257)
+  kQAll = kQdQEmpty + 1,               // every MMA of the run complete
+  kQBars = kQAll + 1
 };
 
-// One CTA of the dQ pass for forward tile `tile`.
+// One dQ tile (as in the forward): H heads x P positions of one group, and the 64-key blocks
+// j0 .. j0 + nb - 1 its rows see.
+struct DqTile {
+  int b, g, hb, q0, nh, kv, qs, j0, nb;
+  long long pos_min, pos_max;
+};
+
+__device__ __forceinline__ DqTile dq_tile(const BArgs& a, int tile) {
+  DqTile t;
+  const int per = a.B * a.h_kv * a.hblocks;
+  const int qd = a.div_per.div(tile);
+  const int qt = a.n_qt - 1 - qd;  // heaviest (latest positions) first
+  const int rem = tile - qd * per;
+  t.b = a.div_gh.div(rem);
+  const int gh = rem - t.b * (a.h_kv * a.hblocks);
+  t.g = a.div_hb.div(gh);
+  t.hb = gh - t.g * a.hblocks;
+  t.q0 = qt * a.P;
+  t.nh = min(a.H, a.r - t.hb * a.H);
+  t.kv = a.kv_len ? a.kv_len[t.b] : a.T_max;
+  t.qs = a.q_start ? a.q_start[t.b] : 0;
+  const bool valid = t.kv >= 1 && t.kv <= a.T_max && t.qs >= 0;
+  t.pos_min = (long long)t.qs + t.q0;
+  t.pos_max = (long long)t.qs + min(t.q0 + a.P, a.S_q) - 1;
+  t.j0 = 0;
+  t.nb = 0;
+  if (valid) {
+    int end = (t.kv + kQBK - 1) / kQBK;
+    if (a.causal) {
+      const long long last_key = t.pos_max < t.kv - 1 ? t.pos_max : (long long)(t.kv - 1);
+      end = (int)(last_key / kQBK) + 1;
+      if (a.window > 0) {
+        const long long lo = t.pos_min - a.window + 1;
+        if (lo > 0) t.j0 = (int)(lo / kQBK);
+      }
+    }
+    t.nb = end > t.j0 ? end - t.j0 : 0;
+  }
+  return t;
+}
+
+// The dQ pass from item `item0` on: every item after the first dQ tile is a dQ tile, so the CTA
+// takes them all here from the work counter, with its pipelines running on from one tile into the
+// next. The producer loads a tile's Q and dO rows as soon as the elementwise warps have copied the
+// previous tile's into TMEM (that copy follows the previous tile's last S / dP, the MMAs that read
+// them), and its K/V blocks through the ring; the MMA warp issues the new tile's first S and dP
+// while the elementwise warps write out the previous tile's dQ; the new tile's first dQ += dS K,
+// which overwrites the accumulator, waits for dS that those warps produce after reading it out.
+// The producer hands each tile's number to the other roles through `s_items` (two slots), and a
+// number past the last item ends the run.
 template <int D>
-__device__ __forceinline__ void dq_cta(const CUtensorMap& tmq, const CUtensorMap& tmdo,
+__device__ __forceinline__ void dq_run(const CUtensorMap& tmq, const CUtensorMap& tmdo,
                                        const CUtensorMap& tmk, const CUtensorMap& tmv, const BArgs& a,
-                                       int tile, uint32_t tmem) {
+                                       int item0, int n_dkdv, uint32_t tmem, volatile int* s_items) {
   using C = QCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kQBars);
-  volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* abort = reinterpret_cast<volatile int*>(bars + kQBars) + 1;  // after the barriers
   const uint32_t sQ = smem_u32(smem + C::kOffQ), sDO = smem_u32(smem + C::kOffDO);
   auto sK = [&](int st) { return smem_u32(smem + C::kOffK + st * 2 * C::kKTile); };
   auto sV = [&](int st) { return smem_u32(smem + C::kOffK + st * 2 * C::kKTile + C::kKTile); };
   auto bar = [&](int i) { return smem_u32(&bars[i]); };
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // ---- the tile (as in the forward): H heads x P positions of one group, heaviest first
-  const int per = a.B * a.h_kv * a.hblocks;
-  const int qt = a.n_qt - 1 - tile / per;
-  const int rem = tile - (tile / per) * per;
-  const int b = rem / (a.h_kv * a.hblocks);
-  const int gh = rem - b * (a.h_kv * a.hblocks);
-  const int g = gh / a.hblocks, hb = gh - g * a.hblocks;
-  const int q0 = qt * a.P;
-  const int nh = min(a.H, a.r - hb * a.H);
-  const int kv = a.kv_len ? a.kv_len[b] : a.T_max;
-  const int qs = a.q_start ? a.q_start[b] : 0;
-  const bool valid = kv >= 1 && kv <= a.T_max && qs >= 0;
-  const long long pos_min = (long long)qs + q0;
-  const long long pos_max = (long long)qs + min(q0 + a.P, a.S_q) - 1;
-  int j0 = 0, nb = 0;  // 64-key blocks j0 .. j0 + nb - 1
-  if (valid) {
-    int end = (kv + kQBK - 1) / kQBK;
-    if (a.causal) {
-      const long long last_key = pos_max < kv - 1 ? pos_max : (long long)(kv - 1);
-      end = (int)(last_key / kQBK) + 1;
-      if (a.window > 0) {
-        const long long lo = pos_min - a.window + 1;
-        if (lo > 0) j0 = (int)(lo / kQBK);
-      }
-    }
-    nb = end > j0 ? end - j0 : 0;
-  }
-
   if (threadIdx.x == 0) {
     mbar_init(bar(kQdQ), 1);
+    mbar_init(bar(kQdQEmpty), 256 + 1);  // the elementwise threads and the MMA warp's lane
     mbar_init(bar(kQT), 256);
     for (int st = 0; st < kQStages; ++st) {
       mbar_init(bar(kQKvFull + st), 1);
@@ -617,54 +642,76 @@ __device__ __forceinline__ void dq_cta(const CUtensorMap& tmq, const CUtensorMap
       mbar_init(bar(kQP + bf), 256);
     }
     mbar_init(bar(kQDone), 1);
+    mbar_init(bar(kQAll), 1);
     *abort = 0;
     fence_barrier_init();
   }
-  (void)tmem_slot;
   tc::fence_before_sync();
   cta_sync();
   tc::fence_after_sync();
-  const int row0 = (b * a.h_kv + g) * a.T_max;
 
-  if (warp == 0 && lane == 0 && nb > 0) {
+  // the tile number of the run's n-th item, or -1 at the end (after its Q/dO barrier phase n)
+  auto item_at = [&](int n) { return s_items[n & 1]; };
+
+  if (warp == 0 && lane == 0) {
     // ------------------------------ TMA producer ------------------------------------------
     tma_prefetch_desc(&tmq);
     tma_prefetch_desc(&tmdo);
     tma_prefetch_desc(&tmk);
     tma_prefetch_desc(&tmv);
-    const int zq = b * a.h_q + g * a.r + hb * a.H;
-    mbar_arrive_expect_tx(bar(kQdQ), (uint32_t)(2 * C::kNch * a.H * a.P * 128));
-    for (int ch = 0; ch < C::kNch; ++ch) {
-      tma_load_3d(sQ + ch * 128 * 128, &tmq, bar(kQdQ), ch * 64, q0, zq);
-      tma_load_3d(sDO + ch * 128 * 128, &tmdo, bar(kQdQ), ch * 64, q0, zq);
-    }
-    int last[kQStages];
-    for (int st = 0; st < kQStages; ++st) last[st] = -1;
-    for (int j = 0; j < nb; ++j) {
-      const int st = j % kQStages, n = j / kQStages;
-      if (n > 0 && !wait_bar(bar(kQKvEmpty + st), (uint32_t)((n - 1) & 1), abort, a.err)) break;
-      mbar_arrive_expect_tx(bar(kQKvFull + st), 2 * C::kKTile);
-      for (int ch = 0; ch < C::kNch; ++ch) {
-        tma_load_2d(sK(st) + ch * C::kKChunk, &tmk, bar(kQKvFull + st), ch * 64, row0 + (j0 + j) * kQBK);
-        tma_load_2d(sV(st) + ch * C::kKChunk, &tmv, bar(kQKvFull + st), ch * 64, row0 + (j0 + j) * kQBK);
+    int item = item0, n = 0, J = 0, nk = 0;  // J: K/V blocks loaded (nk: issued, for the drain)
+    bool ok = true;
+    while (ok) {
+      // the slot of item n held item n - 2; item n - 1's Q/dO rows are in TMEM and its number
+      // has been read
+      if (n > 0 && !(ok = wait_bar(bar(kQdQEmpty), (uint32_t)((n - 1) & 1), abort, a.err))) break;
+      if (item >= a.n_items) {
+        s_items[n & 1] = -1;
+        mbar_arrive(bar(kQdQ));  // completes phase n with no bytes: the end
+        break;
       }
-      last[st] = n;
+      const int tile = item - n_dkdv;
+      const DqTile t = dq_tile(a, tile);
+      s_items[n & 1] = tile;
+      const int next = (int)gridDim.x + atomicAdd(a.ticket, 1);  // the next item, fetched early
+      const int zq = t.b * a.h_q + t.g * a.r + t.hb * a.H;
+      mbar_arrive_expect_tx(bar(kQdQ), (uint32_t)(2 * C::kNch * a.H * a.P * 128));
+      for (int ch = 0; ch < C::kNch; ++ch) {
+        tma_load_3d(sQ + ch * 128 * 128, &tmq, bar(kQdQ), ch * 64, t.q0, zq);
+        tma_load_3d(sDO + ch * 128 * 128, &tmdo, bar(kQdQ), ch * 64, t.q0, zq);
+      }
+      const int row0 = (t.b * a.h_kv + t.g) * a.T_max;
+      for (int j = 0; j < t.nb && ok; ++j) {
+        const int jg = J + j, st = jg % kQStages, f = jg / kQStages;
+        if (f > 0 && !(ok = wait_bar(bar(kQKvEmpty + st), (uint32_t)((f - 1) & 1), abort, a.err))) break;
+        mbar_arrive_expect_tx(bar(kQKvFull + st), 2 * C::kKTile);
+        for (int ch = 0; ch < C::kNch; ++ch) {
+          tma_load_2d(sK(st) + ch * C::kKChunk, &tmk, bar(kQKvFull + st), ch * 64, row0 + (t.j0 + j) * kQBK);
+          tma_load_2d(sV(st) + ch * C::kKChunk, &tmv, bar(kQKvFull + st), ch * 64, row0 + (t.j0 + j) * kQBK);
+        }
+        ++nk;
+      }
+      J += t.nb;
+      ++n;
+      item = next;
     }
-    volatile int no_abort = 0;  // drain (bounded)
-    wait_bar(bar(kQdQ), 0, &no_abort, a.err);
-    for (int st = 0; st < kQStages; ++st)
-      if (last[st] >= 0) wait_bar(bar(kQKvFull + st), (uint32_t)(last[st] & 1), &no_abort, a.err);
-  } else if (warp == 1 && nb > 0) {
+    // Drain (bounded): no copy may still land in shared memory when the run ends. The Q/dO rows
+    // of every item were copied into TMEM before the end (or the run gave up); the K/V fills:
+    volatile int no_abort = 0;
+    if (!ok && n > 0) wait_bar(bar(kQdQ), (uint32_t)((n - 1) & 1), &no_abort, a.err);
+#pragma unroll
+    for (int s = 0; s < kQStages; ++s)
+      if (nk > s) wait_bar(bar(kQKvFull + s), (uint32_t)(((nk - 1 - s) / kQStages) & 1), &no_abort, a.err);
+  } else if (warp == 1) {
     // ------------------------------ MMA issuer ---------------------------------------------
-    // whole warp, one elected lane per batch of MMAs and its commit (as in the dK / dV pass)
     constexpr uint32_t idesc_s = tc::idesc_bf16(128, kQBK, false);  // S, dP: M rows, N keys
     constexpr uint32_t idesc_acc = tc::idesc_bf16(128, D, true);    // dQ: M rows, N = d_h
     constexpr uint32_t kColQ = kColAcc0 + D, kColDO = kColAcc0 + D + D / 2;
     auto wait = [&](int b_, uint32_t parity) {
       return __all_sync(0xffffffffu, wait_bar(bar(b_), parity, abort, a.err));
     };
-    auto issue_s = [&](int j) {
-      const int st = j % kQStages, bf = j & 1;
+    auto issue_s = [&](int jg) {  // the run's block jg: K/V stage jg % 3 into score buffer jg & 1
+      const int st = jg % kQStages, bf = jg & 1;
       const uint64_t dk = tc::smem_desc(sK(st), 16, 1024), dv = tc::smem_desc(sV(st), 16, 1024);
       if (elect_one()) {
 #pragma unroll
@@ -677,34 +724,55 @@ __device__ __forceinline__ void dq_cta(const CUtensorMap& tmq, const CUtensorMap
       }
       __syncwarp();
     };
-    bool ok = wait(kQT, 0) && wait(kQKvFull, 0);
-    if (ok) {
-      tc::fence_after_sync();
-      issue_s(0);
-    }
-    for (int j = 0; j < nb && ok; ++j) {
-      const int st = j % kQStages, bf = j & 1;
-      if (j + 1 < nb) {
-        if (!(ok = wait(kQKvFull + (j + 1) % kQStages, (uint32_t)(((j + 1) / kQStages) & 1)))) break;
-        tc::fence_after_sync();
-        issue_s(j + 1);
-      }
-      if (!(ok = wait(kQP + bf, (uint32_t)((j >> 1) & 1)))) break;
-      tc::fence_after_sync();
-      const uint64_t dk_mn = tc::smem_desc(sK(st), C::kKChunk, 1024);
-      if (elect_one()) {
-#pragma unroll
-        for (int kk = 0; kk < kQBK / 16; ++kk)
-          tc::mma_ts(tmem + kColAcc0, tmem + (uint32_t)(64 * bf + (kk >> 1) * 32 + (kk & 1) * 8),
-                     dk_mn + mnoff(kk), idesc_acc, (j > 0 || kk > 0) ? 1u : 0u);
-        tc::commit(bar(kQKvEmpty + st));
-      }
+    int n = 0, J = 0;  // items, K/V blocks (= score blocks) so far
+    bool ok = true;
+    while (ok) {
+      if (!(ok = wait(kQdQ, (uint32_t)(n & 1)))) break;
+      const int tile = item_at(n);
+      if (tile < 0) break;
+      const DqTile t = dq_tile(a, tile);
+      // this tile's Q and dO in TMEM; only then is the release below allowed: it lets the
+      // elementwise warps reach the next tile's copy, and this warp must not be two phases of
+      // kQT behind when they do
+      if (!(ok = wait(kQT, (uint32_t)(n & 1)))) break;
+      if (elect_one()) mbar_arrive(bar(kQdQEmpty));
       __syncwarp();
+      if (t.nb > 0) {
+        if (!(ok = wait(kQKvFull + J % kQStages, (uint32_t)((J / kQStages) & 1)))) break;
+        tc::fence_after_sync();
+        issue_s(J);
+        for (int j = 0; j < t.nb && ok; ++j) {
+          const int jg = J + j, st = jg % kQStages, bf = jg & 1;
+          if (j + 1 < t.nb) {
+            const int jn = jg + 1;
+            if (!(ok = wait(kQKvFull + jn % kQStages, (uint32_t)((jn / kQStages) & 1)))) break;
+            tc::fence_after_sync();
+            issue_s(jn);
+          }
+          if (!(ok = wait(kQP + bf, (uint32_t)((jg >> 1) & 1)))) break;
+          tc::fence_after_sync();
+          const uint64_t dk_mn = tc::smem_desc(sK(st), C::kKChunk, 1024);
+          if (elect_one()) {
+#pragma unroll
+            for (int kk = 0; kk < kQBK / 16; ++kk)
+              tc::mma_ts(tmem + kColAcc0, tmem + (uint32_t)(64 * bf + (kk >> 1) * 32 + (kk & 1) * 8),
+                         dk_mn + mnoff(kk), idesc_acc, (j > 0 || kk > 0) ? 1u : 0u);
+            tc::commit(bar(kQKvEmpty + st));
+          }
+          __syncwarp();
+        }
+        if (!ok) break;
+        if (elect_one()) tc::commit(bar(kQDone));  // this tile's dQ is complete
+        __syncwarp();
+      }
+      J += t.nb;
+      ++n;
     }
-    if (elect_one()) tc::commit(bar(kQDone));
+    // every MMA issued above has completed before the run ends
+    if (elect_one()) tc::commit(bar(kQAll));
     __syncwarp();
     volatile int no_abort = 0;
-    wait_bar(bar(kQDone), 0, &no_abort, a.err);
+    wait_bar(bar(kQAll), 0, &no_abort, a.err);
   } else if (warp >= 2) {
     // ------------------------------ elementwise: one query row, 32 keys per thread ----------
     const int quarter = warp & 3;
@@ -713,116 +781,150 @@ __device__ __forceinline__ void dq_cta(const CUtensorMap& tmq, const CUtensorMap
     const int row = quarter * 32 + lane;  // TMEM lane = tile row (head h, position p)
     const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
     const int h = row / a.P, p = row - h * a.P;
-    const int qi = q0 + p;
-    const bool store_row = h < nh && row < a.H * a.P && qi < a.S_q;
-    const int head = g * a.r + hb * a.H + h;
-    const long long srow = ((long long)b * a.h_q + head) * a.S_q + qi;
-    const long long pos = (long long)qs + qi;
-    const float lse2 = store_row ? a.lse2[srow] : INFINITY;
-    const float dr = store_row ? a.drow[srow] : 0.f;
-    // keys [k_first, k_last] this row sees (length, causal and window limits as 32-bit bounds)
-    const long long kl = a.causal && pos < kv - 1 ? pos : (long long)kv - 1;
-    const int k_last = (int)kl;
-    const long long kf = a.window > 0 ? pos - a.window + 1 : 0;
-    const int k_first = kf < 0 ? 0 : (kf > 0x7fffffffLL ? 0x7fffffff : (int)kf);
-    // this row of Q (half 0) or dO (half 1): shared memory (128-byte swizzled) -> TMEM
-    bool ok = nb > 0 && wait_bar(bar(kQdQ), 0, abort, a.err);
-    ok = __all_sync(0xffffffffu, ok);
-    if (ok) {
-      const uint32_t src = half == 0 ? sQ : sDO;
-      const uint32_t dst = lane_addr + kColAcc0 + D + half * (D / 2);
-#pragma unroll
-      for (int ch = 0; ch < C::kNch; ++ch) {
-        uint32_t r[32];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const uint32_t addr = swz128(src + ch * 128 * 128, row, k);
-          asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                       : "=r"(r[4 * k]), "=r"(r[4 * k + 1]), "=r"(r[4 * k + 2]), "=r"(r[4 * k + 3])
-                       : "r"(addr));
-        }
-        tc::st32(dst + ch * 32, r);
-      }
-      tc::wait_st();
-    }
-    tc::fence_before_sync();
-    if (nb > 0) mbar_arrive(bar(kQT));
-    for (int j = 0; j < nb; ++j) {
-      const int st = j % kQStages, bf = j & 1;
-      if (ok) ok = wait_bar(bar(kQS + bf), (uint32_t)((j >> 1) & 1), abort, a.err);
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) break;
-      const int blk0 = (j0 + j) * kQBK;
-      const int key0 = blk0 + half * 32;  // first key of this half
-      const bool need_mask = (a.causal && (long long)key0 + 31 > pos_min) || key0 + 32 > kv ||
-                             (a.window > 0 && (long long)key0 <= pos_max - a.window);
-      tc::fence_after_sync();
-      uint32_t sv[32], dv[32];
-      tc::ld32(lane_addr + 64 * bf + 32 * half, sv);
-      tc::ld32(lane_addr + 128 + 64 * bf + 32 * half, dv);
-      tc::wait_ld();
-      uint32_t pd[16];
-      const float2 c2 = make_float2(a.sl2, a.sl2), nl = make_float2(-lse2, -lse2), nd = make_float2(-dr, -dr);
-#pragma unroll
-      for (int x = 0; x < 32; x += 2) {
-        const float2 arg = fma2(make_float2(__uint_as_float(sv[x]), __uint_as_float(sv[x + 1])), c2, nl);
-        const float2 pr = make_float2(fast_exp2(arg.x), fast_exp2(arg.y));
-        float2 ds = mul2(pr, add2(make_float2(__uint_as_float(dv[x]), __uint_as_float(dv[x + 1])), nd));
-        if (need_mask) {
-          if (key0 + x < k_first || key0 + x > k_last) ds.x = 0.f;
-          if (key0 + x + 1 < k_first || key0 + x + 1 > k_last) ds.y = 0.f;
-        }
-        pd[x / 2] = pack_bf16x2(ds.x, ds.y);
-      }
-      tc::st16(lane_addr + 64 * bf + 32 * half, pd);  // dS over this half's first columns of S
-      // K rows no row of the tile may see (past kv_len: last block; below every row's window:
-      // first block) get dS = 0 but may hold anything: zero them before dQ += dS K
-      const bool zero_tail = j == nb - 1 && blk0 + kQBK > kv;
-      const bool zero_head = j == 0 && a.window > 0 && (long long)blk0 < pos_min - a.window + 1;
-      if ((zero_tail || zero_head) && et < kQBK) {
-        const long long key = (long long)blk0 + et;  // this thread's K row of the block
-        if ((zero_tail && key >= kv) || (zero_head && key <= pos_min - a.window)) {
-          for (int ch = 0; ch < C::kNch; ++ch)
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-              const uint32_t addr = sK(st) + ch * C::kKChunk + et * 128 + k * 16;
-              asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(addr), "r"(0u) : "memory");
-            }
-        }
-        tc::fence_proxy_async_smem();
-      }
-      tc::wait_st();
-      tc::fence_before_sync();
-      mbar_arrive(bar(kQP + bf));
-    }
-    // ---- epilogue: scale * dQ -> bf16; each half writes half of the columns
-    bool have = nb > 0 && ok;
-    if (have) {
-      have = wait_bar(bar(kQDone), 0, abort, a.err);
-      have = __all_sync(0xffffffffu, have);
-      if (have) tc::fence_after_sync();
-    }
-    uint4* out = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.dq) + srow * D);
-    if (have) {
+    // dQ of the previous tile -> bf16 rows (or zeros when it had no block or gave up)
+    auto epilogue = [&](bool have, long long srow, bool store_row) {
+      uint4* out = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.dq) + srow * D);
+      if (have) {
 #pragma unroll 1
-      for (int c = half * (D / 64); c < (half + 1) * (D / 64); ++c) {
-        uint32_t v[32];
-        tc::ld32(lane_addr + kColAcc0 + c * 32, v);
-        tc::wait_ld();
-        uint32_t pk[16];
+        for (int c = half * (D / 64); c < (half + 1) * (D / 64); ++c) {
+          uint32_t v[32];
+          tc::ld32(lane_addr + kColAcc0 + c * 32, v);
+          tc::wait_ld();
+          uint32_t pk[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
-          pk[i] = pack_bf16x2(__uint_as_float(v[2 * i]) * a.scale, __uint_as_float(v[2 * i + 1]) * a.scale);
-        if (store_row) {
+          for (int i = 0; i < 16; ++i)
+            pk[i] = pack_bf16x2(__uint_as_float(v[2 * i]) * a.scale, __uint_as_float(v[2 * i + 1]) * a.scale);
+          if (store_row) {
 #pragma unroll
-          for (int q = 0; q < 4; ++q) out[c * 4 + q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+            for (int q = 0; q < 4; ++q) out[c * 4 + q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+          }
         }
+      } else if (store_row) {
+        for (int v = half * (D / 16); v < (half + 1) * (D / 16); ++v) out[v] = make_uint4(0u, 0u, 0u, 0u);
       }
-    } else if (store_row) {
-      for (int v = half * (D / 16); v < (half + 1) * (D / 16); ++v) out[v] = make_uint4(0u, 0u, 0u, 0u);
+    };
+    int n = 0, J = 0, nd = 0;  // items, K/V blocks, items whose dQ the MMA warp completed
+    bool ok = true;
+    bool prev = false, prev_blocks = false, prev_store = false;  // the previous tile's epilogue
+    long long prev_srow = 0;
+    while (true) {
+      if (ok) ok = wait_bar(bar(kQdQ), (uint32_t)(n & 1), abort, a.err);
+      ok = __all_sync(0xffffffffu, ok);
+      const int tile = ok ? item_at(n) : -1;
+      if (tile < 0) break;
+      const DqTile t = dq_tile(a, tile);
+      const int qi = t.q0 + p;
+      const bool store_row = h < t.nh && row < a.H * a.P && qi < a.S_q;
+      const long long srow = ((long long)t.b * a.h_q + t.g * a.r + t.hb * a.H + h) * a.S_q + qi;
+      const long long pos = (long long)t.qs + qi;
+      const float lse2 = store_row ? a.lse2[srow] : INFINITY;
+      const float dr = store_row ? a.drow[srow] : 0.f;
+      // keys [k_first, k_last] this row sees (length, causal and window limits as 32-bit bounds)
+      const long long kl = a.causal && pos < t.kv - 1 ? pos : (long long)t.kv - 1;
+      const int k_last = (int)kl;
+      const long long kf = a.window > 0 ? pos - a.window + 1 : 0;
+      const int k_first = kf < 0 ? 0 : (kf > 0x7fffffffLL ? 0x7fffffff : (int)kf);
+      // this row of Q (half 0) or dO (half 1): shared memory (128-byte swizzled) -> TMEM. The
+      // previous tile's S and dP MMAs, which read these columns, are complete (this warp saw the
+      // scores of its last block).
+      {
+        const uint32_t src = half == 0 ? sQ : sDO;
+        const uint32_t dst = lane_addr + kColAcc0 + D + half * (D / 2);
+#pragma unroll
+        for (int ch = 0; ch < C::kNch; ++ch) {
+          uint32_t r[32];
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const uint32_t addr = swz128(src + ch * 128 * 128, row, k);
+            asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(r[4 * k]), "=r"(r[4 * k + 1]), "=r"(r[4 * k + 2]), "=r"(r[4 * k + 3])
+                         : "r"(addr));
+          }
+          tc::st32(dst + ch * 32, r);
+        }
+        tc::wait_st();
+      }
+      tc::fence_before_sync();
+      mbar_arrive(bar(kQT));
+      mbar_arrive(bar(kQdQEmpty));
+      // the previous tile's dQ (the MMA warp can start this tile's scores meanwhile)
+      if (prev) {
+        bool have = prev_blocks && ok;
+        if (have) {
+          have = wait_bar(bar(kQDone), (uint32_t)((nd - 1) & 1), abort, a.err);
+          have = __all_sync(0xffffffffu, have);
+          if (have) tc::fence_after_sync();
+          else ok = false;
+        }
+        epilogue(have, prev_srow, prev_store);
+      }
+      for (int j = 0; j < t.nb; ++j) {
+        const int jg = J + j, st = jg % kQStages, bf = jg & 1;
+        if (ok) ok = wait_bar(bar(kQS + bf), (uint32_t)((jg >> 1) & 1), abort, a.err);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        const int blk0 = (t.j0 + j) * kQBK;
+        const int key0 = blk0 + half * 32;  // first key of this half
+        const bool need_mask = (a.causal && (long long)key0 + 31 > t.pos_min) || key0 + 32 > t.kv ||
+                               (a.window > 0 && (long long)key0 <= t.pos_max - a.window);
+        tc::fence_after_sync();
+        uint32_t sv[32], dv[32];
+        tc::ld32(lane_addr + 64 * bf + 32 * half, sv);
+        tc::ld32(lane_addr + 128 + 64 * bf + 32 * half, dv);
+        tc::wait_ld();
+        uint32_t pd[16];
+        const float2 c2 = make_float2(a.sl2, a.sl2), nl = make_float2(-lse2, -lse2), nd2 = make_float2(-dr, -dr);
+#pragma unroll
+        for (int x = 0; x < 32; x += 2) {
+          const float2 arg = fma2(make_float2(__uint_as_float(sv[x]), __uint_as_float(sv[x + 1])), c2, nl);
+          const float2 pr = make_float2(fast_exp2(arg.x), fast_exp2(arg.y));
+          float2 ds = mul2(pr, add2(make_float2(__uint_as_float(dv[x]), __uint_as_float(dv[x + 1])), nd2));
+          if (need_mask) {
+            if (key0 + x < k_first || key0 + x > k_last) ds.x = 0.f;
+            if (key0 + x + 1 < k_first || key0 + x + 1 > k_last) ds.y = 0.f;
+          }
+          pd[x / 2] = pack_bf16x2(ds.x, ds.y);
+        }
+        tc::st16(lane_addr + 64 * bf + 32 * half, pd);  // dS over this half's first columns of S
+        // K rows no row of the tile may see (past kv_len: last block; below every row's window:
+        // first block) get dS = 0 but may hold anything: zero them before dQ += dS K
+        const bool zero_tail = j == t.nb - 1 && blk0 + kQBK > t.kv;
+        const bool zero_head = j == 0 && a.window > 0 && (long long)blk0 < t.pos_min - a.window + 1;
+        if ((zero_tail || zero_head) && et < kQBK) {
+          const long long key = (long long)blk0 + et;  // this thread's K row of the block
+          if ((zero_tail && key >= t.kv) || (zero_head && key <= t.pos_min - a.window)) {
+            for (int ch = 0; ch < C::kNch; ++ch)
+#pragma unroll
+              for (int k = 0; k < 8; ++k) {
+                const uint32_t addr = sK(st) + ch * C::kKChunk + et * 128 + k * 16;
+                asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(addr), "r"(0u) : "memory");
+              }
+          }
+          tc::fence_proxy_async_smem();
+        }
+        tc::wait_st();
+        tc::fence_before_sync();
+        mbar_arrive(bar(kQP + bf));
+      }
+      prev = true;
+      prev_blocks = t.nb > 0;
+      prev_store = store_row;
+      prev_srow = srow;
+      if (t.nb > 0) ++nd;
+      J += t.nb;
+      ++n;
+    }
+    if (prev) {  // the last tile's dQ
+      bool have = prev_blocks && ok;
+      if (have) {
+        have = wait_bar(bar(kQDone), (uint32_t)((nd - 1) & 1), abort, a.err);
+        have = __all_sync(0xffffffffu, have);
+        if (have) tc::fence_after_sync();
+      }
+      epilogue(have, prev_srow, prev_store);
     }
   }
-  // every role is done with the item (copies landed, MMAs complete, TMEM read): its barriers go
+  // every role is done (copies landed, MMAs complete, TMEM read): the barriers go
   tc::fence_before_sync();
   cta_sync();
   if (threadIdx.x == 0)
@@ -848,6 +950,7 @@ __global__ void __launch_bounds__(kKvThreads, 1)
                     BArgs a, int n_dkdv) {
   __shared__ uint32_t s_tmem;
   __shared__ int s_next;
+  __shared__ int s_items[2];
   const int warp = threadIdx.x >> 5;
   if (warp == 1) {  // all 512 columns, held across the CTA's items
     tc::tmem_alloc(smem_u32(&s_tmem), kTmemCols);
@@ -858,11 +961,14 @@ __global__ void __launch_bounds__(kKvThreads, 1)
   tc::fence_after_sync();
   const uint32_t tmem = s_tmem;
   for (int item = blockIdx.x; item < a.n_items;) {
+    if (item >= n_dkdv) {  // tickets only grow: every later item of this CTA is a dq tile too
+      dq_run<D>(tmq_tile, tmdo_tile, tmk64, tmv64, a, item, n_dkdv, tmem, s_items);
+      break;
+    }
     // the next item's ticket, fetched while this item runs by a thread of the elementwise warps
     // (which wait for the first scores anyway); the item's closing barrier publishes it
     if (threadIdx.x == 64) s_next = (int)gridDim.x + atomicAdd(a.ticket, 1);
-    if (item < n_dkdv) dkdv_cta<D>(tmq_rows, tmdo_rows, tmk128, tmv128, a, item, tmem);
-    else dq_cta<D>(tmq_tile, tmdo_tile, tmk64, tmv64, a, item - n_dkdv, tmem);
+    dkdv_cta<D>(tmq_rows, tmdo_rows, tmk128, tmv128, a, item, tmem);
     item = s_next;
     cta_sync();  // every thread has read s_next before the next item writes it
   }
@@ -937,6 +1043,9 @@ cudaError_t launch_backward_bf16(const BackwardArgs& a, const CUtensorMap* tmaps
   p.hblocks = (p.r + p.H - 1) / p.H;
   p.n_qt = (a.S_q + p.P - 1) / p.P;
   p.n_kb = (a.T_max + bw::kBK - 1) / bw::kBK;
+  p.div_per = FastDiv::make((uint32_t)(a.B * a.h_kv * p.hblocks));
+  p.div_gh = FastDiv::make((uint32_t)(a.h_kv * p.hblocks));
+  p.div_hb = FastDiv::make((uint32_t)p.hblocks);
   p.scale = a.scale;
   p.sl2 = a.scale * bw::kLog2e;
   p.causal = a.causal;

@@ -119,6 +119,25 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
+// n / d for 0 <= n < 2^31 and 1 <= d < 2^31 by a multiply and a shift (division by an invariant
+// integer, Granlund and Montgomery 1994): q = (umulhi(n, m) + n) >> s with s = ceil(log2 d) and
+// m = floor(2^32 (2^s - d) / d) + 1. An integer divide by a run-time value is a chain of a few
+// dozen instructions through the reciprocal unit, which the exponential-heavy warps of the same
+// SM keep busy; the persistent kernels' per-item bookkeeping divides with this instead.
+struct FastDiv {
+  uint32_t m, s;
+  static FastDiv make(uint32_t d) {
+    FastDiv f;
+    f.s = 0;
+    while ((1ull << f.s) < d) ++f.s;
+    f.m = (uint32_t)((((1ull << 32) * ((1ull << f.s) - d)) / d) + 1);
+    return f;
+  }
+  __device__ __forceinline__ int div(int n) const {
+    return (int)((__umulhi((uint32_t)n, m) + (uint32_t)n) >> s);
+  }
+};
+
 // ---------------------------------------------------------------------------------------------
 // Warp-level helpers
 // ---------------------------------------------------------------------------------------------

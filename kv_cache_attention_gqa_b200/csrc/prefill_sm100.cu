@@ -94,25 +94,6 @@ struct Cfg {
   static constexpr uint32_t colO(int t) { return (uint32_t)(256 * t + 128); }
 };
 
-// n / d for 0 <= n < 2^31 and 1 <= d < 2^31 by a multiply and a shift (division by an invariant
-// integer, Granlund and Montgomery 1994): q = (umulhi(n, m) + n) >> s with s = ceil(log2 d) and
-// m = floor(2^32 (2^s - d) / d) + 1. An integer divide by a run-time value goes through the
-// reciprocal unit, which the softmax warps keep busy with exponentials: the control warps' item
-// bookkeeping measured over a microsecond per item with it.
-struct FastDiv {
-  uint32_t m, s;
-  static FastDiv make(uint32_t d) {
-    FastDiv f;
-    f.s = 0;
-    while ((1ull << f.s) < d) ++f.s;
-    f.m = (uint32_t)((((1ull << 32) * ((1ull << f.s) - d)) / d) + 1);
-    return f;
-  }
-  __device__ __forceinline__ int div(int n) const {
-    return (int)((__umulhi((uint32_t)n, m) + (uint32_t)n) >> s);
-  }
-};
-
 struct PArgs {
   void* o;
   float* lse;
@@ -945,9 +926,9 @@ cudaError_t launch_prefill_bf16(const PrefillArgs& a, const CUtensorMap* tmaps, 
   if (items <= 0) return cudaSuccess;
   if (items > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
   p.n_items = (int)items;
-  p.div_per = pf::FastDiv::make((uint32_t)units);
-  p.div_gh = pf::FastDiv::make((uint32_t)(a.h_kv * p.hblocks));
-  p.div_hb = pf::FastDiv::make((uint32_t)p.hblocks);
+  p.div_per = FastDiv::make((uint32_t)units);
+  p.div_gh = FastDiv::make((uint32_t)(a.h_kv * p.hblocks));
+  p.div_hb = FastDiv::make((uint32_t)p.hblocks);
   // pair mode: one persistent CTA per SM (it holds all 512 TMEM columns), or one per item when
   // fewer; split mode (chosen when the items barely fill the SMs): one CTA per item
   const long long ctas = p.split || items < num_sms ? items : num_sms;

@@ -137,3 +137,49 @@ def test_backward_bf16_unaligned_o(d):
         assert_grad_close(_f64(dq), rq, f"dQ {what} d={d}", False)
         assert_grad_close(_f64(dk), rk, f"dK {what} d={d}", False)
         assert_grad_close(_f64(dv), rv, f"dV {what} d={d}", False)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_backward_dq_runs_mha_ragged(d):
+    """More dQ tiles than SMs (320 tiles of one head x 128 positions, after 512 dK/dV tiles), so
+    CTAs run several dQ tiles back to back, the next tile's loads and first scores overlapping the
+    previous tile's dQ write-out; per-sequence offsets and lengths make consecutive tiles of a CTA
+    differ in block count and mask, and NaN sits past every length."""
+    rng = np.random.default_rng(37)
+    kv = rng.integers(650, 900, size=8)
+    qs = (kv - 600 - rng.integers(0, 40, size=8)).clip(0, None)
+    _run(8, 8, 8, 600, 900, d, q_start=qs.tolist(), kv_len=kv.tolist(), nan_tail=True, seed=41 + d)
+
+
+def test_backward_dq_runs_window_gqa():
+    """416 dQ tiles of 4 heads x 32 positions under a 100-key window: tiles whose first K/V block
+    is partly below every row's window (K rows zeroed in the ring) follow one another on a CTA."""
+    _run(16, 8, 2, 400, 400, 128, window=100, seed=43)
+
+
+def test_backward_dq_runs_with_an_invalid_sequence():
+    """A sequence with kv_len = 0 among 12 (384 dQ tiles): its tiles see no key block, so a CTA's
+    run passes tiles with no MMA between ones with; their dQ, dK and dV are zero, the device
+    error reads GQA_DEVERR_KV_LEN, and every other sequence matches the oracle."""
+    import kv_cache_attention_gqa_b200 as gqa
+
+    B, h_q, h_kv, S, T, d, bad = 12, 16, 4, 256, 256, 64, 5
+    g = torch.Generator().manual_seed(47)
+    q = (torch.randn(B, h_q, S, d, generator=g) * 0.5).to(torch.bfloat16)
+    k = (torch.randn(B, h_kv, T, d, generator=g) * 0.5).to(torch.bfloat16)
+    v = torch.randn(B, h_kv, T, d, generator=g).to(torch.bfloat16)
+    d_o = torch.randn(B, h_q, S, d, generator=g).to(torch.bfloat16)
+    kl = [T] * B
+    kl[bad] = 0
+    qd, kd, vd, dod = q.cuda(), k.cuda(), v.cuda(), d_o.cuda()
+    o, lse = gqa.prefill(qd, kd, vd, kv_len=kl, return_lse=True)
+    assert gqa.get_device_error() == 1
+    dq, dk, dv = gqa.prefill_backward(qd, kd, vd, o, dod, lse, kv_len=kl)
+    assert gqa.get_device_error() == 1
+    assert dq[bad].abs().sum().item() == 0
+    assert dk[bad].abs().sum().item() == 0 and dv[bad].abs().sum().item() == 0
+    keep = [b for b in range(B) if b != bad]
+    rq, rk, rv = oracle.attention_backward_ref(_f64(q[keep]), _f64(k[keep]), _f64(v[keep]), _f64(d_o[keep]))
+    assert_grad_close(_f64(dq[keep]), rq, "dQ, the valid sequences")
+    assert_grad_close(_f64(dk[keep]), rk, "dK, the valid sequences")
+    assert_grad_close(_f64(dv[keep]), rv, "dV, the valid sequences")

@@ -423,7 +423,7 @@ size_t gqa_mla_decode_workspace_size(int B, int h_q, int T_max, int d_v, gqa_dty
   if (dtype != GQA_BF16 && dtype != GQA_FP32) return 0;
   const int sms = num_splits > 0 ? 1 : sm_count();
   if (sms <= 0) return 0;
-  return decode_workspace_bytes(B, h_q, 1, T_max, d_v, num_splits, sms, true);
+  return decode_workspace_bytes(B, h_q, 1, T_max, d_v, num_splits, sms, true, mla_uses_tc(h_q, dtype) != 0);
 }
 
 gqa_status gqa_mla_decode(const void* q, const void* cache, void* o, float* lse,
@@ -441,11 +441,12 @@ gqa_status gqa_mla_decode(const void* q, const void* cache, void* o, float* lse,
   if (B > decode_max_batch()) return GQA_ERR_UNSUPPORTED;
   if ((long long)B * T_max >= (1ll << 31) || (long long)B * h_q >= (1ll << 31)) return GQA_ERR_UNSUPPORTED;
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return GQA_ERR_WORKSPACE;
-  if (num_splits > 0 && workspace_bytes < decode_workspace_bytes(B, h_q, 1, T_max, d_v, num_splits, 1, true))
+  const bool tc = mla_uses_tc(h_q, dtype) != 0;
+  if (num_splits > 0 && workspace_bytes < decode_workspace_bytes(B, h_q, 1, T_max, d_v, num_splits, 1, true, tc))
     return GQA_ERR_WORKSPACE;
   const int sms = sm_count();
   if (sms <= 0) return GQA_ERR_CUDA;
-  if (workspace_bytes < decode_workspace_bytes(B, h_q, 1, T_max, d_v, num_splits, sms, true))
+  if (workspace_bytes < decode_workspace_bytes(B, h_q, 1, T_max, d_v, num_splits, sms, true, tc))
     return GQA_ERR_WORKSPACE;
   DecodeArgs a;
   a.q = q;
@@ -462,6 +463,7 @@ gqa_status gqa_mla_decode(const void* q, const void* cache, void* o, float* lse,
   a.d_h = d_qk;
   a.d_v = d_v;
   a.mla = 1;
+  a.mla_tc = tc ? 1 : 0;
   a.scale = scale;
   a.window = 0;
   a.workspace = workspace;
@@ -472,14 +474,18 @@ gqa_status gqa_mla_decode(const void* q, const void* cache, void* o, float* lse,
   if (!a.err) return GQA_ERR_CUDA;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (dtype == GQA_FP32) return from_cuda(launch_decode_fp32(a, s));
-  CUtensorMap maps[2];
+  CUtensorMap maps[4];
   const uint64_t cdims[2] = {(uint64_t)d_qk, (uint64_t)B * T_max};
   const uint64_t qdims[2] = {(uint64_t)d_qk, (uint64_t)B * h_q};
   const uint64_t strides[1] = {(uint64_t)d_qk * 2};
   const uint32_t cbox[2] = {64, 64};
   const uint32_t qbox[2] = {64, 16};
+  const uint32_t qbox_tc[2] = {64, 128};  // the tensor-core kernel: 128 heads, 32-key tiles
+  const uint32_t cbox_tc[2] = {64, 32};
   if (!encode_bf16(&maps[0], cache, 2, cdims, strides, cbox) ||
-      !encode_bf16(&maps[1], q, 2, qdims, strides, qbox))
+      !encode_bf16(&maps[1], q, 2, qdims, strides, qbox) ||
+      (tc && (!encode_bf16(&maps[2], q, 2, qdims, strides, qbox_tc) ||
+              !encode_bf16(&maps[3], cache, 2, cdims, strides, cbox_tc))))
     return GQA_ERR_CUDA;
   return from_cuda(launch_mla_bf16(a, maps, s));
 }

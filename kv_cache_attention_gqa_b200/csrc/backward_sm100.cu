@@ -200,20 +200,9 @@ __device__ __forceinline__ uint64_t desc_k(uint32_t tile, int k, uint32_t chunk)
 __device__ __forceinline__ uint64_t desc_mn(uint32_t tile, int kk, uint32_t chunk) {
   return tc::smem_desc(tile + (uint32_t)(kk * 2048), chunk, 1024);
 }
-// The same descriptors as a base plus a constant: the start address sits in the low 14 bits
-// (address >> 4, below 2^14 for any shared-memory address), so the descriptor of tile + offset is
-// the tile's descriptor plus offset >> 4. The MMA issuers build the bases once per stage and add
-// compile-time offsets inside their unrolled loops.
-__device__ __forceinline__ uint64_t koff(int k, uint32_t chunk) {
-  return (uint64_t)(((k >> 2) * chunk + (k & 3) * 32) >> 4);
-}
-__device__ __forceinline__ uint64_t mnoff(int kk) { return (uint64_t)((kk * 2048) >> 4); }
-
-__device__ __forceinline__ bool elect_one() {
-  uint32_t p;
-  asm volatile("{\n\t.reg .pred q;\n\telect.sync _|q, 0xffffffff;\n\tselp.u32 %0, 1, 0, q;\n\t}" : "=r"(p));
-  return p != 0;
-}
+using tc::elect_one;
+using tc::koff;
+using tc::mnoff;
 
 // ---- dkdv: key-stationary dK / dV -------------------------------------------------------------
 // Query blocks of 64 rows, so S^T and dP^T are double-buffered in TMEM next to the dV / dK

@@ -45,6 +45,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "tcgen05.cuh"
 
 namespace gqa {
 namespace dec {
@@ -124,7 +125,8 @@ struct KArgs {
   int hpu, hblocks;
   float scale;     // natural-log scale; the bf16 core folds log2(e) in
   int n_max;       // upper bound on the number of chunks (workspace slots)
-  int auto_chunk;  // 1: chunks hold at least kMinChunkAuto keys
+  int auto_chunk;  // 1: chunks hold at least min_chunk keys
+  int min_chunk;   // keys
   int window;      // 0: none; W > 0: the query at q_pos sees keys q_pos - W < j <= q_pos
   Header* hdr;
   long long* pre;
@@ -252,8 +254,7 @@ __device__ void build_plan(const KArgs& a, Plan& p, long long* pre, int* nlen, i
   if (a.auto_chunk) {
     // at least kMinChunkAuto keys, and at least 16 keys per query row, so the partial written per
     // chunk (hpu x d_h fp32) stays small against the chunk's K/V bytes (2 x C x d_h bf16)
-    const long long lo_keys = 16LL * a.hpu > kMinChunkAuto ? 16LL * a.hpu : kMinChunkAuto;
-    const long long lo = udiv(lo_keys + a.gran - 1, a.gran);
+    const long long lo = udiv((long long)a.min_chunk + a.gran - 1, a.gran);
     if (C < lo) C = lo;
   }
   if (C < 1) C = 1;
@@ -1229,6 +1230,422 @@ __global__ void __launch_bounds__(MlaCfg::kThreads, 1)
 }
 
 // =============================================================================================
+// MLA decode on the tensor cores (bf16, 128 heads per unit)
+// =============================================================================================
+// With 128 heads the score and value products are dense enough for tcgen05: the unit's 128
+// heads sit on the 128 TMEM lanes (M = 128) and each 32-key tile of latent rows is the B operand
+//   S  = Q C^T   (M 128, N 32 keys, K 576)   into TMEM columns [0, 32)
+//   O += P C_v   (M 128, N 256, K 32 keys)   into TMEM columns [64, 320)
+// The 512-wide latent accumulator is twice what TMEM holds next to S, so a unit's chunk is run by
+// two CTAs, each owning 256 of the latent columns (d_v half); both compute the same S (the same
+// bits: the same MMAs on the same inputs), and each writes its half of the piece output.
+// TMEM: S [0, 32), O half [64, 320), the query's first 384 columns [320, 512) (the A operand of
+// the first 24 k-steps of S); the query's last 192 columns stay in shared memory (the A operand of
+// the other 12). P (bf16) goes to shared memory, so the next tile's S overwrites the scores as soon
+// as the softmax warps have read them and runs while they compute P. The tiles pass through a
+// 4-deep ring of 36 KiB stages, so a tile's copy starts three tiles ahead of its use.
+// Warps: 0 TMA producer, 1 MMA issuer (and TMEM owner), 2..5 softmax, one TMEM lane quarter each
+// (warp w reads lanes 32 (w % 4) ..), one head per thread.
+// Chunks: CTAs 2p and 2p + 1 take chunks p, p + G/2, ... of the same split-KV plan as the other
+// decode kernels; partials and the merge kernel are shared with them.
+constexpr int kMlaTcHeads = 128;
+constexpr int kMlaTcMinChunk = 256;  // keys; the automatic chunking never goes below this
+constexpr int kMlaTcKeys = 32;       // keys per tile
+struct MlaTcCfg {
+  static constexpr int kStages = 4;
+  static constexpr int kNch = kMlaDqk / 64;                // 9 column chunks of a latent row
+  static constexpr int kChunkBytes = kMlaTcKeys * 128;     // 32 rows x 128 B
+  static constexpr int kTileBytes = kNch * kChunkBytes;    // 36 KiB
+  static constexpr int kQTmemCh = 6;                       // query chunks held in TMEM (384 columns)
+  static constexpr int kQSmemCh = kNch - kQTmemCh;         // 3 in shared memory
+  static constexpr int kQChunkBytes = kMlaTcHeads * 128;   // 128 rows x 128 B
+  static constexpr int kQBytes = kQSmemCh * kQChunkBytes;  // 48 KiB
+  static constexpr int kPBytes = kMlaTcHeads * 128;        // 128 rows of 128 B; a tile's P uses 64 B
+  static constexpr int kThreads = 192;
+  static constexpr uint32_t kColS = 0, kColO = 64, kColQ = 320;
+  static constexpr int kHalf = kMlaDv / 2;                 // latent columns per CTA
+  enum { kFull = 0, kEmpty = kFull + kStages, kQInfo = kEmpty + kStages, kQFull, kQTmem, kSFull, kSFree,
+         kPFull, kPvDone, kPieceDone, kAll, kBars };
+  static constexpr size_t kOffQ = (size_t)kStages * kTileBytes;
+  static constexpr size_t kOffP = kOffQ + kQBytes;
+  static constexpr size_t kOffPre = kOffP + kPBytes;
+  static constexpr size_t kOffNlen = kOffPre + (kMaxBatch + 1) * 8;
+  static constexpr size_t kOffWlo = kOffNlen + kMaxBatch * 4;
+  static constexpr size_t kOffMeta = kOffWlo + kMaxBatch * 4;
+  static constexpr size_t kOffBar = kOffMeta + kStages * sizeof(TileMeta);
+  static constexpr size_t kSmem = kOffBar + kBars * 8 + 1024;  // + alignment of the base
+  static_assert(kSmem + 16 <= 227 * 1024, "shared memory budget");
+};
+
+__global__ void __launch_bounds__(MlaTcCfg::kThreads, 1)
+    mla_tc_kernel(const __grid_constant__ CUtensorMap tmc, const __grid_constant__ CUtensorMap tmq,
+                  KArgs a) {
+  using C = MlaTcCfg;
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ uint32_t s_tmem;
+  __shared__ int s_qrow;  // the current piece's first query row (b * h_q + first head), -1: the end
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  long long* pre = reinterpret_cast<long long*>(smem + C::kOffPre);
+  int* nlen = reinterpret_cast<int*>(smem + C::kOffNlen);
+  int* wlo = reinterpret_cast<int*>(smem + C::kOffWlo);
+  TileMeta* meta = reinterpret_cast<TileMeta*>(smem + C::kOffMeta);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
+  volatile int* qrow_slot = &s_qrow;
+  auto bar = [&](int i) { return smem_u32(&bars[i]); };
+  const uint32_t sQ = smem_u32(smem + C::kOffQ), sP = smem_u32(smem + C::kOffP);
+  auto sC = [&](int st) { return smem_u32(smem + st * C::kTileBytes); };
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int half = blockIdx.x & 1;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(bar(C::kFull + s), 1);
+      mbar_init(bar(C::kEmpty + s), 1);
+    }
+    mbar_init(bar(C::kQInfo), 1);
+    mbar_init(bar(C::kQFull), 1);
+    mbar_init(bar(C::kQTmem), 128);
+    mbar_init(bar(C::kSFull), 1);
+    mbar_init(bar(C::kSFree), 128);
+    mbar_init(bar(C::kPFull), 128);
+    mbar_init(bar(C::kPvDone), 1);
+    mbar_init(bar(C::kPieceDone), 1);
+    mbar_init(bar(C::kAll), 1);
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmc);
+    tma_prefetch_desc(&tmq);
+  }
+  if (warp == 1) {  // all 512 columns (one CTA per SM: the shared memory sees to that)
+    tc::tmem_alloc(smem_u32(&s_tmem), 512);
+    tc::tmem_relinquish();
+    tc::fence_before_sync();
+  }
+  pdl_wait();  // launched as a programmatic dependent: no input is read before this
+  Plan plan;
+  build_plan<__nv_bfloat16>(a, plan, pre, nlen, wlo, warp, lane, 0);  // ends with a CTA barrier
+  pdl_launch_dependents();
+  tc::fence_after_sync();
+  const uint32_t tmem = s_tmem;
+  const int pairs = (int)(gridDim.x >> 1);
+
+  if (warp == 0) {
+    // ------------------------------ TMA producer (lane 0) --------------------------------------
+    if (lane == 0) {
+      int stage = 0, issued = 0, pieces = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int chunk = (int)(blockIdx.x >> 1); ok && chunk < plan.n_chunks; chunk += pairs) {
+        const long long x1 = min((long long)(chunk + 1) * plan.C, plan.K);
+        for (long long x = (long long)chunk * plan.C; x < x1 && ok;) {
+          const Piece pc = locate(plan, a.B, a.hblocks, x, x1);
+          const int slot = pc.n_pieces == 1 ? -1 : chunk + pc.unit;
+          const int row0 = pc.b * a.T_max;
+          const int qrow = pc.b * a.h_q + pc.hb * kMlaTcHeads;
+          // The previous piece's MMAs (the last readers of the query buffers) are complete, and
+          // every consumer has passed its piece start (so no barrier phase below is skipped).
+          if (pieces > 0 && !(ok = mbar_wait(bar(C::kPieceDone), (uint32_t)((pieces - 1) & 1), a.err))) break;
+          *qrow_slot = qrow;
+          mbar_arrive(bar(C::kQInfo));  // the softmax warps start the query's TMEM copy now
+          mbar_arrive_expect_tx(bar(C::kQFull), (uint32_t)C::kQBytes);
+#pragma unroll
+          for (int ch = 0; ch < C::kQSmemCh; ++ch)
+            tma_load_2d(sQ + ch * C::kQChunkBytes, &tmq, bar(C::kQFull), (C::kQTmemCh + ch) * 64, qrow);
+          ++pieces;
+          for (int t = pc.k0; t < pc.k1; t += kMlaTcKeys) {
+            if (!(ok = mbar_wait(bar(C::kEmpty + stage), phase ^ 1u, a.err))) break;
+            TileMeta m;
+            m.b = pc.b;
+            m.g = 0;
+            m.hb = pc.hb;
+            m.nvalid = min(kMlaTcKeys, pc.k1 - t);
+            m.flags = (t == pc.k0 ? kFirst : 0) | (t + kMlaTcKeys >= pc.k1 ? kLast : 0);
+            m.slot = slot;
+            m.nh = kMlaTcHeads;
+            m.nskip = 0;
+            meta[stage] = m;
+            mbar_arrive_expect_tx(bar(C::kFull + stage), (uint32_t)C::kTileBytes);
+#pragma unroll
+            for (int ch = 0; ch < C::kNch; ++ch)
+              tma_load_2d(sC(stage) + ch * C::kChunkBytes, &tmc, bar(C::kFull + stage), ch * 64, row0 + t);
+            ++issued;
+            if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
+          }
+          x = pc.end;
+        }
+      }
+      // Drain (bounded) before the end markers: every copy issued has landed, so none can reach
+      // shared memory after the CTA is gone. Fill f of stage f % 4 completes phase f / 4 of its
+      // full barrier and no later fill follows the last four; the query rows complete phase
+      // pieces - 1 of theirs.
+      for (int f = issued > C::kStages ? issued - C::kStages : 0; f < issued; ++f)
+        mbar_wait(bar(C::kFull + f % C::kStages), (uint32_t)(f / C::kStages) & 1u, a.err);
+      if (pieces > 0) mbar_wait(bar(C::kQFull), (uint32_t)((pieces - 1) & 1), a.err);
+      if (ok) {
+        // the end: a piece with no rows for the softmax warps, a marker tile for the MMA warp
+        if (pieces == 0 || mbar_wait(bar(C::kPieceDone), (uint32_t)((pieces - 1) & 1), a.err)) {
+          *qrow_slot = -1;
+          mbar_arrive(bar(C::kQInfo));
+        }
+        if (mbar_wait(bar(C::kEmpty + stage), phase ^ 1u, a.err)) {
+          meta[stage].flags = kEnd;
+          mbar_arrive(bar(C::kFull + stage));
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------ MMA issuer (one elected lane) ------------------------------
+    constexpr uint32_t idesc_s = tc::idesc_bf16(128, kMlaTcKeys, false);  // S: 128 heads x 32 keys
+    constexpr uint32_t idesc_o = tc::idesc_bf16(128, C::kHalf, true);     // O: 128 x 256, B MN-major
+    auto wait = [&](int b_, uint32_t parity) {
+      return __all_sync(0xffffffffu, mbar_wait(bar(b_), parity, a.err));
+    };
+    auto issue_s = [&](int st) {  // S = Q C^T over all 576 columns of the tile in stage st
+      const uint64_t dc = tc::smem_desc(sC(st), 16, 1024), dq = tc::smem_desc(sQ, 16, 1024);
+      if (tc::elect_one()) {
+#pragma unroll
+        for (int k = 0; k < 4 * C::kQTmemCh; ++k)  // query columns [0, 384) from TMEM
+          tc::mma_ts(tmem + C::kColS, tmem + C::kColQ + k * 8, dc + tc::koff(k, C::kChunkBytes), idesc_s,
+                     k > 0 ? 1u : 0u);
+#pragma unroll
+        for (int k = 0; k < 4 * C::kQSmemCh; ++k)  // [384, 576) from shared memory
+          tc::mma_ss(tmem + C::kColS, dq + tc::koff(k, C::kQChunkBytes),
+                     dc + tc::koff(4 * C::kQTmemCh + k, C::kChunkBytes), idesc_s, 1u);
+        tc::commit(bar(C::kSFull));
+      }
+      __syncwarp();
+    };
+    int stage = 0, jg = 0, piece = 0;
+    uint32_t phase = 0;
+    bool pre_issued = false;  // S of the current tile was issued with the previous tile
+    bool ok = true;
+    while (ok) {
+      if (!(ok = wait(C::kFull + stage, phase))) break;
+      const TileMeta m = meta[stage];
+      if (m.flags & kEnd) break;
+      if (m.flags & kFirst) {
+        if (!(ok = wait(C::kQFull, (uint32_t)(piece & 1)) && wait(C::kQTmem, (uint32_t)(piece & 1)))) break;
+      }
+      if (!pre_issued) {
+        if (jg > 0 && !(ok = wait(C::kSFree, (uint32_t)((jg - 1) & 1)))) break;
+        tc::fence_after_sync();
+        issue_s(stage);
+      }
+      pre_issued = false;
+      const int nstage = stage + 1 == C::kStages ? 0 : stage + 1;
+      const uint32_t nphase = stage + 1 == C::kStages ? phase ^ 1u : phase;
+      if (!(m.flags & kLast)) {
+        // the piece's next tile, if it has landed: its scores overlap this tile's softmax; if
+        // not, this tile's P V goes first, so its stage refills sooner
+        if (!(ok = wait(C::kSFree, (uint32_t)(jg & 1)))) break;
+        int landed = lane == 0 ? (int)mbar_test(bar(C::kFull + nstage), nphase) : 0;
+        landed = __shfl_sync(0xffffffffu, landed, 0);
+        if (landed) {
+          tc::fence_after_sync();
+          issue_s(nstage);
+          pre_issued = true;
+        }
+      }
+      if (!(ok = wait(C::kPFull, (uint32_t)(jg & 1)))) break;
+      tc::fence_after_sync();
+      const uint64_t dp = tc::smem_desc(sP, 16, 1024);
+      const uint64_t dv = tc::smem_desc(sC(stage) + half * 4 * C::kChunkBytes, C::kChunkBytes, 1024);
+      if (tc::elect_one()) {
+#pragma unroll
+        for (int kk = 0; kk < kMlaTcKeys / 16; ++kk)
+          tc::mma_ss(tmem + C::kColO, dp + tc::koff(kk, C::kPBytes), dv + tc::mnoff(kk), idesc_o,
+                     ((m.flags & kFirst) && kk == 0) ? 0u : 1u);
+        tc::commit(bar(C::kPvDone));
+        tc::commit(bar(C::kEmpty + stage));
+        if (m.flags & kLast) tc::commit(bar(C::kPieceDone));
+      }
+      __syncwarp();
+      if (m.flags & kLast) ++piece;
+      ++jg;
+      stage = nstage;
+      phase = nphase;
+    }
+    // every MMA issued above has completed before TMEM is released
+    if (tc::elect_one()) tc::commit(bar(C::kAll));
+    __syncwarp();
+    mbar_wait(bar(C::kAll), 0, a.err);
+  } else {
+    // ------------------------------ softmax: one head (TMEM lane) per thread --------------------
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
+    const int et = (warp - 2) * 32 + lane;  // 0..127, for the V-row zeroing
+    const float sl2 = a.scale * kLog2e;
+    int stage = 0, jg = 0, piece = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    while (ok) {
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(C::kQInfo), (uint32_t)(piece & 1), a.err));
+      if (!ok) break;
+      const int qrow = *qrow_slot;
+      if (qrow < 0) break;
+      // this head's query columns [0, 384) -> TMEM, two 64-column chunks per round of loads (the
+      // previous piece's scores are all read, so no MMA still reads these columns)
+      {
+        const uint4* qg = reinterpret_cast<const uint4*>(a.q) + (long long)(qrow + row) * (kMlaDqk / 8);
+#pragma unroll
+        for (int bc = 0; bc < C::kQTmemCh; bc += 2) {
+          uint4 v[16];
+#pragma unroll
+          for (int u = 0; u < 16; ++u) v[u] = __ldg(qg + bc * 8 + u);
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            uint32_t r[32];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              r[4 * u] = v[8 * c + u].x;
+              r[4 * u + 1] = v[8 * c + u].y;
+              r[4 * u + 2] = v[8 * c + u].z;
+              r[4 * u + 3] = v[8 * c + u].w;
+            }
+            tc::st32(lane_addr + C::kColQ + (bc + c) * 32, r);
+          }
+        }
+        tc::wait_st();
+        tc::fence_before_sync();
+        mbar_arrive(bar(C::kQTmem));
+      }
+      float m_run = -INFINITY, l_run = 0.f;
+      bool last = false;
+      while (!last) {
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(C::kFull + stage), phase, a.err));
+        if (!ok) break;
+        const TileMeta m = meta[stage];
+        const bool first = (m.flags & kFirst) != 0;
+        last = (m.flags & kLast) != 0;
+        // ---- scores of this tile
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(C::kSFull), (uint32_t)(jg & 1), a.err));
+        if (!ok) break;
+        tc::fence_after_sync();
+        float s[kMlaTcKeys];
+        tc::ld32f(lane_addr + C::kColS, s);
+        tc::wait_ld();
+        tc::fence_before_sync();
+        mbar_arrive(bar(C::kSFree));  // the next tile's scores may overwrite them
+        const int nvalid = m.nvalid;
+        float bm = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < kMlaTcKeys; ++i) {
+          s[i] = i < nvalid ? s[i] * sl2 : -INFINITY;
+          bm = fmaxf(bm, s[i]);
+        }
+        // running maximum, raised lazily: the accumulator is rescaled only when the tile's
+        // maximum passes the running one by more than 2^8 (P then stays below 2^8); the piece's
+        // first tile sets it (its P V overwrites the accumulator)
+        float alpha = 1.f;
+        const bool raise = first || bm > m_run + 8.f;
+        if (raise) {
+          alpha = first ? 0.f : fast_exp2(m_run - bm);
+          m_run = bm;
+        }
+        // the previous tile's P V has completed: P may be rewritten and O rescaled
+        if (jg > 0) {
+          ok = __all_sync(0xffffffffu, mbar_wait(bar(C::kPvDone), (uint32_t)((jg - 1) & 1), a.err));
+          if (!ok) break;
+          tc::fence_after_sync();
+        }
+        if (__any_sync(0xffffffffu, raise && !first)) {  // `first` is the same for the whole warp
+#pragma unroll 1
+          for (int c = 0; c < C::kHalf / 32; ++c) {
+            float o[32];
+            tc::ld32f(lane_addr + C::kColO + c * 32, o);
+            tc::wait_ld();
+            uint32_t w[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) w[i] = __float_as_uint(o[i] * alpha);
+            tc::st32(lane_addr + C::kColO + c * 32, w);
+          }
+          tc::wait_st();
+        }
+        l_run *= alpha;
+        float ls = 0.f;
+        uint32_t pk[kMlaTcKeys / 2];
+#pragma unroll
+        for (int i = 0; i < kMlaTcKeys; i += 2) {
+          const float p0 = fast_exp2(s[i] - m_run), p1 = fast_exp2(s[i + 1] - m_run);
+          ls += p0 + p1;
+          pk[i / 2] = pack_bf16x2(p0, p1);
+        }
+        l_run += ls;
+#pragma unroll
+        for (int u = 0; u < kMlaTcKeys / 8; ++u)
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(swz128(sP, row, u)), "r"(pk[4 * u]),
+                       "r"(pk[4 * u + 1]), "r"(pk[4 * u + 2]), "r"(pk[4 * u + 3])
+                       : "memory");
+        // rows past the piece's last key may hold anything (NaN past a length): their P is 0,
+        // but 0 * NaN is NaN, so this CTA's value columns of those rows are zeroed before P V
+        if (nvalid < kMlaTcKeys) {
+          const int units = (kMlaTcKeys - nvalid) * 4 * 8;  // rows x 4 chunks x 8 16-byte units
+          for (int e = et; e < units; e += 128) {
+            const int rr = nvalid + e / 32, ch = (e / 8) & 3, u = e & 7;
+            const uint32_t addr = sC(stage) + (half * 4 + ch) * C::kChunkBytes + rr * 128 + u * 16;
+            asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(addr), "r"(0u) : "memory");
+          }
+        }
+        tc::fence_proxy_async_smem();
+        tc::fence_before_sync();
+        mbar_arrive(bar(C::kPFull));
+        if (last) {
+          // ---- piece end: O / l -> the output (one piece) or a partial, this CTA's columns
+          ok = __all_sync(0xffffffffu, mbar_wait(bar(C::kPvDone), (uint32_t)(jg & 1), a.err));
+          if (!ok) break;
+          tc::fence_after_sync();
+          const float inv = 1.f / l_run;
+          const float lse2 = m_run + __log2f(l_run);
+          const int head = m.hb * kMlaTcHeads + row;
+#pragma unroll 1
+          for (int c = 0; c < C::kHalf / 32; ++c) {
+            float o[32];
+            tc::ld32f(lane_addr + C::kColO + c * 32, o);
+            tc::wait_ld();
+            const int col = half * C::kHalf + c * 32;
+            if (m.slot < 0) {
+              uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.o) +
+                                                    ((long long)m.b * a.h_q + head) * kMlaDv + col);
+#pragma unroll
+              for (int q = 0; q < 4; ++q)
+                dst[q] = make_uint4(pack_bf16x2(o[8 * q] * inv, o[8 * q + 1] * inv),
+                                    pack_bf16x2(o[8 * q + 2] * inv, o[8 * q + 3] * inv),
+                                    pack_bf16x2(o[8 * q + 4] * inv, o[8 * q + 5] * inv),
+                                    pack_bf16x2(o[8 * q + 6] * inv, o[8 * q + 7] * inv));
+            } else {
+              float4* dst = reinterpret_cast<float4*>(a.part_o + ((long long)m.slot * a.hpu + row) * kMlaDv + col);
+#pragma unroll
+              for (int q = 0; q < 8; ++q)
+                dst[q] = make_float4(o[4 * q] * inv, o[4 * q + 1] * inv, o[4 * q + 2] * inv, o[4 * q + 3] * inv);
+            }
+          }
+          if (half == 0) {
+            if (m.slot < 0) {
+              if (a.lse) a.lse[(long long)m.b * a.h_q + head] = lse2 * kLn2;
+            } else {
+              a.part_lse[(long long)m.slot * a.hpu + row] = lse2;
+            }
+          }
+        }
+        ++jg;
+        if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
+      }
+      ++piece;
+    }
+  }
+  // every role is done: copies landed, MMAs complete, TMEM read
+  tc::fence_before_sync();
+  cta_sync();
+  if (warp == 1) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, 512);
+  }
+}
+
+// =============================================================================================
 // fp32 check-mode kernel
 // =============================================================================================
 constexpr int kF32Warps = 4;
@@ -1401,14 +1818,28 @@ int auto_n_max(long long K_max, int sms) {
   return (int)(n < 1 ? 1 : n);
 }
 
+// The tensor-core MLA kernel runs each chunk on two CTAs: at most one chunk per pair of SMs.
+int auto_n_max_mla_tc(long long K_max, int sms) {
+  long long n = (K_max + kMlaTcMinChunk - 1) / kMlaTcMinChunk;
+  const long long cap = sms / 2 > 0 ? sms / 2 : 1;
+  if (n > cap) n = cap;
+  return (int)(n < 1 ? 1 : n);
+}
+
+int mla_heads_per_unit(bool mla, bool mla_tc) {
+  return mla ? (mla_tc ? kMlaTcHeads : kMlaHeads) : kHeadsPerUnitMax;
+}
+
 KArgs make_kargs(const DecodeArgs& a) {
   const bool auto_chunk = a.num_splits == 0;
   const int r = a.h_q / a.h_kv;
-  const int hpu_max = a.mla ? kMlaHeads : kHeadsPerUnitMax;
+  const int hpu_max = mla_heads_per_unit(a.mla != 0, a.mla_tc != 0);
   const int hpu = r < hpu_max ? r : hpu_max;
   const int d_out = a.d_v > 0 ? a.d_v : a.d_h;
   const long long K_max = (long long)a.B * a.h_kv * ((r + hpu - 1) / hpu) * a.T_max;
-  const int n_max = auto_chunk ? auto_n_max(K_max, a.num_sms) : a.num_splits;
+  const int n_max = !auto_chunk ? a.num_splits
+                    : a.mla_tc  ? auto_n_max_mla_tc(K_max, a.num_sms)
+                                : auto_n_max(K_max, a.num_sms);
   const Layout L = make_layout(a.B, a.h_q, a.h_kv, d_out, n_max, hpu_max);
   KArgs k;
   k.q = a.q;
@@ -1430,6 +1861,10 @@ KArgs make_kargs(const DecodeArgs& a) {
   k.scale = a.scale;
   k.n_max = n_max;
   k.auto_chunk = auto_chunk ? 1 : 0;
+  // at least 16 keys per query row, so the partial written per chunk (hpu x d_out fp32) stays
+  // small against the chunk's K/V bytes; the tensor-core MLA kernel is bound by its MMAs instead
+  // and wants every pair of SMs busy
+  k.min_chunk = a.mla_tc ? kMlaTcMinChunk : (16 * L.hpu > kMinChunkAuto ? 16 * L.hpu : kMinChunkAuto);
   k.window = a.window;
   uint8_t* ws = reinterpret_cast<uint8_t*>(a.workspace);
   k.hdr = reinterpret_cast<Header*>(ws);
@@ -1450,12 +1885,14 @@ KArgs make_kargs(const DecodeArgs& a) {
 }  // namespace dec
 
 size_t decode_workspace_bytes(int B, int h_q, int h_kv, int T_max, int d_h, int num_splits,
-                              int num_sms, bool mla) {
+                              int num_sms, bool mla, bool mla_tc) {
   const int r = h_q / h_kv;
-  const int hpu_max = mla ? dec::kMlaHeads : dec::kHeadsPerUnitMax;
+  const int hpu_max = dec::mla_heads_per_unit(mla, mla_tc);
   const int hpu = r < hpu_max ? r : hpu_max;
   const long long K_max = (long long)B * h_kv * ((r + hpu - 1) / hpu) * T_max;
-  const int n_max = num_splits == 0 ? dec::auto_n_max(K_max, num_sms) : num_splits;
+  const int n_max = num_splits != 0 ? num_splits
+                    : mla_tc        ? dec::auto_n_max_mla_tc(K_max, num_sms)
+                                    : dec::auto_n_max(K_max, num_sms);
   return dec::make_layout(B, h_q, h_kv, d_h, n_max, hpu_max).total;
 }
 
@@ -1496,6 +1933,23 @@ cudaError_t launch_decode_bf16(const DecodeArgs& a, const CUtensorMap* tmaps, cu
 
 cudaError_t launch_mla_bf16(const DecodeArgs& a, const CUtensorMap* tmaps, cudaStream_t s) {
   const dec::KArgs k = dec::make_kargs(a);
+  if (a.mla_tc) {
+    using T = dec::MlaTcCfg;
+    static bool tc_attr_set[64] = {false};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64 || !tc_attr_set[dev]) {
+      e = cudaFuncSetAttribute(dec::mla_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)T::kSmem);
+      if (e != cudaSuccess) return e;
+      if (dev >= 0 && dev < 64) tc_attr_set[dev] = true;
+    }
+    const int pairs = k.n_max < a.num_sms / 2 ? k.n_max : a.num_sms / 2;
+    if (pairs < 1) return cudaErrorInvalidConfiguration;
+    e = dec::launch_dependent(dec::mla_tc_kernel, 2 * pairs, T::kThreads, T::kSmem, s, tmaps[3], tmaps[2], k);
+    if (e != cudaSuccess) return e;
+    return dec::launch_merge<__nv_bfloat16, true>(k, s);
+  }
   using C = dec::MlaCfg;
   static bool attr_set[64] = {false};
   int dev = 0;
@@ -1512,5 +1966,7 @@ cudaError_t launch_mla_bf16(const DecodeArgs& a, const CUtensorMap* tmaps, cudaS
 }
 
 int mla_dims_supported_bf16(int d_qk, int d_v) { return d_qk == dec::kMlaDqk && d_v == dec::kMlaDv; }
+
+int mla_uses_tc(int h_q, gqa_dtype dtype) { return dtype == GQA_BF16 && h_q % dec::kMlaTcHeads == 0; }
 
 }  // namespace gqa

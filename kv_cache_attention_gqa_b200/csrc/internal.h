@@ -104,6 +104,9 @@ struct DecodeArgs {
   // width (576), d_v = the value / output width (the row's first 512 entries); 16 heads per unit
   int mla = 0;
   int d_v = 0;
+  // MLA with a multiple of 128 heads (bf16): the tensor-core kernel, 128 heads per unit, each
+  // chunk on two CTAs (one per half of the 512 value columns)
+  int mla_tc = 0;
   int expire_wait = 0;  // test hook (gqa_debug_expire_waits), contiguous bf16 decode only
 };
 
@@ -115,7 +118,7 @@ gqa_status decode_check_args(const void* q, const void* k_cache, const void* v_c
 
 // Workspace bytes for a decode of this shape (layout in decode.cu).
 size_t decode_workspace_bytes(int B, int h_q, int h_kv, int T_max, int d_h, int num_splits,
-                              int num_sms, bool mla = false);
+                              int num_sms, bool mla = false, bool mla_tc = false);
 int decode_max_batch();
 
 cudaError_t launch_decode_fp32(const DecodeArgs& a, cudaStream_t s);
@@ -124,8 +127,11 @@ cudaError_t launch_decode_fp32(const DecodeArgs& a, cudaStream_t s);
 // [2] = queries as (d_h, B*h_q) with box (64, 16 or 32 rows: 32 when r > 16); SWIZZLE_128B.
 cudaError_t launch_decode_bf16(const DecodeArgs& a, const CUtensorMap* tmaps, cudaStream_t s);
 // MLA (bf16, d_h = 576, d_v = 512): tmaps [0] = the cache as (576, B*T_max) with box (64, 64),
-// [1] = the queries as (576, B*h_q) with box (64, 16); SWIZZLE_128B.
+// [1] = the queries as (576, B*h_q) with box (64, 16); when a.mla_tc, [2] the queries with box
+// (64, 128) and [3] the cache with box (64, 32); SWIZZLE_128B.
 cudaError_t launch_mla_bf16(const DecodeArgs& a, const CUtensorMap* tmaps, cudaStream_t s);
 int mla_dims_supported_bf16(int d_qk, int d_v);
+// 1 when gqa_mla_decode runs the tensor-core kernel for this head count and dtype
+int mla_uses_tc(int h_q, gqa_dtype dtype);
 
 }  // namespace gqa

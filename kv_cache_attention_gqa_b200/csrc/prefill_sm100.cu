@@ -593,11 +593,7 @@ __device__ __forceinline__ void softmax_role(const PArgs& a, int t, int wq, int 
   }
 }
 
-__device__ __forceinline__ bool elect_one() {
-  uint32_t p;
-  asm volatile("{\n\t.reg .pred q;\n\telect.sync _|q, 0xffffffff;\n\tselp.u32 %0, 1, 0, q;\n\t}" : "=r"(p));
-  return p != 0;
-}
+using tc::elect_one;
 
 // MMA issuer of tile t over the CTA's items: the whole warp runs the loop; one elected lane issues
 // each batch of MMAs and the commits that follow it (a commit tracks the MMAs of the thread that

@@ -136,5 +136,23 @@ __device__ __forceinline__ void st32(uint32_t taddr, const uint32_t (&r)[32]) {
 __device__ __forceinline__ void wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
+// ---- offsets of a tile's descriptor (128-byte swizzle, tiles of 64-column chunks) -------------
+// The start address sits in the low 14 bits (address >> 4, below 2^14 for any shared-memory
+// address), so the descriptor of tile + offset is the tile's descriptor plus offset >> 4; MMA
+// issuers build a base once per stage and add compile-time offsets in their unrolled loops.
+// K-major operand, k-th 16-column step (chunk: bytes of one 64-column chunk of the tile).
+__device__ __forceinline__ uint64_t koff(int k, uint32_t chunk) {
+  return (uint64_t)(((k >> 2) * chunk + (k & 3) * 32) >> 4);
+}
+// MN-major operand, kk-th 16-row step.
+__device__ __forceinline__ uint64_t mnoff(int kk) { return (uint64_t)((kk * 2048) >> 4); }
+
+// One lane of a converged warp (the same lane every time), for the single-thread MMA issue.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t p;
+  asm volatile("{\n\t.reg .pred q;\n\telect.sync _|q, 0xffffffff;\n\tselp.u32 %0, 1, 0, q;\n\t}" : "=r"(p));
+  return p != 0;
+}
+
 }  // namespace tc
 }  // namespace gqa

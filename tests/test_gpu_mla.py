@@ -105,3 +105,33 @@ def test_mla_decode_8k_full_size(h_q):
     assert gqa.get_device_error() == 0
     ref, _ = mla_ref.mla_decode_ref(_f64(q), _f64(cache), 512, kv_len=kl.cpu().numpy(), scale=shape.scale)
     assert_bf16_close(_f64(o), ref, f"mla decode_8k h_q={h_q}")
+
+
+@pytest.mark.parametrize("splits", [3, 0])
+def test_mla_decode_bf16_two_units_per_sequence(splits):
+    """256 heads: two 128-head units per sequence on the tensor-core kernel, ragged lengths with
+    NaN past each, chunks that cut through units and sequences."""
+    import kv_cache_attention_gqa_b200 as gqa
+
+    shape = workloads.MlaShape(B=2, h_q=256, T_max=1500)
+    lens = [1500, 901]
+    q, cache, kl = workloads.mla_decode_inputs(shape, seed=256 + splits, lengths=lens)
+    ref, lref = mla_ref.mla_decode_ref(_f64(q), _f64(cache), 512, kv_len=np.array(lens), scale=shape.scale)
+    o, lse = gqa.mla_decode(q.cuda(), cache.cuda(), kv_len=lens, scale=shape.scale, num_splits=splits,
+                            return_lse=True)
+    assert gqa.get_device_error() == 0
+    assert_bf16_close(_f64(o), ref, f"mla h_q=256 splits={splits}")
+    assert np.abs(lse.cpu().double().numpy() - lref).max() < 2e-2
+
+
+def test_mla_decode_128_heads_query_position_inside_the_cache():
+    import kv_cache_attention_gqa_b200 as gqa
+
+    shape = workloads.MlaShape(B=3, h_q=128, T_max=1000)
+    q, cache, _ = workloads.mla_decode_inputs(shape, seed=5, nan_tail=False)
+    q_pos = np.array([0, 611, 64], np.int32)
+    ref, _ = mla_ref.mla_decode_ref(_f64(q), _f64(cache), 512, q_pos=q_pos, scale=shape.scale)
+    for splits in (5, 0):
+        o = gqa.mla_decode(q.cuda(), cache.cuda(), q_pos=q_pos.tolist(), scale=shape.scale, num_splits=splits)
+        assert gqa.get_device_error() == 0
+        assert_bf16_close(_f64(o), ref, f"mla 128 heads q_pos splits={splits}")

@@ -480,12 +480,18 @@ gqa_status gqa_mla_decode(const void* q, const void* cache, void* o, float* lse,
   const uint64_t strides[1] = {(uint64_t)d_qk * 2};
   const uint32_t cbox[2] = {64, 64};
   const uint32_t qbox[2] = {64, 16};
-  const uint32_t qbox_tc[2] = {64, 128};  // the tensor-core kernel: 128 heads, 32-key tiles
-  const uint32_t cbox_tc[2] = {64, 32};
+  // The tensor-core kernel reads rows as (64 columns, rows, 9 column chunks): one copy brings a
+  // tile's chunks (the chunk dimension outermost in shared memory, one 128-byte row per key and
+  // chunk) -- 32-key cache tiles, and the query's last 3 chunks of 128 heads.
+  const uint64_t cdims3[3] = {64, (uint64_t)B * T_max, (uint64_t)d_qk / 64};
+  const uint64_t qdims3[3] = {64, (uint64_t)B * h_q, (uint64_t)d_qk / 64};
+  const uint64_t strides3[2] = {(uint64_t)d_qk * 2, 128};
+  const uint32_t cbox_tc[3] = {64, 32, (uint32_t)d_qk / 64};
+  const uint32_t qbox_tc[3] = {64, 128, 3};
   if (!encode_bf16(&maps[0], cache, 2, cdims, strides, cbox) ||
       !encode_bf16(&maps[1], q, 2, qdims, strides, qbox) ||
-      (tc && (!encode_bf16(&maps[2], q, 2, qdims, strides, qbox_tc) ||
-              !encode_bf16(&maps[3], cache, 2, cdims, strides, cbox_tc))))
+      (tc && (!encode_bf16(&maps[2], q, 3, qdims3, strides3, qbox_tc) ||
+              !encode_bf16(&maps[3], cache, 3, cdims3, strides3, cbox_tc))))
     return GQA_ERR_CUDA;
   return from_cuda(launch_mla_bf16(a, maps, s));
 }

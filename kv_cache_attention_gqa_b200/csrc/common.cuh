@@ -106,6 +106,12 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigne
 // ---------------------------------------------------------------------------------------------
 // TMA (cp.async.bulk.tensor), no multicast
 // ---------------------------------------------------------------------------------------------
+// Ask for `bytes` of global memory at `p` to be brought into L2 (both 16-byte aligned/multiples);
+// nothing waits for it.
+__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(__cvta_generic_to_global(p)), "r"(bytes)
+               : "memory");
+}
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }

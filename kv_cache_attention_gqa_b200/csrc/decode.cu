@@ -317,11 +317,10 @@ __device__ __forceinline__ float ex2(float x) {
 
 // Running-maximum merge of the partials of one row. Each lane owns kV consecutive columns
 // (kV = 4: 16-byte loads; lanes past d_h idle) and keeps kU pieces' loads in flight.
-template <typename OutT, bool kFast, int kV>
+template <typename OutT, bool kFast, int kV, int kU>
 __device__ __forceinline__ void merge_row(const KArgs& a, int lane, int unit, int h,
                                           long long c0, long long c1, long long out_base,
                                           long long lse_index, int col_base) {
-  constexpr int kU = 16;
   const int D = a.D;
   const int col0 = col_base + lane * kV;
   const bool active = col0 < D;
@@ -371,8 +370,13 @@ __device__ __forceinline__ void merge_row(const KArgs& a, int lane, int unit, in
 // Rows wider than 256 (the MLA latent) are merged by one warp per 128-column slice.
 __host__ __device__ inline int merge_slices(int D) { return D > 256 ? (D + 127) / 128 : 1; }
 
-template <typename OutT, bool kFast>
-__global__ void __launch_bounds__(256) merge_kernel(KArgs a) {
+// Merge paths by row width, one kernel each so that each carries only its own registers (the
+// 8-column path keeps twice the loads in flight): 0 for d <= 128 (4 columns per lane), 1 for
+// d <= 256 (8, lane-strided), 2 for wider rows (4 columns per lane, one warp per 128-column slice).
+__host__ __device__ inline int merge_path(int D) { return D % 4 == 0 && D <= 128 ? 0 : D <= 256 ? 1 : 2; }
+
+template <typename OutT, bool kFast, int kPath>
+__global__ void __launch_bounds__(256, kPath == 2 ? 4 : 1) merge_kernel(KArgs a) {
   // The row's place (unit, head, output offsets) depends only on the arguments, so it is worked
   // out before the wait (units number fewer than 2^31: B * h_q is below it).
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -386,14 +390,26 @@ __global__ void __launch_bounds__(256) merge_kernel(KArgs a) {
   const int b = unit / UPB, ui = unit - b * UPB;
   const int g = ui / a.hblocks, hb = ui - g * a.hblocks;
   const int nh = min(a.hpu, a.r - hb * a.hpu);
+  // The chunk size and the length and prefix of the block's sequences (its 8 rows span at most
+  // 8 of them) are loaded once per block, one round trip, into shared memory: every warp loading
+  // its own made a few addresses hot (thousands of warps requesting the same words).
+  __shared__ long long s_pre[8];
+  __shared__ int s_n[8];
+  __shared__ long long s_C;
+  const long long row_first = udiv((long long)blockIdx.x * 8, slices);
+  const int b_first = (int)udiv(udiv(row_first, a.hpu), UPB);
   pdl_wait();  // the decode grid has completed and its writes are visible
   if (blockIdx.x == 0 && threadIdx.x == 0) a.hdr->ticket = 0;  // ready for the next call
+  if (threadIdx.x < 8 && b_first + (int)threadIdx.x < a.B) {
+    s_n[threadIdx.x] = __ldcg(&a.nlen[b_first + threadIdx.x]);
+    s_pre[threadIdx.x] = __ldcg(&a.pre[b_first + threadIdx.x]);
+  }
+  if (threadIdx.x == 32) s_C = __ldcg(&a.hdr->chunk);
+  __syncthreads();
   if (row >= rows || h >= nh) return;
-  // the chunk size, the unit's length and its sequence's prefix: three independent loads, one
-  // round trip
-  const long long C = __ldcg(&a.hdr->chunk);
-  const int n = __ldcg(&a.nlen[b]);
-  const long long pre_b = __ldcg(&a.pre[b]);
+  const long long C = s_C;
+  const int n = s_n[b - b_first];
+  const long long pre_b = s_pre[b - b_first];
   if (n == 0) return;
   const long long ng = (n + a.gran - 1) / a.gran;
   const long long P = pre_b * UPB + (long long)ui * ng;
@@ -402,9 +418,9 @@ __global__ void __launch_bounds__(256) merge_kernel(KArgs a) {
   const int head = g * a.r + hb * a.hpu + h;
   const long long ob = ((long long)b * a.h_q + head) * a.D;
   const long long li = (long long)b * a.h_q + head;
-  if (a.D % 4 == 0 && a.D <= 128) merge_row<OutT, kFast, 4>(a, lane, unit, h, c0, c1, ob, li, 0);
-  else if (a.D <= 256) merge_row<OutT, kFast, 8>(a, lane, unit, h, c0, c1, ob, li, 0);  // lane-strided
-  else merge_row<OutT, kFast, 4>(a, lane, unit, h, c0, c1, ob, li, slice * 128);  // wide rows
+  if constexpr (kPath == 0) merge_row<OutT, kFast, 4, 16>(a, lane, unit, h, c0, c1, ob, li, 0);
+  else if constexpr (kPath == 1) merge_row<OutT, kFast, 8, 16>(a, lane, unit, h, c0, c1, ob, li, 0);
+  else merge_row<OutT, kFast, 4, 8>(a, lane, unit, h, c0, c1, ob, li, slice * 128);
 }
 
 // =============================================================================================
@@ -1344,35 +1360,45 @@ __global__ void __launch_bounds__(MlaTcCfg::kThreads, 1)
           const int slot = pc.n_pieces == 1 ? -1 : chunk + pc.unit;
           const int row0 = pc.b * a.T_max;
           const int qrow = pc.b * a.h_q + pc.hb * kMlaTcHeads;
+          const int ntiles = (pc.k1 - pc.k0 + kMlaTcKeys - 1) / kMlaTcKeys;
+          // the piece's 128 query rows (contiguous) into L2 now: the softmax warps read their
+          // first 384 columns with plain loads once the previous piece is done
+          prefetch_l2(reinterpret_cast<const uint8_t*>(a.q) + (long long)qrow * (kMlaDqk * 2),
+                      (uint32_t)(kMlaTcHeads * kMlaDqk * 2));
+          // tile i of the piece: all 9 column chunks in one 3-D copy (chunk-major in the stage)
+          auto issue_tile = [&](int i) -> bool {
+            if (!mbar_wait(bar(C::kEmpty + stage), phase ^ 1u, a.err)) return false;
+            const int t = pc.k0 + i * kMlaTcKeys;
+            TileMeta m;
+            m.b = pc.b;
+            m.g = 0;
+            m.hb = pc.hb;
+            m.nvalid = min(kMlaTcKeys, pc.k1 - t);
+            m.flags = (i == 0 ? kFirst : 0) | (i == ntiles - 1 ? kLast : 0);
+            m.slot = slot;
+            m.nh = kMlaTcHeads;
+            m.nskip = 0;
+            meta[stage] = m;
+            mbar_arrive_expect_tx(bar(C::kFull + stage), (uint32_t)C::kTileBytes);
+            tma_load_3d(sC(stage), &tmc, bar(C::kFull + stage), 0, row0 + t, 0);
+            ++issued;
+            if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
+            return true;
+          };
+          // Up to kStages tiles of a later piece go out before its query: the stages they take
+          // were held by earlier pieces' tiles, whose consumption needs nothing of this piece.
+          const int early = pieces > 0 ? min(C::kStages, ntiles) : 0;
+          for (int i = 0; i < early && ok; ++i) ok = issue_tile(i);
+          if (!ok) break;
           // The previous piece's MMAs (the last readers of the query buffers) are complete, and
           // every consumer has passed its piece start (so no barrier phase below is skipped).
           if (pieces > 0 && !(ok = mbar_wait(bar(C::kPieceDone), (uint32_t)((pieces - 1) & 1), a.err))) break;
           *qrow_slot = qrow;
           mbar_arrive(bar(C::kQInfo));  // the softmax warps start the query's TMEM copy now
           mbar_arrive_expect_tx(bar(C::kQFull), (uint32_t)C::kQBytes);
-#pragma unroll
-          for (int ch = 0; ch < C::kQSmemCh; ++ch)
-            tma_load_2d(sQ + ch * C::kQChunkBytes, &tmq, bar(C::kQFull), (C::kQTmemCh + ch) * 64, qrow);
+          tma_load_3d(sQ, &tmq, bar(C::kQFull), 0, qrow, C::kQTmemCh);
           ++pieces;
-          for (int t = pc.k0; t < pc.k1; t += kMlaTcKeys) {
-            if (!(ok = mbar_wait(bar(C::kEmpty + stage), phase ^ 1u, a.err))) break;
-            TileMeta m;
-            m.b = pc.b;
-            m.g = 0;
-            m.hb = pc.hb;
-            m.nvalid = min(kMlaTcKeys, pc.k1 - t);
-            m.flags = (t == pc.k0 ? kFirst : 0) | (t + kMlaTcKeys >= pc.k1 ? kLast : 0);
-            m.slot = slot;
-            m.nh = kMlaTcHeads;
-            m.nskip = 0;
-            meta[stage] = m;
-            mbar_arrive_expect_tx(bar(C::kFull + stage), (uint32_t)C::kTileBytes);
-#pragma unroll
-            for (int ch = 0; ch < C::kNch; ++ch)
-              tma_load_2d(sC(stage) + ch * C::kChunkBytes, &tmc, bar(C::kFull + stage), ch * 64, row0 + t);
-            ++issued;
-            if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
-          }
+          for (int i = early; i < ntiles && ok; ++i) ok = issue_tile(i);
           x = pc.end;
         }
       }
@@ -1478,46 +1504,45 @@ __global__ void __launch_bounds__(MlaTcCfg::kThreads, 1)
     const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
     const int et = (warp - 2) * 32 + lane;  // 0..127, for the V-row zeroing
     const float sl2 = a.scale * kLog2e;
+    // this head's query columns [0, 384) -> TMEM, two 64-column chunks per round of loads; the
+    // caller has seen every score of the previous piece, so no MMA still reads these columns
+    auto copy_query = [&](int qrow) {
+      const uint4* qg = reinterpret_cast<const uint4*>(a.q) + (long long)(qrow + row) * (kMlaDqk / 8);
+#pragma unroll
+      for (int bc = 0; bc < C::kQTmemCh; bc += 2) {
+        uint4 v[16];
+#pragma unroll
+        for (int u = 0; u < 16; ++u) v[u] = __ldg(qg + bc * 8 + u);
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          uint32_t r[32];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            r[4 * u] = v[8 * c + u].x;
+            r[4 * u + 1] = v[8 * c + u].y;
+            r[4 * u + 2] = v[8 * c + u].z;
+            r[4 * u + 3] = v[8 * c + u].w;
+          }
+          tc::st32(lane_addr + C::kColQ + (bc + c) * 32, r);
+        }
+      }
+      tc::wait_st();
+      tc::fence_before_sync();
+      mbar_arrive(bar(C::kQTmem));
+    };
     int stage = 0, jg = 0, piece = 0;
     uint32_t phase = 0;
-    bool ok = true;
-    while (ok) {
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(C::kQInfo), (uint32_t)(piece & 1), a.err));
-      if (!ok) break;
-      const int qrow = *qrow_slot;
-      if (qrow < 0) break;
-      // this head's query columns [0, 384) -> TMEM, two 64-column chunks per round of loads (the
-      // previous piece's scores are all read, so no MMA still reads these columns)
-      {
-        const uint4* qg = reinterpret_cast<const uint4*>(a.q) + (long long)(qrow + row) * (kMlaDqk / 8);
-#pragma unroll
-        for (int bc = 0; bc < C::kQTmemCh; bc += 2) {
-          uint4 v[16];
-#pragma unroll
-          for (int u = 0; u < 16; ++u) v[u] = __ldg(qg + bc * 8 + u);
-#pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            uint32_t r[32];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-              r[4 * u] = v[8 * c + u].x;
-              r[4 * u + 1] = v[8 * c + u].y;
-              r[4 * u + 2] = v[8 * c + u].z;
-              r[4 * u + 3] = v[8 * c + u].w;
-            }
-            tc::st32(lane_addr + C::kColQ + (bc + c) * 32, r);
-          }
-        }
-        tc::wait_st();
-        tc::fence_before_sync();
-        mbar_arrive(bar(C::kQTmem));
-      }
+    bool ok = __all_sync(0xffffffffu, mbar_wait(bar(C::kQInfo), 0u, a.err));
+    int qrow = ok ? *qrow_slot : -1;
+    if (qrow >= 0) copy_query(qrow);
+    while (qrow >= 0) {
       float m_run = -INFINITY, l_run = 0.f;
       bool last = false;
+      TileMeta m;
       while (!last) {
         ok = __all_sync(0xffffffffu, mbar_wait(bar(C::kFull + stage), phase, a.err));
         if (!ok) break;
-        const TileMeta m = meta[stage];
+        m = meta[stage];
         const bool first = (m.flags & kFirst) != 0;
         last = (m.flags & kLast) != 0;
         // ---- scores of this tile
@@ -1592,47 +1617,72 @@ __global__ void __launch_bounds__(MlaTcCfg::kThreads, 1)
         tc::fence_proxy_async_smem();
         tc::fence_before_sync();
         mbar_arrive(bar(C::kPFull));
-        if (last) {
-          // ---- piece end: O / l -> the output (one piece) or a partial, this CTA's columns
-          ok = __all_sync(0xffffffffu, mbar_wait(bar(C::kPvDone), (uint32_t)(jg & 1), a.err));
-          if (!ok) break;
-          tc::fence_after_sync();
-          const float inv = 1.f / l_run;
-          const float lse2 = m_run + __log2f(l_run);
-          const int head = m.hb * kMlaTcHeads + row;
-#pragma unroll 1
-          for (int c = 0; c < C::kHalf / 32; ++c) {
-            float o[32];
-            tc::ld32f(lane_addr + C::kColO + c * 32, o);
-            tc::wait_ld();
-            const int col = half * C::kHalf + c * 32;
-            if (m.slot < 0) {
-              uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.o) +
-                                                    ((long long)m.b * a.h_q + head) * kMlaDv + col);
-#pragma unroll
-              for (int q = 0; q < 4; ++q)
-                dst[q] = make_uint4(pack_bf16x2(o[8 * q] * inv, o[8 * q + 1] * inv),
-                                    pack_bf16x2(o[8 * q + 2] * inv, o[8 * q + 3] * inv),
-                                    pack_bf16x2(o[8 * q + 4] * inv, o[8 * q + 5] * inv),
-                                    pack_bf16x2(o[8 * q + 6] * inv, o[8 * q + 7] * inv));
-            } else {
-              float4* dst = reinterpret_cast<float4*>(a.part_o + ((long long)m.slot * a.hpu + row) * kMlaDv + col);
-#pragma unroll
-              for (int q = 0; q < 8; ++q)
-                dst[q] = make_float4(o[4 * q] * inv, o[4 * q + 1] * inv, o[4 * q + 2] * inv, o[4 * q + 3] * inv);
-            }
-          }
-          if (half == 0) {
-            if (m.slot < 0) {
-              if (a.lse) a.lse[(long long)m.b * a.h_q + head] = lse2 * kLn2;
-            } else {
-              a.part_lse[(long long)m.slot * a.hpu + row] = lse2;
-            }
-          }
-        }
         ++jg;
         if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
       }
+      if (!ok) break;
+      // The next piece's query goes into TMEM first (this piece's scores are all read), so its
+      // first scores run while this piece's output is written out.
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(C::kQInfo), (uint32_t)((piece + 1) & 1), a.err));
+      const int next = ok ? *qrow_slot : -1;
+      if (next >= 0) copy_query(next);
+      // ---- piece end: O / l -> the output (one piece) or a partial, this CTA's columns; the
+      // next piece's first P V, which overwrites the accumulator, waits for this warp's P
+      const bool done = __all_sync(0xffffffffu, mbar_wait(bar(C::kPvDone), (uint32_t)((jg - 1) & 1), a.err));
+      if (done) {
+        tc::fence_after_sync();
+        const float inv = 1.f / l_run;
+        const float lse2 = m_run + __log2f(l_run);
+        const int head = m.hb * kMlaTcHeads + row;
+#pragma unroll 1
+        for (int c = 0; c < C::kHalf / 32; ++c) {
+          float o[32];
+          tc::ld32f(lane_addr + C::kColO + c * 32, o);
+          tc::wait_ld();
+          const int col = half * C::kHalf + c * 32;
+          if (m.slot < 0) {
+            uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.o) +
+                                                  ((long long)m.b * a.h_q + head) * kMlaDv + col);
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              dst[q] = make_uint4(pack_bf16x2(o[8 * q] * inv, o[8 * q + 1] * inv),
+                                  pack_bf16x2(o[8 * q + 2] * inv, o[8 * q + 3] * inv),
+                                  pack_bf16x2(o[8 * q + 4] * inv, o[8 * q + 5] * inv),
+                                  pack_bf16x2(o[8 * q + 6] * inv, o[8 * q + 7] * inv));
+          } else {
+            // The warp's 32 rows x 32 columns pass through its quarter of the P buffer (free: the
+            // piece's last P V has completed; 128-byte rows, 16-byte units swizzled by row), so
+            // each store below writes 128 contiguous bytes of 4 rows, not 16 bytes of 32.
+            const uint32_t stg = sP + quarter * 4096;
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+              asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(stg + lane * 128 + ((u ^ (lane & 7)) << 4)),
+                           "f"(o[4 * u] * inv), "f"(o[4 * u + 1] * inv), "f"(o[4 * u + 2] * inv), "f"(o[4 * u + 3] * inv)
+                           : "memory");
+            __syncwarp();
+            float* rows = a.part_o + ((long long)m.slot * a.hpu + quarter * 32) * kMlaDv + col;
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+              const int r = k * 4 + (lane >> 3), u = lane & 7;
+              float4 v;
+              asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                           : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                           : "r"(stg + r * 128 + ((u ^ (r & 7)) << 4)));
+              *reinterpret_cast<float4*>(rows + (long long)r * kMlaDv + u * 4) = v;
+            }
+            __syncwarp();
+          }
+        }
+        if (half == 0) {
+          if (m.slot < 0) {
+            if (a.lse) a.lse[(long long)m.b * a.h_q + head] = lse2 * kLn2;
+          } else {
+            a.part_lse[(long long)m.slot * a.hpu + row] = lse2;
+          }
+        }
+      }
+      if (!done) break;
+      qrow = next;
       ++piece;
     }
   }
@@ -1757,13 +1807,17 @@ cudaError_t launch_merge(const KArgs& ka, cudaStream_t s) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, merge_kernel<OutT, kFast>, ka);
+  const int path = merge_path(ka.D);
+  void (*kern)(KArgs) = path == 0 ? merge_kernel<OutT, kFast, 0>
+                        : path == 1 ? merge_kernel<OutT, kFast, 1>
+                                    : merge_kernel<OutT, kFast, 2>;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, ka);
   if (e != cudaSuccess) {
     // programmatic dependent launch refused (e.g. on a stream that does not support it): fall
     // back to an ordinary launch ordered after the decode kernel
     (void)cudaGetLastError();
     cfg.numAttrs = 0;
-    e = cudaLaunchKernelEx(&cfg, merge_kernel<OutT, kFast>, ka);
+    e = cudaLaunchKernelEx(&cfg, kern, ka);
   }
   return e;
 }

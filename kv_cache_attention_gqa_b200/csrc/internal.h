@@ -127,8 +127,9 @@ cudaError_t launch_decode_fp32(const DecodeArgs& a, cudaStream_t s);
 // [2] = queries as (d_h, B*h_q) with box (64, 16 or 32 rows: 32 when r > 16); SWIZZLE_128B.
 cudaError_t launch_decode_bf16(const DecodeArgs& a, const CUtensorMap* tmaps, cudaStream_t s);
 // MLA (bf16, d_h = 576, d_v = 512): tmaps [0] = the cache as (576, B*T_max) with box (64, 64),
-// [1] = the queries as (576, B*h_q) with box (64, 16); when a.mla_tc, [2] the queries with box
-// (64, 128) and [3] the cache with box (64, 32); SWIZZLE_128B.
+// [1] = the queries as (576, B*h_q) with box (64, 16); when a.mla_tc, [2] the queries and [3]
+// the cache as (64, rows, 9 chunks) with strides (1152, 128) bytes and boxes (64, 128, 3) and
+// (64, 32, 9); SWIZZLE_128B.
 cudaError_t launch_mla_bf16(const DecodeArgs& a, const CUtensorMap* tmaps, cudaStream_t s);
 int mla_dims_supported_bf16(int d_qk, int d_v);
 // 1 when gqa_mla_decode runs the tensor-core kernel for this head count and dtype

@@ -1277,11 +1277,12 @@ struct MlaTcCfg {
   static constexpr int kQChunkBytes = kMlaTcHeads * 128;   // 128 rows x 128 B
   static constexpr int kQBytes = kQSmemCh * kQChunkBytes;  // 48 KiB
   static constexpr int kPBytes = kMlaTcHeads * 128;        // 128 rows of 128 B; a tile's P uses 64 B
-  static constexpr int kThreads = 192;
-  static constexpr uint32_t kColS = 0, kColO = 64, kColQ = 320;
+  static constexpr int kThreads = 224;
+  static constexpr int kKSplit = 18;  // k-steps of S issued by warp 1; warp 6 issues the other 18
+  static constexpr uint32_t kColS = 0, kColS2 = 32, kColO = 64, kColQ = 320;
   static constexpr int kHalf = kMlaDv / 2;                 // latent columns per CTA
-  enum { kFull = 0, kEmpty = kFull + kStages, kQInfo = kEmpty + kStages, kQFull, kQTmem, kSFull, kSFree,
-         kPFull, kPvDone, kPieceDone, kAll, kBars };
+  enum { kFull = 0, kEmpty = kFull + kStages, kQInfo = kEmpty + kStages, kQFull, kQTmem, kSFull, kSFull2,
+         kSFree, kPFull, kPvDone, kPieceDone, kAll, kAll2, kBars };
   static constexpr size_t kOffQ = (size_t)kStages * kTileBytes;
   static constexpr size_t kOffP = kOffQ + kQBytes;
   static constexpr size_t kOffPre = kOffP + kPBytes;
@@ -1323,11 +1324,13 @@ __global__ void __launch_bounds__(MlaTcCfg::kThreads, 1)
     mbar_init(bar(C::kQFull), 1);
     mbar_init(bar(C::kQTmem), 128);
     mbar_init(bar(C::kSFull), 1);
+    mbar_init(bar(C::kSFull2), 1);
     mbar_init(bar(C::kSFree), 128);
     mbar_init(bar(C::kPFull), 128);
     mbar_init(bar(C::kPvDone), 1);
     mbar_init(bar(C::kPieceDone), 1);
     mbar_init(bar(C::kAll), 1);
+    mbar_init(bar(C::kAll2), 1);
     fence_barrier_init();
   }
   if (warp == 0 && lane == 0) {
@@ -1428,17 +1431,13 @@ __global__ void __launch_bounds__(MlaTcCfg::kThreads, 1)
     auto wait = [&](int b_, uint32_t parity) {
       return __all_sync(0xffffffffu, mbar_wait(bar(b_), parity, a.err));
     };
-    auto issue_s = [&](int st) {  // S = Q C^T over all 576 columns of the tile in stage st
-      const uint64_t dc = tc::smem_desc(sC(st), 16, 1024), dq = tc::smem_desc(sQ, 16, 1024);
+    auto issue_s = [&](int st) {  // S_a = Q C^T over the tile's columns [0, 288) (query from TMEM)
+      const uint64_t dc = tc::smem_desc(sC(st), 16, 1024);
       if (tc::elect_one()) {
 #pragma unroll
-        for (int k = 0; k < 4 * C::kQTmemCh; ++k)  // query columns [0, 384) from TMEM
+        for (int k = 0; k < C::kKSplit; ++k)
           tc::mma_ts(tmem + C::kColS, tmem + C::kColQ + k * 8, dc + tc::koff(k, C::kChunkBytes), idesc_s,
                      k > 0 ? 1u : 0u);
-#pragma unroll
-        for (int k = 0; k < 4 * C::kQSmemCh; ++k)  // [384, 576) from shared memory
-          tc::mma_ss(tmem + C::kColS, dq + tc::koff(k, C::kQChunkBytes),
-                     dc + tc::koff(4 * C::kQTmemCh + k, C::kChunkBytes), idesc_s, 1u);
         tc::commit(bar(C::kSFull));
       }
       __syncwarp();
@@ -1497,6 +1496,47 @@ __global__ void __launch_bounds__(MlaTcCfg::kThreads, 1)
     if (tc::elect_one()) tc::commit(bar(C::kAll));
     __syncwarp();
     mbar_wait(bar(C::kAll), 0, a.err);
+  } else if (warp == 6) {
+    // ------------------------------ second score issuer (one elected lane) ---------------------
+    // S_b = Q C^T over the tile's columns [288, 576): an MMA issue returns only after tens of
+    // cycles, so at N = 32 one thread issuing all 36 k-steps left the tensor pipe mostly idle; two
+    // threads issue half each, into separate accumulators that the softmax warps add.
+    constexpr uint32_t idesc_s = tc::idesc_bf16(128, kMlaTcKeys, false);
+    auto wait = [&](int b_, uint32_t parity) {
+      return __all_sync(0xffffffffu, mbar_wait(bar(b_), parity, a.err));
+    };
+    int stage = 0, jg = 0, piece = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    while (ok) {
+      if (!(ok = wait(C::kFull + stage, phase))) break;
+      const TileMeta m = meta[stage];
+      if (m.flags & kEnd) break;
+      if (m.flags & kFirst) {
+        if (!(ok = wait(C::kQFull, (uint32_t)(piece & 1)) && wait(C::kQTmem, (uint32_t)(piece & 1)))) break;
+      }
+      if (jg > 0 && !(ok = wait(C::kSFree, (uint32_t)((jg - 1) & 1)))) break;  // S_b(jg - 1) read
+      tc::fence_after_sync();
+      const uint64_t dc = tc::smem_desc(sC(stage), 16, 1024), dq = tc::smem_desc(sQ, 16, 1024);
+      if (tc::elect_one()) {
+#pragma unroll
+        for (int k = C::kKSplit; k < 4 * C::kQTmemCh; ++k)  // query columns [288, 384) from TMEM
+          tc::mma_ts(tmem + C::kColS2, tmem + C::kColQ + k * 8, dc + tc::koff(k, C::kChunkBytes), idesc_s,
+                     k > C::kKSplit ? 1u : 0u);
+#pragma unroll
+        for (int k = 0; k < 4 * C::kQSmemCh; ++k)  // [384, 576) from shared memory
+          tc::mma_ss(tmem + C::kColS2, dq + tc::koff(k, C::kQChunkBytes),
+                     dc + tc::koff(4 * C::kQTmemCh + k, C::kChunkBytes), idesc_s, 1u);
+        tc::commit(bar(C::kSFull2));
+      }
+      __syncwarp();
+      if (m.flags & kLast) ++piece;
+      ++jg;
+      if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
+    }
+    if (tc::elect_one()) tc::commit(bar(C::kAll2));
+    __syncwarp();
+    mbar_wait(bar(C::kAll2), 0, a.err);
   } else {
     // ------------------------------ softmax: one head (TMEM lane) per thread --------------------
     const int quarter = warp & 3;
@@ -1546,12 +1586,16 @@ __global__ void __launch_bounds__(MlaTcCfg::kThreads, 1)
         const bool first = (m.flags & kFirst) != 0;
         last = (m.flags & kLast) != 0;
         // ---- scores of this tile
-        ok = __all_sync(0xffffffffu, mbar_wait(bar(C::kSFull), (uint32_t)(jg & 1), a.err));
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(C::kSFull), (uint32_t)(jg & 1), a.err) &&
+                                         mbar_wait(bar(C::kSFull2), (uint32_t)(jg & 1), a.err));
         if (!ok) break;
         tc::fence_after_sync();
-        float s[kMlaTcKeys];
+        float s[kMlaTcKeys], s2[kMlaTcKeys];
         tc::ld32f(lane_addr + C::kColS, s);
+        tc::ld32f(lane_addr + C::kColS2, s2);
         tc::wait_ld();
+#pragma unroll
+        for (int i = 0; i < kMlaTcKeys; ++i) s[i] += s2[i];
         tc::fence_before_sync();
         mbar_arrive(bar(C::kSFree));  // the next tile's scores may overwrite them
         const int nvalid = m.nvalid;

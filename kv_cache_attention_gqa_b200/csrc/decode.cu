@@ -127,6 +127,7 @@ struct KArgs {
   int n_max;       // upper bound on the number of chunks (workspace slots)
   int auto_chunk;  // 1: chunks hold at least min_chunk keys
   int min_chunk;   // keys
+  int align_units;  // 1: when every unit has the same length, chunks do not straddle units
   int window;      // 0: none; W > 0: the query at q_pos sees keys q_pos - W < j <= q_pos
   Header* hdr;
   long long* pre;
@@ -226,12 +227,16 @@ __device__ void build_plan(const KArgs& a, Plan& p, long long* pre, int* nlen, i
     wlo[b] = lo;
   }
   cta_sync();
-  // ... then one warp turns them into prefix sums in granules, from shared memory
+  // ... then one warp turns them into prefix sums in granules, from shared memory (and notes
+  // whether every sequence has the same visible length)
+  __shared__ int s_same_len;
   if (warp == w0) {
     long long run = 0;
+    bool same = true;
     for (int base = 0; base < a.B; base += 32) {
       const int b = base + lane;
       const long long ngr = b < a.B ? (nlen[b] + a.gran - 1) / a.gran : 0;  // granules
+      same = same && __all_sync(0xffffffffu, b >= a.B || nlen[b] == nlen[0]);
       long long s = ngr;  // inclusive warp scan
 #pragma unroll
       for (int off = 1; off < 32; off <<= 1) {
@@ -241,7 +246,10 @@ __device__ void build_plan(const KArgs& a, Plan& p, long long* pre, int* nlen, i
       if (b < a.B) pre[b] = run + s - ngr;
       run += __shfl_sync(0xffffffffu, s, 31);
     }
-    if (lane == 0) pre[a.B] = run;
+    if (lane == 0) {
+      pre[a.B] = run;
+      s_same_len = same ? 1 : 0;
+    }
   }
   cta_sync();
   p.pre = pre;
@@ -258,6 +266,20 @@ __device__ void build_plan(const KArgs& a, Plan& p, long long* pre, int* nlen, i
     if (C < lo) C = lo;
   }
   if (C < 1) C = 1;
+  if (a.align_units && s_same_len && nlen[0] > 0) {
+    // Every unit has the same length N (in granules): cut each into m equal chunks, m dividing N
+    // and as large as the chunk bound allows (down to half of it), so that no chunk holds the end
+    // of one unit and the start of the next (a second piece costs a CTA its start-up again).
+    const long long N = (nlen[0] + a.gran - 1) / a.gran;
+    const long long units = (long long)a.B * p.UPB;
+    const long long m_hi = udiv(a.n_max, units);
+    for (long long m = m_hi; m >= 1 && 2 * m >= m_hi; --m) {
+      if (N % m == 0 && N / m >= C) {
+        C = N / m;
+        break;
+      }
+    }
+  }
   p.C = C;
   p.n_chunks = (int)udiv(p.K + C - 1, C);
 
@@ -1963,6 +1985,9 @@ KArgs make_kargs(const DecodeArgs& a) {
   // small against the chunk's K/V bytes; the tensor-core MLA kernel is bound by its MMAs instead
   // and wants every pair of SMs busy
   k.min_chunk = a.mla_tc ? kMlaTcMinChunk : (16 * L.hpu > kMinChunkAuto ? 16 * L.hpu : kMinChunkAuto);
+  // the compute-bound tensor-core MLA kernel gives up a few idle SMs for chunks that never hold
+  // two pieces; the HBM-bound kernels keep every SM streaming
+  k.align_units = a.mla_tc && auto_chunk ? 1 : 0;
   k.window = a.window;
   uint8_t* ws = reinterpret_cast<uint8_t*>(a.workspace);
   k.hdr = reinterpret_cast<Header*>(ws);

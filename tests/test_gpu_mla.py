@@ -135,3 +135,18 @@ def test_mla_decode_128_heads_query_position_inside_the_cache():
         o = gqa.mla_decode(q.cuda(), cache.cuda(), q_pos=q_pos.tolist(), scale=shape.scale, num_splits=splits)
         assert gqa.get_device_error() == 0
         assert_bf16_close(_f64(o), ref, f"mla 128 heads q_pos splits={splits}")
+
+
+def test_mla_decode_128_heads_equal_lengths_aligned_chunks():
+    """Every sequence at the same length (1000 keys, 4 sequences): the automatic plan cuts each
+    unit into equal chunks that never straddle two sequences (here 2 chunks of 500 keys each, not
+    16 of 256), so every CTA pair has one piece and every row two partials."""
+    import kv_cache_attention_gqa_b200 as gqa
+
+    shape = workloads.MlaShape(B=4, h_q=128, T_max=1000)
+    q, cache, kl = workloads.mla_decode_inputs(shape, seed=11)
+    ref, lref = mla_ref.mla_decode_ref(_f64(q), _f64(cache), 512, kv_len=kl.numpy(), scale=shape.scale)
+    o, lse = gqa.mla_decode(q.cuda(), cache.cuda(), kv_len=kl.cuda(), scale=shape.scale, return_lse=True)
+    assert gqa.get_device_error() == 0
+    assert_bf16_close(_f64(o), ref, "mla 128 heads, equal lengths")
+    assert np.abs(lse.cpu().double().numpy() - lref).max() < 2e-2

@@ -320,11 +320,11 @@ const char* gqa_version(void);
  * gqa_debug_expire_waits - failure-detection test hook; never needed in normal use.
  * Every pipeline wait of the kernels is bounded (about 2 s of %globaltimer); when one runs out the
  * kernel records GQA_DEVERR_TIMEOUT and returns instead of spinning, so the context stays usable.
- * With enable = 1, every later bf16 gqa_prefill and contiguous bf16 gqa_decode on any device makes
- * CTA 0 wait on a barrier that nothing signals, so that bound is reached on purpose: the call
- * takes about 2 s longer, the error word reads GQA_DEVERR_TIMEOUT, prefill writes the rows of the
- * tile that gave up as zeros (lse = -inf), and decode leaves the rows of CTA 0's first chunk
- * unspecified. A following call with the hook off is unaffected (a decode workspace stays
+ * With enable = 1, every later bf16 gqa_prefill, contiguous bf16 gqa_decode and tensor-core
+ * gqa_mla_decode (bf16, a multiple of 128 heads) on any device makes CTA 0 wait on a barrier that
+ * nothing signals, so that bound is reached on purpose: the call takes about 2 s longer, the error
+ * word reads GQA_DEVERR_TIMEOUT, prefill writes the rows of the tile that gave up as zeros
+ * (lse = -inf), and decode and MLA decode leave the rows of CTA 0's first chunk unspecified. A following call with the hook off is unaffected (a decode workspace stays
  * reusable). enable = 0 (the default) turns it off. Other calls ignore it. Not thread-safe with
  * respect to concurrent launches: set it only while no other thread calls the library.
  * Errors: INVALID_ARG (enable not 0 or 1).

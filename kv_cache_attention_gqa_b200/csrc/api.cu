@@ -19,8 +19,9 @@ namespace {
 
 constexpr int kMaxDevices = 64;
 
-// Test hook set by gqa_debug_expire_waits: the bf16 prefill and the contiguous bf16 decode pass
-// it to their kernels, whose CTA 0 then waits on a barrier that nothing signals.
+// Test hook set by gqa_debug_expire_waits: the bf16 prefill, the contiguous bf16 decode and the
+// tensor-core MLA decode pass it to their kernels, whose CTA 0 then waits on a barrier that nothing
+// signals.
 std::atomic<int> g_expire_waits{0};
 
 unsigned* device_error_ptr() {
@@ -464,6 +465,7 @@ gqa_status gqa_mla_decode(const void* q, const void* cache, void* o, float* lse,
   a.d_v = d_v;
   a.mla = 1;
   a.mla_tc = tc ? 1 : 0;
+  a.expire_wait = g_expire_waits.load(std::memory_order_relaxed);
   a.scale = scale;
   a.window = 0;
   a.workspace = workspace;

@@ -1304,7 +1304,7 @@ struct MlaTcCfg {
   static constexpr uint32_t kColS = 0, kColS2 = 32, kColO = 64, kColQ = 320;
   static constexpr int kHalf = kMlaDv / 2;                 // latent columns per CTA
   enum { kFull = 0, kEmpty = kFull + kStages, kQInfo = kEmpty + kStages, kQFull, kQTmem, kSFull, kSFull2,
-         kSFree, kPFull, kPvDone, kPieceDone, kAll, kAll2, kBars };
+         kSFree, kPFull, kPvDone, kPieceDone, kAll, kAll2, kNever, kBars };
   static constexpr size_t kOffQ = (size_t)kStages * kTileBytes;
   static constexpr size_t kOffP = kOffQ + kQBytes;
   static constexpr size_t kOffPre = kOffP + kPBytes;
@@ -1353,6 +1353,7 @@ __global__ void __launch_bounds__(MlaTcCfg::kThreads, 1)
     mbar_init(bar(C::kPieceDone), 1);
     mbar_init(bar(C::kAll), 1);
     mbar_init(bar(C::kAll2), 1);
+    mbar_init(bar(C::kNever), 1);  // nothing arrives: the expired-wait test hook waits on it
     fence_barrier_init();
   }
   if (warp == 0 && lane == 0) {
@@ -1377,7 +1378,9 @@ __global__ void __launch_bounds__(MlaTcCfg::kThreads, 1)
     if (lane == 0) {
       int stage = 0, issued = 0, pieces = 0;
       uint32_t phase = 0;
-      bool ok = true;
+      // test hook: CTA 0 first waits on a barrier that nothing signals, runs out after the bound
+      // and gives up (its rows are left unspecified; every other role's first wait runs out too)
+      bool ok = !(a.expire_wait && blockIdx.x == 0) || mbar_wait(bar(C::kNever), 0, a.err);
       for (int chunk = (int)(blockIdx.x >> 1); ok && chunk < plan.n_chunks; chunk += pairs) {
         const long long x1 = min((long long)(chunk + 1) * plan.C, plan.K);
         for (long long x = (long long)chunk * plan.C; x < x1 && ok;) {
@@ -2001,7 +2004,7 @@ KArgs make_kargs(const DecodeArgs& a) {
   k.page_size = a.page_size;
   k.num_pages = a.num_pages;
   k.gran = a.block_table ? (a.page_size % kTile == 0 ? kTile : 16) : 1;
-  k.expire_wait = a.block_table || a.mla ? 0 : a.expire_wait;
+  k.expire_wait = a.block_table || (a.mla && !a.mla_tc) ? 0 : a.expire_wait;
   return k;
 }
 

@@ -84,3 +84,28 @@ def test_decode_expired_wait_reports_timeout_and_workspace_stays_usable(splits):
         o = gqa.decode(qd, kd, vd, kv_len=lens.tolist(), num_splits=splits, ws=ws)
         assert gqa.get_device_error() == 0
         assert_bf16_close(_f64(o), ref, f"decode after the expired wait, rep {rep}")
+
+
+def test_mla_tensor_core_expired_wait_reports_timeout():
+    """The tensor-core MLA kernel (128 heads): CTA 0's producer waits on a barrier nothing signals;
+    every other role of that CTA finds its first wait running out as well, the CTA releases its
+    TMEM and ends, the call reports GQA_DEVERR_TIMEOUT, and the next call matches the oracle."""
+    import kv_cache_attention_gqa_b200 as gqa
+    from oracle import mla as mla_ref
+
+    shape = workloads.MlaShape(B=2, h_q=128, T_max=1000)
+    lens = [1000, 700]
+    q, cache, _ = workloads.mla_decode_inputs(shape, seed=43, lengths=lens)
+    ref, _ = mla_ref.mla_decode_ref(_f64(q), _f64(cache), 512, kv_len=np.array(lens), scale=shape.scale)
+    qd, cd = q.cuda(), cache.cuda()
+    assert gqa.get_device_error() == 0
+    gqa.debug_expire_waits(True)
+    try:
+        gqa.mla_decode(qd, cd, kv_len=lens, scale=shape.scale)
+        code = gqa.get_device_error()
+    finally:
+        gqa.debug_expire_waits(False)
+    assert code == 4  # GQA_DEVERR_TIMEOUT
+    o = gqa.mla_decode(qd, cd, kv_len=lens, scale=shape.scale)
+    assert gqa.get_device_error() == 0
+    assert_bf16_close(_f64(o), ref, "MLA decode after the expired wait")

@@ -1272,20 +1272,24 @@ __global__ void __launch_bounds__(MlaCfg::kThreads, 1)
 // =============================================================================================
 // With 128 heads the score and value products are dense enough for tcgen05: the unit's 128
 // heads sit on the 128 TMEM lanes (M = 128) and each 32-key tile of latent rows is the B operand
-//   S  = Q C^T   (M 128, N 32 keys, K 576)   into TMEM columns [0, 32)
+//   S  = Q C^T   (M 128, N 32 keys, K 576)   into TMEM columns [0, 32) and [32, 64) (two halves
+//                                            of the contraction, added by the softmax warps)
 //   O += P C_v   (M 128, N 256, K 32 keys)   into TMEM columns [64, 320)
 // The 512-wide latent accumulator is twice what TMEM holds next to S, so a unit's chunk is run by
 // two CTAs, each owning 256 of the latent columns (d_v half); both compute the same S (the same
 // bits: the same MMAs on the same inputs), and each writes its half of the piece output.
-// TMEM: S [0, 32), O half [64, 320), the query's first 384 columns [320, 512) (the A operand of
+// TMEM: S [0, 64), O half [64, 320), the query's first 384 columns [320, 512) (the A operand of
 // the first 24 k-steps of S); the query's last 192 columns stay in shared memory (the A operand of
 // the other 12). P (bf16) goes to shared memory, so the next tile's S overwrites the scores as soon
 // as the softmax warps have read them and runs while they compute P. The tiles pass through a
 // 4-deep ring of 36 KiB stages, so a tile's copy starts three tiles ahead of its use.
-// Warps: 0 TMA producer, 1 MMA issuer (and TMEM owner), 2..5 softmax, one TMEM lane quarter each
-// (warp w reads lanes 32 (w % 4) ..), one head per thread.
+// Warps: 0 TMA producer; 1 issues k-steps 0-17 of S and P V (and owns TMEM); 6 issues k-steps
+// 18-35 of S (an MMA issue returns only after tens of cycles, and at N = 32 one issuing thread
+// left the tensor pipe mostly idle); 2..5 softmax, one TMEM lane quarter each (warp w reads lanes
+// 32 (w % 4) ..), one head per thread.
 // Chunks: CTAs 2p and 2p + 1 take chunks p, p + G/2, ... of the same split-KV plan as the other
-// decode kernels; partials and the merge kernel are shared with them.
+// decode kernels (with equal-length sequences, chunks that divide each sequence: see the plan);
+// partials and the merge kernel are shared with them.
 constexpr int kMlaTcHeads = 128;
 constexpr int kMlaTcMinChunk = 256;  // keys; the automatic chunking never goes below this
 constexpr int kMlaTcKeys = 32;       // keys per tile

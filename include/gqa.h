@@ -129,8 +129,14 @@ gqa_status gqa_prefill(const void* q, const void* k_cache, const void* v_cache, 
  *   dtype  GQA_BF16: d_qk = 576 and d_v = 512 (the DeepSeek-V2/V3 latent and rotary widths);
  *          GQA_FP32: d_qk <= 768, d_v <= min(d_qk, 512) (check mode).
  *   workspace: >= gqa_mla_decode_workspace_size(B, h_q, T_max, d_v, dtype, num_splits) bytes,
- *          256-byte aligned, zero-filled before first use, as for gqa_decode (same reuse rules).
- *   num_splits: as gqa_decode. A unit is 16 heads of one sequence.
+ *          256-byte aligned, zero-filled before first use, as for gqa_decode (same reuse rules);
+ *          the size depends on dtype and h_q because they select the kernel (below).
+ *   num_splits: as gqa_decode.
+ * Kernels: bf16 with h_q a multiple of 128 runs on the tensor cores (tcgen05): a unit is 128 heads
+ * of one sequence, and each chunk of keys runs on two CTAs, one per half of the d_v value columns.
+ * With automatic chunking and every sequence at the same visible length, each sequence is cut into
+ * equal chunks that divide it (no chunk holds parts of two sequences). Otherwise a unit is 16 heads
+ * (m16n8k16 tensor-core MMAs). The fp32 check mode uses 16-head units too.
  * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA.
  */
 size_t gqa_mla_decode_workspace_size(int B, int h_q, int T_max, int d_v, gqa_dtype dtype,

@@ -150,3 +150,22 @@ def test_mla_decode_128_heads_equal_lengths_aligned_chunks():
     assert gqa.get_device_error() == 0
     assert_bf16_close(_f64(o), ref, "mla 128 heads, equal lengths")
     assert np.abs(lse.cpu().double().numpy() - lref).max() < 2e-2
+
+
+def test_mla_decode_128_heads_more_chunks_than_pairs():
+    """200 explicit splits of 2 ragged sequences (NaN past each length) on the tensor-core kernel:
+    more chunks than CTA pairs, so each pair walks several chunks in turn, every chunk a piece of
+    its own with a query copy, early tiles and a partial epilogue, and rows merge up to ~120
+    partials."""
+    import kv_cache_attention_gqa_b200 as gqa
+
+    shape = workloads.MlaShape(B=2, h_q=128, T_max=2500)
+    lens = [2500, 1733]
+    q, cache, kl = workloads.mla_decode_inputs(shape, seed=57, lengths=lens)
+    ref, lref = mla_ref.mla_decode_ref(_f64(q), _f64(cache), 512, kv_len=np.array(lens), scale=shape.scale)
+    for rep in range(2):
+        o, lse = gqa.mla_decode(q.cuda(), cache.cuda(), kv_len=lens, scale=shape.scale, num_splits=200,
+                                return_lse=True)
+        assert gqa.get_device_error() == 0
+        assert_bf16_close(_f64(o), ref, f"mla 128 heads, 200 splits, call {rep}")
+        assert np.abs(lse.cpu().double().numpy() - lref).max() < 2e-2

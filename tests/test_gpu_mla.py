@@ -169,3 +169,26 @@ def test_mla_decode_128_heads_more_chunks_than_pairs():
         assert gqa.get_device_error() == 0
         assert_bf16_close(_f64(o), ref, f"mla 128 heads, 200 splits, call {rep}")
         assert np.abs(lse.cpu().double().numpy() - lref).max() < 2e-2
+
+
+def test_mla_decode_128_heads_many_short_sequences_and_an_empty_one():
+    """40 sequences of 1-120 visible keys on the tensor-core kernel: chunks of at least 256 keys hold
+    several sequences each, so a CTA pair runs piece after piece (its next piece's tiles issued
+    early, its query copied before the previous piece's epilogue). One sequence has kv_len = 0: its
+    rows are zeros with lse = -inf and the device error reads GQA_DEVERR_KV_LEN; every other row
+    matches the oracle."""
+    import kv_cache_attention_gqa_b200 as gqa
+
+    rng = np.random.default_rng(61)
+    B, bad = 40, 17
+    lens = rng.integers(1, 121, size=B).astype(np.int32)
+    lens[bad] = 0
+    shape = workloads.MlaShape(B=B, h_q=128, T_max=120)
+    q, cache, _ = workloads.mla_decode_inputs(shape, seed=61, lengths=lens)
+    o, lse = gqa.mla_decode(q.cuda(), cache.cuda(), kv_len=lens.tolist(), scale=shape.scale, return_lse=True)
+    assert gqa.get_device_error() == 1  # GQA_DEVERR_KV_LEN
+    assert o[bad].abs().sum().item() == 0 and torch.isneginf(lse[bad]).all()
+    keep = [b for b in range(B) if b != bad]
+    ref, lref = mla_ref.mla_decode_ref(_f64(q[keep]), _f64(cache[keep]), 512, kv_len=lens[keep], scale=shape.scale)
+    assert_bf16_close(_f64(o[keep]), ref, "mla 128 heads, 39 short sequences")
+    assert np.abs(lse[keep].cpu().double().numpy() - lref).max() < 2e-2

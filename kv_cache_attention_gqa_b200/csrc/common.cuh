@@ -104,7 +104,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigne
 }
 
 // ---------------------------------------------------------------------------------------------
-// TMA (cp.async.bulk.tensor), no multicast
+// TMA (cp.async.bulk.tensor): each CTA loads its own tiles
 // ---------------------------------------------------------------------------------------------
 // Ask for `bytes` of global memory at `p` to be brought into L2 (both 16-byte aligned/multiples);
 // nothing waits for it.

@@ -21,7 +21,7 @@
 //
 // bf16 kernel, warp-specialised. One producer warp takes chunks, writes one small descriptor per
 // 64-key tile into shared memory, and streams the tile's K and V (and, on the first tile of a
-// piece, the unit's query rows) with TMA (cp.async.bulk.tensor, 128-byte swizzle, no multicast)
+// piece, the unit's query rows) with TMA (cp.async.bulk.tensor, 128-byte swizzle, each CTA its own copies)
 // into a 5-stage (one m-tile) or 4-stage (two) ring guarded by mbarriers. Four consumer warps per
 // 16-row m-tile each take 16 keys
 // of every tile: S = Q K^T and O += P V run on the tensor cores as m16n8k16 bf16 MMAs with fp32

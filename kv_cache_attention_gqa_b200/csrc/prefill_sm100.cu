@@ -23,7 +23,7 @@
 //
 // Roles (384 threads, three warpgroups):
 //   warp 0      TMA producer: the Q rows once, then 128-key K blocks into a 3-deep ring and
-//               V blocks into a 2-deep ring (cp.async.bulk.tensor, 128-byte swizzle, no multicast).
+//               V blocks into a 2-deep ring (cp.async.bulk.tensor, 128-byte swizzle, each CTA its own copies).
 //   warp 1+t    issues the MMAs of tile t (warp 1 also allocates the 512 TMEM columns):
 //               S_t = Q_t K_j^T (tcgen05.mma kind::f16, A = Q_t and B = K_j from shared memory),
 //               O_t += P_t V_j  (A = P_t from TMEM, B = V_j from shared memory, MN-major).

@@ -394,7 +394,9 @@ __host__ __device__ inline int merge_slices(int D) { return D > 256 ? (D + 127) 
 
 // Merge paths by row width, one kernel each so that each carries only its own registers (the
 // 8-column path keeps twice the loads in flight): 0 for d <= 128 (4 columns per lane), 1 for
-// d <= 256 (8, lane-strided), 2 for wider rows (4 columns per lane, one warp per 128-column slice).
+// d <= 256 (8, lane-strided), 2 for wider rows (4 columns per lane, one warp per 128-column slice,
+// 8 partials per round so that four blocks fit an SM), 3 the same with 16 partials per round for
+// launches small enough to fit one wave anyway (rows with many partials then take fewer rounds).
 __host__ __device__ inline int merge_path(int D) { return D % 4 == 0 && D <= 128 ? 0 : D <= 256 ? 1 : 2; }
 
 template <typename OutT, bool kFast, int kPath>
@@ -442,7 +444,8 @@ __global__ void __launch_bounds__(256, kPath == 2 ? 4 : 1) merge_kernel(KArgs a)
   const long long li = (long long)b * a.h_q + head;
   if constexpr (kPath == 0) merge_row<OutT, kFast, 4, 16>(a, lane, unit, h, c0, c1, ob, li, 0);
   else if constexpr (kPath == 1) merge_row<OutT, kFast, 8, 16>(a, lane, unit, h, c0, c1, ob, li, 0);
-  else merge_row<OutT, kFast, 4, 8>(a, lane, unit, h, c0, c1, ob, li, slice * 128);
+  else if constexpr (kPath == 2) merge_row<OutT, kFast, 4, 8>(a, lane, unit, h, c0, c1, ob, li, slice * 128);
+  else merge_row<OutT, kFast, 4, 16>(a, lane, unit, h, c0, c1, ob, li, slice * 128);
 }
 
 // =============================================================================================
@@ -1880,10 +1883,12 @@ cudaError_t launch_merge(const KArgs& ka, cudaStream_t s) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  const int path = merge_path(ka.D);
-  void (*kern)(KArgs) = path == 0 ? merge_kernel<OutT, kFast, 0>
+  int path = merge_path(ka.D);
+  if (path == 2 && rows <= 2048) path = 3;  // 256 blocks: one wave at two blocks per SM
+  void (*kern)(KArgs) = path == 0   ? merge_kernel<OutT, kFast, 0>
                         : path == 1 ? merge_kernel<OutT, kFast, 1>
-                                    : merge_kernel<OutT, kFast, 2>;
+                        : path == 2 ? merge_kernel<OutT, kFast, 2>
+                                    : merge_kernel<OutT, kFast, 3>;
   cudaError_t e = cudaLaunchKernelEx(&cfg, kern, ka);
   if (e != cudaSuccess) {
     // programmatic dependent launch refused (e.g. on a stream that does not support it): fall

@@ -132,6 +132,24 @@ def test_workspace_size(lib):
     assert a >= (148 + 64) * 4 * 129 * 4 + 64 * 4
 
 
+def test_mla_workspace_size_follows_the_kernel_the_call_selects(lib):
+    """With explicit splits the size needs no device. bf16 with a multiple of 128 heads runs the
+    tensor-core kernel (units of 128 heads, one partial row per head of a unit); fp32 and other
+    head counts run 16-head units. Layout: a 256-byte header, the prefix sums and lengths of the
+    sequences, then (splits + units) partial slots of lse and of d_v floats per unit head, each
+    region 256-byte aligned."""
+    def expected(B, units, hpu, d_v, splits):
+        al = lambda x: (x + 255) // 256 * 256  # noqa: E731
+        slots = splits + units
+        return 256 + al((B + 1) * 8) + al(B * 4) + al(slots * hpu * 4) + slots * hpu * d_v * 4
+
+    bf16, fp32 = 0, 1
+    assert lib.gqa_mla_decode_workspace_size(8, 128, 8192, 512, bf16, 200) == expected(8, 8, 128, 512, 200)
+    assert lib.gqa_mla_decode_workspace_size(8, 256, 8192, 512, bf16, 7) == expected(8, 16, 128, 512, 7)
+    assert lib.gqa_mla_decode_workspace_size(8, 16, 8192, 512, bf16, 7) == expected(8, 8, 16, 512, 7)
+    assert lib.gqa_mla_decode_workspace_size(8, 128, 8192, 512, fp32, 7) == expected(8, 64, 16, 512, 7)
+
+
 def test_paged_host_side_argument_errors(lib):
     """gqa_decode_paged / kv_append_paged reject bad page geometry before any CUDA call."""
     P = ctypes.c_void_p
